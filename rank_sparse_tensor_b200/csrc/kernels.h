@@ -1,0 +1,63 @@
+// Host-side launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tgd {
+
+struct AdamConst;
+
+// ---- select.cu: Omega selection and index structures
+size_t select_workspace_bytes(int64_t n);
+cudaError_t select_topk(const void* g, int dt, int64_t n, int64_t k, int64_t* out_idx,
+                        float* out_val, void* ws, cudaStream_t s);
+cudaError_t select_random(uint64_t seed, uint64_t ordinal, const void* g, int dt, int64_t n,
+                          int64_t k, int64_t* out_idx, float* out_val, void* ws,
+                          cudaStream_t s);
+cudaError_t build_mask_bits(const int64_t* omega, int64_t k, int64_t n, uint32_t* bits,
+                            cudaStream_t s);
+cudaError_t build_tile_index(const int64_t* omega, int64_t k, int64_t tile_elems,
+                             int64_t n_tiles, int64_t* tile_off, uint16_t* loc, cudaStream_t s);
+
+// ---- gram_eig.cu: refresh of the factors
+// Gram of mode n of the masked gradient (shape dims[0..nd), storage dtype dt,
+// Omega bitmask `bits`), accumulated in fp32 partials and summed in fp64
+// into gram (I_n x I_n complex, interleaved doubles).
+size_t gram_partial_bytes(int nd, const int64_t* dims, int n);
+cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
+                      int n, float* partial, double* gram, cudaStream_t s);
+
+struct EigJob {
+  const double* gram;  // n x n complex (interleaved doubles)
+  double* work;        // 2 * n * n complex doubles of global scratch (used when n > 64)
+  float* U;            // out: n x r complex fp32, row-major
+  double* evals;       // out: n eigenvalues, descending
+  int n, r;
+};
+size_t eig_work_doubles(int n);
+cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
+
+// ---- step_generic.cu: CUDA-core path of the step
+cudaError_t sparse_adam(const void* g, int dt, const int64_t* omega, int64_t k, float* m,
+                        float* v, const AdamConst& a, float* upd, cudaStream_t s);
+// Y = X x_n M: X (A, K, B), M (J x K) row-major complex or real, Y (A, J, B).
+// src_dt >= 0: X is the storage-typed gradient, masked by `bits`; src_dt < 0:
+// X is fp32 (float2 when cplx).
+cudaError_t mode_product(const void* X, int src_dt, const uint32_t* bits, bool cplx, int64_t A,
+                         int64_t K, int64_t B, const float* M, int64_t J, float* Y,
+                         cudaStream_t s);
+cudaError_t masked_copy(const void* g, int dt, const uint32_t* bits, int64_t n, float* out,
+                        cudaStream_t s);
+cudaError_t core_adam(float* c, int64_t n, float* m, float* v, const AdamConst& a,
+                      cudaStream_t s);
+cudaError_t scatter_add(float* L, bool cplx, const int64_t* omega, int64_t k, const float* upd,
+                        cudaStream_t s);
+cudaError_t weight_update(void* w, int dt, const float* L, int64_t n, float decay, float lr,
+                          cudaStream_t s);
+// Projection (r x I, conj(U)^T) and expansion (I x r, U) coefficient matrices
+// from U (I x r, complex fp32); real tensors get real matrices.
+cudaError_t coef_matrices(const float* U, int64_t I, int64_t r, bool cplx, float* P, float* E,
+                          cudaStream_t s);
+
+}  // namespace tgd

@@ -1,0 +1,37 @@
+// Tensor-core (tcgen05) path of the TensorGRaD step for complex fp16 tensors.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tgd {
+
+struct AdamConst;
+
+typedef bool (*AllocFn)(void* ctx, void** p, size_t bytes);
+
+// Geometry and device buffers of the tensor-core path (see step_tc.cu).
+struct TcPlan {
+  int d = 0;
+  int64_t I[8] = {}, r[8] = {};
+  int64_t N = 0, k = 0, ncore = 0;
+  int gdt = 0, wdt = 0;
+  bool ready = false;
+  void* impl = nullptr;  // owned by step_tc.cu (host-side description)
+};
+
+bool tc_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt);
+bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
+             int wdt, AllocFn alloc, void* ctx);
+void tc_release(TcPlan& p);
+cudaError_t tc_rebuild(TcPlan& p, const int64_t* omega, int64_t k, const float* const* U,
+                       cudaStream_t s);
+cudaError_t tc_step(TcPlan& p, const void* g, void* w, float* sp_m, float* sp_v, float* core_m,
+                    float* core_v, const AdamConst& asp, const AdamConst& acore, float decay,
+                    float lr, int* d_err, cudaStream_t s);
+// Core moments are stored in the path's internal layout; these convert
+// to/from the canonical row-major r_1 x ... x r_d layout (host buffers).
+cudaError_t tc_core_to_canonical(const TcPlan& p, const float* dev, int comps, float* host_out);
+cudaError_t tc_core_from_canonical(const TcPlan& p, const float* host_in, int comps, float* dev);
+
+}  // namespace tgd
