@@ -74,6 +74,7 @@ struct tgd_ctx {
   std::vector<cudaEvent_t> ev_pool;
   size_t ev_used = 0;
   std::vector<std::pair<std::string, std::pair<cudaEvent_t, cudaEvent_t>>> prof;
+  cudaEvent_t hook_start = nullptr;
 };
 
 namespace {
@@ -106,6 +107,23 @@ struct KTimer {
     h->prof.push_back({name, {a, b}});
   }
 };
+// Timing hook for launch sequences that live in other translation units.
+void timer_hook(void* ctx, int phase, const char* name, cudaStream_t s) {
+  tgd_ctx* h = (tgd_ctx*)ctx;
+  if (!h->prof_on) return;
+  if (phase == 0) {
+    h->hook_start = next_event(h);
+    if (h->hook_start) cudaEventRecord(h->hook_start, s);
+  } else if (h->hook_start) {
+    cudaEvent_t b = next_event(h);
+    if (b) {
+      cudaEventRecord(b, s);
+      h->prof.push_back({name, {h->hook_start, b}});
+    }
+    h->hook_start = nullptr;
+  }
+}
+
 #define TGD_CAT2(a, b) a##b
 #define TGD_CAT(a, b) TGD_CAT2(a, b)
 #define TIMED(h, s, name) KTimer TGD_CAT(kt_, __LINE__)((h), (s), (name))
@@ -160,6 +178,7 @@ bool dalloc_t(tgd_ctx* h, T** p, size_t count) {
 }
 
 void free_all(tgd_ctx* h) {
+  tc_release(h->tc);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   h->ev_pool.clear();
   for (void* p : h->allocs) cudaFree(p);
@@ -492,7 +511,7 @@ tgd_status tgd_step(tgd_handle h, const void* grad, void* weight, void* stream) 
     AdamConst acore = adam_const(h, 1.0);
     float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
     cudaError_t e = tc_step(h->tc, grad, weight, h->sp_m, h->sp_v, h->core_m, h->core_v, asp, acore,
-                            decay, h->lr, h->d_err, s);
+                            decay, h->lr, h->d_err, s, timer_hook, h);
     st = e == cudaSuccess ? TGD_OK : cuda_fail(h, e, "tensor-core step");
   }
   if (st != TGD_OK) return st;

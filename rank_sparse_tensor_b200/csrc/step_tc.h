@@ -9,6 +9,8 @@ namespace tgd {
 struct AdamConst;
 
 typedef bool (*AllocFn)(void* ctx, void** p, size_t bytes);
+// Called before (phase 0) and after (phase 1) each kernel launch, for timing.
+typedef void (*TimerHook)(void* ctx, int phase, const char* name, cudaStream_t s);
 
 // Geometry and device buffers of the tensor-core path (see step_tc.cu).
 struct TcPlan {
@@ -28,7 +30,7 @@ cudaError_t tc_rebuild(TcPlan& p, const int64_t* omega, int64_t k, const float* 
                        cudaStream_t s);
 cudaError_t tc_step(TcPlan& p, const void* g, void* w, float* sp_m, float* sp_v, float* core_m,
                     float* core_v, const AdamConst& asp, const AdamConst& acore, float decay,
-                    float lr, int* d_err, cudaStream_t s);
+                    float lr, int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx);
 // Core moments are stored in the path's internal layout; these convert
 // to/from the canonical row-major r_1 x ... x r_d layout (host buffers).
 cudaError_t tc_core_to_canonical(const TcPlan& p, const float* dev, int comps, float* host_out);
