@@ -202,11 +202,22 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "generic", "tcgen05"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide the leading mode (and its rank) by this factor: small "
+                         "cases of the same kernels, for profiler captures only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    import dataclasses
     from rank_sparse_tensor_b200.synth import WORKLOADS
     wl = WORKLOADS[args.workload]
+    if args.shrink > 1:
+        sh, rk, gr = list(wl.shape), list(wl.ranks), list(wl.gen_ranks)
+        sh[0] //= args.shrink
+        rk[0] = max(1, rk[0] // args.shrink)
+        gr[0] = max(1, gr[0] // args.shrink)
+        wl = dataclasses.replace(wl, name=f"{wl.name}/shrink{args.shrink}", shape=tuple(sh),
+                                 ranks=tuple(rk), gen_ranks=tuple(gr))
     if args.impl == "reference":
         return run_reference(args, wl)
 

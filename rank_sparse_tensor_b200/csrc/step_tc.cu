@@ -71,18 +71,50 @@ __host__ __device__ __forceinline__ uint32_t kmaj_off(uint32_t row, uint32_t k, 
 }
 
 constexpr uint32_t LBO_M128 = 2048;         // 128 rows: 16 groups x 128 B
-constexpr uint32_t LBO_M128_PAD = 2048 + 16; // the same plus 16 B: spreads banks
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 
 // ----------------------------------------------------------- projection
-constexpr int P1T = 128;
-constexpr int PF = 4;
+// Bounded wait for one thread. Gives up when another role has aborted or
+// after WAIT_NS, setting the CTA's abort flag and the device error word.
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  // sleep in the barrier (no issue slots) until the phase completes
+  while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
+    if (*abort) return false;
+    if (global_ns() - t0 > WAIT_NS) {
+      *abort = 1;
+      atomicOr(err, DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// The same for a whole warp: lane 0 polls, the warp re-converges after.
+__device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait1(bar, parity, abort, err) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+constexpr int P1T = 512;
+constexpr int PF = 4;  // Omega entries per converter thread prefetched for the next tile
 
 struct P1Args {
   const uint32_t* G;
   int64_t N, n_slabs, n_tiles, n_groups, tile_elems;
-  int Ia, Ib, ra, rb, spb, q, sg;
+  int Ia, Ib, ra, rb, spb, q, sg, log2Ia;
   int K1, N1, K2, N2;
+  uint32_t lbo_a2;  // GEMM2's A: 64 or 128 physical rows (see geometry)
+  uint32_t d1_col[2], d2_col;
   const int64_t* tile_off;
   const uint16_t* loc;
   float* sp_m;
@@ -94,48 +126,85 @@ struct P1Args {
   void* Y;
   int y_f32;
   int* err;
-  uint32_t off_stage0, off_stage1, off_A1, off_A2, off_B1, off_B2, off_bar;
+  int nstage;
+  uint32_t off_stage, stage_bytes, off_A1, off_A2, off_B1, off_B2, off_bar;
 };
 
+// Position in this CTA's tile sequence: groups blockIdx.x, +gridDim.x, ...,
+// q tiles each; advanced incrementally (no divisions).
+struct TileCursor {
+  int64_t g;
+  int i;
+  __device__ __forceinline__ int64_t tile(int q) const { return g * q + i; }
+  __device__ __forceinline__ void next(int q) {
+    if (++i == q) {
+      i = 0;
+      g += gridDim.x;
+    }
+  }
+};
+
+// Warp-specialised projection stream, one CTA per SM, persistent over groups
+// of q tiles:
+//   warp 0   producer: bulk copies of G tiles into a ring of stages;
+//   warp 1   MMA issuer: GEMM1(t) = A1 x B1 -> D1[t&1]; per group GEMM2 =
+//            A2 x B2 -> D2;
+//   warps 4-11  converters: sparse pass on Omega (gather, zero the entry,
+//            sparse AdamW) and the residual tile into GEMM1's A operand;
+//   warps 12-15 epilogue: P(t) from D1 into the group's GEMM2 operand; Y of
+//            the group from D2 to global memory.
+// Roles hand off through mbarriers.
 __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* stage[2] = {smem + p.off_stage0, smem + p.off_stage1};
   uint8_t* A1 = smem + p.off_A1;
   uint8_t* A2 = smem + p.off_A2;
   uint8_t* B1 = smem + p.off_B1;
   uint8_t* B2 = smem + p.off_B2;
-  uint64_t* bars = (uint64_t*)(smem + p.off_bar);  // 0 factors, 1-2 stages, 3 gemm1, 4 gemm2
-  uint32_t* tslot = (uint32_t*)(bars + 8);
-  __shared__ int s_abort;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  uint64_t* bars = (uint64_t*)(smem + p.off_bar);
+  uint64_t* full = bars;          // [4] stage loaded (1 + tx)
+  uint64_t* sempty = bars + 4;    // [4] stage consumed (256)
+  uint64_t* opnd = bars + 8;      // B1 + B2 loaded
+  uint64_t* a1full = bars + 9;    // (256)
+  uint64_t* a1empty = bars + 10;  // (commit)
+  uint64_t* d1full = bars + 11;   // [2] (commit)
+  uint64_t* d1empty = bars + 13;  // [2] (128)
+  uint64_t* a2full = bars + 15;   // (128)
+  uint64_t* d2full = bars + 16;   // (commit)
+  uint32_t* tslot = (uint32_t*)(bars + 18);
+  __shared__ int s_abort_storage;
+  volatile int* s_abort = &s_abort_storage;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q = p.q, ns = p.nstage;
 
   const int64_t my_groups =
       p.n_groups > (int64_t)blockIdx.x ? (p.n_groups - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  int64_t n_it = my_groups * p.q;
+  int64_t n_it = my_groups * q;
   if (my_groups > 0) {
     int64_t last_g = blockIdx.x + (my_groups - 1) * gridDim.x;
-    int64_t last_tiles = p.n_tiles - last_g * p.q;
-    if (last_tiles < p.q) n_it -= p.q - last_tiles;
+    int64_t last_tiles = p.n_tiles - last_g * q;
+    if (last_tiles < q) n_it -= q - last_tiles;
   }
-  auto tile_at = [&](int64_t it) -> int64_t {
-    return (blockIdx.x + (it / p.q) * gridDim.x) * p.q + it % p.q;
-  };
-  auto group_at = [&](int64_t it) -> int64_t { return blockIdx.x + (it / p.q) * gridDim.x; };
-  auto is_last = [&](int64_t it) -> bool { return (it % p.q == p.q - 1) || (it == n_it - 1); };
-  auto tile_bytes = [&](int64_t t) -> uint32_t {
-    int64_t rem = p.N - t * p.tile_elems;
-    return (uint32_t)((rem < p.tile_elems ? rem : p.tile_elems) * 4);
-  };
+  auto stage = [&](int s) { return smem + p.off_stage + (uint32_t)s * p.stage_bytes; };
 
   if (tid == 0) {
-    s_abort = 0;
-    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+    *s_abort = 0;
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&sempty[i], 256);
+    }
+    mbar_init(opnd, 1);
+    mbar_init(a1full, 256);
+    mbar_init(a1empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&d1full[b], 1);
+      mbar_init(&d1empty[b], 128);
+    }
+    mbar_init(a2full, 128);
+    mbar_init(d2full, 1);
     fence_mbar_init();
   }
   {
-    const uint32_t a1b = (uint32_t)(p.K1 / 8) * LBO_M128, a2b = (uint32_t)(p.K2 / 8) * LBO_M128_PAD;
-    for (uint32_t i = tid; i < a1b / 16; i += P1T) ((uint4*)A1)[i] = make_uint4(0, 0, 0, 0);
+    const uint32_t a2b = (uint32_t)(p.K2 / 8) * p.lbo_a2;
     for (uint32_t i = tid; i < a2b / 16; i += P1T) ((uint4*)A2)[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
@@ -144,236 +213,264 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t d1 = tmem, d2 = tmem + 256;
 
-  // thread 0's record of outstanding asynchronous work, for a bounded drain
-  uint32_t ld_issued[2] = {0, 0}, ld_waited[2] = {0, 0};
-  uint32_t m1_issued = 0, m2_issued = 0;
-  if (tid == 0) {
-    uint32_t b1 = (uint32_t)(p.N1 * p.K1 * 2), b2 = (uint32_t)(p.N2 * p.K2 * 2);
-    mbar_expect_tx(&bars[0], b1 + b2);
-    bulk_g2s(B1, p.B1img, b1, &bars[0]);
-    bulk_g2s(B2, p.B2img, b2, &bars[0]);
-    for (int s = 0; s < 2 && s < n_it; ++s) {
-      int64_t t = tile_at(s);
-      uint32_t nb = tile_bytes(t);
-      mbar_expect_tx(&bars[1 + s], nb);
-      bulk_g2s(stage[s], p.G + t * p.tile_elems, nb, &bars[1 + s]);
-      ld_issued[s]++;
-    }
-  }
-  // Every wait is bounded; the abort decision is made uniform by a barrier so
-  // that warp-collective tcgen05 instructions never run in a divergent warp.
-  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (!mbar_wait(bar, parity, WAIT_NS)) {
-      atomicOr(p.err, DEV_ERR_TIMEOUT);
-      s_abort = 1;
-    }
-    __syncthreads();
-    return s_abort == 0;
-  };
-  wait_all(&bars[0], 0);
-
-  const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
-  const uint32_t id1 = idesc_f16(0, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
-  const uint32_t sA1 = smem_u32(A1), sA2 = smem_u32(A2), sB1 = smem_u32(B1), sB2 = smem_u32(B2);
-  const int vc = p.asp.cmode == 1 ? 2 : 1;
-
-  // Omega entries of the next tile, prefetched into registers one tile ahead.
-  int64_t pf_e0 = 0, pf_e1 = 0;
-  uint32_t pf_loc[PF];
-  float2 pf_m[PF], pf_v[PF];
-  auto load_pf = [&](int64_t t) {
-    pf_e0 = p.tile_off[t];
-    pf_e1 = p.tile_off[t + 1];
-#pragma unroll
-    for (int j = 0; j < PF; ++j) {
-      int64_t e = pf_e0 + tid + (int64_t)P1T * j;
-      if (e < pf_e1) {
-        pf_loc[j] = p.loc[e];
-        pf_m[j] = ((const float2*)p.sp_m)[e];
-        pf_v[j] = vc == 2 ? ((const float2*)p.sp_v)[e] : make_float2(p.sp_v[e], 0.f);
-      }
-    }
-  };
-  auto apply_sparse = [&](uint32_t* sw, int64_t e, uint32_t l, float2 m, float2 v) {
-    uint32_t u = sw[l];
-    sw[l] = 0u;
-    float mm[2] = {m.x, m.y}, vv[2] = {v.x, v.y};
-    float2 upd = adam_elem(h2_to_f2(u), mm, vv, p.asp);
-    ((float2*)p.sp_m)[e] = make_float2(mm[0], mm[1]);
-    if (vc == 2)
-      ((float2*)p.sp_v)[e] = make_float2(vv[0], vv[1]);
-    else
-      p.sp_v[e] = vv[0];
-    p.sp_upd[e] = f2_to_h2(upd);
-  };
-
-  auto epilogue1 = [&](int64_t it) {
-    const int64_t t = tile_at(it);
-    const int i = (int)(it % p.q);
-    const int m = tid, sl = m / p.Ia, ia = m - sl * p.Ia;
-    const bool valid = t * p.spb + sl < p.n_slabs;
-    const int m2base = (i * p.spb + sl) * p.rb;
-    for (int c0 = 0; c0 < p.N1; c0 += 16) {
-      float v[16];
-      tmem_ld16(d1 + lane_base + c0, v);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        int jb = c0 / 2 + u;
-        if (valid && jb < p.rb) {
-          uint32_t off = kmaj_off((uint32_t)(m2base + jb), (uint32_t)(2 * ia), LBO_M128_PAD);
-          *(uint32_t*)(A2 + off) = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t b1 = (uint32_t)(p.N1 * p.K1 * 2), b2 = (uint32_t)(p.N2 * p.K2 * 2);
+      mbar_expect_tx(opnd, b1 + b2);
+      bulk_g2s(B1, p.B1img, b1, opnd);
+      bulk_g2s(B2, p.B2img, b2, opnd);
+      TileCursor c{(int64_t)blockIdx.x, 0};
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t it = 0; it < n_it; ++it) {
+        if (!wait1(&sempty[s], ph ^ 1u, s_abort, p.err)) break;
+        const int64_t t = c.tile(q);
+        const int64_t rem = p.N - t * p.tile_elems;
+        const uint32_t nb = (uint32_t)((rem < p.tile_elems ? rem : p.tile_elems) * 4);
+        mbar_expect_tx(&full[s], nb);
+        bulk_g2s(stage(s), p.G + t * p.tile_elems, nb, &full[s]);
+        ++issued;
+        c.next(q);
+        if (++s == ns) {
+          s = 0;
+          ph ^= 1u;
         }
       }
-    }
-  };
-  auto epilogue2 = [&](int64_t g) {
-    const int m2 = tid, sb = m2 / p.rb, jb = m2 - sb * p.rb;
-    const int64_t slab = g * p.sg + sb;
-    const bool valid = m2 < p.sg * p.rb && slab < p.n_slabs;
-    const int64_t ybase = (slab * p.rb + jb) * p.ra;
-    for (int c0 = 0; c0 < p.N2; c0 += 16) {
-      float v[16];
-      tmem_ld16(d2 + lane_base + c0, v);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        int ja = c0 / 2 + u;
-        if (valid && ja < p.ra) {
-          if (p.y_f32)
-            ((float2*)p.Y)[ybase + ja] = make_float2(v[2 * u], v[2 * u + 1]);
-          else
-            ((uint32_t*)p.Y)[ybase + ja] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
-        }
+      if (*s_abort) {
+        // wait (bounded) for the copies still in flight before the CTA exits
+        for (int64_t it = 0; it < issued; ++it) mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
       }
     }
-  };
-  auto issue_gemm1 = [&]() {
-    for (int kk = 0; kk < p.K1 / 16; ++kk)
-      mma_f16(d1, sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
-              sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
-    mma_commit(&bars[3]);
-  };
-  auto issue_gemm2 = [&]() {
-    for (int kk = 0; kk < p.K2 / 16; ++kk)
-      mma_f16(d2, sdesc(sA2 + kk * 2 * LBO_M128_PAD, LBO_M128_PAD, 128),
-              sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
-    mma_commit(&bars[4]);
-  };
-
-  uint32_t m1_waited = 0, m2_waited = 0;
-  if (n_it > 0 && !s_abort) load_pf(tile_at(0));
-  __syncthreads();
-  for (int64_t it = 0; it < n_it && !s_abort; ++it) {
-    const int s = (int)(it & 1);
-    const int64_t t = tile_at(it);
-    uint32_t* sw = (uint32_t*)stage[s];
-    const bool got = wait_all(&bars[1 + s], (uint32_t)((it >> 1) & 1));
-    if (tid == 0) ld_waited[s]++;
-    if (!got) break;
-    {
-      // sparse pass: gather, residual, sparse AdamW
-      const int64_t e0 = pf_e0, e1 = pf_e1;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
+      const uint32_t id1 = idesc_f16(0, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
+      const uint32_t sA1 = smem_u32(A1), sA2 = smem_u32(A2), sB1 = smem_u32(B1), sB2 = smem_u32(B2);
+      bool ok = wait1(opnd, 0, s_abort, p.err);
+      TileCursor c{(int64_t)blockIdx.x, 0};
+      int64_t g1_next = 0;      // next tile to run GEMM1 on
+      int64_t groups_done = 0;  // GEMM2s issued
+      int64_t groups_ready = 0; // groups whose last GEMM1 is issued
+      uint32_t a2par = 0;
+      uint64_t t0 = global_ns();
+      while (ok && (g1_next < n_it || groups_done < groups_ready)) {
+        bool progressed = false;
+        // GEMM2 of a complete group, as soon as its operand is written
+        if (groups_done < groups_ready && mbar_try_wait(a2full, a2par)) {
+          tc_fence_after();
+          for (int kk = 0; kk < p.K2 / 16; ++kk)
+            mma_f16(tmem + p.d2_col, sdesc(sA2 + kk * 2 * p.lbo_a2, p.lbo_a2, 128),
+                    sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
+          mma_commit(d2full);
+          a2par ^= 1u;
+          ++groups_done;
+          progressed = true;
+        }
+        if (g1_next < n_it) {
+          const int b = (int)(g1_next & 1);
+          const uint32_t par = (uint32_t)((g1_next >> 1) & 1);
+          if (mbar_try_wait(a1full, (uint32_t)(g1_next & 1)) && mbar_try_wait(&d1empty[b], par ^ 1u)) {
+            tc_fence_after();
+            for (int kk = 0; kk < p.K1 / 16; ++kk)
+              mma_f16(tmem + p.d1_col[b], sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
+                      sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
+            mma_commit(&d1full[b]);
+            mma_commit(a1empty);
+            const bool last = c.i == q - 1 || g1_next == n_it - 1;
+            if (last) ++groups_ready;
+            ++g1_next;
+            c.next(q);
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t0 = global_ns();
+        } else {
+          __nanosleep(64);
+          if (*s_abort) break;
+          if (global_ns() - t0 > WAIT_NS) {  // no progress for WAIT_NS
+            *s_abort = 1;
+            atomicOr(p.err, DEV_ERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+      if (*s_abort) {
+        // bounded wait for the last MMAs before TMEM is released
+        if (g1_next > 0) mbar_wait(&d1full[(g1_next - 1) & 1], (uint32_t)(((g1_next - 1) >> 1) & 1), WAIT_NS / 4);
+        if (groups_done > 0) mbar_wait(d2full, (a2par ^ 1u), WAIT_NS / 4);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ converters
+    const int ct = tid - 128;  // 0..255
+    const int row = ct & 127, half = ct >> 7;
+    const int vc = p.asp.cmode == 1 ? 2 : 1;
+    const int sl_row = row >> p.log2Ia;
+    const int Ib = p.Ib, nk = p.K1 / 8;
+    int64_t cur_e0 = 0, cur_e1 = 0, nx_e0 = 0, nx_e1 = 0, nn_e0 = 0, nn_e1 = 0;
+    uint32_t pf_loc[PF];
+    float2 pf_m[PF], pf_v[PF];
+    auto load_entries = [&](int64_t e0, int64_t e1) {
 #pragma unroll
       for (int j = 0; j < PF; ++j) {
-        int64_t e = e0 + tid + (int64_t)P1T * j;
-        if (e < e1) apply_sparse(sw, e, pf_loc[j], pf_m[j], pf_v[j]);
+        int64_t e = e0 + ct + 256 * j;
+        if (e < e1) {
+          pf_loc[j] = p.loc[e];
+          pf_m[j] = ((const float2*)p.sp_m)[e];
+          pf_v[j] = vc == 2 ? ((const float2*)p.sp_v)[e] : make_float2(p.sp_v[e], 0.f);
+        }
       }
-      for (int64_t e = e0 + (int64_t)P1T * PF + tid; e < e1; e += P1T) {
+    };
+    auto apply_sparse = [&](uint32_t* sw, int64_t e, uint32_t l, float2 m, float2 v) {
+      uint32_t u = sw[l];
+      sw[l] = 0u;
+      float mm[2] = {m.x, m.y}, vv[2] = {v.x, v.y};
+      float2 upd = adam_elem(h2_to_f2(u), mm, vv, p.asp);
+      ((float2*)p.sp_m)[e] = make_float2(mm[0], mm[1]);
+      if (vc == 2)
+        ((float2*)p.sp_v)[e] = make_float2(vv[0], vv[1]);
+      else
+        p.sp_v[e] = vv[0];
+      p.sp_upd[e] = f2_to_h2(upd);
+    };
+    TileCursor cur{(int64_t)blockIdx.x, 0}, ahead{(int64_t)blockIdx.x, 0};
+    if (n_it > 0) {
+      int64_t t0 = cur.tile(q);
+      cur_e0 = p.tile_off[t0];
+      cur_e1 = p.tile_off[t0 + 1];
+      ahead.next(q);
+      if (n_it > 1) {
+        int64_t t1 = ahead.tile(q);
+        nx_e0 = p.tile_off[t1];
+        nx_e1 = p.tile_off[t1 + 1];
+      }
+      ahead.next(q);
+      load_entries(cur_e0, cur_e1);
+    }
+    int s = 0;
+    uint32_t ph = 0;
+    for (int64_t it = 0; it < n_it; ++it) {
+      const int64_t t = cur.tile(q);
+      if (it + 2 < n_it) {
+        const int64_t t2 = ahead.tile(q);
+        nn_e0 = p.tile_off[t2];
+        nn_e1 = p.tile_off[t2 + 1];
+      }
+      if (!waitw(&full[s], ph, s_abort, p.err)) break;
+      uint32_t* sw = (uint32_t*)stage(s);
+#pragma unroll
+      for (int j = 0; j < PF; ++j) {
+        int64_t e = cur_e0 + ct + 256 * j;
+        if (e < cur_e1) apply_sparse(sw, e, pf_loc[j], pf_m[j], pf_v[j]);
+      }
+      for (int64_t e = cur_e0 + 256 * PF + ct; e < cur_e1; e += 256) {
         float2 m = ((const float2*)p.sp_m)[e];
         float2 v = vc == 2 ? ((const float2*)p.sp_v)[e] : make_float2(p.sp_v[e], 0.f);
         apply_sparse(sw, e, p.loc[e], m, v);
       }
-      if (it + 1 < n_it) load_pf(tile_at(it + 1));
-    }
-    if (it > 0) {
-      const bool ok1 = wait_all(&bars[3], (uint32_t)((it - 1) & 1));
-      m1_waited++;
-      if (!ok1) break;
-      tc_fence_after();
-      epilogue1(it - 1);
-    } else {
-      __syncthreads();
-    }
-    // residual tile -> GEMM1's A operand (row = i_a of a slab, K = (i_b, re/im))
-    {
-      const int m = tid, sl = m / p.Ia;
-      const bool valid = t * p.spb + sl < p.n_slabs;
-      const uint32_t* src = sw + (int64_t)m * p.Ib;
-      for (int kc = 0; kc < p.K1 / 8; ++kc) {
-        uint32_t v[4];
+      if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
+      cur_e0 = nx_e0;
+      cur_e1 = nx_e1;
+      nx_e0 = nn_e0;
+      nx_e1 = nn_e1;
+      named_sync(1, 256);  // every zeroed entry is in place before conversion
+      if (!waitw(a1empty, (uint32_t)((it & 1) ^ 1), s_abort, p.err)) break;
+      // residual tile -> GEMM1's A operand (row = (slab, i_a), K = (i_b, re/im))
+      const bool valid = t * p.spb + sl_row < p.n_slabs;
+      const uint32_t* src = sw + row * Ib;
+      uint8_t* dst = A1 + row * 16;
+      if (valid) {
+        int kc = half;
+        for (; 4 * kc + 3 < Ib; kc += 2)
+          *(uint4*)(dst + kc * LBO_M128) = make_uint4(src[4 * kc], src[4 * kc + 1], src[4 * kc + 2], src[4 * kc + 3]);
+        for (; kc < nk; kc += 2) {
+          uint32_t v[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          int ib = 4 * kc + u;
-          v[u] = (valid && ib < p.Ib) ? src[ib] : 0u;
+          for (int u = 0; u < 4; ++u) v[u] = 4 * kc + u < Ib ? src[4 * kc + u] : 0u;
+          *(uint4*)(dst + kc * LBO_M128) = make_uint4(v[0], v[1], v[2], v[3]);
         }
-        *(uint4*)(A1 + kc * LBO_M128 + m * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+      } else {
+        for (int kc = half; kc < nk; kc += 2) *(uint4*)(dst + kc * LBO_M128) = make_uint4(0, 0, 0, 0);
       }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (s_abort) break;
-    const bool prev_last = it > 0 && is_last(it - 1);
-    if (tid == 0) {
-      if (it + 2 < n_it) {
-        int64_t t2 = tile_at(it + 2);
-        uint32_t nb = tile_bytes(t2);
-        mbar_expect_tx(&bars[1 + s], nb);
-        bulk_g2s(stage[s], p.G + t2 * p.tile_elems, nb, &bars[1 + s]);
-        ld_issued[s]++;
-      }
-      if (prev_last) {
-        issue_gemm2();
-        m2_issued++;
-      }
-      issue_gemm1();
-      m1_issued++;
-    }
-    if (prev_last) {
-      const bool ok2 = wait_all(&bars[4], m2_waited & 1u);
-      m2_waited++;
-      if (!ok2) break;
-      tc_fence_after();
-      epilogue2(group_at(it - 1));
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-    }
-  }
-  __syncthreads();
-  if (n_it > 0 && !s_abort) {
-    const bool ok1 = wait_all(&bars[3], (uint32_t)((n_it - 1) & 1));
-    m1_waited++;
-    if (ok1) {
-      tc_fence_after();
-      epilogue1(n_it - 1);
       fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      if (tid == 0) {
-        issue_gemm2();
-        m2_issued++;
-      }
-      const bool ok2 = wait_all(&bars[4], m2_waited & 1u);
-      m2_waited++;
-      if (ok2) {
-        tc_fence_after();
-        epilogue2(group_at(n_it - 1));
+      mbar_arrive(a1full);
+      mbar_arrive(&sempty[s]);
+      cur.next(q);
+      ahead.next(q);
+      if (++s == ns) {
+        s = 0;
+        ph ^= 1u;
       }
     }
-  }
-  // Bounded drain of anything still in flight (only after a timeout).
-  if (tid == 0 && s_abort) {
-    for (int s = 0; s < 2; ++s)
-      while (ld_waited[s] < ld_issued[s]) {
-        mbar_wait(&bars[1 + s], ld_waited[s] & 1u, WAIT_NS / 4);
-        ld_waited[s]++;
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ epilogue
+    const int row = tid & 127;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int sl_row = row >> p.log2Ia, ia_row = row & (p.Ia - 1);
+    TileCursor c{(int64_t)blockIdx.x, 0};
+    uint32_t d2par = 0;
+    for (int64_t it = 0; it < n_it; ++it) {
+      const int b = (int)(it & 1);
+      const int64_t t = c.tile(q);
+      if (!waitw(&d1full[b], (uint32_t)((it >> 1) & 1), s_abort, p.err)) break;
+      tc_fence_after();
+      // P (fp32, TMEM) -> GEMM2's A operand (bf16), rows (slab in group,
+      // j_b), K = (i_a, re/im)
+      const bool valid = t * p.spb + sl_row < p.n_slabs;
+      const int m2base = (c.i * p.spb + sl_row) * p.rb;
+      for (int c0 = 0; c0 < p.N1; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            int jb = c0 / 2 + u;
+            if (jb < p.rb) {
+              uint32_t off = kmaj_off((uint32_t)(m2base + jb), (uint32_t)(2 * ia_row), p.lbo_a2);
+              *(uint32_t*)(A2 + off) = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+            }
+          }
+        }
       }
-    if (m1_issued > m1_waited) mbar_wait(&bars[3], (m1_issued - 1) & 1u, WAIT_NS / 4);
-    if (m2_issued > m2_waited) mbar_wait(&bars[4], (m2_issued - 1) & 1u, WAIT_NS / 4);
+      tc_fence_before();
+      mbar_arrive(&d1empty[b]);
+      const bool last = c.i == q - 1 || it == n_it - 1;
+      if (last) {
+        fence_async_smem();
+        mbar_arrive(a2full);
+        if (!waitw(d2full, d2par, s_abort, p.err)) break;
+        d2par ^= 1u;
+        tc_fence_after();
+        // Y (row = (slab in group, j_b)) -> global, j_a contiguous
+        const int sb = row / p.rb, jb = row - sb * p.rb;
+        const int64_t slab = c.g * p.sg + sb;
+        const bool yvalid = row < p.sg * p.rb && slab < p.n_slabs;
+        const int64_t ybase = (slab * p.rb + jb) * p.ra;
+        for (int c0 = 0; c0 < p.N2; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + p.d2_col + lane_base + c0, v);
+          if (yvalid) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              int ja = c0 / 2 + u;
+              if (ja < p.ra) {
+                if (p.y_f32)
+                  ((float2*)p.Y)[ybase + ja] = make_float2(v[2 * u], v[2 * u + 1]);
+                else
+                  ((uint32_t*)p.Y)[ybase + ja] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+      }
+      c.next(q);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -430,8 +527,9 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
   const uint32_t idesc = idesc_f16(1, 128, p.NT);
   const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * b_bytes;
   uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
+  // One thread polls (bounded), the rest sleep in the barrier.
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (!mbar_wait(bar, parity, WAIT_NS)) {
+    if (tid == 0 && !mbar_wait(bar, parity, WAIT_NS)) {
       atomicOr(p.err, DEV_ERR_TIMEOUT);
       s_abort = 1;
     }
@@ -525,7 +623,13 @@ __global__ void core_adam_tc_kernel(const float2* C, int64_t n, int64_t blk, int
 }
 
 // ------------------------------------------------------- reconstruction
-constexpr int R3T = 256;
+__device__ __forceinline__ float2 wload(const __half2* p) { return __half22float2(*p); }
+__device__ __forceinline__ void wstore(__half2* p, float x, float y) { *p = __floats2half2_rn(x, y); }
+__device__ __forceinline__ float2 wload(const float2* p) { return *p; }
+__device__ __forceinline__ void wstore(float2* p, float x, float y) { *p = make_float2(x, y); }
+
+constexpr int R3T = 512;
+constexpr int EPF = 4;  // Omega entries per epilogue thread prefetched for the next tile
 
 struct R3Args {
   const uint32_t* Yp;
@@ -533,8 +637,9 @@ struct R3Args {
   void* W;
   int w_c64;
   int64_t N, n_slabs, n_tiles, tile_elems;
-  int Ia, Ib, ra, rb, spb;
+  int Ia, Ib, ra, rb, spb, log2Ia;
   int K1, N1, K2, N2;
+  uint32_t d1_col[2], d2_col[2];
   const int64_t* tile_off;
   const uint16_t* loc;
   const uint32_t* sp_upd;
@@ -544,28 +649,52 @@ struct R3Args {
   int* err;
   int nstage, cap;
   uint32_t w_tile_bytes, y_tile_bytes;
-  uint32_t off_w, off_y, off_A1, off_B1, off_A2, off_B2, off_lloc, off_lval, off_bar;
+  uint32_t off_w, off_y, off_A1, off_B1, off_A2, off_B2, off_ds, off_bar;
 };
 
+// Warp-specialised reconstruction stream, one CTA per SM, persistent over
+// tiles (t = blockIdx.x, +gridDim.x, ...):
+//   warp 0   producer: bulk copies W(t), Y'(t) into a ring of stages, and
+//            bulk-stores each W tile once its epilogue is done;
+//   warp 1   MMA issuer: GEMM1(t) = A1 x B1(t) -> D1[t&1], GEMM2(t) =
+//            A2(t) x B2 -> D2[t&1];
+//   warps 4-7   prep: B1(t+1) from Y'(t+1), the tile's Omega list and
+//            per-row start table, then P'(t) from D1 into A2[t&1];
+//   warps 8-15  epilogue: Delta(t) from D2 + lambda S~ on Omega, AdamW on
+//            the staged W tile (column halves per warpgroup).
+// Roles hand off through mbarriers; operands, lists and accumulators are
+// double-buffered, so consecutive tiles overlap.
+template <class WT>
 __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* A1 = smem + p.off_A1;
-  uint8_t* B1 = smem + p.off_B1;
-  uint8_t* A2 = smem + p.off_A2;
   uint8_t* B2 = smem + p.off_B2;
-  uint16_t* lloc = (uint16_t*)(smem + p.off_lloc);
-  uint32_t* lval = (uint32_t*)(smem + p.off_lval);
-  uint64_t* bars = (uint64_t*)(smem + p.off_bar);  // 0..2 stages, 3 operands, 4 gemm1, 5 gemm2
-  uint32_t* tslot = (uint32_t*)(bars + 8);
-  __shared__ int s_abort;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  uint64_t* bars = (uint64_t*)(smem + p.off_bar);
+  // barrier map
+  uint64_t* full = bars;           // [4] stage loaded
+  uint64_t* wdone = bars + 4;      // [4] W tile updated (256 arrivals)
+  uint64_t* opnd = bars + 8;       // A1 + B2 loaded
+  uint64_t* b1full = bars + 9;     // [2] (128)
+  uint64_t* b1empty = bars + 11;   // [2] (commit)
+  uint64_t* d1full = bars + 13;    // [2] (commit)
+  uint64_t* d1empty = bars + 15;   // [2] (128)
+  uint64_t* a2full = bars + 17;    // [2] (128)
+  uint64_t* a2empty = bars + 19;   // [2] (commit)
+  uint64_t* d2full = bars + 21;    // [2] (commit)
+  uint64_t* d2empty = bars + 23;   // [2] (256)
+  uint32_t* tslot = (uint32_t*)(bars + 26);
+  __shared__ int s_abort_storage;
+  volatile int* s_abort = &s_abort_storage;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_it =
       p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  auto tile_at = [&](int64_t it) -> int64_t { return blockIdx.x + it * gridDim.x; };
+  const int64_t G = gridDim.x;
+  const int ns = p.nstage;
   auto wst = [&](int s) { return smem + p.off_w + (uint32_t)s * p.w_tile_bytes; };
   auto yst = [&](int s) { return smem + p.off_y + (uint32_t)s * p.y_tile_bytes; };
-  const int wb = p.w_c64 ? 8 : 4;
+  auto B1b = [&](int b) { return smem + p.off_B1 + (uint32_t)b * (uint32_t)(p.N1 * p.K1 * 2); };
+  auto A2b = [&](int b) { return smem + p.off_A2 + (uint32_t)b * (uint32_t)(p.K2 / 8) * LBO_M128; };
+  const int wb = (int)sizeof(WT);
   auto tile_wbytes = [&](int64_t t) -> uint32_t {
     int64_t rem = p.N - t * p.tile_elems;
     return (uint32_t)((rem < p.tile_elems ? rem : p.tile_elems) * wb);
@@ -574,15 +703,27 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     int64_t rem = p.n_slabs - t * p.spb;
     return (uint32_t)((rem < p.spb ? rem : p.spb) * p.yp_bs * 4);
   };
+
   if (tid == 0) {
-    s_abort = 0;
-    for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+    *s_abort = 0;
+    for (int i = 0; i < 4; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&wdone[i], 256);
+    mbar_init(opnd, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&b1full[b], 128);
+      mbar_init(&b1empty[b], 1);
+      mbar_init(&d1full[b], 1);
+      mbar_init(&d1empty[b], 128);
+      mbar_init(&a2full[b], 128);
+      mbar_init(&a2empty[b], 1);
+      mbar_init(&d2full[b], 1);
+      mbar_init(&d2empty[b], 256);
+    }
     fence_mbar_init();
   }
   {
-    const uint32_t b1b = (uint32_t)(p.N1 * p.K1 * 2), a2b = (uint32_t)(p.K2 / 8) * LBO_M128;
-    for (uint32_t i = tid; i < b1b / 16; i += R3T) ((uint4*)B1)[i] = make_uint4(0, 0, 0, 0);
-    for (uint32_t i = tid; i < a2b / 16; i += R3T) ((uint4*)A2)[i] = make_uint4(0, 0, 0, 0);
+    const uint32_t b1b = (uint32_t)(2 * p.N1 * p.K1 * 2);
+    for (uint32_t i = tid; i < b1b / 16; i += R3T) ((uint4*)(smem + p.off_B1))[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   if (warp == 0) tmem_alloc(tslot, 512);
@@ -590,184 +731,262 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t d1 = tmem, d2 = tmem + 256;
-  uint32_t ld_issued[3] = {0, 0, 0}, ld_waited[3] = {0, 0, 0};
-  auto issue_loads = [&](int64_t it) {
-    const int s = (int)(it % p.nstage);
-    const int64_t t = tile_at(it);
-    const uint32_t nw = tile_wbytes(t), ny = tile_ybytes(t);
-    mbar_expect_tx(&bars[s], nw + ny);
-    bulk_g2s(wst(s), (const uint8_t*)p.W + t * p.tile_elems * wb, nw, &bars[s]);
-    bulk_g2s(yst(s), p.Yp + t * p.spb * p.yp_bs, ny, &bars[s]);
-    ld_issued[s]++;
-  };
-  if (tid == 0) {
-    const uint32_t a1b = (uint32_t)(p.K1 / 8) * LBO_M128, b2b = (uint32_t)(p.N2 * p.K2 * 2);
-    mbar_expect_tx(&bars[3], a1b + b2b);
-    bulk_g2s(A1, p.A1img, a1b, &bars[3]);
-    bulk_g2s(B2, p.B2img, b2b, &bars[3]);
-    for (int64_t it = 0; it < p.nstage - 1 && it < n_it; ++it) issue_loads(it);
-  }
-  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (!mbar_wait(bar, parity, WAIT_NS)) {
-      atomicOr(p.err, DEV_ERR_TIMEOUT);
-      s_abort = 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t a1b = (uint32_t)(p.K1 / 8) * LBO_M128, b2b = (uint32_t)(p.N2 * p.K2 * 2);
+      mbar_expect_tx(opnd, a1b + b2b);
+      bulk_g2s(A1, p.A1img, a1b, opnd);
+      bulk_g2s(B2, p.B2img, b2b, opnd);
+      auto load = [&](int64_t it) {
+        const int s = (int)(it % ns);
+        const int64_t t = blockIdx.x + it * G;
+        const uint32_t nw = tile_wbytes(t), ny = tile_ybytes(t);
+        mbar_expect_tx(&full[s], nw + ny);
+        bulk_g2s(wst(s), (const uint8_t*)p.W + t * p.tile_elems * wb, nw, &full[s]);
+        bulk_g2s(yst(s), p.Yp + t * p.spb * p.yp_bs, ny, &full[s]);
+      };
+      int64_t loaded = 0;
+      for (; loaded < ns && loaded < n_it; ++loaded) load(loaded);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t it = 0; it < n_it; ++it) {
+        if (!wait1(&wdone[s], ph, s_abort, p.err)) break;
+        const int64_t t = blockIdx.x + it * G;
+        bulk_s2g((uint8_t*)p.W + t * p.tile_elems * wb, wst(s), tile_wbytes(t));
+        bulk_commit();
+        if (loaded < n_it) {
+          bulk_wait_read0();  // the stage's last store has been read out
+          load(loaded++);
+        }
+        if (++s == ns) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (*s_abort) {
+        // wait (bounded) for loads still in flight before the CTA exits
+        for (int64_t it = 0; it < loaded; ++it) mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
+      }
+      bulk_wait_all0();
     }
-    __syncthreads();
-    return s_abort == 0;
-  };
-  wait_all(&bars[3], 0);
-  const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
-  const uint32_t id1 = idesc_f16(1, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
-  const uint32_t sA1 = smem_u32(A1), sB1 = smem_u32(B1), sA2 = smem_u32(A2), sB2 = smem_u32(B2);
-  const int blk = p.rb * p.ra;
-  uint32_t m1_waited = 0, m2_waited = 0, m1_issued = 0, m2_issued = 0;
-  __syncthreads();
-  for (int64_t it = 0; it < n_it && !s_abort; ++it) {
-    const int s = (int)(it % p.nstage);
-    const int64_t t = tile_at(it);
-    const bool got = wait_all(&bars[s], (uint32_t)((it / p.nstage) & 1));
-    if (tid == 0) ld_waited[s]++;
-    if (!got) break;
-    const int64_t e0 = p.tile_off[t], e1 = p.tile_off[t + 1];
-    const int cnt = (int)(e1 - e0);
-    // GEMM1's B operand: the tile's Y' slabs in the embedding [[Yr, Yi], [-Yi, Yr]]
-    {
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
+      const uint32_t id1 = idesc_f16(1, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
+      const uint32_t sA1 = smem_u32(A1), sB2 = smem_u32(B2);
+      bool ok = wait1(opnd, 0, s_abort, p.err);
+      auto gemm1 = [&](int64_t it) -> bool {
+        const int b = (int)(it & 1);
+        const uint32_t par = (uint32_t)((it >> 1) & 1);
+        if (!wait1(&b1full[b], par, s_abort, p.err)) return false;
+        if (!wait1(&d1empty[b], par ^ 1u, s_abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t sB1 = smem_u32(B1b(b));
+        for (int kk = 0; kk < p.K1 / 16; ++kk)
+          mma_f16(tmem + p.d1_col[b], sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
+                  sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
+        mma_commit(&d1full[b]);
+        mma_commit(&b1empty[b]);
+        return true;
+      };
+      int64_t g1_done = 0, g2_done = 0;
+      if (ok && n_it > 0) {
+        ok = gemm1(0);
+        if (ok) g1_done = 1;
+      }
+      for (int64_t it = 0; ok && it < n_it; ++it) {
+        if (it + 1 < n_it) {
+          if (!gemm1(it + 1)) break;
+          g1_done = it + 2;
+        }
+        const int b = (int)(it & 1);
+        const uint32_t par = (uint32_t)((it >> 1) & 1);
+        if (!wait1(&a2full[b], par, s_abort, p.err)) break;
+        if (!wait1(&d2empty[b], par ^ 1u, s_abort, p.err)) break;
+        tc_fence_after();
+        const uint32_t sA2 = smem_u32(A2b(b));
+        for (int kk = 0; kk < p.K2 / 16; ++kk)
+          mma_f16(tmem + p.d2_col[b], sdesc(sA2 + kk * 2 * LBO_M128, LBO_M128, 128),
+                  sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
+        mma_commit(&d2full[b]);
+        mma_commit(&a2empty[b]);
+        g2_done = it + 1;
+      }
+      if (*s_abort) {
+        // bounded wait for the last MMAs before TMEM is released
+        if (g1_done > 0) mbar_wait(&d1full[(g1_done - 1) & 1], (uint32_t)(((g1_done - 1) >> 1) & 1), WAIT_NS / 4);
+        if (g2_done > 0) mbar_wait(&d2full[(g2_done - 1) & 1], (uint32_t)(((g2_done - 1) >> 1) & 1), WAIT_NS / 4);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ prep
+    const int row = tid - 128;  // 0..127, TMEM lane of warps 4-7
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128;
+    const int blk = p.rb * p.ra;
+    bool ok = true;
+    auto build = [&](int64_t it) -> bool {
+      const int b = (int)(it & 1), s = (int)(it % ns);
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
+      const int64_t t = blockIdx.x + it * G;
+      if (!waitw(&full[s], (uint32_t)((it / ns) & 1), s_abort, p.err)) return false;
+      if (!waitw(&b1empty[b], par ^ 1u, s_abort, p.err)) return false;
+      // B1: rows (j_b, re/im), K = (slab, j_a, re/im), entries [[Yr, -Yi], [Yi, Yr]]
+      uint8_t* B1 = B1b(b);
       const uint32_t* ys = (const uint32_t*)yst(s);
       const int64_t vslabs = p.n_slabs - t * p.spb;
-      for (int e = tid; e < p.spb * blk; e += R3T) {
+      for (int e = row; e < p.spb * blk; e += 128) {
         const int sl = e / blk, r2 = e - sl * blk, jb = r2 / p.ra, ja = r2 - jb * p.ra;
         float2 y = sl < vslabs ? bf2_to_f2(ys[sl * p.yp_bs + r2]) : make_float2(0.f, 0.f);
         const uint32_t k = (uint32_t)(sl * 2 * p.ra + 2 * ja);
         *(uint32_t*)(B1 + kmaj_off((uint32_t)(2 * jb), k, lbo_b1)) = f2_to_bf2(y.x, -y.y);
         *(uint32_t*)(B1 + kmaj_off((uint32_t)(2 * jb + 1), k, lbo_b1)) = f2_to_bf2(y.y, y.x);
       }
-    }
-    // Omega entries of the tile (local index and fp16 S~) into shared memory
-    if (cnt <= p.cap) {
-      for (int j = tid; j < cnt; j += R3T) {
-        lloc[j] = p.loc[e0 + j];
-        lval[j] = p.sp_upd[e0 + j];
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (s_abort) break;
-    if (tid == 0) {
-      for (int kk = 0; kk < p.K1 / 16; ++kk)
-        mma_f16(d1, sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
-                sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
-      mma_commit(&bars[4]);
-      m1_issued++;
-      if (it + p.nstage - 1 < n_it) {
-        bulk_wait_read0();  // the stage being refilled was last stored from
-        issue_loads(it + p.nstage - 1);
-      }
-    }
-    const bool ok1 = wait_all(&bars[4], m1_waited & 1u);
-    m1_waited++;
-    if (!ok1) break;
-    tc_fence_after();
-    if (warp < 4) {
-      // P' row (this thread's i_a) -> GEMM2's A operand
+      fence_async_smem();
+      mbar_arrive(&b1full[b]);
+      return true;
+    };
+    if (n_it > 0) ok = build(0);
+    for (int64_t it = 0; ok && it < n_it; ++it) {
+      if (it + 1 < n_it && !build(it + 1)) break;
+      // P'(t): D1 -> A2 (rows (slab, i_a), K = (j_b, re/im))
+      const int b = (int)(it & 1);
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
+      if (!waitw(&d1full[b], par, s_abort, p.err)) break;
+      if (!waitw(&a2empty[b], par ^ 1u, s_abort, p.err)) break;
+      tc_fence_after();
+      uint8_t* A2 = A2b(b);
       for (int c0 = 0; c0 < p.N1; c0 += 16) {
         float v[16];
-        tmem_ld16(d1 + lane_base + c0, v);
+        tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
         uint32_t w[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) w[u] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
-        *(uint4*)(A2 + (c0 / 8) * LBO_M128 + tid * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *(uint4*)(A2 + (c0 / 8 + 1) * LBO_M128 + tid * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        *(uint4*)(A2 + (c0 / 8) * LBO_M128 + row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *(uint4*)(A2 + (c0 / 8 + 1) * LBO_M128 + row * 16) = make_uint4(w[4], w[5], w[6], w[7]);
       }
+      tc_fence_before();
+      mbar_arrive(&d1empty[b]);
+      fence_async_smem();
+      mbar_arrive(&a2full[b]);
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (s_abort) break;
-    if (tid == 0) {
-      for (int kk = 0; kk < p.K2 / 16; ++kk)
-        mma_f16(d2, sdesc(sA2 + kk * 2 * LBO_M128, LBO_M128, 128),
-                sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
-      mma_commit(&bars[5]);
-      m2_issued++;
-    }
-    const bool ok2 = wait_all(&bars[5], m2_waited & 1u);
-    m2_waited++;
-    if (!ok2) break;
-    tc_fence_after();
-    {
-      // Delta row + lambda S~ on Omega, then the AdamW weight update in place.
-      const int m = tid & 127, h = tid >> 7;
-      const int sl = m / p.Ia;
-      const bool valid = t * p.spb + sl < p.n_slabs;
-      const int nch = p.N2 / 16, nch0 = (nch + 1) / 2;
-      const int c_lo = h ? nch0 : 0, c_hi = h ? nch : nch0;
-      const uint32_t erow = (uint32_t)m * p.Ib;
-      const uint16_t* L = cnt <= p.cap ? lloc : p.loc + e0;
-      const uint32_t* V = cnt <= p.cap ? lval : p.sp_upd + e0;
-      int lo = 0, hi = cnt;
-      const uint32_t first = erow + (uint32_t)c_lo * 8;
-      while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if ((uint32_t)L[mid] < first)
-          lo = mid + 1;
-        else
-          hi = mid;
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue
+    // lambda S~ of the tile is scattered into a zeroed tile-sized buffer
+    // (fp16 pairs, the precision S~ is kept in), so the weight pass is dense
+    // and branch-free: W <- W (1 - lr wd) - lr (Delta + S), one rounding.
+    const int et = tid - 256;  // 0..255
+    const int row = et & 127, half = et >> 7;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int nch = p.N2 / 16, nch0 = (nch + 1) / 2;
+    const int c_lo = half ? nch0 : 0, c_hi = half ? nch : nch0;
+    const int sl_row = row >> p.log2Ia;
+    const uint32_t erow = (uint32_t)row * p.Ib;
+    const float nlr = -p.lr, decay = p.decay;
+    const int Ib = p.Ib;
+    uint32_t* ds = (uint32_t*)(smem + p.off_ds);
+    // Omega ranges two tiles ahead, entries one tile ahead (registers)
+    int64_t cur_e0 = 0, cur_e1 = 0, nx_e0 = 0, nx_e1 = 0, nn_e0 = 0, nn_e1 = 0;
+    uint32_t pf_loc[EPF], pf_val[EPF];
+    auto load_entries = [&](int64_t e0, int64_t e1) {
+#pragma unroll
+      for (int j = 0; j < EPF; ++j) {
+        int64_t e = e0 + et + 256 * j;
+        if (e < e1) {
+          pf_loc[j] = p.loc[e];
+          pf_val[j] = p.sp_upd[e];
+        }
       }
-      int ptr = lo;
-      uint8_t* ws = wst(s);
+    };
+    if (n_it > 0) {
+      cur_e0 = p.tile_off[blockIdx.x];
+      cur_e1 = p.tile_off[blockIdx.x + 1];
+      if (n_it > 1) {
+        nx_e0 = p.tile_off[blockIdx.x + G];
+        nx_e1 = p.tile_off[blockIdx.x + G + 1];
+      }
+      load_entries(cur_e0, cur_e1);
+    }
+    for (uint32_t i = et; i < (uint32_t)(128 * Ib); i += 256) ds[i] = 0u;
+    named_sync(2, 256);
+    int s = 0;
+    uint32_t sph = 0;
+    for (int64_t it = 0; it < n_it; ++it) {
+      const int b = (int)(it & 1);
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
+      const int64_t t = blockIdx.x + it * G;
+      if (it + 2 < n_it) {
+        nn_e0 = p.tile_off[t + 2 * G];
+        nn_e1 = p.tile_off[t + 2 * G + 1];
+      }
+      // scatter lambda S~ of this tile
+#pragma unroll
+      for (int j = 0; j < EPF; ++j) {
+        int64_t e = cur_e0 + et + 256 * j;
+        if (e < cur_e1) ds[pf_loc[j]] = pf_val[j];
+      }
+      for (int64_t e = cur_e0 + 256 * EPF + et; e < cur_e1; e += 256) ds[p.loc[e]] = p.sp_upd[e];
+      named_sync(2, 256);
+      if (!waitw(&d2full[b], par, s_abort, p.err)) break;
+      if (!waitw(&full[s], sph, s_abort, p.err)) break;
+      tc_fence_after();
+      const bool valid = t * p.spb + sl_row < p.n_slabs;
+      WT* wrow = (WT*)wst(s) + erow;
+      const uint32_t* drow = ds + erow;
+      const uint32_t dbase = tmem + p.d2_col[b] + lane_base;
       for (int c = c_lo; c < c_hi; ++c) {
         float v[16];
-        tmem_ld16(d2 + lane_base + c * 16, v);
+        tmem_ld16(dbase + c * 16, v);
+        if (!valid) continue;
+        const int ib0 = c * 8;
+        if (ib0 + 8 <= Ib) {
+          float2 w[8], d[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int ib = c * 8 + u;
-          if (valid && ib < p.Ib) {
-            const uint32_t le = erow + (uint32_t)ib;
-            float dx = v[2 * u], dy = v[2 * u + 1];
-            while (ptr < cnt && (uint32_t)L[ptr] == le) {
-              float2 su = h2_to_f2(V[ptr]);
-              dx += su.x;
-              dy += su.y;
-              ++ptr;
-            }
-            if (p.w_c64) {
-              float2* wp = (float2*)ws + le;
-              float2 w = *wp;
-              *wp = make_float2(__fmaf_rn(-p.lr, dx, w.x * p.decay), __fmaf_rn(-p.lr, dy, w.y * p.decay));
-            } else {
-              uint32_t* wp = (uint32_t*)ws + le;
-              float2 w = h2_to_f2(*wp);
-              *wp = f2_to_h2(make_float2(__fmaf_rn(-p.lr, dx, w.x * p.decay),
-                                         __fmaf_rn(-p.lr, dy, w.y * p.decay)));
+          for (int u = 0; u < 8; ++u) {
+            w[u] = wload(wrow + ib0 + u);
+            d[u] = h2_to_f2(drow[ib0 + u]);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            wstore(wrow + ib0 + u, __fmaf_rn(nlr, v[2 * u] + d[u].x, w[u].x * decay),
+                   __fmaf_rn(nlr, v[2 * u + 1] + d[u].y, w[u].y * decay));
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (ib0 + u < Ib) {
+              float2 w = wload(wrow + ib0 + u), d = h2_to_f2(drow[ib0 + u]);
+              wstore(wrow + ib0 + u, __fmaf_rn(nlr, v[2 * u] + d.x, w.x * decay),
+                     __fmaf_rn(nlr, v[2 * u + 1] + d.y, w.y * decay));
             }
           }
         }
       }
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(&d2empty[b]);
+      mbar_arrive(&wdone[s]);
+      named_sync(2, 256);  // every read of the scattered buffer is done
+      // zero the scattered slots again, then move to the next tile's entries
+#pragma unroll
+      for (int j = 0; j < EPF; ++j) {
+        int64_t e = cur_e0 + et + 256 * j;
+        if (e < cur_e1) ds[pf_loc[j]] = 0u;
+      }
+      for (int64_t e = cur_e0 + 256 * EPF + et; e < cur_e1; e += 256) ds[p.loc[e]] = 0u;
+      named_sync(2, 256);  // zeroed before the next tile scatters
+      if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
+      cur_e0 = nx_e0;
+      cur_e1 = nx_e1;
+      nx_e0 = nn_e0;
+      nx_e1 = nn_e1;
+      if (++s == ns) {
+        s = 0;
+        sph ^= 1u;
+      }
     }
-    fence_async_smem();
-    __syncthreads();
-    if (s_abort) break;
-    if (tid == 0) {
-      bulk_s2g((uint8_t*)p.W + t * p.tile_elems * wb, wst(s), tile_wbytes(t));
-      bulk_commit();
-    }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    if (s_abort) {
-      for (int s = 0; s < p.nstage; ++s)
-        while (ld_waited[s] < ld_issued[s]) {
-          mbar_wait(&bars[s], ld_waited[s] & 1u, WAIT_NS / 4);
-          ld_waited[s]++;
-        }
-      if (m1_issued > m1_waited) mbar_wait(&bars[4], (m1_issued - 1) & 1u, WAIT_NS / 4);
-      if (m2_issued > m2_waited) mbar_wait(&bars[5], (m2_issued - 1) & 1u, WAIT_NS / 4);
-    }
-    bulk_wait_all0();
   }
   tc_fence_before();
   __syncthreads();
@@ -853,6 +1072,7 @@ struct TcImpl {
   int64_t n_slabs = 0, n_tiles = 0, n_groups = 0, tile_elems = 0, blk = 0, bs_pad = 0;
   int K1 = 0, N1 = 0, K2 = 0, N2 = 0;
   int rK1 = 0, rN1 = 0, rK2 = 0, rN2 = 0;
+  int a2_rows = 128;
   int wdt = 0;
   std::vector<InnerMode> inner;
   int64_t* tile_off = nullptr;
@@ -868,25 +1088,28 @@ struct TcImpl {
   P1Args p1{};
   R3Args r3{};
   size_t p1_smem = 0, r3_smem = 0, mg_smem_max = 0;
+  int r3_nstage = 3, p1_nstage = 3;
   int num_sms = 148;
   const float* U[8] = {};
 };
 
-size_t p1_smem_bytes(int Ib, int K1, int K2, int N1, int N2, P1Args* a) {
+size_t p1_smem_bytes(int Ib, int ns, int K1, int K2, int N1, int N2, uint32_t lbo_a2, P1Args* a) {
   size_t off = 0;
   auto take = [&](size_t b) {
     size_t o = off;
     off += (b + 127) / 128 * 128;
     return (uint32_t)o;
   };
-  size_t tile = (size_t)128 * Ib * 4;
-  uint32_t s0 = take(tile), s1 = take(tile);
-  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), a2 = take((size_t)(K2 / 8) * LBO_M128_PAD);
+  const size_t tile = ((size_t)128 * Ib * 4 + 127) / 128 * 128;
+  uint32_t st = take(tile * ns);
+  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), a2 = take((size_t)(K2 / 8) * lbo_a2);
   uint32_t b1 = take((size_t)N1 * K1 * 2), b2 = take((size_t)N2 * K2 * 2);
-  uint32_t bar = take(128);
+  uint32_t bar = take(256);
   if (a) {
-    a->off_stage0 = s0;
-    a->off_stage1 = s1;
+    a->lbo_a2 = lbo_a2;
+    a->nstage = ns;
+    a->off_stage = st;
+    a->stage_bytes = (uint32_t)tile;
     a->off_A1 = a1;
     a->off_A2 = a2;
     a->off_B1 = b1;
@@ -908,9 +1131,9 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
   wt = (wt + 127) / 128 * 128;
   yt = (yt + 127) / 128 * 128;
   uint32_t w = take(wt * nstage), y = take(yt * nstage);
-  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), b1 = take((size_t)N1 * K1 * 2);
-  uint32_t a2 = take((size_t)(K2 / 8) * LBO_M128), b2 = take((size_t)N2 * K2 * 2);
-  uint32_t ll = take((size_t)cap * 2), lv = take((size_t)cap * 4), bar = take(128);
+  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), b1 = take((size_t)2 * N1 * K1 * 2);
+  uint32_t a2 = take((size_t)2 * (K2 / 8) * LBO_M128), b2 = take((size_t)N2 * K2 * 2);
+  uint32_t dsb = take((size_t)128 * Ib * 4), bar = take(256);
   if (a) {
     a->w_tile_bytes = (uint32_t)wt;
     a->y_tile_bytes = (uint32_t)yt;
@@ -920,8 +1143,7 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
     a->off_B1 = b1;
     a->off_A2 = a2;
     a->off_B2 = b2;
-    a->off_lloc = ll;
-    a->off_lval = lv;
+    a->off_ds = dsb;
     a->off_bar = bar;
   }
   return off;
@@ -929,7 +1151,7 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
 
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 constexpr size_t ONE_CTA_SMEM = 120 * 1024;
-constexpr int R3_CAP = 2048;
+constexpr int R3_CAP = 1024;
 
 bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int wdt) {
   if (nd < 3) return false;
@@ -942,7 +1164,16 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
   if (g.Ib < 1 || g.Ib > 120) return false;
   if (g.rb > g.Ia) return false;
   g.spb = 128 / g.Ia;
-  g.q = std::max(1, 128 / (g.rb * g.spb));
+  // GEMM2 groups at most 64 valid rows when a slab's rows allow it; its A
+  // operand then holds 64 physical rows and the MMA's rows 64-127 read
+  // in-bounds shared memory whose results are never used.
+  if (g.rb * g.spb <= 64) {
+    g.q = 64 / (g.rb * g.spb);
+    g.a2_rows = 64;
+  } else {
+    g.q = 1;
+    g.a2_rows = 128;
+  }
   g.sg = g.spb * g.q;
   g.n_slabs = 1;
   for (int n = 0; n < nd - 2; ++n) g.n_slabs *= shape[n];
@@ -961,11 +1192,20 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
   g.blk = (int64_t)g.rb * g.ra;
   g.bs_pad = (g.blk + 3) / 4 * 4;
   g.wdt = wdt;
-  g.p1_smem = p1_smem_bytes(g.Ib, g.K1, g.K2, g.N1, g.N2, nullptr);
+  const uint32_t lbo_a2 = (uint32_t)(g.a2_rows / 8) * 128 + 16;
+  for (g.p1_nstage = 4; g.p1_nstage >= 2; --g.p1_nstage) {
+    g.p1_smem = p1_smem_bytes(g.Ib, g.p1_nstage, g.K1, g.K2, g.N1, g.N2, lbo_a2, nullptr);
+    if (g.p1_smem <= SMEM_LIMIT) break;
+  }
   if (g.p1_smem > SMEM_LIMIT) return false;
+  // TMEM (512 columns): P1 holds D1 twice and D2; R3 holds D1 and D2 twice.
+  auto r32 = [](int x) { return (x + 31) / 32 * 32; };
+  if (2 * r32(g.N1) + g.N2 > 512) return false;
+  if (2 * r32(g.rN1) + r32(g.rN2) + g.rN2 > 512) return false;
   int wbytes = wdt == TGD_C64 ? 8 : 4;
-  size_t r3a = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 3, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
-  size_t r3b = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 2, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
+  size_t r3a = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 4, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
+  size_t r3b = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 3, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
+  g.r3_nstage = r3a <= SMEM_LIMIT ? 4 : 3;
   g.r3_smem = r3a <= SMEM_LIMIT ? r3a : r3b;
   if (g.r3_smem > SMEM_LIMIT) return false;
   g.inner.clear();
@@ -1148,7 +1388,13 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
     }
   // ---- projection stream over G
   P1Args& a = g->p1;
-  p1_smem_bytes(g->Ib, g->K1, g->K2, g->N1, g->N2, &a);
+  p1_smem_bytes(g->Ib, g->p1_nstage, g->K1, g->K2, g->N1, g->N2, (uint32_t)(g->a2_rows / 8) * 128 + 16, &a);
+  {
+    const uint32_t n1 = (uint32_t)((g->N1 + 31) / 32 * 32);
+    a.d1_col[0] = 0;
+    a.d1_col[1] = n1;
+    a.d2_col = 2 * n1;
+  }
   a.G = (const uint32_t*)grad;
   a.N = p.N;
   a.n_slabs = g->n_slabs;
@@ -1160,6 +1406,7 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   a.ra = g->ra;
   a.rb = g->rb;
   a.spb = g->spb;
+  a.log2Ia = __builtin_ctz((unsigned)g->Ia);
   a.q = g->q;
   a.sg = g->sg;
   a.K1 = g->K1;
@@ -1249,8 +1496,14 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   // ---- reconstruction stream over W
   R3Args& r = g->r3;
   const int wbytes = g->wdt == TGD_C64 ? 8 : 4;
-  size_t need3 = r3_smem_bytes(g->Ib, g->spb, g->bs_pad, wbytes, 3, g->rK1, g->rN1, g->rK2, g->rN2, R3_CAP, nullptr);
-  r.nstage = need3 <= SMEM_LIMIT ? 3 : 2;
+  r.nstage = g->r3_nstage;
+  {
+    const uint32_t n1 = (uint32_t)((g->rN1 + 31) / 32 * 32), n2 = (uint32_t)((g->rN2 + 31) / 32 * 32);
+    r.d1_col[0] = 0;
+    r.d1_col[1] = n1;
+    r.d2_col[0] = 2 * n1;
+    r.d2_col[1] = 2 * n1 + n2;
+  }
   r3_smem_bytes(g->Ib, g->spb, g->bs_pad, wbytes, r.nstage, g->rK1, g->rN1, g->rK2, g->rN2, R3_CAP, &r);
   r.cap = R3_CAP;
   r.Yp = g->Yp;
@@ -1266,6 +1519,7 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   r.ra = g->ra;
   r.rb = g->rb;
   r.spb = g->spb;
+  r.log2Ia = __builtin_ctz((unsigned)g->Ia);
   r.K1 = g->rK1;
   r.N1 = g->rN1;
   r.K2 = g->rK2;
@@ -1279,10 +1533,20 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   r.lr = lr;
   r.err = d_err;
   const size_t r3_launch_smem = std::max(g->r3_smem, ONE_CTA_SMEM);
-  e = cudaFuncSetAttribute(recon_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r3_launch_smem);
-  if (e != cudaSuccess) return e;
-  H(0, "recon_stream");
-  recon_stream_kernel<<<(unsigned)std::min<int64_t>(g->n_tiles, g->num_sms), R3T, r3_launch_smem, s>>>(r);
+  const unsigned r3_grid = (unsigned)std::min<int64_t>(g->n_tiles, g->num_sms);
+  if (r.w_c64) {
+    e = cudaFuncSetAttribute(recon_stream_kernel<float2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)r3_launch_smem);
+    if (e != cudaSuccess) return e;
+    H(0, "recon_stream");
+    recon_stream_kernel<float2><<<r3_grid, R3T, r3_launch_smem, s>>>(r);
+  } else {
+    e = cudaFuncSetAttribute(recon_stream_kernel<__half2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)r3_launch_smem);
+    if (e != cudaSuccess) return e;
+    H(0, "recon_stream");
+    recon_stream_kernel<__half2><<<r3_grid, R3T, r3_launch_smem, s>>>(r);
+  }
   H(1, "recon_stream");
   return cudaGetLastError();
 }

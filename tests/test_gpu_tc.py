@@ -98,11 +98,19 @@ def test_tc_complex_adam_view_as_real(lib, orc, name):
     assert rel_err(w, w_ref, "c32h") <= TOL["c32h"]
 
 
-@pytest.mark.parametrize("name", ["4way_spb2_partial_group", "spectral_slice"])
+@pytest.mark.parametrize("name", ["4way_spb2_partial_group", "4way_spb4", "5way"])
 def test_tc_fp32_weights(lib, orc, name):
     shape, ranks, gen_ranks, rho = SHAPES[name]
     o, g, st, w, w_ref = _run(lib, orc, shape, ranks, gen_ranks, rho, "tcgen05", wdt="c64")
     assert rel_err(w, w_ref, "c64") <= TOL["c32h"]
+
+
+def test_tc_fp32_weights_large_slab_routes_generic(lib):
+    """fp32 weight tiles of 128 x 65 do not fit the reconstruction's load
+    ring in shared memory; such tensors take the CUDA-core path."""
+    g = lib.TensorGRaD((4, 8, 128, 65), (2, 4, 32, 16), 0.05, 0, grad_dtype="c32h",
+                       weight_dtype="c64")
+    assert g.info["path"] == "generic"
 
 
 def test_tc_paths_agree_over_steps(lib):
