@@ -194,6 +194,29 @@ TGD_API tgd_status tgd_topk_select(const void* grad, tgd_dtype dtype, int64_t n,
                            int64_t* omega_out, float* val_out, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Top-k selection that allocates nothing (no counterpart in the paper: an
+ *  interface for callers that cannot allocate device memory). The same
+ *  selection and output as tgd_topk_select, but its scratch space is a
+ *  fixed array compiled into the library instead of a caller workspace, so
+ *  a caller that only holds its input and output buffers can use it: for
+ *  example a plugin inside a framework whose allocator owns all device
+ *  memory, or a loop that must not call cudaMalloc because cudaMalloc may
+ *  synchronise the device.
+ *  - n must not exceed TGD_TOPK_STATIC_MAX_N, else TGD_ERR_INVALID_ARG.
+ *  - The array (TGD_TOPK_STATIC_SCRATCH_BYTES bytes) exists once per GPU
+ *    that loads the library and stays allocated until the process exits.
+ *  - The first call on each device looks up the array's device address on
+ *    that device (the current device); make that first call before any
+ *    stream capture.
+ *  - All calls share the array: calls whose work overlaps on the GPU (on
+ *    different streams, or from different threads) race and give wrong
+ *    results. Calls in one stream are ordered and safe; the array keeps the
+ *    last call's contents, and every call clears what it needs itself. */
+#define TGD_TOPK_STATIC_MAX_N ((int64_t)1 << 28)
+#define TGD_TOPK_STATIC_SCRATCH_BYTES ((size_t)2 << 20)
+TGD_API tgd_status tgd_topk_select_static(const void* grad, tgd_dtype dtype, int64_t n, int64_t k,
+                                          int64_t* omega_out, float* val_out, void* stream);
+
 /* Per-kernel timing with CUDA events recorded on the launching stream around
  *  every kernel the handle launches (no effect on results). enable = 1 clears
  *  the record and starts timing; enable = 0 stops it. */

@@ -21,7 +21,7 @@ import numpy as np
 from . import native
 from .native import TgdError, check, lib
 
-__all__ = ["TensorGRaD", "TgdError", "topk_select"]
+__all__ = ["TensorGRaD", "TgdError", "topk_select", "topk_select_static"]
 
 
 def _stream_ptr(stream) -> Optional[int]:
@@ -203,5 +203,23 @@ def topk_select(grad, dtype: str, k: int, stream=None):
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=grad.device)
     check(lib().tgd_topk_select(grad.data_ptr(), native.DTYPES[dtype], n, k, omega.data_ptr(),
                                 vals.data_ptr(), ws.data_ptr(), wsb, _stream_ptr(stream)))
+    vals = vals[: k * (2 if cplx else 1)]
+    return omega[:k], (vals.view(k, 2) if cplx else vals)
+
+
+def topk_select_static(grad, dtype: str, k: int, stream=None):
+    """The same selection as topk_select, for callers that cannot allocate
+    device scratch memory: the library uses a fixed array of its own (one per
+    device, n <= 2**28). Only the outputs are allocated here, by the caller's
+    framework. Calls that overlap on the GPU share that array and must not
+    run concurrently."""
+    import torch
+    n = grad.numel() * grad.element_size() // native.ELEM_BYTES[dtype]
+    _check_tensor(grad, dtype, n, "grad")
+    cplx = dtype in ("c64", "c32h")
+    omega = torch.empty(max(k, 1), dtype=torch.int64, device=grad.device)
+    vals = torch.empty(max(k, 1) * (2 if cplx else 1), dtype=torch.float32, device=grad.device)
+    check(lib().tgd_topk_select_static(grad.data_ptr(), native.DTYPES[dtype], n, k, omega.data_ptr(),
+                                       vals.data_ptr(), _stream_ptr(stream)))
     vals = vals[: k * (2 if cplx else 1)]
     return omega[:k], (vals.view(k, 2) if cplx else vals)

@@ -335,6 +335,9 @@ __global__ void identity_kernel(float2* U, int64_t n) {
 
 }  // namespace
 
+// Global (handle-less) error message, shared with other translation units.
+void tgd::set_global_error(const std::string& msg) { g_last_error = msg; }
+
 extern "C" {
 
 void tgd_default_options(tgd_options* opt) {

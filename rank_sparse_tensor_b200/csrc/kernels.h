@@ -4,9 +4,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string>
+
 namespace tgd {
 
 struct AdamConst;
+
+// Sets the message tgd_last_error(NULL) returns.
+void set_global_error(const std::string& msg);
 
 // ---- select.cu: Omega selection and index structures
 size_t select_workspace_bytes(int64_t n);

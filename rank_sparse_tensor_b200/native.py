@@ -14,6 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtgd.so")
 
 MAX_NDIM = 8
+TOPK_STATIC_MAX_N = 1 << 28  # TGD_TOPK_STATIC_MAX_N
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "OOM", 4: "CUDA", 5: "TIMEOUT",
           6: "STATE", 7: "NONFINITE"}
@@ -75,6 +76,8 @@ SIGNATURES = {
     "tgd_topk_workspace_bytes": (C.c_size_t, [C.c_int64]),
     "tgd_topk_select": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
                                   C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "tgd_topk_select_static": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
+                                         C.c_void_p, C.c_void_p]),
     "tgd_profile": (C.c_int, [C.c_void_p, C.c_int]),
     "tgd_profile_read": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.POINTER(C.c_int)]),
     "tgd_last_error": (C.c_char_p, [C.c_void_p]),
