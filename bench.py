@@ -70,14 +70,17 @@ def kernel_algorithmic_bytes(name: str, wl) -> float:
     step's algorithmic bytes (the parts of the step it alone moves)."""
     a = algorithmic_bytes(wl)
     N = wl.N
+    cplx = wl.dtype in ("c64", "c32h")
+    moments = wl.k * 2 * ((8, 4) if cplx else (4, 4))[0] + wl.k * 2 * 4
     table = {
-        # tensor-core path: G stream (mask, gather, sparse AdamW) and W stream
-        "proj_stream": a["grad"] + a["sparse"] - wl.k * 0,  # reads G once; sparse moments r/w
-        "recon_stream": a["weight"],                          # reads and writes W once
+        # tensor-core path: G stream (mask, gather, Omega's index read once),
+        # sparse AdamW stream (moments read and written), W stream
+        "proj_stream": a["grad"] + 8 * wl.k,
+        "sparse_adam": moments,
+        "recon_stream": a["weight"],
         # CUDA-core path
         "weight_update": a["weight"],
         "mode_product": a["grad"],
-        "sparse_adam": a["sparse"],
     }
     return float(table.get(name, 0.0))
 

@@ -106,7 +106,9 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 }
 
 constexpr int P1T = 512;
-constexpr int PF = 4;  // Omega entries per converter thread prefetched for the next tile
+constexpr int PF = 4;     // Omega indices per converter thread prefetched for the next tile
+constexpr int P1_NS_MAX = 4;
+constexpr int P1_CONV_UNROLL = 5;  // 8-column chunks a converter loads before storing
 
 struct P1Args {
   const uint32_t* G;
@@ -114,20 +116,17 @@ struct P1Args {
   int Ia, Ib, ra, rb, spb, q, sg, log2Ia;
   int K1, N1, K2, N2;
   uint32_t lbo_a2;  // GEMM2's A: 64 or 128 physical rows (see geometry)
-  uint32_t d1_col[2], d2_col;
+  uint32_t d1_col[2], d2_col, a1_col[2];  // TMEM columns
   const int64_t* tile_off;
   const uint16_t* loc;
-  float* sp_m;
-  float* sp_v;
-  uint32_t* sp_upd;
-  AdamConst asp;
+  uint32_t* gs;  // out: g_s = G[Omega] (fp16 pairs), Omega order
   const uint8_t* B1img;
   const uint8_t* B2img;
   void* Y;
-  int y_f32;
+  int y_f32, y_vec;  // fp32 (else bf16) Y; rows 16-byte aligned (ra % 4 == 0, or even for fp32)
   int* err;
-  int nstage;
-  uint32_t off_stage, stage_bytes, off_A1, off_A2, off_B1, off_B2, off_bar;
+  int nstage;  // load stages
+  uint32_t stage_bytes, off_stage, off_A2, off_B1, off_B2, off_bar;
 };
 
 // Position in this CTA's tile sequence: groups blockIdx.x, +gridDim.x, ...,
@@ -145,32 +144,33 @@ struct TileCursor {
 };
 
 // Warp-specialised projection stream, one CTA per SM, persistent over groups
-// of q tiles:
+// of q tiles (a tile = 128 rows (slab, i_a) x I_b, contiguous in G):
 //   warp 0   producer: bulk copies of G tiles into a ring of stages;
-//   warp 1   MMA issuer: GEMM1(t) = A1 x B1 -> D1[t&1]; per group GEMM2 =
-//            A2 x B2 -> D2;
-//   warps 4-11  converters: sparse pass on Omega (gather, zero the entry,
-//            sparse AdamW) and the residual tile into GEMM1's A operand;
-//   warps 12-15 epilogue: P(t) from D1 into the group's GEMM2 operand; Y of
-//            the group from D2 to global memory.
+//   warps 4-11  converters: gather Omega's values (g_s, written out for
+//            the sparse AdamW) and zero them in the staged tile (R = G - S),
+//            then write the residual rows into TMEM as GEMM1's A operand
+//            (tcgen05.st), two buffers;
+//   warp 1   MMA issuer: GEMM1(t) = A1[t & 1] (TMEM) x B1 -> D1[t & 1];
+//            per group GEMM2 = A2 x B2 -> D2;
+//   warps 12-15 epilogue: P(t) from D1 into the group's GEMM2 operand, Y of
+//            the group from D2.
 // Roles hand off through mbarriers.
 __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* A1 = smem + p.off_A1;
   uint8_t* A2 = smem + p.off_A2;
   uint8_t* B1 = smem + p.off_B1;
   uint8_t* B2 = smem + p.off_B2;
   uint64_t* bars = (uint64_t*)(smem + p.off_bar);
   uint64_t* full = bars;          // [4] stage loaded (1 + tx)
   uint64_t* sempty = bars + 4;    // [4] stage consumed (256)
-  uint64_t* opnd = bars + 8;      // B1 + B2 loaded
-  uint64_t* a1full = bars + 9;    // (256)
-  uint64_t* a1empty = bars + 10;  // (commit)
-  uint64_t* d1full = bars + 11;   // [2] (commit)
-  uint64_t* d1empty = bars + 13;  // [2] (128)
-  uint64_t* a2full = bars + 15;   // (128)
-  uint64_t* d2full = bars + 16;   // (commit)
-  uint32_t* tslot = (uint32_t*)(bars + 18);
+  uint64_t* a1full = bars + 8;    // [2] A1 written to TMEM (256)
+  uint64_t* a1empty = bars + 10;  // [2] GEMM1 done reading A1 (commit)
+  uint64_t* d1full = bars + 12;   // [2] (commit)
+  uint64_t* d1empty = bars + 14;  // [2] (128)
+  uint64_t* opnd = bars + 16;     // B1 + B2 loaded
+  uint64_t* a2full = bars + 17;   // (128)
+  uint64_t* d2full = bars + 18;   // (commit)
+  uint32_t* tslot = (uint32_t*)(bars + 19);
   __shared__ int s_abort_storage;
   volatile int* s_abort = &s_abort_storage;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -188,17 +188,17 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
 
   if (tid == 0) {
     *s_abort = 0;
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < P1_NS_MAX; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&sempty[i], 256);
     }
-    mbar_init(opnd, 1);
-    mbar_init(a1full, 256);
-    mbar_init(a1empty, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&a1full[b], 256);
+      mbar_init(&a1empty[b], 1);
       mbar_init(&d1full[b], 1);
       mbar_init(&d1empty[b], 128);
     }
+    mbar_init(opnd, 1);
     mbar_init(a2full, 128);
     mbar_init(d2full, 1);
     fence_mbar_init();
@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   {
     const uint32_t a2b = (uint32_t)(p.K2 / 8) * p.lbo_a2;
     for (uint32_t i = tid; i < a2b / 16; i += P1T) ((uint4*)A2)[i] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
   }
   __syncthreads();
   if (warp == 0) tmem_alloc(tslot, 512);
@@ -239,8 +240,10 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
           ph ^= 1u;
         }
       }
+      // wait (bounded) for the operand copies and for tile copies still in
+      // flight before the CTA exits
+      mbar_wait(opnd, 0, WAIT_NS / 4);
       if (*s_abort) {
-        // wait (bounded) for the copies still in flight before the CTA exits
         for (int64_t it = 0; it < issued; ++it) mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
       }
     }
@@ -249,94 +252,78 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     if (lane == 0) {
       const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
       const uint32_t id1 = idesc_f16(0, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
-      const uint32_t sA1 = smem_u32(A1), sA2 = smem_u32(A2), sB1 = smem_u32(B1), sB2 = smem_u32(B2);
+      const uint32_t sA2 = smem_u32(A2), sB1 = smem_u32(B1), sB2 = smem_u32(B2);
       bool ok = wait1(opnd, 0, s_abort, p.err);
       TileCursor c{(int64_t)blockIdx.x, 0};
-      int64_t g1_next = 0;      // next tile to run GEMM1 on
-      int64_t groups_done = 0;  // GEMM2s issued
-      int64_t groups_ready = 0; // groups whose last GEMM1 is issued
       uint32_t a2par = 0;
-      uint64_t t0 = global_ns();
-      while (ok && (g1_next < n_it || groups_done < groups_ready)) {
-        bool progressed = false;
-        // GEMM2 of a complete group, as soon as its operand is written
-        if (groups_done < groups_ready && mbar_try_wait(a2full, a2par)) {
-          tc_fence_after();
-          for (int kk = 0; kk < p.K2 / 16; ++kk)
-            mma_f16(tmem + p.d2_col, sdesc(sA2 + kk * 2 * p.lbo_a2, p.lbo_a2, 128),
-                    sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
-          mma_commit(d2full);
-          a2par ^= 1u;
-          ++groups_done;
-          progressed = true;
+      int64_t it = 0, g2_issued = 0;
+      bool pending = false;  // a group whose GEMM1s are all issued awaits its GEMM2
+      auto gemm2 = [&]() -> bool {
+        if (!wait1(a2full, a2par, s_abort, p.err)) return false;
+        tc_fence_after();
+        for (int kk = 0; kk < p.K2 / 16; ++kk)
+          mma_f16(tmem + p.d2_col, sdesc(sA2 + kk * 2 * p.lbo_a2, p.lbo_a2, 128),
+                  sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
+        mma_commit(d2full);
+        a2par ^= 1u;
+        ++g2_issued;
+        return true;
+      };
+      // Fixed issue order with sleeping waits: GEMM1 of every tile; a
+      // group's GEMM2 right after the next group's first GEMM1 (its
+      // operand is complete about when that tile's D1 buffer frees up).
+      for (; ok && it < n_it; ++it) {
+        const int b = (int)(it & 1);
+        const uint32_t par = (uint32_t)((it >> 1) & 1);
+        if (!wait1(&a1full[b], par, s_abort, p.err) || !wait1(&d1empty[b], par ^ 1u, s_abort, p.err)) {
+          ok = false;
+          break;
         }
-        if (g1_next < n_it) {
-          const int b = (int)(g1_next & 1);
-          const uint32_t par = (uint32_t)((g1_next >> 1) & 1);
-          if (mbar_try_wait(a1full, (uint32_t)(g1_next & 1)) && mbar_try_wait(&d1empty[b], par ^ 1u)) {
-            tc_fence_after();
-            for (int kk = 0; kk < p.K1 / 16; ++kk)
-              mma_f16(tmem + p.d1_col[b], sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
-                      sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
-            mma_commit(&d1full[b]);
-            mma_commit(a1empty);
-            const bool last = c.i == q - 1 || g1_next == n_it - 1;
-            if (last) ++groups_ready;
-            ++g1_next;
-            c.next(q);
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          t0 = global_ns();
-        } else {
-          __nanosleep(64);
-          if (*s_abort) break;
-          if (global_ns() - t0 > WAIT_NS) {  // no progress for WAIT_NS
-            *s_abort = 1;
-            atomicOr(p.err, DEV_ERR_TIMEOUT);
+        tc_fence_after();
+        // A from TMEM: 16 K values = 8 columns per MMA
+        for (int kk = 0; kk < p.K1 / 16; ++kk)
+          mma_f16_ts(tmem + p.d1_col[b], tmem + p.a1_col[b] + kk * 8, sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128),
+                     id1, kk > 0);
+        mma_commit(&d1full[b]);
+        mma_commit(&a1empty[b]);
+        if (pending) {
+          pending = false;
+          if (!gemm2()) {
+            ok = false;
+            ++it;
             break;
           }
         }
+        if (c.i == q - 1 || it == n_it - 1) pending = true;
+        c.next(q);
       }
+      if (ok && pending) ok = gemm2();
       if (*s_abort) {
         // bounded wait for the last MMAs before TMEM is released
-        if (g1_next > 0) mbar_wait(&d1full[(g1_next - 1) & 1], (uint32_t)(((g1_next - 1) >> 1) & 1), WAIT_NS / 4);
-        if (groups_done > 0) mbar_wait(d2full, (a2par ^ 1u), WAIT_NS / 4);
+        if (it > 0) mbar_wait(&d1full[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), WAIT_NS / 4);
+        if (g2_issued > 0) mbar_wait(d2full, (a2par ^ 1u), WAIT_NS / 4);
       }
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ converters
     const int ct = tid - 128;  // 0..255
     const int row = ct & 127, half = ct >> 7;
-    const int vc = p.asp.cmode == 1 ? 2 : 1;
     const int sl_row = row >> p.log2Ia;
-    const int Ib = p.Ib, nk = p.K1 / 8;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int Ib = p.Ib;
+    // GEMM1's A row in TMEM: K1 / 2 columns (one complex fp16 pair each) in
+    // chunks of 8; the two halves of the converters take alternate ranges
+    const int nch = p.K1 / 16, nch0 = (nch + 1) / 2;
+    const int ch_lo = half ? nch0 : 0, ch_hi = half ? nch : nch0;
     int64_t cur_e0 = 0, cur_e1 = 0, nx_e0 = 0, nx_e1 = 0, nn_e0 = 0, nn_e1 = 0;
     uint32_t pf_loc[PF];
-    float2 pf_m[PF], pf_v[PF];
     auto load_entries = [&](int64_t e0, int64_t e1) {
 #pragma unroll
       for (int j = 0; j < PF; ++j) {
-        int64_t e = e0 + ct + 256 * j;
-        if (e < e1) {
-          pf_loc[j] = p.loc[e];
-          pf_m[j] = ((const float2*)p.sp_m)[e];
-          pf_v[j] = vc == 2 ? ((const float2*)p.sp_v)[e] : make_float2(p.sp_v[e], 0.f);
-        }
+        const int64_t e = e0 + ct + 256 * j;
+        if (e >= e1) break;
+        pf_loc[j] = p.loc[e];
       }
-    };
-    auto apply_sparse = [&](uint32_t* sw, int64_t e, uint32_t l, float2 m, float2 v) {
-      uint32_t u = sw[l];
-      sw[l] = 0u;
-      float mm[2] = {m.x, m.y}, vv[2] = {v.x, v.y};
-      float2 upd = adam_elem(h2_to_f2(u), mm, vv, p.asp);
-      ((float2*)p.sp_m)[e] = make_float2(mm[0], mm[1]);
-      if (vc == 2)
-        ((float2*)p.sp_v)[e] = make_float2(vv[0], vv[1]);
-      else
-        p.sp_v[e] = vv[0];
-      p.sp_upd[e] = f2_to_h2(upd);
     };
     TileCursor cur{(int64_t)blockIdx.x, 0}, ahead{(int64_t)blockIdx.x, 0};
     if (n_it > 0) {
@@ -356,6 +343,8 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     uint32_t ph = 0;
     for (int64_t it = 0; it < n_it; ++it) {
       const int64_t t = cur.tile(q);
+      const int b = (int)(it & 1);
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
       if (it + 2 < n_it) {
         const int64_t t2 = ahead.tile(q);
         nn_e0 = p.tile_off[t2];
@@ -363,15 +352,28 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       }
       if (!waitw(&full[s], ph, s_abort, p.err)) break;
       uint32_t* sw = (uint32_t*)stage(s);
+      // gather g_s (coalesced stores, Omega order) and zero it in the tile
+      // (R = G - S)
+      const int cnt = (int)(cur_e1 - cur_e0);
+      {
+        uint32_t u[PF];
 #pragma unroll
-      for (int j = 0; j < PF; ++j) {
-        int64_t e = cur_e0 + ct + 256 * j;
-        if (e < cur_e1) apply_sparse(sw, e, pf_loc[j], pf_m[j], pf_v[j]);
+        for (int j = 0; j < PF; ++j)
+          if (ct + 256 * j < cnt) u[j] = sw[pf_loc[j]];
+#pragma unroll
+        for (int j = 0; j < PF; ++j) {
+          const int jj = ct + 256 * j;
+          if (jj < cnt) {
+            sw[pf_loc[j]] = 0u;
+            p.gs[cur_e0 + jj] = u[j];
+          }
+        }
       }
-      for (int64_t e = cur_e0 + 256 * PF + ct; e < cur_e1; e += 256) {
-        float2 m = ((const float2*)p.sp_m)[e];
-        float2 v = vc == 2 ? ((const float2*)p.sp_v)[e] : make_float2(p.sp_v[e], 0.f);
-        apply_sparse(sw, e, p.loc[e], m, v);
+      for (int jj = 256 * PF + ct; jj < cnt; jj += 256) {
+        const int64_t e = cur_e0 + jj;
+        const uint32_t l = p.loc[e];
+        p.gs[e] = sw[l];
+        sw[l] = 0u;
       }
       if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
       cur_e0 = nx_e0;
@@ -379,26 +381,31 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       nx_e0 = nn_e0;
       nx_e1 = nn_e1;
       named_sync(1, 256);  // every zeroed entry is in place before conversion
-      if (!waitw(a1empty, (uint32_t)((it & 1) ^ 1), s_abort, p.err)) break;
-      // residual tile -> GEMM1's A operand (row = (slab, i_a), K = (i_b, re/im))
+      if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err)) break;
+      tc_fence_after();
+      // residual row -> TMEM (K = (i_b, re/im): one complex pair per column)
       const bool valid = t * p.spb + sl_row < p.n_slabs;
       const uint32_t* src = sw + row * Ib;
-      uint8_t* dst = A1 + row * 16;
-      if (valid) {
-        int kc = half;
-        for (; 4 * kc + 3 < Ib; kc += 2)
-          *(uint4*)(dst + kc * LBO_M128) = make_uint4(src[4 * kc], src[4 * kc + 1], src[4 * kc + 2], src[4 * kc + 3]);
-        for (; kc < nk; kc += 2) {
-          uint32_t v[4];
+      const uint32_t taddr = tmem + lane_base + p.a1_col[b];
+      // all loads of up to P1_CONV_UNROLL chunks before their stores
+      for (int ch0 = ch_lo; ch0 < ch_hi; ch0 += P1_CONV_UNROLL) {
+        const int nc = ch_hi - ch0 < P1_CONV_UNROLL ? ch_hi - ch0 : P1_CONV_UNROLL;
+        uint32_t v[8 * P1_CONV_UNROLL];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) v[u] = 4 * kc + u < Ib ? src[4 * kc + u] : 0u;
-          *(uint4*)(dst + kc * LBO_M128) = make_uint4(v[0], v[1], v[2], v[3]);
+        for (int i = 0; i < P1_CONV_UNROLL; ++i) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int cc = 8 * (ch0 + i) + u;
+            v[8 * i + u] = i < nc && valid && cc < Ib ? src[cc] : 0u;
+          }
         }
-      } else {
-        for (int kc = half; kc < nk; kc += 2) *(uint4*)(dst + kc * LBO_M128) = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < P1_CONV_UNROLL; ++i)
+          if (i < nc) tmem_st8(taddr + 8 * (ch0 + i), v + 8 * i);  // nc is warp-uniform
       }
-      fence_async_smem();
-      mbar_arrive(a1full);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&a1full[b]);
       mbar_arrive(&sempty[s]);
       cur.next(q);
       ahead.next(q);
@@ -416,19 +423,23 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     uint32_t d2par = 0;
     for (int64_t it = 0; it < n_it; ++it) {
       const int b = (int)(it & 1);
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
       const int64_t t = c.tile(q);
-      if (!waitw(&d1full[b], (uint32_t)((it >> 1) & 1), s_abort, p.err)) break;
+      if (!waitw(&d1full[b], par, s_abort, p.err)) break;
       tc_fence_after();
       // P (fp32, TMEM) -> GEMM2's A operand (bf16), rows (slab in group,
       // j_b), K = (i_a, re/im)
       const bool valid = t * p.spb + sl_row < p.n_slabs;
       const int m2base = (c.i * p.spb + sl_row) * p.rb;
-      for (int c0 = 0; c0 < p.N1; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
+      for (int c0 = 0; c0 < p.N1; c0 += 32) {
+        float v[32];
+        if (c0 + 32 <= p.N1)
+          tmem_ld32(tmem + p.d1_col[b] + lane_base + c0, v);
+        else
+          tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int u = 0; u < 16; ++u) {
             int jb = c0 / 2 + u;
             if (jb < p.rb) {
               uint32_t off = kmaj_off((uint32_t)(m2base + jb), (uint32_t)(2 * ia_row), p.lbo_a2);
@@ -451,12 +462,29 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
         const int64_t slab = c.g * p.sg + sb;
         const bool yvalid = row < p.sg * p.rb && slab < p.n_slabs;
         const int64_t ybase = (slab * p.rb + jb) * p.ra;
-        for (int c0 = 0; c0 < p.N2; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + p.d2_col + lane_base + c0, v);
-          if (yvalid) {
+        for (int c0 = 0; c0 < p.N2; c0 += 32) {
+          float v[32];
+          if (c0 + 32 <= p.N2)
+            tmem_ld32(tmem + p.d2_col + lane_base + c0, v);
+          else
+            tmem_ld16(tmem + p.d2_col + lane_base + c0, v);
+          // a thread owns one Y row: 16-byte stores where the row allows
+          // them (one warp store touches 32 rows, so wider is cheaper)
+          if (yvalid && p.y_vec && c0 / 2 + 16 <= p.ra) {
+            if (p.y_f32) {
+              float4* y4 = (float4*)((float2*)p.Y + ybase + c0 / 2);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+              for (int u = 0; u < 8; ++u) y4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            } else {
+              uint4* y4 = (uint4*)((uint32_t*)p.Y + ybase + c0 / 2);
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                y4[u] = make_uint4(f2_to_bf2(v[8 * u], v[8 * u + 1]), f2_to_bf2(v[8 * u + 2], v[8 * u + 3]),
+                                   f2_to_bf2(v[8 * u + 4], v[8 * u + 5]), f2_to_bf2(v[8 * u + 6], v[8 * u + 7]));
+            }
+          } else if (yvalid) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
               int ja = c0 / 2 + u;
               if (ja < p.ra) {
                 if (p.y_f32)
@@ -619,6 +647,26 @@ __global__ void core_adam_tc_kernel(const float2* C, int64_t n, int64_t blk, int
     m[2 * j + 1] = mm[1];
     for (int q = 0; q < vc; ++q) v[j * vc + q] = vv[q];
     out[(j / blk) * out_bs + j % blk] = f2_to_bf2(u.x, u.y);
+  }
+}
+
+// S~ = lambda * Adam(g_s), in place of the gathered g_s (fp16 pairs in and
+// out; fp32 moments: m complex, v one or two floats). A plain stream over
+// the k entries in Omega order.
+__global__ void sparse_adam_tc_kernel(uint32_t* gs, int64_t k, float* m, float* v, AdamConst a) {
+  const int vc = a.cmode == 1 ? 2 : 1;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < k;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    const float2 m2 = ((const float2*)m)[j];
+    const float2 v2 = vc == 2 ? ((const float2*)v)[j] : make_float2(v[j], 0.f);
+    float mm[2] = {m2.x, m2.y}, vv[2] = {v2.x, v2.y};
+    const float2 u = adam_elem(h2_to_f2(gs[j]), mm, vv, a);
+    ((float2*)m)[j] = make_float2(mm[0], mm[1]);
+    if (vc == 2)
+      ((float2*)v)[j] = make_float2(vv[0], vv[1]);
+    else
+      v[j] = vv[0];
+    gs[j] = f2_to_h2(u);
   }
 }
 
@@ -1093,7 +1141,8 @@ struct TcImpl {
   const float* U[8] = {};
 };
 
-size_t p1_smem_bytes(int Ib, int ns, int K1, int K2, int N1, int N2, uint32_t lbo_a2, P1Args* a) {
+// Projection shared memory: nstage tile stages, A2, B1, B2, barriers.
+size_t p1_smem_bytes(int Ib, int ns, int K2, int K1, int N1, int N2, uint32_t lbo_a2, P1Args* a) {
   size_t off = 0;
   auto take = [&](size_t b) {
     size_t o = off;
@@ -1101,16 +1150,14 @@ size_t p1_smem_bytes(int Ib, int ns, int K1, int K2, int N1, int N2, uint32_t lb
     return (uint32_t)o;
   };
   const size_t tile = ((size_t)128 * Ib * 4 + 127) / 128 * 128;
-  uint32_t st = take(tile * ns);
-  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), a2 = take((size_t)(K2 / 8) * lbo_a2);
+  uint32_t st = take(tile * ns), a2 = take((size_t)(K2 / 8) * lbo_a2);
   uint32_t b1 = take((size_t)N1 * K1 * 2), b2 = take((size_t)N2 * K2 * 2);
   uint32_t bar = take(256);
   if (a) {
-    a->lbo_a2 = lbo_a2;
     a->nstage = ns;
-    a->off_stage = st;
     a->stage_bytes = (uint32_t)tile;
-    a->off_A1 = a1;
+    a->lbo_a2 = lbo_a2;
+    a->off_stage = st;
     a->off_A2 = a2;
     a->off_B1 = b1;
     a->off_B2 = b2;
@@ -1149,7 +1196,9 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
   return off;
 }
 
-constexpr size_t SMEM_LIMIT = 227 * 1024;
+// Dynamic shared memory per CTA: the 227 KB opt-in maximum less 1 KB for the
+// kernels' static shared variables (the launch fails if the sum exceeds it).
+constexpr size_t SMEM_LIMIT = 227 * 1024 - 1024;
 constexpr size_t ONE_CTA_SMEM = 120 * 1024;
 constexpr int R3_CAP = 1024;
 
@@ -1193,14 +1242,16 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
   g.bs_pad = (g.blk + 3) / 4 * 4;
   g.wdt = wdt;
   const uint32_t lbo_a2 = (uint32_t)(g.a2_rows / 8) * 128 + 16;
-  for (g.p1_nstage = 4; g.p1_nstage >= 2; --g.p1_nstage) {
-    g.p1_smem = p1_smem_bytes(g.Ib, g.p1_nstage, g.K1, g.K2, g.N1, g.N2, lbo_a2, nullptr);
+  // Projection shared memory: as many load stages as fit.
+  for (g.p1_nstage = P1_NS_MAX; g.p1_nstage >= 2; --g.p1_nstage) {
+    g.p1_smem = p1_smem_bytes(g.Ib, g.p1_nstage, g.K2, g.K1, g.N1, g.N2, lbo_a2, nullptr);
     if (g.p1_smem <= SMEM_LIMIT) break;
   }
   if (g.p1_smem > SMEM_LIMIT) return false;
-  // TMEM (512 columns): P1 holds D1 twice and D2; R3 holds D1 and D2 twice.
+  // TMEM (512 columns): P1 holds D1 twice, D2 and GEMM1's A twice (K1 / 2
+  // columns each); R3 holds D1 and D2 twice.
   auto r32 = [](int x) { return (x + 31) / 32 * 32; };
-  if (2 * r32(g.N1) + g.N2 > 512) return false;
+  if (2 * r32(g.N1) + r32(g.N2) + 2 * r32(g.K1 / 2) > 512) return false;
   if (2 * r32(g.rN1) + r32(g.rN2) + g.rN2 > 512) return false;
   int wbytes = wdt == TGD_C64 ? 8 : 4;
   size_t r3a = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 4, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
@@ -1388,12 +1439,16 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
     }
   // ---- projection stream over G
   P1Args& a = g->p1;
-  p1_smem_bytes(g->Ib, g->p1_nstage, g->K1, g->K2, g->N1, g->N2, (uint32_t)(g->a2_rows / 8) * 128 + 16, &a);
+  p1_smem_bytes(g->Ib, g->p1_nstage, g->K2, g->K1, g->N1, g->N2, (uint32_t)(g->a2_rows / 8) * 128 + 16, &a);
   {
-    const uint32_t n1 = (uint32_t)((g->N1 + 31) / 32 * 32);
+    // TMEM columns: D1 x2, D2, GEMM1's A x2 (each 32-column aligned)
+    const uint32_t n1 = (uint32_t)((g->N1 + 31) / 32 * 32), n2 = (uint32_t)((g->N2 + 31) / 32 * 32);
+    const uint32_t na = (uint32_t)((g->K1 / 2 + 31) / 32 * 32);
     a.d1_col[0] = 0;
     a.d1_col[1] = n1;
     a.d2_col = 2 * n1;
+    a.a1_col[0] = 2 * n1 + n2;
+    a.a1_col[1] = 2 * n1 + n2 + na;
   }
   a.G = (const uint32_t*)grad;
   a.N = p.N;
@@ -1415,15 +1470,13 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   a.N2 = g->N2;
   a.tile_off = g->tile_off;
   a.loc = g->loc;
-  a.sp_m = sp_m;
-  a.sp_v = sp_v;
-  a.sp_upd = g->sp_upd;
-  a.asp = asp;
+  a.gs = g->sp_upd;  // g_s, replaced in place by S~ below
   a.B1img = (const uint8_t*)g->B1img;
   a.B2img = (const uint8_t*)g->B2img;
   const bool no_inner = first_active < 0;
   a.Y = no_inner ? (void*)g->C : (void*)g->Y;
   a.y_f32 = no_inner ? 1 : 0;
+  a.y_vec = a.y_f32 ? (g->ra % 2 == 0) : (g->ra % 4 == 0);
   a.err = d_err;
   // At least half the shared memory of an SM, so one CTA (and its 512 TMEM
   // columns) per SM.
@@ -1435,6 +1488,13 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   proj_stream_kernel<<<(unsigned)std::min<int64_t>(g->n_groups, g->num_sms), P1T, p1_launch_smem, s>>>(a);
   H(1, "proj_stream");
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p.k > 0) {
+    H(0, "sparse_adam");
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(p.k, 256), (int64_t)g->num_sms * 8);
+    sparse_adam_tc_kernel<<<blocks, 256, 0, s>>>(g->sp_upd, p.k, sp_m, sp_v, asp);
+    H(1, "sparse_adam");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   // ---- inner modes, innermost first; dims of the current tensor
   int64_t dims[8];
   for (int n = 0; n < d - 2; ++n) dims[n] = p.I[n];
