@@ -86,13 +86,48 @@ def kernel_algorithmic_bytes(name: str, wl) -> float:
 
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled during the timed region: an
+    NVML polling thread (read-only queries, every 2 ms), else nvidia-smi at
+    its 100 ms minimum. The samples are also written to gpurun_out/."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
+
     def __init__(self, index: int):
+        import threading
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        self.samples, self.proc, self.nv = [], None, None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.stop_ev = threading.Event()
+            self.th = threading.Thread(target=self._poll, daemon=True)
+            self.th.start()
+        except Exception:
+            self.nv = None
+            self._start_smi(index)
+
+    def _poll(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     int(get_reasons(self.h)),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1e3))
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def _start_smi(self, index):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-        self.proc = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
@@ -102,6 +137,18 @@ class ClockSampler:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.nv is not None:
+            self.stop_ev.set()
+            self.th.join(timeout=5)
+            with open(self.path, "w") as f:
+                f.write("time,sm_mhz,reasons_bits,power_w\n")
+                for t, mhz, bits, pw in self.samples:
+                    f.write(f"{t:.4f},{mhz},{bits:#x},{pw:.1f}\n")
+            sm = [x[1] for x in self.samples]
+            reasons = sorted({nm for _, _, bits, _ in self.samples
+                              for b, nm in self.REASONS.items() if bits & b})
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -126,79 +173,130 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
-def cpu_baseline_sample(wl, seed=0):
-    """The oracle, as it stands, on a bounded sample of the workload: the same
-    trailing modes and rank ratios with the leading modes cut down so that one
-    step takes seconds; one timed step after one untimed refresh."""
-    import numpy as np
-    import oracle
-    from rank_sparse_tensor_b200.synth import GradientStream, weights
-    shape, ranks = list(wl.shape), list(wl.ranks)
-    budget = 2_500_000
-    n = 0
-    while math.prod(shape) > budget and n < len(shape) - 2:
-        f = max(1, math.prod(shape) // budget)
-        new = max(1, shape[n] // min(f, shape[n]))
-        if new == shape[n]:
-            n += 1
-            continue
-        ratio = ranks[n] / shape[n]
-        shape[n] = new
-        ranks[n] = max(1, min(new, math.ceil(ratio * new)))
+def oracle_sample(wl, factor: int):
+    """The workload with its leading mode divided by `factor` (rank scaled
+    with it): the same trailing modes, ranks, dtype and generator."""
+    import dataclasses
+    sh, rk, gr = list(wl.shape), list(wl.ranks), list(wl.gen_ranks)
+    f = max(1, min(factor, sh[0]))
+    ratio = rk[0] / sh[0]
+    sh[0] //= f
+    rk[0] = max(1, min(sh[0], math.ceil(ratio * sh[0])))
+    gr[0] = max(1, min(sh[0], math.ceil(gr[0] / f)))
+    return dataclasses.replace(wl, name=f"{wl.name}/leading-mode/{f}", shape=tuple(sh),
+                               ranks=tuple(rk), gen_ranks=tuple(gr))
+
+
+class OracleRun:
+    """The oracle, as it stands (test infrastructure, never tuned for this),
+    on a sample of the workload: one untimed refresh, then timed steps."""
+
+    def __init__(self, wl, seed=0):
+        import oracle
+        from rank_sparse_tensor_b200.synth import GradientStream, weights
+        self.wl = wl
+        gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed, outlier_frac=wl.outlier_frac,
+                            outlier_scale=wl.outlier_scale)
+        self.g = [gs.next().numpy() for _ in range(2)]
+        self.w = weights(wl.shape, wl.weight_dtype, seed).numpy()
+        self.o = oracle.Oracle(wl.shape, wl.ranks, wl.sparse_ratio, 0, wl.lr, wl.betas, wl.eps,
+                               wl.wd, wl.dtype, wl.weight_dtype, auto_refresh=0)
+        self.o.refresh(self.g[0])
+        self.i = 0
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        self.o.step(self.g[1 - self.i % 2], self.w)
+        self.i += 1
+        return time.perf_counter() - t0
+
+    def describe(self, steps, seconds):
+        wl = self.wl
+        return (f"{steps} oracle steps (after one untimed refresh) on shape {tuple(wl.shape)} ranks "
+                f"{tuple(wl.ranks)}, {wl.dtype} gradients, rho {wl.sparse_ratio}: the workload with "
+                f"its leading mode cut down; {seconds:.1f} s of step time")
+
+
+def oracle_threads() -> int:
+    return int(os.environ.get("TGD_ORACLE_THREADS", "0")) or (os.cpu_count() or 1)
+
+
+def cpu_baseline(wl, target_s=10.0):
+    """Oracle throughput on a bounded sample (about `target_s` of step time)."""
+    run = OracleRun(oracle_sample(wl, 16), seed=0)
+    n, tot = 0, 0.0
+    while tot < target_s and n < 64:
+        tot += run.step()
         n += 1
-    gen = [min(g, s) for g, s in zip(wl.gen_ranks, shape)]
-    gs = GradientStream(shape, gen, wl.dtype, seed, outlier_frac=wl.outlier_frac,
-                        outlier_scale=wl.outlier_scale)
-    g0 = gs.next().numpy()
-    g1 = gs.next().numpy()
-    w = weights(shape, wl.weight_dtype, seed).numpy()
-    o = oracle.Oracle(shape, ranks, wl.sparse_ratio, 0, wl.lr, wl.betas, wl.eps, wl.wd,
-                      wl.dtype, wl.weight_dtype, auto_refresh=0)
-    o.refresh(g0)
-    t0 = time.perf_counter()
-    o.step(g1, w)
-    dt = time.perf_counter() - t0
-    N = math.prod(shape)
-    threads = int(os.environ.get("TGD_ORACLE_THREADS", "0")) or (os.cpu_count() or 1)
-    return {"value": N / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "_seconds": dt, "_elements": N,
-            "sample": f"one oracle step (after an untimed refresh) on shape {tuple(shape)} "
-                      f"ranks {tuple(ranks)}, {wl.dtype}, rho {wl.sparse_ratio}: the workload "
-                      f"with its leading modes cut down; {dt:.2f} s"}
+    N = math.prod(run.wl.shape)
+    return {"value": N * n / tot, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": run.describe(n, tot)}
 
 
 def run_reference(args, wl):
-    rank = int(os.environ.get("RANK", "0"))
+    """The reference arm: the oracle on the host cores, on this arm's metric,
+    each step a bounded sample of the workload (leading mode / 16). Under a
+    multi-rank launch rank 0 alone runs and prints; the others exit."""
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
-    samples = []
+    run = OracleRun(oracle_sample(wl, 16), seed=1)
     for _ in range(args.warmup):
-        cpu_baseline_sample(wl, seed=1)
-    for s in range(args.steps):
-        samples.append(cpu_baseline_sample(wl, seed=2 + s))
-    tot_elems = sum(x["_elements"] for x in samples)
-    tot_time = sum(x["_seconds"] for x in samples)
-    value = tot_elems / tot_time
+        run.step()
+    tot = sum(run.step() for _ in range(args.steps))
+    N = math.prod(run.wl.shape)
+    value = N * args.steps / tot
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * tot_time / max(1, args.steps), "higher_is_better": True,
+            "ms_per_step": 1e3 * tot / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "shape": list(wl.shape), "ranks": list(wl.ranks),
-                       "sparse_ratio": wl.sparse_ratio},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[0]["cores"],
-                             "kind": "oracle", "sample": samples[0]["sample"]},
+                       "sparse_ratio": wl.sparse_ratio, "sample_shape": list(run.wl.shape),
+                       "sample_ranks": list(run.wl.ranks)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(),
+                             "kind": "oracle", "sample": run.describe(args.steps, tot)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
+# ---------------------------------------------------------------- ranks
+def rank_env():
+    """(world, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def tensor_seeds(rank: int, n_tensors: int):
+    """Seeds of the independent tensors a rank steps (gradient, weight):
+    disjoint across ranks, so no two ranks hold the same problem."""
+    return [(1000 * rank + 17 * j + 1, 1000 * rank + j) for j in range(n_tensors)]
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's value (all ranks take this collective)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, elems_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job gradient elements/s: every rank's elements over the slowest
+    rank's time (weak scaling: each rank has its own tensors)."""
+    return world * elems_per_rank * steps / (max_ms / 1e3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -230,9 +328,7 @@ def main():
     import rank_sparse_tensor_b200 as rst
     from rank_sparse_tensor_b200.synth import GradientStream, weights
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -247,12 +343,12 @@ def main():
     # Inputs resident in HBM before the timed region.
     nt = wl.n_tensors if args.workload != DEFAULT_WORKLOAD else 1
     tensors = []
-    for j in range(nt):
-        gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=1000 * rank + 17 * j + 1,
+    for gseed, wseed in tensor_seeds(rank, nt):
+        gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=gseed,
                             outlier_frac=wl.outlier_frac, outlier_scale=wl.outlier_scale,
                             noise=wl.noise, drift=0.0, device=str(dev))
         grads = [gs.next() for _ in range(2)]
-        w = weights(wl.shape, wl.weight_dtype, seed=1000 * rank + j, device=str(dev))
+        w = weights(wl.shape, wl.weight_dtype, seed=wseed, device=str(dev))
         T = wl.T
         opt = rst.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, T, wl.lr, wl.betas, wl.eps, wl.wd,
                              wl.dtype, wl.weight_dtype, path=args.path)
@@ -274,37 +370,46 @@ def main():
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local)
-    for opt, _, _ in tensors:
-        opt.profile(True)
     stream = torch.cuda.current_stream()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        evs[i][0].record(stream)
-        one_step(i)
-        evs[i][1].record(stream)
-        if flush:
-            scratch.add_(1.0)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
+
+    def timed_steps(profile: bool):
+        """K steps between barriers, each bracketed by CUDA events on the
+        launching stream (L2 flushed between steps when inputs fit in it)."""
+        for opt, _, _ in tensors:
+            opt.profile(profile)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            one_step(i)
+            evs[i][1].record(stream)
+            if flush:
+                scratch.add_(1.0)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        prof = {}
+        for opt, _, _ in tensors:
+            opt.profile(False)
+            if profile:
+                for kname, (n, ms) in opt.profile_read().items():
+                    a = prof.setdefault(kname, [0, 0.0])
+                    a[0] += n
+                    a[1] += ms
+        return sum(a.elapsed_time(b) for a, b in evs), prof
+
+    # the metric: K steps without per-kernel events; then K more with them,
+    # for the per-kernel launch times of the roofline
+    sampler = ClockSampler(local)
+    total_ms, _ = timed_steps(False)
     clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    prof = {}
-    for opt, _, _ in tensors:
-        opt.profile(False)
-        for kname, (n, ms) in opt.profile_read().items():
-            a = prof.setdefault(kname, [0, 0.0])
-            a[0] += n
-            a[1] += ms
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    _, prof = timed_steps(True)
+    max_ms = max_over_ranks(total_ms, world, dev)
     n_elems = wl.N * len(tensors)
-    value = world * n_elems * args.steps / (max_ms / 1e3)
+    value = job_throughput(world, n_elems, args.steps, max_ms)
 
     # End to end through the host-buffer entry point: H2D of the gradient and
     # the weights, the step, D2H of the updated weights, every step.
@@ -321,10 +426,8 @@ def main():
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
             opt.step_host(gh_np, wh_np)
-        el = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(el, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * wl.N * args.e2e_steps / float(el.item()), "unit": UNIT,
+        el = max_over_ranks(time.perf_counter() - t0, world, dev)
+        e2e = {"value": job_throughput(world, wl.N, args.e2e_steps, 1e3 * el), "unit": UNIT,
                "h2d_bytes_per_step": gh.numel() * gh.element_size() + wh.numel() * wh.element_size(),
                "d2h_bytes_per_step": wh.numel() * wh.element_size()}
 
@@ -360,13 +463,12 @@ def main():
                      "step_achieved_gbs": ab["total"] / (step_ms / 1e3) / 1e9,
                      "step_frac": ab["total"] / (step_ms / 1e3) / 1e9 / hbm_gbs},
         "kernels": {k: {"launches": v[0], "ms_total": round(v[1], 4)} for k, v in prof.items()},
-        "gpu_launches": int(sum(v[0] for v in prof.values())),
+        "gpu_launches": int(sum(v[0] for v in prof.values())),  # per K steps (profiled pass)
         "clocks": clocks,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline_sample(wl)
-        line["cpu_baseline"] = {k: v for k, v in cb.items() if not k.startswith("_")}
+        line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
     for opt, _, _ in tensors:
