@@ -523,14 +523,16 @@ struct MGArgs {
 // Y[a][j][b] = sum_k X[a][k][b] M[k][j] (complex, bf16 in, fp32 accumulate).
 // Rows of the GEMM are 128 consecutive (a, b) positions; each thread gathers
 // its row's K values (coalesced across threads), so any mode is contracted
-// without a transpose in memory.
+// without a transpose in memory. K advances in chunks of 32 complex values:
+// the next chunk's values are loaded into registers while the current
+// chunk's MMAs run, and the operand image chunk arrives by bulk copy.
 __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t a_bytes = 8 * LBO_M128;               // 128 rows x 64 K
   const uint32_t b_bytes = (uint32_t)p.NT * 64 * 2;
   uint8_t* As[2] = {smem, smem + a_bytes};
   uint8_t* Bs[2] = {smem + 2 * a_bytes, smem + 2 * a_bytes + b_bytes};
-  uint64_t* bars = (uint64_t*)(smem + 2 * a_bytes + 2 * b_bytes);
+  uint64_t* bars = (uint64_t*)(smem + 2 * a_bytes + 2 * b_bytes);  // [0,1] MMA done, [2,3] B landed
   uint32_t* tslot = (uint32_t*)(bars + 4);
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -541,8 +543,7 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
   const uint32_t* xrow = p.X + a * p.K * p.in_bs + b;
   if (tid == 0) {
     s_abort = 0;
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -554,8 +555,8 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
   const uint32_t lbo_b = (uint32_t)(p.NT / 8) * 128;
   const uint32_t idesc = idesc_f16(1, 128, p.NT);
   const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * b_bytes;
-  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
-  // One thread polls (bounded), the rest sleep in the barrier.
+  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0}, bloaded[2] = {0, 0};
+  // One thread waits (bounded), the rest sleep in the barrier.
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (tid == 0 && !mbar_wait(bar, parity, WAIT_NS)) {
       atomicOr(p.err, DEV_ERR_TIMEOUT);
@@ -564,6 +565,15 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
     __syncthreads();
     return s_abort == 0;
   };
+  uint32_t v[32];
+  auto load_x = [&](int kc) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t k = (int64_t)kc * 32 + i;
+      v[i] = (valid && k < p.K) ? __ldg(xrow + k * p.in_bs) : 0u;
+    }
+  };
+  load_x(0);
   for (int kc = 0; kc < p.nkc; ++kc) {
     const int s = kc & 1;
     if (kc >= 2) {
@@ -572,31 +582,33 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
       if (!ok) break;
       tc_fence_after();
     }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        int64_t k = (int64_t)kc * 32 + 4 * q + u;
-        v[u] = (valid && k < p.K) ? __ldg(xrow + k * p.in_bs) : 0u;
-      }
-      *(uint4*)(As[s] + q * LBO_M128 + tid * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+    if (tid == 0) {
+      mbar_expect_tx(&bars[2 + s], b_bytes);
+      bulk_g2s(Bs[s], img + (int64_t)kc * b_bytes, b_bytes, &bars[2 + s]);
+      bloaded[s]++;
     }
-    const uint4* src = (const uint4*)(img + (int64_t)kc * b_bytes);
-    for (uint32_t i = tid; i < b_bytes / 16; i += MGT) ((uint4*)Bs[s])[i] = __ldg(src + i);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      *(uint4*)(As[s] + q * LBO_M128 + tid * 16) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    if (kc + 1 < p.nkc) load_x(kc + 1);  // in flight during this chunk's MMAs
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (s_abort) break;
     if (tid == 0) {
-      const uint32_t sa = smem_u32(As[s]), sb = smem_u32(Bs[s]);
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(dt, sdesc(sa + kk * 2 * LBO_M128, LBO_M128, 128), sdesc(sb + kk * 2 * lbo_b, lbo_b, 128),
-                idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(&bars[s]);
+      if (!mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, WAIT_NS)) {
+        atomicOr(p.err, DEV_ERR_TIMEOUT);
+        s_abort = 1;
+      } else {
+        const uint32_t sa = smem_u32(As[s]), sb = smem_u32(Bs[s]);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(dt, sdesc(sa + kk * 2 * LBO_M128, LBO_M128, 128), sdesc(sb + kk * 2 * lbo_b, lbo_b, 128),
+                  idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[s]);
+        issued[s]++;
+      }
     }
-    issued[s]++;
   }
   __syncthreads();
   if (!s_abort) {
@@ -608,23 +620,26 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
   if (!s_abort) {
     const int64_t j0 = (int64_t)blockIdx.y * (p.NT / 2);
     for (int c0 = 0; c0 < p.NT; c0 += 16) {
-      float v[16];
-      tmem_ld16(dt + lane_base + c0, v);
+      float y[16];
+      tmem_ld16(dt + lane_base + c0, y);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         int64_t j = j0 + c0 / 2 + u;
         if (valid && j < p.J) {
           int64_t o = (a * p.J + j) * p.out_bs + b;
           if (p.y_f32)
-            ((float2*)p.Y)[o] = make_float2(v[2 * u], v[2 * u + 1]);
+            ((float2*)p.Y)[o] = make_float2(y[2 * u], y[2 * u + 1]);
           else
-            ((uint32_t*)p.Y)[o] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+            ((uint32_t*)p.Y)[o] = f2_to_bf2(y[2 * u], y[2 * u + 1]);
         }
       }
     }
   } else if (tid == 0) {
-    for (int s = 0; s < 2; ++s)
+    // bounded waits for the copies and MMAs still in flight
+    for (int s = 0; s < 2; ++s) {
       if (issued[s] > waited[s]) mbar_wait(&bars[s], (issued[s] - 1) & 1u, WAIT_NS / 4);
+      if (bloaded[s] > 0) mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, WAIT_NS / 4);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -696,6 +711,7 @@ struct R3Args {
   float decay, lr;
   int* err;
   int nstage, cap;
+  uint32_t lbo_b1;  // GEMM1's B: K-adjacent core matrices N1 / 8 * 128 + 16 B apart
   uint32_t w_tile_bytes, y_tile_bytes;
   uint32_t off_w, off_y, off_A1, off_B1, off_A2, off_B2, off_ds, off_bar;
 };
@@ -740,7 +756,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   const int ns = p.nstage;
   auto wst = [&](int s) { return smem + p.off_w + (uint32_t)s * p.w_tile_bytes; };
   auto yst = [&](int s) { return smem + p.off_y + (uint32_t)s * p.y_tile_bytes; };
-  auto B1b = [&](int b) { return smem + p.off_B1 + (uint32_t)b * (uint32_t)(p.N1 * p.K1 * 2); };
+  auto B1b = [&](int b) { return smem + p.off_B1 + (uint32_t)b * (uint32_t)(p.K1 / 8) * p.lbo_b1; };
   auto A2b = [&](int b) { return smem + p.off_A2 + (uint32_t)b * (uint32_t)(p.K2 / 8) * LBO_M128; };
   const int wb = (int)sizeof(WT);
   auto tile_wbytes = [&](int64_t t) -> uint32_t {
@@ -770,7 +786,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     fence_mbar_init();
   }
   {
-    const uint32_t b1b = (uint32_t)(2 * p.N1 * p.K1 * 2);
+    const uint32_t b1b = (uint32_t)(2 * (p.K1 / 8)) * p.lbo_b1;
     for (uint32_t i = tid; i < b1b / 16; i += R3T) ((uint4*)(smem + p.off_B1))[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
@@ -822,7 +838,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
+      const uint32_t lbo_b1 = p.lbo_b1, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
       const uint32_t id1 = idesc_f16(1, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
       const uint32_t sA1 = smem_u32(A1), sB2 = smem_u32(B2);
       bool ok = wait1(opnd, 0, s_abort, p.err);
@@ -873,8 +889,8 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     // ------------------------------------------------------------ prep
     const int row = tid - 128;  // 0..127, TMEM lane of warps 4-7
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128;
-    const int blk = p.rb * p.ra;
+    const int nkc = p.K1 / 8;  // 16-byte K chunks of a B1 row (4 complex j_a each)
+    const bool vec = (p.ra & 3) == 0;  // a chunk's 4 j_a lie in one slab, 16-byte aligned
     bool ok = true;
     auto build = [&](int64_t it) -> bool {
       const int b = (int)(it & 1), s = (int)(it % ns);
@@ -882,16 +898,41 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       const int64_t t = blockIdx.x + it * G;
       if (!waitw(&full[s], (uint32_t)((it / ns) & 1), s_abort, p.err)) return false;
       if (!waitw(&b1empty[b], par ^ 1u, s_abort, p.err)) return false;
-      // B1: rows (j_b, re/im), K = (slab, j_a, re/im), entries [[Yr, -Yi], [Yi, Yr]]
+      // B1: rows (j_b, re/im), K = (slab, j_a, re/im), entries [[Yr, -Yi], [Yi, Yr]];
+      // one item = one K chunk of rows 2 j_b and 2 j_b + 1 (two 16-byte stores)
       uint8_t* B1 = B1b(b);
       const uint32_t* ys = (const uint32_t*)yst(s);
-      const int64_t vslabs = p.n_slabs - t * p.spb;
-      for (int e = row; e < p.spb * blk; e += 128) {
-        const int sl = e / blk, r2 = e - sl * blk, jb = r2 / p.ra, ja = r2 - jb * p.ra;
-        float2 y = sl < vslabs ? bf2_to_f2(ys[sl * p.yp_bs + r2]) : make_float2(0.f, 0.f);
-        const uint32_t k = (uint32_t)(sl * 2 * p.ra + 2 * ja);
-        *(uint32_t*)(B1 + kmaj_off((uint32_t)(2 * jb), k, lbo_b1)) = f2_to_bf2(y.x, -y.y);
-        *(uint32_t*)(B1 + kmaj_off((uint32_t)(2 * jb + 1), k, lbo_b1)) = f2_to_bf2(y.y, y.x);
+      const int64_t vs = p.n_slabs - t * p.spb;
+      const int vslabs = vs < p.spb ? (int)vs : p.spb;
+      for (int e = row; e < p.rb * nkc; e += 128) {
+        const int kc = e % nkc, jb = e / nkc;
+        uint32_t yv[4];
+        if (vec) {
+          const int sl = 4 * kc / p.ra, ja0 = 4 * kc - sl * p.ra;
+          uint4 y4 = make_uint4(0, 0, 0, 0);
+          if (sl < vslabs) y4 = *(const uint4*)(ys + sl * p.yp_bs + jb * p.ra + ja0);
+          yv[0] = y4.x;
+          yv[1] = y4.y;
+          yv[2] = y4.z;
+          yv[3] = y4.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int kp = 4 * kc + u, sl = kp / p.ra, ja = kp - sl * p.ra;
+            yv[u] = sl < vslabs ? ys[sl * p.yp_bs + jb * p.ra + ja] : 0u;
+          }
+        }
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 y = bf2_to_f2(yv[u]);
+          lo[u] = f2_to_bf2(y.x, -y.y);
+          hi[u] = f2_to_bf2(y.y, y.x);
+        }
+        *(uint4*)(B1 + kmaj_off((uint32_t)(2 * jb), (uint32_t)(8 * kc), p.lbo_b1)) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *(uint4*)(B1 + kmaj_off((uint32_t)(2 * jb + 1), (uint32_t)(8 * kc), p.lbo_b1)) =
+            make_uint4(hi[0], hi[1], hi[2], hi[3]);
       }
       fence_async_smem();
       mbar_arrive(&b1full[b]);
@@ -1178,10 +1219,12 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
   wt = (wt + 127) / 128 * 128;
   yt = (yt + 127) / 128 * 128;
   uint32_t w = take(wt * nstage), y = take(yt * nstage);
-  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), b1 = take((size_t)2 * N1 * K1 * 2);
+  const uint32_t lbo_b1 = (uint32_t)(N1 / 8) * 128 + 16;
+  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), b1 = take((size_t)2 * (K1 / 8) * lbo_b1);
   uint32_t a2 = take((size_t)2 * (K2 / 8) * LBO_M128), b2 = take((size_t)N2 * K2 * 2);
   uint32_t dsb = take((size_t)128 * Ib * 4), bar = take(256);
   if (a) {
+    a->lbo_b1 = lbo_b1;
     a->w_tile_bytes = (uint32_t)wt;
     a->y_tile_bytes = (uint32_t)yt;
     a->off_w = w;
