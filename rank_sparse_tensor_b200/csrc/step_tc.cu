@@ -728,7 +728,8 @@ struct R3Args {
 //            the staged W tile (column halves per warpgroup).
 // Roles hand off through mbarriers; operands, lists and accumulators are
 // double-buffered, so consecutive tiles overlap.
-template <class WT>
+// UNIT_DECAY: lr * wd == 0, so W (1 - lr wd) is W itself (no multiply).
+template <class WT, bool UNIT_DECAY>
 __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* A1 = smem + p.off_A1;
@@ -1039,9 +1040,13 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
             d[u] = h2_to_f2(drow[ib0 + u]);
           }
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            wstore(wrow + ib0 + u, __fmaf_rn(nlr, v[2 * u] + d[u].x, w[u].x * decay),
-                   __fmaf_rn(nlr, v[2 * u + 1] + d[u].y, w[u].y * decay));
+          for (int u = 0; u < 8; ++u) {
+            const float xr = v[2 * u] + d[u].x, xi = v[2 * u + 1] + d[u].y;
+            if (UNIT_DECAY)
+              wstore(wrow + ib0 + u, __fmaf_rn(nlr, xr, w[u].x), __fmaf_rn(nlr, xi, w[u].y));
+            else
+              wstore(wrow + ib0 + u, __fmaf_rn(nlr, xr, w[u].x * decay), __fmaf_rn(nlr, xi, w[u].y * decay));
+          }
         } else {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -1637,19 +1642,19 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   r.err = d_err;
   const size_t r3_launch_smem = std::max(g->r3_smem, ONE_CTA_SMEM);
   const unsigned r3_grid = (unsigned)std::min<int64_t>(g->n_tiles, g->num_sms);
-  if (r.w_c64) {
-    e = cudaFuncSetAttribute(recon_stream_kernel<float2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)r3_launch_smem);
-    if (e != cudaSuccess) return e;
+  auto launch_r3 = [&](auto kern) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r3_launch_smem);
+    if (err != cudaSuccess) return err;
     H(0, "recon_stream");
-    recon_stream_kernel<float2><<<r3_grid, R3T, r3_launch_smem, s>>>(r);
-  } else {
-    e = cudaFuncSetAttribute(recon_stream_kernel<__half2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)r3_launch_smem);
-    if (e != cudaSuccess) return e;
-    H(0, "recon_stream");
-    recon_stream_kernel<__half2><<<r3_grid, R3T, r3_launch_smem, s>>>(r);
-  }
+    kern<<<r3_grid, R3T, r3_launch_smem, s>>>(r);
+    return cudaSuccess;
+  };
+  const bool unit = decay == 1.0f;
+  if (r.w_c64)
+    e = unit ? launch_r3(recon_stream_kernel<float2, true>) : launch_r3(recon_stream_kernel<float2, false>);
+  else
+    e = unit ? launch_r3(recon_stream_kernel<__half2, true>) : launch_r3(recon_stream_kernel<__half2, false>);
+  if (e != cudaSuccess) return e;
   H(1, "recon_stream");
   return cudaGetLastError();
 }
