@@ -692,6 +692,7 @@ __device__ __forceinline__ float2 wload(const float2* p) { return *p; }
 __device__ __forceinline__ void wstore(float2* p, float x, float y) { *p = make_float2(x, y); }
 
 constexpr int R3T = 512;
+constexpr int R3_NS_MAX = 6;  // W stages
 constexpr int EPF = 4;  // Omega entries per epilogue thread prefetched for the next tile
 
 struct R3Args {
@@ -702,7 +703,7 @@ struct R3Args {
   int64_t N, n_slabs, n_tiles, tile_elems;
   int Ia, Ib, ra, rb, spb, log2Ia;
   int K1, N1, K2, N2;
-  uint32_t d1_col[2], d2_col[2];
+  uint32_t d1_col[2], d2_col[2], a1_col, a2_col[2];  // TMEM columns
   const int64_t* tile_off;
   const uint16_t* loc;
   const uint32_t* sp_upd;
@@ -713,7 +714,7 @@ struct R3Args {
   int nstage, cap;
   uint32_t lbo_b1;  // GEMM1's B: K-adjacent core matrices N1 / 8 * 128 + 16 B apart
   uint32_t w_tile_bytes, y_tile_bytes;
-  uint32_t off_w, off_y, off_A1, off_B1, off_A2, off_B2, off_ds, off_bar;
+  uint32_t off_w, off_y, off_B1, off_B2, off_ds, off_bar;
 };
 
 // Warp-specialised reconstruction stream, one CTA per SM, persistent over
@@ -721,7 +722,9 @@ struct R3Args {
 //   warp 0   producer: bulk copies W(t), Y'(t) into a ring of stages, and
 //            bulk-stores each W tile once its epilogue is done;
 //   warp 1   MMA issuer: GEMM1(t) = A1 x B1(t) -> D1[t&1], GEMM2(t) =
-//            A2(t) x B2 -> D2[t&1];
+//            A2(t) x B2 -> D2[t&1]; both A operands live in TMEM (A1 the
+//            constant U_a image, written once; A2 = P'(t), two buffers), so
+//            shared memory holds up to six W stages;
 //   warps 4-7   prep: B1(t+1) from Y'(t+1), the tile's Omega list and
 //            per-row start table, then P'(t) from D1 into A2[t&1];
 //   warps 8-15  epilogue: Delta(t) from D2 + lambda S~ on Omega, AdamW on
@@ -732,22 +735,21 @@ struct R3Args {
 template <class WT, bool UNIT_DECAY>
 __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* A1 = smem + p.off_A1;
   uint8_t* B2 = smem + p.off_B2;
   uint64_t* bars = (uint64_t*)(smem + p.off_bar);
   // barrier map
-  uint64_t* full = bars;           // [4] stage loaded
-  uint64_t* wdone = bars + 4;      // [4] W tile updated (256 arrivals)
-  uint64_t* opnd = bars + 8;       // A1 + B2 loaded
-  uint64_t* b1full = bars + 9;     // [2] (128)
-  uint64_t* b1empty = bars + 11;   // [2] (commit)
-  uint64_t* d1full = bars + 13;    // [2] (commit)
-  uint64_t* d1empty = bars + 15;   // [2] (128)
-  uint64_t* a2full = bars + 17;    // [2] (128)
-  uint64_t* a2empty = bars + 19;   // [2] (commit)
-  uint64_t* d2full = bars + 21;    // [2] (commit)
-  uint64_t* d2empty = bars + 23;   // [2] (256)
-  uint32_t* tslot = (uint32_t*)(bars + 26);
+  uint64_t* full = bars;           // [6] stage loaded
+  uint64_t* wdone = bars + 6;      // [6] W tile updated (256 arrivals)
+  uint64_t* opnd = bars + 12;      // B2 loaded
+  uint64_t* b1full = bars + 13;    // [2] (128)
+  uint64_t* b1empty = bars + 15;   // [2] (commit)
+  uint64_t* d1full = bars + 17;    // [2] (commit)
+  uint64_t* d1empty = bars + 19;   // [2] (128)
+  uint64_t* a2full = bars + 21;    // [2] (128)
+  uint64_t* a2empty = bars + 23;   // [2] (commit)
+  uint64_t* d2full = bars + 25;    // [2] (commit)
+  uint64_t* d2empty = bars + 27;   // [2] (256)
+  uint32_t* tslot = (uint32_t*)(bars + 29);
   __shared__ int s_abort_storage;
   volatile int* s_abort = &s_abort_storage;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -758,7 +760,6 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   auto wst = [&](int s) { return smem + p.off_w + (uint32_t)s * p.w_tile_bytes; };
   auto yst = [&](int s) { return smem + p.off_y + (uint32_t)s * p.y_tile_bytes; };
   auto B1b = [&](int b) { return smem + p.off_B1 + (uint32_t)b * (uint32_t)(p.K1 / 8) * p.lbo_b1; };
-  auto A2b = [&](int b) { return smem + p.off_A2 + (uint32_t)b * (uint32_t)(p.K2 / 8) * LBO_M128; };
   const int wb = (int)sizeof(WT);
   auto tile_wbytes = [&](int64_t t) -> uint32_t {
     int64_t rem = p.N - t * p.tile_elems;
@@ -771,8 +772,8 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
 
   if (tid == 0) {
     *s_abort = 0;
-    for (int i = 0; i < 4; ++i) mbar_init(&full[i], 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&wdone[i], 256);
+    for (int i = 0; i < R3_NS_MAX; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < R3_NS_MAX; ++i) mbar_init(&wdone[i], 256);
     mbar_init(opnd, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&b1full[b], 128);
@@ -796,13 +797,27 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  if (warp >= 4 && warp < 8) {
+    // GEMM1's A (the U_a image, K-major in global memory) -> TMEM, row per lane
+    const int row = tid - 128;
+    const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + p.a1_col;
+    for (int kc = 0; kc < p.K1 / 8; kc += 2) {
+      const uint4 x = __ldg((const uint4*)(p.A1img + kmaj_off((uint32_t)row, (uint32_t)(8 * kc), LBO_M128)));
+      const uint4 y = __ldg((const uint4*)(p.A1img + kmaj_off((uint32_t)row, (uint32_t)(8 * kc + 8), LBO_M128)));
+      const uint32_t w[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+      tmem_st8(taddr + 4 * kc, w);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t a1b = (uint32_t)(p.K1 / 8) * LBO_M128, b2b = (uint32_t)(p.N2 * p.K2 * 2);
-      mbar_expect_tx(opnd, a1b + b2b);
-      bulk_g2s(A1, p.A1img, a1b, opnd);
+      const uint32_t b2b = (uint32_t)(p.N2 * p.K2 * 2);
+      mbar_expect_tx(opnd, b2b);
       bulk_g2s(B2, p.B2img, b2b, opnd);
       auto load = [&](int64_t it) {
         const int s = (int)(it % ns);
@@ -841,7 +856,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     if (lane == 0) {
       const uint32_t lbo_b1 = p.lbo_b1, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
       const uint32_t id1 = idesc_f16(1, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
-      const uint32_t sA1 = smem_u32(A1), sB2 = smem_u32(B2);
+      const uint32_t sB2 = smem_u32(B2);
       bool ok = wait1(opnd, 0, s_abort, p.err);
       auto gemm1 = [&](int64_t it) -> bool {
         const int b = (int)(it & 1);
@@ -851,8 +866,8 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
         tc_fence_after();
         const uint32_t sB1 = smem_u32(B1b(b));
         for (int kk = 0; kk < p.K1 / 16; ++kk)
-          mma_f16(tmem + p.d1_col[b], sdesc(sA1 + kk * 2 * LBO_M128, LBO_M128, 128),
-                  sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128), id1, kk > 0);
+          mma_f16_ts(tmem + p.d1_col[b], tmem + p.a1_col + kk * 8, sdesc(sB1 + kk * 2 * lbo_b1, lbo_b1, 128),
+                     id1, kk > 0);
         mma_commit(&d1full[b]);
         mma_commit(&b1empty[b]);
         return true;
@@ -872,10 +887,9 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
         if (!wait1(&a2full[b], par, s_abort, p.err)) break;
         if (!wait1(&d2empty[b], par ^ 1u, s_abort, p.err)) break;
         tc_fence_after();
-        const uint32_t sA2 = smem_u32(A2b(b));
         for (int kk = 0; kk < p.K2 / 16; ++kk)
-          mma_f16(tmem + p.d2_col[b], sdesc(sA2 + kk * 2 * LBO_M128, LBO_M128, 128),
-                  sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
+          mma_f16_ts(tmem + p.d2_col[b], tmem + p.a2_col[b] + kk * 8, sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128),
+                     id2, kk > 0);
         mma_commit(&d2full[b]);
         mma_commit(&a2empty[b]);
         g2_done = it + 1;
@@ -948,19 +962,18 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       if (!waitw(&d1full[b], par, s_abort, p.err)) break;
       if (!waitw(&a2empty[b], par ^ 1u, s_abort, p.err)) break;
       tc_fence_after();
-      uint8_t* A2 = A2b(b);
+      // P' row (bf16 pairs) -> TMEM, the A operand of GEMM2
       for (int c0 = 0; c0 < p.N1; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
         uint32_t w[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) w[u] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
-        *(uint4*)(A2 + (c0 / 8) * LBO_M128 + row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *(uint4*)(A2 + (c0 / 8 + 1) * LBO_M128 + row * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        tmem_st8(tmem + p.a2_col[b] + lane_base + c0 / 2, w);
       }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&d1empty[b]);
-      fence_async_smem();
       mbar_arrive(&a2full[b]);
     }
   } else if (warp >= 8) {
@@ -1223,20 +1236,18 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
   size_t wt = (size_t)128 * Ib * wbytes, yt = (size_t)spb * yp_bs * 4;
   wt = (wt + 127) / 128 * 128;
   yt = (yt + 127) / 128 * 128;
-  uint32_t w = take(wt * nstage), y = take(yt * nstage);
   const uint32_t lbo_b1 = (uint32_t)(N1 / 8) * 128 + 16;
-  uint32_t a1 = take((size_t)(K1 / 8) * LBO_M128), b1 = take((size_t)2 * (K1 / 8) * lbo_b1);
-  uint32_t a2 = take((size_t)2 * (K2 / 8) * LBO_M128), b2 = take((size_t)N2 * K2 * 2);
+  uint32_t w = take(wt * nstage), y = take(yt * nstage);
+  uint32_t b1 = take((size_t)2 * (K1 / 8) * lbo_b1), b2 = take((size_t)N2 * K2 * 2);
   uint32_t dsb = take((size_t)128 * Ib * 4), bar = take(256);
+  (void)K2;
   if (a) {
     a->lbo_b1 = lbo_b1;
     a->w_tile_bytes = (uint32_t)wt;
     a->y_tile_bytes = (uint32_t)yt;
     a->off_w = w;
     a->off_y = y;
-    a->off_A1 = a1;
     a->off_B1 = b1;
-    a->off_A2 = a2;
     a->off_B2 = b2;
     a->off_ds = dsb;
     a->off_bar = bar;
@@ -1244,8 +1255,6 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
   return off;
 }
 
-// Dynamic shared memory per CTA: the 227 KB opt-in maximum less 1 KB for the
-// kernels' static shared variables (the launch fails if the sum exceeds it).
 constexpr size_t SMEM_LIMIT = 227 * 1024 - 1024;
 constexpr size_t ONE_CTA_SMEM = 120 * 1024;
 constexpr int R3_CAP = 1024;
@@ -1297,15 +1306,19 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
   }
   if (g.p1_smem > SMEM_LIMIT) return false;
   // TMEM (512 columns): P1 holds D1 twice, D2 and GEMM1's A twice (K1 / 2
-  // columns each); R3 holds D1 and D2 twice.
+  // columns each); R3 holds D1 and D2 twice, its GEMM1's A once and its
+  // GEMM2's A twice.
   auto r32 = [](int x) { return (x + 31) / 32 * 32; };
   if (2 * r32(g.N1) + r32(g.N2) + 2 * r32(g.K1 / 2) > 512) return false;
-  if (2 * r32(g.rN1) + r32(g.rN2) + g.rN2 > 512) return false;
+  if (2 * r32(g.rN1) + 2 * r32(g.rN2) + r32(g.rK1 / 2) + 2 * r32(g.rK2 / 2) > 512) return false;
+  // Reconstruction: as many W stages as fit (it is bound by the bytes it
+  // keeps in flight), at least three.
   int wbytes = wdt == TGD_C64 ? 8 : 4;
-  size_t r3a = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 4, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
-  size_t r3b = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, 3, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP, nullptr);
-  g.r3_nstage = r3a <= SMEM_LIMIT ? 4 : 3;
-  g.r3_smem = r3a <= SMEM_LIMIT ? r3a : r3b;
+  for (g.r3_nstage = R3_NS_MAX; g.r3_nstage >= 3; --g.r3_nstage) {
+    g.r3_smem = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, g.r3_nstage, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP,
+                              nullptr);
+    if (g.r3_smem <= SMEM_LIMIT) break;
+  }
   if (g.r3_smem > SMEM_LIMIT) return false;
   g.inner.clear();
   for (int n = 0; n < nd - 2; ++n) {
@@ -1606,11 +1619,16 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   const int wbytes = g->wdt == TGD_C64 ? 8 : 4;
   r.nstage = g->r3_nstage;
   {
-    const uint32_t n1 = (uint32_t)((g->rN1 + 31) / 32 * 32), n2 = (uint32_t)((g->rN2 + 31) / 32 * 32);
+    // TMEM columns: D1 x2, D2 x2, A1 (the U_a image), A2 x2; 32-column aligned
+    auto r32c = [](int x) { return (uint32_t)((x + 31) / 32 * 32); };
+    const uint32_t n1 = r32c(g->rN1), n2 = r32c(g->rN2), na1 = r32c(g->rK1 / 2), na2 = r32c(g->rK2 / 2);
     r.d1_col[0] = 0;
     r.d1_col[1] = n1;
     r.d2_col[0] = 2 * n1;
     r.d2_col[1] = 2 * n1 + n2;
+    r.a1_col = 2 * n1 + 2 * n2;
+    r.a2_col[0] = r.a1_col + na1;
+    r.a2_col[1] = r.a1_col + na1 + na2;
   }
   r3_smem_bytes(g->Ib, g->spb, g->bs_pad, wbytes, r.nstage, g->rK1, g->rN1, g->rK2, g->rN2, R3_CAP, &r);
   r.cap = R3_CAP;
