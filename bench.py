@@ -136,10 +136,21 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def mark(self, start: bool):
+        """Bounds of the timed region (samples outside it are dropped)."""
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
     def stop(self) -> dict:
         if self.nv is not None:
             self.stop_ev.set()
             self.th.join(timeout=5)
+            t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+            inside = [x for x in self.samples if t0 <= x[0] <= t1]
+            # the nearest samples on either side when the region is shorter than the period
+            self.samples = inside or self.samples[-2:]
             with open(self.path, "w") as f:
                 f.write("time,sm_mhz,reasons_bits,power_w\n")
                 for t, mhz, bits, pw in self.samples:
@@ -404,7 +415,10 @@ def main():
     # the metric: K steps without per-kernel events; then K more with them,
     # for the per-kernel launch times of the roofline
     sampler = ClockSampler(local)
+    time.sleep(0.05)  # the polling thread is running before the timed region
+    sampler.mark(True)
     total_ms, _ = timed_steps(False)
+    sampler.mark(False)
     clocks = sampler.stop()
     _, prof = timed_steps(True)
     max_ms = max_over_ranks(total_ms, world, dev)

@@ -116,7 +116,7 @@ struct P1Args {
   int Ia, Ib, ra, rb, spb, q, sg, log2Ia;
   int K1, N1, K2, N2;
   uint32_t lbo_a2;  // GEMM2's A: 64 or 128 physical rows (see geometry)
-  uint32_t d1_col[2], d2_col, a1_col[2];  // TMEM columns
+  uint32_t d1_col[2], d2_col[2], a1_col[2];  // TMEM columns
   const int64_t* tile_off;
   const uint16_t* loc;
   uint32_t* gs;  // out: g_s = G[Omega] (fp16 pairs), Omega order
@@ -151,13 +151,15 @@ struct TileCursor {
 //            then write the residual rows into TMEM as GEMM1's A operand
 //            (tcgen05.st), two buffers;
 //   warp 1   MMA issuer: GEMM1(t) = A1[t & 1] (TMEM) x B1 -> D1[t & 1];
-//            per group GEMM2 = A2 x B2 -> D2;
-//   warps 12-15 epilogue: P(t) from D1 into the group's GEMM2 operand, Y of
-//            the group from D2.
+//            per group g GEMM2 = A2[g & 1] x B2 -> D2[g & 1];
+//   warps 12-15 epilogue: P(t) from D1 into the group's GEMM2 operand; Y
+//            of group g from D2 once the first tile of group g + 1 is
+//            drained (so the wait for GEMM2 never stalls the D1 drain).
 // Roles hand off through mbarriers.
 __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* A2 = smem + p.off_A2;
+  const uint32_t a2_bytes = (uint32_t)(p.K2 / 8) * p.lbo_a2;
+  auto A2b = [&](int64_t g) { return smem + p.off_A2 + (uint32_t)(g & 1) * a2_bytes; };
   uint8_t* B1 = smem + p.off_B1;
   uint8_t* B2 = smem + p.off_B2;
   uint64_t* bars = (uint64_t*)(smem + p.off_bar);
@@ -168,9 +170,10 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
   uint64_t* d1full = bars + 12;   // [2] (commit)
   uint64_t* d1empty = bars + 14;  // [2] (128)
   uint64_t* opnd = bars + 16;     // B1 + B2 loaded
-  uint64_t* a2full = bars + 17;   // (128)
-  uint64_t* d2full = bars + 18;   // (commit)
-  uint32_t* tslot = (uint32_t*)(bars + 19);
+  uint64_t* a2full = bars + 17;   // [2] (128)
+  uint64_t* d2full = bars + 19;   // [2] (commit)
+  uint64_t* d2empty = bars + 21;  // [2] (128)
+  uint32_t* tslot = (uint32_t*)(bars + 23);
   __shared__ int s_abort_storage;
   volatile int* s_abort = &s_abort_storage;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -199,13 +202,15 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       mbar_init(&d1empty[b], 128);
     }
     mbar_init(opnd, 1);
-    mbar_init(a2full, 128);
-    mbar_init(d2full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&a2full[b], 128);
+      mbar_init(&d2full[b], 1);
+      mbar_init(&d2empty[b], 128);
+    }
     fence_mbar_init();
   }
   {
-    const uint32_t a2b = (uint32_t)(p.K2 / 8) * p.lbo_a2;
-    for (uint32_t i = tid; i < a2b / 16; i += P1T) ((uint4*)A2)[i] = make_uint4(0, 0, 0, 0);
+    for (uint32_t i = tid; i < 2 * a2_bytes / 16; i += P1T) ((uint4*)(smem + p.off_A2))[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
   }
   __syncthreads();
@@ -252,20 +257,22 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     if (lane == 0) {
       const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
       const uint32_t id1 = idesc_f16(0, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
-      const uint32_t sA2 = smem_u32(A2), sB1 = smem_u32(B1), sB2 = smem_u32(B2);
+      const uint32_t sB1 = smem_u32(B1), sB2 = smem_u32(B2);
       bool ok = wait1(opnd, 0, s_abort, p.err);
       TileCursor c{(int64_t)blockIdx.x, 0};
-      uint32_t a2par = 0;
       int64_t it = 0, g2_issued = 0;
       bool pending = false;  // a group whose GEMM1s are all issued awaits its GEMM2
       auto gemm2 = [&]() -> bool {
-        if (!wait1(a2full, a2par, s_abort, p.err)) return false;
+        const int gb = (int)(g2_issued & 1);
+        const uint32_t gpar = (uint32_t)((g2_issued >> 1) & 1);
+        if (!wait1(&a2full[gb], gpar, s_abort, p.err) || !wait1(&d2empty[gb], gpar ^ 1u, s_abort, p.err))
+          return false;
         tc_fence_after();
+        const uint32_t sA2 = smem_u32(A2b(gb));
         for (int kk = 0; kk < p.K2 / 16; ++kk)
-          mma_f16(tmem + p.d2_col, sdesc(sA2 + kk * 2 * p.lbo_a2, p.lbo_a2, 128),
+          mma_f16(tmem + p.d2_col[gb], sdesc(sA2 + kk * 2 * p.lbo_a2, p.lbo_a2, 128),
                   sdesc(sB2 + kk * 2 * lbo_b2, lbo_b2, 128), id2, kk > 0);
-        mma_commit(d2full);
-        a2par ^= 1u;
+        mma_commit(&d2full[gb]);
         ++g2_issued;
         return true;
       };
@@ -301,7 +308,8 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       if (*s_abort) {
         // bounded wait for the last MMAs before TMEM is released
         if (it > 0) mbar_wait(&d1full[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), WAIT_NS / 4);
-        if (g2_issued > 0) mbar_wait(d2full, (a2par ^ 1u), WAIT_NS / 4);
+        if (g2_issued > 0)
+          mbar_wait(&d2full[(g2_issued - 1) & 1], (uint32_t)(((g2_issued - 1) >> 1) & 1), WAIT_NS / 4);
       }
     }
   } else if (warp >= 4 && warp < 12) {
@@ -420,15 +428,69 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int sl_row = row >> p.log2Ia, ia_row = row & (p.Ia - 1);
     TileCursor c{(int64_t)blockIdx.x, 0};
-    uint32_t d2par = 0;
+    int64_t g_done = 0;        // groups whose Y has been written
+    int64_t g_pending = -1;    // group (index in this CTA) whose Y is ready to read
+    int64_t g_pending_abs = 0; // its group number
+    // Y of one group from D2[gi & 1] (row = (slab in group, j_b)), j_a contiguous
+    auto write_y = [&](int64_t gi, int64_t gabs) -> bool {
+      const int gb = (int)(gi & 1);
+      if (!waitw(&d2full[gb], (uint32_t)((gi >> 1) & 1), s_abort, p.err)) return false;
+      tc_fence_after();
+      const int sb = row / p.rb, jb = row - sb * p.rb;
+      const int64_t slab = gabs * p.sg + sb;
+      const bool yvalid = row < p.sg * p.rb && slab < p.n_slabs;
+      const int64_t ybase = (slab * p.rb + jb) * p.ra;
+      for (int c0 = 0; c0 < p.N2; c0 += 32) {
+        float v[32];
+        if (c0 + 32 <= p.N2)
+          tmem_ld32(tmem + p.d2_col[gb] + lane_base + c0, v);
+        else
+          tmem_ld16(tmem + p.d2_col[gb] + lane_base + c0, v);
+        // a thread owns one Y row: 16-byte stores where the row allows
+        // them (one warp store touches 32 rows, so wider is cheaper)
+        if (yvalid && p.y_vec && c0 / 2 + 16 <= p.ra) {
+          if (p.y_f32) {
+            float4* y4 = (float4*)((float2*)p.Y + ybase + c0 / 2);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) y4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          } else {
+            uint4* y4 = (uint4*)((uint32_t*)p.Y + ybase + c0 / 2);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              y4[u] = make_uint4(f2_to_bf2(v[8 * u], v[8 * u + 1]), f2_to_bf2(v[8 * u + 2], v[8 * u + 3]),
+                                 f2_to_bf2(v[8 * u + 4], v[8 * u + 5]), f2_to_bf2(v[8 * u + 6], v[8 * u + 7]));
+          }
+        } else if (yvalid) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            int ja = c0 / 2 + u;
+            if (ja < p.ra) {
+              if (p.y_f32)
+                ((float2*)p.Y)[ybase + ja] = make_float2(v[2 * u], v[2 * u + 1]);
+              else
+                ((uint32_t*)p.Y)[ybase + ja] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&d2empty[gb]);
+      return true;
+    };
+    bool ok = true;
+    int64_t gi = 0;  // index of the current group in this CTA
     for (int64_t it = 0; it < n_it; ++it) {
       const int b = (int)(it & 1);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
       const int64_t t = c.tile(q);
-      if (!waitw(&d1full[b], par, s_abort, p.err)) break;
+      if (!waitw(&d1full[b], par, s_abort, p.err)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       // P (fp32, TMEM) -> GEMM2's A operand (bf16), rows (slab in group,
       // j_b), K = (i_a, re/im)
+      uint8_t* A2 = A2b(gi);
       const bool valid = t * p.spb + sl_row < p.n_slabs;
       const int m2base = (c.i * p.spb + sl_row) * p.rb;
       for (int c0 = 0; c0 < p.N1; c0 += 32) {
@@ -450,55 +512,26 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       }
       tc_fence_before();
       mbar_arrive(&d1empty[b]);
+      // the previous group's Y, now that this tile's D1 is drained
+      if (g_pending >= 0) {
+        if (!write_y(g_pending, g_pending_abs)) {
+          ok = false;
+          break;
+        }
+        g_pending = -1;
+        ++g_done;
+      }
       const bool last = c.i == q - 1 || it == n_it - 1;
       if (last) {
         fence_async_smem();
-        mbar_arrive(a2full);
-        if (!waitw(d2full, d2par, s_abort, p.err)) break;
-        d2par ^= 1u;
-        tc_fence_after();
-        // Y (row = (slab in group, j_b)) -> global, j_a contiguous
-        const int sb = row / p.rb, jb = row - sb * p.rb;
-        const int64_t slab = c.g * p.sg + sb;
-        const bool yvalid = row < p.sg * p.rb && slab < p.n_slabs;
-        const int64_t ybase = (slab * p.rb + jb) * p.ra;
-        for (int c0 = 0; c0 < p.N2; c0 += 32) {
-          float v[32];
-          if (c0 + 32 <= p.N2)
-            tmem_ld32(tmem + p.d2_col + lane_base + c0, v);
-          else
-            tmem_ld16(tmem + p.d2_col + lane_base + c0, v);
-          // a thread owns one Y row: 16-byte stores where the row allows
-          // them (one warp store touches 32 rows, so wider is cheaper)
-          if (yvalid && p.y_vec && c0 / 2 + 16 <= p.ra) {
-            if (p.y_f32) {
-              float4* y4 = (float4*)((float2*)p.Y + ybase + c0 / 2);
-#pragma unroll
-              for (int u = 0; u < 8; ++u) y4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-            } else {
-              uint4* y4 = (uint4*)((uint32_t*)p.Y + ybase + c0 / 2);
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                y4[u] = make_uint4(f2_to_bf2(v[8 * u], v[8 * u + 1]), f2_to_bf2(v[8 * u + 2], v[8 * u + 3]),
-                                   f2_to_bf2(v[8 * u + 4], v[8 * u + 5]), f2_to_bf2(v[8 * u + 6], v[8 * u + 7]));
-            }
-          } else if (yvalid) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              int ja = c0 / 2 + u;
-              if (ja < p.ra) {
-                if (p.y_f32)
-                  ((float2*)p.Y)[ybase + ja] = make_float2(v[2 * u], v[2 * u + 1]);
-                else
-                  ((uint32_t*)p.Y)[ybase + ja] = f2_to_bf2(v[2 * u], v[2 * u + 1]);
-              }
-            }
-          }
-        }
-        tc_fence_before();
+        mbar_arrive(&a2full[gi & 1]);
+        g_pending = gi;
+        g_pending_abs = c.g;
+        ++gi;
       }
       c.next(q);
     }
+    if (ok && g_pending >= 0) write_y(g_pending, g_pending_abs);
   }
   tc_fence_before();
   __syncthreads();
@@ -1200,7 +1233,7 @@ struct TcImpl {
   const float* U[8] = {};
 };
 
-// Projection shared memory: nstage tile stages, A2, B1, B2, barriers.
+// Projection shared memory: nstage tile stages, A2 twice, B1, B2, barriers.
 size_t p1_smem_bytes(int Ib, int ns, int K2, int K1, int N1, int N2, uint32_t lbo_a2, P1Args* a) {
   size_t off = 0;
   auto take = [&](size_t b) {
@@ -1209,7 +1242,7 @@ size_t p1_smem_bytes(int Ib, int ns, int K2, int K1, int N1, int N2, uint32_t lb
     return (uint32_t)o;
   };
   const size_t tile = ((size_t)128 * Ib * 4 + 127) / 128 * 128;
-  uint32_t st = take(tile * ns), a2 = take((size_t)(K2 / 8) * lbo_a2);
+  uint32_t st = take(tile * ns), a2 = take((size_t)2 * (K2 / 8) * lbo_a2);
   uint32_t b1 = take((size_t)N1 * K1 * 2), b2 = take((size_t)N2 * K2 * 2);
   uint32_t bar = take(256);
   if (a) {
@@ -1305,11 +1338,11 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
     if (g.p1_smem <= SMEM_LIMIT) break;
   }
   if (g.p1_smem > SMEM_LIMIT) return false;
-  // TMEM (512 columns): P1 holds D1 twice, D2 and GEMM1's A twice (K1 / 2
-  // columns each); R3 holds D1 and D2 twice, its GEMM1's A once and its
+  // TMEM (512 columns): P1 holds D1 twice, D2 twice and GEMM1's A twice
+  // (K1 / 2 columns each); R3 holds D1 and D2 twice, its GEMM1's A once and its
   // GEMM2's A twice.
   auto r32 = [](int x) { return (x + 31) / 32 * 32; };
-  if (2 * r32(g.N1) + r32(g.N2) + 2 * r32(g.K1 / 2) > 512) return false;
+  if (2 * r32(g.N1) + 2 * r32(g.N2) + 2 * r32(g.K1 / 2) > 512) return false;
   if (2 * r32(g.rN1) + 2 * r32(g.rN2) + r32(g.rK1 / 2) + 2 * r32(g.rK2 / 2) > 512) return false;
   // Reconstruction: as many W stages as fit (it is bound by the bytes it
   // keeps in flight), at least three.
@@ -1502,14 +1535,15 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   P1Args& a = g->p1;
   p1_smem_bytes(g->Ib, g->p1_nstage, g->K2, g->K1, g->N1, g->N2, (uint32_t)(g->a2_rows / 8) * 128 + 16, &a);
   {
-    // TMEM columns: D1 x2, D2, GEMM1's A x2 (each 32-column aligned)
+    // TMEM columns: D1 x2, D2 x2, GEMM1's A x2 (each 32-column aligned)
     const uint32_t n1 = (uint32_t)((g->N1 + 31) / 32 * 32), n2 = (uint32_t)((g->N2 + 31) / 32 * 32);
     const uint32_t na = (uint32_t)((g->K1 / 2 + 31) / 32 * 32);
     a.d1_col[0] = 0;
     a.d1_col[1] = n1;
-    a.d2_col = 2 * n1;
-    a.a1_col[0] = 2 * n1 + n2;
-    a.a1_col[1] = 2 * n1 + n2 + na;
+    a.d2_col[0] = 2 * n1;
+    a.d2_col[1] = 2 * n1 + n2;
+    a.a1_col[0] = 2 * n1 + 2 * n2;
+    a.a1_col[1] = 2 * n1 + 2 * n2 + na;
   }
   a.G = (const uint32_t*)grad;
   a.N = p.N;
