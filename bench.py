@@ -85,54 +85,39 @@ def kernel_algorithmic_bytes(name: str, wl) -> float:
     return float(table.get(name, 0.0))
 
 
+POLLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[1]))
+get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    print(f"{time.time():.4f},{pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)},"
+          f"{int(get(h)):#x},{pynvml.nvmlDeviceGetPowerUsage(h) / 1e3:.1f}", flush=True)
+    time.sleep(0.002)
+"""
+
+
 class ClockSampler:
-    """SM clock and clock-event reasons sampled during the timed region: an
-    NVML polling thread (read-only queries, every 2 ms), else nvidia-smi at
-    its 100 ms minimum. The samples are also written to gpurun_out/."""
+    """SM clock and clock-event reasons sampled during the timed region by a
+    separate polling process (read-only NVML queries every 2 ms; a thread in
+    this process would be starved while it launches). The samples inside the
+    timed region are kept, and written to gpurun_out/."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown"}
 
     def __init__(self, index: int):
-        import threading
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
-        self.samples, self.proc, self.nv = [], None, None
+        self.raw = self.path + ".raw"
+        self.t0, self.t1 = 0.0, float("inf")
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.stop_ev = threading.Event()
-            self.th = threading.Thread(target=self._poll, daemon=True)
-            self.th.start()
-        except Exception:
-            self.nv = None
-            self._start_smi(index)
-
-    def _poll(self):
-        nv = self.nv
-        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        while not self.stop_ev.is_set():
-            try:
-                self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
-                                     int(get_reasons(self.h)),
-                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1e3))
-            except Exception:
-                break
-            time.sleep(0.002)
-
-    def _start_smi(self, index):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            self.f = open(self.raw, "w")
+            self.proc = subprocess.Popen([sys.executable, "-c", POLLER, str(index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -144,47 +129,35 @@ class ClockSampler:
             self.t1 = time.time()
 
     def stop(self) -> dict:
-        if self.nv is not None:
-            self.stop_ev.set()
-            self.th.join(timeout=5)
-            t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
-            inside = [x for x in self.samples if t0 <= x[0] <= t1]
-            # the nearest samples on either side when the region is shorter than the period
-            self.samples = inside or self.samples[-2:]
-            with open(self.path, "w") as f:
-                f.write("time,sm_mhz,reasons_bits,power_w\n")
-                for t, mhz, bits, pw in self.samples:
-                    f.write(f"{t:.4f},{mhz},{bits:#x},{pw:.1f}\n")
-            sm = [x[1] for x in self.samples]
-            reasons = sorted({nm for _, _, bits, _ in self.samples
-                              for b, nm in self.REASONS.items() if bits & b})
-            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
-                    "reasons": reasons, "samples": len(sm), "source": "nvml"}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["sampler unavailable"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+        smax, rows = None, []
+        for line in open(self.raw):
+            if line.startswith("max"):
+                smax = float(line.split()[1])
                 continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm), "source": "nvidia-smi"}
+            f = line.strip().split(",")
+            if len(f) == 4:
+                try:
+                    rows.append((float(f[0]), float(f[1]), int(f[2], 16), float(f[3])))
+                except ValueError:
+                    pass
+        os.remove(self.raw)
+        inside = [r for r in rows if self.t0 <= r[0] <= self.t1]
+        with open(self.path, "w") as out:
+            out.write("time,sm_mhz,reasons_bits,power_w\n")
+            for t, mhz, bits, pw in inside:
+                out.write(f"{t:.4f},{mhz:.0f},{bits:#x},{pw:.1f}\n")
+        sm = [r[1] for r in inside]
+        reasons = sorted({nm for r in inside for b, nm in self.REASONS.items() if r[2] & b})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(sm), "source": "nvml (polling process)"}
 
 
 def oracle_sample(wl, factor: int):
@@ -415,7 +388,7 @@ def main():
     # the metric: K steps without per-kernel events; then K more with them,
     # for the per-kernel launch times of the roofline
     sampler = ClockSampler(local)
-    time.sleep(0.05)  # the polling thread is running before the timed region
+    time.sleep(1.0)  # the polling process is up before the timed region
     sampler.mark(True)
     total_ms, _ = timed_steps(False)
     sampler.mark(False)

@@ -598,21 +598,24 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
     __syncthreads();
     return s_abort == 0;
   };
-  uint32_t v[32];
-  auto load_x = [&](int kc) {
+  // two register sets: chunk kc + 2 is in flight while chunk kc is stored
+  // and its MMAs run
+  uint32_t va[32], vb[32];
+  auto load_x = [&](uint32_t(&v)[32], int kc) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int64_t k = (int64_t)kc * 32 + i;
       v[i] = (valid && k < p.K) ? __ldg(xrow + k * p.in_bs) : 0u;
     }
   };
-  load_x(0);
-  for (int kc = 0; kc < p.nkc; ++kc) {
+  // one K chunk: buffers free, operand image by bulk copy, X from registers
+  // (then the registers are refilled with chunk kc + 2), MMAs
+  auto chunk = [&](uint32_t(&v)[32], int kc) -> bool {
     const int s = kc & 1;
     if (kc >= 2) {
       const bool ok = wait_all(&bars[s], waited[s] & 1u);
       waited[s]++;
-      if (!ok) break;
+      if (!ok) return false;
       tc_fence_after();
     }
     if (tid == 0) {
@@ -623,12 +626,12 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
 #pragma unroll
     for (int q = 0; q < 8; ++q)
       *(uint4*)(As[s] + q * LBO_M128 + tid * 16) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    if (kc + 1 < p.nkc) load_x(kc + 1);  // in flight during this chunk's MMAs
+    if (kc + 2 < p.nkc) load_x(v, kc + 2);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (s_abort) break;
+    if (s_abort) return false;
     if (tid == 0) {
       if (!mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, WAIT_NS)) {
         atomicOr(p.err, DEV_ERR_TIMEOUT);
@@ -642,6 +645,13 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
         issued[s]++;
       }
     }
+    return true;
+  };
+  load_x(va, 0);
+  if (p.nkc > 1) load_x(vb, 1);
+  for (int kc = 0; kc < p.nkc; kc += 2) {
+    if (!chunk(va, kc)) break;
+    if (kc + 1 < p.nkc && !chunk(vb, kc + 1)) break;
   }
   __syncthreads();
   if (!s_abort) {
