@@ -11,11 +11,13 @@
 // rows (i_a) of 128 / I_a consecutive slabs:
 //
 //  proj_stream  (one pass over G) per tile: bulk-copy the raw tile to shared
-//     memory; on Omega's entries gather g_s, zero the entry (residual) and
-//     run the sparse AdamW update (S~ kept as fp16 for the reconstruction);
+//     memory; on Omega's entries gather g_s (stored in Omega order) and zero
+//     the entry (residual); the residual rows go to TMEM as GEMM1's A;
 //     GEMM1  P = X conj(U_b)        M = 128 rows (i_a), K = 2 I_b, N = 2 r_b
 //     GEMM2  Y = (U_a^H P)^T        M = 128 rows (slab, j_b), K = 2 I_a, N = 2 r_a
 //     over groups of slabs; Y (bf16) is 1/16 of G for the default shapes.
+//  sparse_adam  S~ = lambda Adam(g_s) with FP32 moments, in place over g_s
+//     (fp16, the precision S~ is kept in for the reconstruction).
 //  mode_gemm    the remaining modes n < a, contracted on Y in place of each
 //     other: rows = 128 consecutive inner positions, K = 2 I_n (or 2 r_n),
 //     N = 2 r_n (or 2 I_n); the last projection writes the core C in fp32.
@@ -24,8 +26,8 @@
 //     GEMM1  P' = U_a Y'^T          M = 128 rows (slab, i_a), K = 2 r_a per slab
 //                                    (block-diagonal over the tile's slabs), N = 2 r_b
 //     GEMM2  Delta = P' U_b^T       M = 128 rows, K = 2 r_b, N = 2 I_b
-//     epilogue: Delta += lambda S~ on Omega (in place), W <- W (1 - lr wd)
-//     - lr Delta rounded once, bulk-copy W back.
+//     (both A operands in TMEM); epilogue: Delta += lambda S~ on Omega,
+//     W <- W (1 - lr wd) - lr Delta rounded once, bulk-copy W back.
 //
 // Complex products run as real GEMMs on an embedding: for y = x M with x a
 // complex row (interleaved re, im along K), the K x N real matrix
@@ -754,7 +756,7 @@ struct R3Args {
   const uint8_t* B2img;
   float decay, lr;
   int* err;
-  int nstage, cap;
+  int nstage;
   uint32_t lbo_b1;  // GEMM1's B: K-adjacent core matrices N1 / 8 * 128 + 16 B apart
   uint32_t w_tile_bytes, y_tile_bytes;
   uint32_t off_w, off_y, off_B1, off_B2, off_ds, off_bar;
@@ -1269,7 +1271,7 @@ size_t p1_smem_bytes(int Ib, int ns, int K2, int K1, int N1, int N2, uint32_t lb
 }
 
 size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int K1, int N1, int K2,
-                     int N2, int cap, R3Args* a) {
+                     int N2, R3Args* a) {
   size_t off = 0;
   auto take = [&](size_t b) {
     size_t o = off;
@@ -1300,7 +1302,6 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
 
 constexpr size_t SMEM_LIMIT = 227 * 1024 - 1024;
 constexpr size_t ONE_CTA_SMEM = 120 * 1024;
-constexpr int R3_CAP = 1024;
 
 bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int wdt) {
   if (nd < 3) return false;
@@ -1358,8 +1359,7 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
   // keeps in flight), at least three.
   int wbytes = wdt == TGD_C64 ? 8 : 4;
   for (g.r3_nstage = R3_NS_MAX; g.r3_nstage >= 3; --g.r3_nstage) {
-    g.r3_smem = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, g.r3_nstage, g.rK1, g.rN1, g.rK2, g.rN2, R3_CAP,
-                              nullptr);
+    g.r3_smem = r3_smem_bytes(g.Ib, g.spb, g.bs_pad, wbytes, g.r3_nstage, g.rK1, g.rN1, g.rK2, g.rN2, nullptr);
     if (g.r3_smem <= SMEM_LIMIT) break;
   }
   if (g.r3_smem > SMEM_LIMIT) return false;
@@ -1674,8 +1674,7 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
     r.a2_col[0] = r.a1_col + na1;
     r.a2_col[1] = r.a1_col + na1 + na2;
   }
-  r3_smem_bytes(g->Ib, g->spb, g->bs_pad, wbytes, r.nstage, g->rK1, g->rN1, g->rK2, g->rN2, R3_CAP, &r);
-  r.cap = R3_CAP;
+  r3_smem_bytes(g->Ib, g->spb, g->bs_pad, wbytes, r.nstage, g->rK1, g->rN1, g->rK2, g->rN2, &r);
   r.Yp = g->Yp;
   r.yp_bs = g->bs_pad;
   r.W = w;
