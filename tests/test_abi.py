@@ -59,11 +59,22 @@ def _create(tgd, shape, ranks, rho=0.05, T=5, gdt=1, wdt=1, opt=None):
     ((4, 4, 4), (2, 2, 2), 0.05, 5, 0, 1),     # real gradient, complex weight
     ((4, 4, 4), (2, 2, 2), 0.05, 5, 9, 9),     # unknown dtype
     ((4,), (2,), 0.05, 5, 1, 1),               # one mode
+    ((4, 0, 4), (2, 0, 2), 0.05, 5, 1, 1),     # empty mode
+    ((2,) * 9, (1,) * 9, 0.05, 5, 1, 1),       # more modes than supported
+    ((1 << 21, 1 << 21), (1 << 21, 1 << 21), 0.05, 5, 1, 1),  # more elements than supported
 ])
 def test_create_rejects_bad_arguments(tgd, shape, ranks, rho, T, gdt, wdt):
     st, h = _create(tgd, shape, ranks, rho, T, gdt, wdt)
     assert st == 1 and not h.value
     assert tgd.lib().tgd_last_error(None)
+
+
+def test_unsupported_projected_mode(tgd):
+    """A projected mode above 256 entries (the eigensolver's limit) is
+    reported as unsupported; the same mode at full rank (identity) is not
+    projected and passes the argument checks."""
+    st, h = _create(tgd, (300, 4, 4), (10, 2, 2))
+    assert st == 2 and not h.value  # TGD_ERR_UNSUPPORTED
 
 
 def test_null_arguments(tgd):
