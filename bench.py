@@ -450,9 +450,10 @@ def main():
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,
                      "traffic": traffic, "peak_source": peak_src,
-                     "step_algorithmic_bytes": ab["total"],
-                     "step_achieved_gbs": ab["total"] / (step_ms / 1e3) / 1e9,
-                     "step_frac": ab["total"] / (step_ms / 1e3) / 1e9 / hbm_gbs},
+                     # a step covers every tensor of this rank
+                     "step_algorithmic_bytes": ab["total"] * len(tensors),
+                     "step_achieved_gbs": ab["total"] * len(tensors) / (step_ms / 1e3) / 1e9,
+                     "step_frac": ab["total"] * len(tensors) / (step_ms / 1e3) / 1e9 / hbm_gbs},
         "kernels": {k: {"launches": v[0], "ms_total": round(v[1], 4)} for k, v in prof.items()},
         "gpu_launches": int(sum(v[0] for v in prof.values())),  # per K steps (profiled pass)
         "clocks": clocks,
