@@ -287,6 +287,9 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "generic", "tcgen05"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--sequential", action="store_true",
+                    help="step the tensors of a multi-tensor workload one after another on one "
+                         "stream (default: each on its own stream with an equal share of the SMs)")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the leading mode (and its rank) by this factor: small "
                          "cases of the same kernels, for profiler captures only")
@@ -326,6 +329,10 @@ def main():
 
     # Inputs resident in HBM before the timed region.
     nt = wl.n_tensors if args.workload != DEFAULT_WORKLOAD else 1
+    concurrent = nt > 1 and not args.sequential
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sm_budget = max(1, n_sms // nt) if concurrent else 0
+    streams = [torch.cuda.Stream(device=dev) for _ in range(nt)] if concurrent else None
     tensors = []
     for gseed, wseed in tensor_seeds(rank, nt):
         gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=gseed,
@@ -335,7 +342,7 @@ def main():
         w = weights(wl.shape, wl.weight_dtype, seed=wseed, device=str(dev))
         T = wl.T
         opt = rst.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, T, wl.lr, wl.betas, wl.eps, wl.wd,
-                             wl.dtype, wl.weight_dtype, path=args.path)
+                             wl.dtype, wl.weight_dtype, path=args.path, sm_budget=sm_budget)
         if T == 0:
             opt.refresh(grads[0])
         tensors.append((opt, grads, w))
@@ -346,8 +353,23 @@ def main():
     scratch = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if flush else None
 
     def one_step(i):
-        for opt, grads, w in tensors:
-            opt.step(grads[i % 2], w)
+        if streams is None:
+            for opt, grads, w in tensors:
+                opt.step(grads[i % 2], w)
+            return
+        # each tensor on its own stream, forked from and joined back into the
+        # timed stream
+        main = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        for (opt, grads, w), st in zip(tensors, streams):
+            st.wait_event(fork)
+            with torch.cuda.stream(st):
+                opt.step(grads[i % 2], w)
+        for st in streams:
+            join = torch.cuda.Event()
+            join.record(st)
+            main.wait_event(join)
 
     for i in range(args.warmup):
         one_step(i)
@@ -446,7 +468,9 @@ def main():
                    "grad_dtype": wl.dtype, "weight_dtype": wl.weight_dtype,
                    "kernel_path": tensors[0][0].info["path"],
                    "l2": "flushed between steps" if flush else "inputs larger than L2",
-                   "parallelism": f"independent tensors per rank x{world}"},
+                   "parallelism": f"independent tensors per rank x{world}",
+                   "tensor_streams": "one stream per tensor, 1/%d of the SMs each" % nt if concurrent
+                   else "one stream"},
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,
                      "traffic": traffic, "peak_source": peak_src,

@@ -88,6 +88,9 @@ typedef struct {
   int moments_on_refresh; /* 0: keep moments across a refresh (default); 1: reset to zero */
   int auto_refresh;       /* 1 (default): tgd_step refreshes first when T > 0 and t % T == 0 */
   int path;               /* tgd_path */
+  int sm_budget;          /* 0 (default): the stream kernels spread over every SM; n > 0: over at
+                             most n SMs, so that several tensors stepped on separate streams run
+                             side by side (tensor-core path; results do not change) */
 } tgd_options;
 
 /* Fills `opt` with the defaults listed above. */

@@ -349,6 +349,7 @@ void tgd_default_options(tgd_options* opt) {
   opt->moments_on_refresh = 0;
   opt->auto_refresh = 1;
   opt->path = TGD_PATH_AUTO;
+  opt->sm_budget = 0;
 }
 
 tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int64_t* ranks,
@@ -374,7 +375,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (opt) o = *opt;
   if (o.omega_mode < 0 || o.omega_mode > 1 || o.complex_adam < 0 || o.complex_adam > 1 ||
       o.moments_on_refresh < 0 || o.moments_on_refresh > 1 || o.path < 0 || o.path > 2 ||
-      !std::isfinite(o.sparse_scale))
+      o.sm_budget < 0 || !std::isfinite(o.sparse_scale))
     return fail(nullptr, TGD_ERR_INVALID_ARG, "bad option value");
   int64_t N = 1, ncore = 1;
   for (int n = 0; n < ndim; ++n) {
@@ -457,6 +458,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   }
   if (ok && h->path == TGD_PATH_TCGEN05) {
     auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
+    h->tc.sm_budget = o.sm_budget;
     ok &= tc_plan(h->tc, ndim, shape, ranks, h->k, grad_dtype, weight_dtype, alloc_fn, h);
   }
   if (!ok) {

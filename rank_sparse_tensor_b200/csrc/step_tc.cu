@@ -1451,6 +1451,7 @@ bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, int6
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&g->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (p.sm_budget > 0 && p.sm_budget < g->num_sms) g->num_sms = p.sm_budget;
   auto A = [&](void** ptr, size_t bytes) { return alloc(ctx, ptr, bytes); };
   bool ok = true;
   ok &= A((void**)&g->tile_off, sizeof(int64_t) * (g->n_tiles + 1));

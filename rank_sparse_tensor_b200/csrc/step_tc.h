@@ -18,6 +18,7 @@ struct TcPlan {
   int64_t I[8] = {}, r[8] = {};
   int64_t N = 0, k = 0, ncore = 0;
   int gdt = 0, wdt = 0;
+  int sm_budget = 0;  // > 0: the persistent kernels use at most this many CTAs
   bool ready = false;
   void* impl = nullptr;  // owned by step_tc.cu (host-side description)
 };

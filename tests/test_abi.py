@@ -91,7 +91,7 @@ def test_default_options(tgd):
     o = tgd.Options()
     tgd.lib().tgd_default_options(C.byref(o))
     assert (o.omega_mode, o.sparse_scale, o.complex_adam, o.moments_on_refresh, o.auto_refresh,
-            o.path) == (0, 1.0, 0, 0, 1, 0)
+            o.path, o.sm_budget) == (0, 1.0, 0, 0, 1, 0, 0)
 
 
 def test_create_without_device_fails_cleanly(tgd):

@@ -140,3 +140,24 @@ def test_tc_selected_automatically(lib):
     with pytest.raises(lib.TgdError) as e:
         lib.TensorGRaD((8, 8, 6, 33), (4, 4, 3, 8), 0.05, 0, grad_dtype="c32h", path="tcgen05")
     assert e.value.name == "UNSUPPORTED"
+
+
+def test_sm_budget_gives_identical_results(lib):
+    """Capping the stream kernels' SMs (for tensors stepped side by side) only
+    changes which CTA takes which tile: the weights are bit-identical."""
+    from rank_sparse_tensor_b200.synth import GradientStream, weights
+    shape, ranks = (8, 16, 64, 33), (4, 8, 16, 8)
+    gs = GradientStream(shape, ranks, "c32h", 4, outlier_frac=0.02)
+    g0, g1 = gs.next().cuda(), gs.next().cuda()
+    w0 = weights(shape, "c32h", 4).cuda()
+    out = []
+    for budget in (0, 7):
+        opt = lib.TensorGRaD(shape, ranks, 0.05, 0, grad_dtype="c32h", sm_budget=budget)
+        assert opt.info["path"] == "tcgen05"
+        opt.refresh(g0)
+        w = w0.clone()
+        opt.step(g1, w)
+        opt.step(g0, w)
+        opt.sync()
+        out.append(w)
+    assert torch.equal(out[0], out[1])
