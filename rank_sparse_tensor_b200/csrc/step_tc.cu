@@ -351,7 +351,14 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     }
     int s = 0;
     uint32_t ph = 0;
+    // After an abort a warp still takes every named barrier of the remaining
+    // tiles (and no other work), so no converter warp waits there forever.
+    int64_t dead_from = n_it;
     for (int64_t it = 0; it < n_it; ++it) {
+      if (it >= dead_from) {
+        named_sync(1, 256);
+        continue;
+      }
       const int64_t t = cur.tile(q);
       const int b = (int)(it & 1);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
@@ -360,7 +367,11 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
         nn_e0 = p.tile_off[t2];
         nn_e1 = p.tile_off[t2 + 1];
       }
-      if (!waitw(&full[s], ph, s_abort, p.err)) break;
+      if (!waitw(&full[s], ph, s_abort, p.err)) {
+        named_sync(1, 256);
+        dead_from = it + 1;
+        continue;
+      }
       uint32_t* sw = (uint32_t*)stage(s);
       // gather g_s (coalesced stores, Omega order) and zero it in the tile
       // (R = G - S)
@@ -391,7 +402,10 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       nx_e0 = nn_e0;
       nx_e1 = nn_e1;
       named_sync(1, 256);  // every zeroed entry is in place before conversion
-      if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err)) break;
+      if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err)) {
+        dead_from = it + 1;
+        continue;
+      }
       tc_fence_after();
       // residual row -> TMEM (K = (i_b, re/im): one complex pair per column)
       const bool valid = t * p.spb + sl_row < p.n_slabs;
@@ -1062,7 +1076,16 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     named_sync(2, 256);
     int s = 0;
     uint32_t sph = 0;
+    // After an abort a warp still takes every named barrier of the remaining
+    // tiles (and no other work), so no epilogue warp waits there forever.
+    int64_t dead_from = n_it;
     for (int64_t it = 0; it < n_it; ++it) {
+      if (it >= dead_from) {
+        named_sync(2, 256);
+        named_sync(2, 256);
+        named_sync(2, 256);
+        continue;
+      }
       const int b = (int)(it & 1);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
       const int64_t t = blockIdx.x + it * G;
@@ -1078,8 +1101,12 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       }
       for (int64_t e = cur_e0 + 256 * EPF + et; e < cur_e1; e += 256) ds[p.loc[e]] = p.sp_upd[e];
       named_sync(2, 256);
-      if (!waitw(&d2full[b], par, s_abort, p.err)) break;
-      if (!waitw(&full[s], sph, s_abort, p.err)) break;
+      if (!waitw(&d2full[b], par, s_abort, p.err) || !waitw(&full[s], sph, s_abort, p.err)) {
+        named_sync(2, 256);
+        named_sync(2, 256);
+        dead_from = it + 1;
+        continue;
+      }
       tc_fence_after();
       const bool valid = t * p.spb + sl_row < p.n_slabs;
       WT* wrow = (WT*)wst(s) + erow;
