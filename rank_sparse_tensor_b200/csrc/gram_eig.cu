@@ -11,7 +11,11 @@
 // Gram: fp32 products accumulated per block over a slice of the unfolding's
 // columns (deterministic split), the partial sums added in fp64 in a fixed
 // order. The residual is never stored: the gradient is read in its storage
-// type and entries of Omega (a bitmask) read as zero.
+// type and entries of Omega (a bitmask) read as zero. A block owns one output
+// tile of edge TI = 4 nb (the smallest multiple of 4 >= I_n, at most 64;
+// upper tile pairs when I_n > 64); each thread keeps a 4 x 4 block of complex
+// sums in registers, and when the tile is small several thread groups take
+// interleaved columns of a chunk and their sums are added in group order.
 //
 // Eigensolver: two-sided Jacobi in fp64 with the round-robin parallel
 // ordering (n/2 disjoint rotations per round), one thread block per matrix,
@@ -26,15 +30,28 @@
 namespace tgd {
 namespace {
 
-constexpr int TI = 32;   // Gram tile edge
-constexpr int CC = 32;   // columns per Gram chunk
-constexpr int GT = 256;  // threads per Gram block
+constexpr int GCC = 32;    // columns of one sub-chunk (one per loader lane)
+constexpr int GMAXT = 256; // threads per Gram block, at most
+constexpr int GEPT = 16;   // elements one loader lane carries per chunk, at most
 
 struct GramGeom {
   int64_t A, I, B, ncol;
+  int TI;      // tile edge, 4 * nb
+  int nb;      // thread grid edge: thread (ty, tx) owns rows ty + nb p, columns tx + nb q
+  int ng;      // thread groups; group g takes chunk columns g, g + ng, ...
+  int nthr;    // ng * nb * nb
+  int nsub;    // sub-chunks of GCC columns per chunk
+  int col_fast;  // loader lanes run along columns (B >= 4) or along rows
   int nti, npairs, nsplit;
   int64_t cols_per_split;
 };
+
+// Loader units of one chunk: (tile, sub-chunk, row) along columns, or
+// (tile, sub-chunk, row half, column) along rows.
+int gram_units(const GramGeom& g, int ntile, int nsub) {
+  const int nrh = (g.TI + 31) / 32;
+  return g.col_fast ? ntile * nsub * g.TI : ntile * nsub * nrh * GCC;
+}
 
 GramGeom gram_geom(int nd, const int64_t* dims, int n) {
   GramGeom g;
@@ -44,16 +61,33 @@ GramGeom gram_geom(int nd, const int64_t* dims, int n) {
   for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
   g.I = dims[n];
   g.ncol = g.A * g.B;
-  g.nti = (int)ceil_div(g.I, TI);
+  g.nb = g.I > 64 ? 16 : (int)ceil_div(g.I, 4);
+  g.TI = 4 * g.nb;
+  g.ng = g.I > 64 ? 1 : std::min(64, GMAXT / (g.nb * g.nb));
+  g.nthr = g.ng * g.nb * g.nb;
+  g.col_fast = g.B >= 4;
+  g.nti = (int)ceil_div(g.I, g.TI);
   g.npairs = g.nti * (g.nti + 1) / 2;
-  int target = 148 * 4;
-  int64_t ns = ceil_div(target, g.npairs);
-  int64_t max_ns = ceil_div(g.ncol, 64);
-  if (ns > max_ns) ns = max_ns;
-  if (ns < 1) ns = 1;
-  g.nsplit = (int)ns;
-  g.cols_per_split = ceil_div(ceil_div(g.ncol, g.nsplit), CC) * CC;
+  const int ntile = g.nti > 1 ? 2 : 1;
+  const int nwl = g.nthr / 32;
+  g.nsub = std::max(1, 64 / g.TI);
+  while (g.nsub > 1 && ceil_div(gram_units(g, ntile, g.nsub), nwl) > GEPT) --g.nsub;
+  const int64_t chunk = (int64_t)GCC * g.nsub;
+  // about six blocks per SM over all tile pairs; the partial sums stay under
+  // 32 MB and every split gets at least two chunks
+  int64_t ns = ceil_div(148 * 6, g.npairs);
+  ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
+  ns = std::min<int64_t>(ns, std::max<int64_t>(1, ceil_div(g.ncol, 2 * chunk)));
+  g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), chunk) * chunk;
+  g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
   return g;
+}
+
+size_t gram_smem_bytes(const GramGeom& g) {
+  const int ntile = g.nti > 1 ? 2 : 1;
+  const size_t x = sizeof(float2) * (size_t)ntile * GCC * g.nsub * (g.TI + 1);
+  const size_t red = sizeof(float2) * (size_t)g.ng * g.TI * g.TI;
+  return std::max(x, red) + sizeof(int64_t) * 2 * GCC * g.nsub;
 }
 
 template <int DT>
@@ -62,11 +96,21 @@ __device__ __forceinline__ float2 masked_elem(const void* g, const uint32_t* bit
   return load_elem<DT>(g, idx);
 }
 
+// One (tile pair, column split) of the mode-n Gram R_(n) R_(n)^H. Column c of
+// the unfolding is (a, b) = (c / B, c mod B); its row i sits at a I B + i B + b.
+// Shared memory: X[tile][chunk column][row] (row stride TI + 1), reused for the
+// group sums at the end, then the start offsets of the chunk's columns (two
+// slots: the next chunk's are written while this one is read).
 template <int DT>
-__global__ void __launch_bounds__(GT) gram_partial_kernel(const void* g, const uint32_t* bits,
-                                                          GramGeom geo, float2* partial) {
-  __shared__ float2 Xi[TI][CC + 1];
-  __shared__ float2 Xj[TI][CC + 1];
+__global__ void __launch_bounds__(GMAXT, 2) gram_partial_kernel(const void* g, const uint32_t* bits,
+                                                                GramGeom geo, float2* partial) {
+  extern __shared__ __align__(16) unsigned char gram_smem[];
+  const int TI = geo.TI, nb = geo.nb, ng = geo.ng, LD = TI + 1;
+  const int CCt = GCC * geo.nsub;
+  const int ntile_max = geo.nti > 1 ? 2 : 1;
+  float2* X = (float2*)gram_smem;
+  const size_t x_elems = (size_t)ntile_max * CCt * LD, red_elems = (size_t)ng * TI * TI;
+  int64_t* colbase = (int64_t*)(X + (x_elems > red_elems ? x_elems : red_elems));
   // tile pair (ti <= tj) from the linear pair index
   int pr = blockIdx.x, ti = 0;
   while (pr >= geo.nti - ti) {
@@ -74,74 +118,165 @@ __global__ void __launch_bounds__(GT) gram_partial_kernel(const void* g, const u
     ++ti;
   }
   const int tj = ti + pr;
-  const int split = blockIdx.y;
-  const int64_t c_begin = (int64_t)split * geo.cols_per_split;
-  int64_t c_end = c_begin + geo.cols_per_split;
-  if (c_end > geo.ncol) c_end = geo.ncol;
-  const int il = threadIdx.x >> 3;  // 0..31
-  const int jl = threadIdx.x & 7;   // + 8q
-  float2 acc[4];
-  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
-  const bool col_fast = geo.B >= CC;
-  for (int64_t c0 = c_begin; c0 < c_end; c0 += CC) {
-    for (int e = threadIdx.x; e < TI * CC; e += GT) {
-      int row, col;
-      if (col_fast) {
-        row = e / CC;
-        col = e % CC;
-      } else {
-        col = e / TI;
-        row = e % TI;
-      }
-      int64_t c = c0 + col;
-      int64_t ri = (int64_t)ti * TI + row, rj = (int64_t)tj * TI + row;
-      float2 vi = make_float2(0.f, 0.f), vj = vi;
+  const int ntile = ti == tj ? 1 : 2;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nwl = geo.nthr >> 5;
+  const int nrh = (TI + 31) >> 5;
+  const int nunits = geo.col_fast ? ntile * geo.nsub * TI : ntile * geo.nsub * nrh * GCC;
+  const int64_t c_begin = (int64_t)blockIdx.y * geo.cols_per_split;
+  const int64_t c_end = c_begin + geo.cols_per_split < geo.ncol ? c_begin + geo.cols_per_split : geo.ncol;
+  const int64_t IB = geo.I * geo.B;
+  auto set_colbase = [&](int slot, int64_t c0) {
+    for (int j = tid; j < CCt; j += geo.nthr) {
+      const int64_t c = c0 + j;
+      int64_t off = -1;
       if (c < c_end) {
-        int64_t a = c / geo.B, b = c - a * geo.B;
-        int64_t base = a * geo.I * geo.B + b;
-        if (ri < geo.I) vi = masked_elem<DT>(g, bits, base + ri * geo.B);
-        if (rj < geo.I) vj = masked_elem<DT>(g, bits, base + rj * geo.B);
+        const int64_t a = c / geo.B;
+        off = a * IB + (c - a * geo.B);
       }
-      Xi[row][col] = vi;
-      Xj[row][col] = vj;
+      colbase[slot * CCt + j] = off;
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int cc = 0; cc < CC; ++cc) {
-      float2 a = Xi[il][cc];
+  };
+  // Loader unit k of this lane, decoded once (the mapping is the same for
+  // every chunk) and packed: bits 0-12 the X index, 13-21 the chunk column,
+  // 22-31 the matrix row (1023: outside the matrix, store zero); all ones: no
+  // unit.
+  uint32_t upk[GEPT];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 b = Xj[jl + 8 * q][cc];
-        // a * conj(b)
-        acc[q].x = __fmaf_rn(a.x, b.x, __fmaf_rn(a.y, b.y, acc[q].x));
-        acc[q].y = __fmaf_rn(a.y, b.x, __fmaf_rn(-a.x, b.y, acc[q].y));
+  for (int k = 0; k < GEPT; ++k) {
+    const int u = w + nwl * k;
+    upk[k] = ~0u;
+    if (w < nwl && u < nunits) {
+      int t, col, row;
+      if (geo.col_fast) {
+        const int sub_t = u / TI;  // (tile, sub-chunk)
+        row = u - sub_t * TI;
+        t = sub_t / geo.nsub;
+        col = (sub_t - t * geo.nsub) * GCC + lane;
+      } else {
+        const int cc = u & (GCC - 1), th = u >> 5;  // th = (tile, sub-chunk, row half)
+        const int h = nrh == 2 ? (th & 1) : 0, ts = nrh == 2 ? (th >> 1) : th;
+        t = ts / geo.nsub;
+        col = (ts - t * geo.nsub) * GCC + cc;
+        row = lane + 32 * h;
       }
+      const int grow = (t ? tj : ti) * TI + row;
+      const uint32_t xi = (uint32_t)((t * CCt + col) * LD + row);
+      if (row < TI)
+        upk[k] = xi | ((uint32_t)col << 13) | ((uint32_t)(grow < geo.I ? grow : 1023) << 22);
+    }
+  }
+  float2 pre[GEPT];
+  auto load = [&](int slot) {
+#pragma unroll
+    for (int k = 0; k < GEPT; ++k) {
+      float2 v = make_float2(0.f, 0.f);
+      const uint32_t pk = upk[k];
+      const uint32_t grow = pk >> 22;
+      if (pk != ~0u && grow != 1023u) {
+        const int64_t cb = colbase[slot * CCt + ((pk >> 13) & 511u)];
+        if (cb >= 0) v = masked_elem<DT>(g, bits, cb + (int64_t)grow * geo.B);
+      }
+      pre[k] = v;
+    }
+  };
+  auto store = [&]() {
+#pragma unroll
+    for (int k = 0; k < GEPT; ++k)
+      if (upk[k] != ~0u) X[upk[k] & 8191u] = pre[k];
+  };
+  const int grp = tid / (nb * nb), l = tid - grp * nb * nb, ty = l / nb, tx = l - ty * nb;
+  const float2* Xa = X + ty;
+  const float2* Xb = X + (size_t)(ntile - 1) * CCt * LD + tx;
+  float2 acc[4][4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[p][q] = make_float2(0.f, 0.f);
+
+  set_colbase(0, c_begin);
+  __syncthreads();
+  load(0);
+  int slot = 0;
+  for (int64_t c0 = c_begin; c0 < c_end; c0 += CCt) {
+    store();
+    set_colbase(slot ^ 1, c0 + CCt);
+    __syncthreads();
+    if (c0 + CCt < c_end) load(slot ^ 1);
+#pragma unroll 4
+    for (int col = grp; col < CCt; col += ng) {
+      float2 a[4], b[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) a[p] = Xa[(size_t)col * LD + nb * p];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) b[q] = Xb[(size_t)col * LD + nb * q];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // a * conj(b)
+          acc[p][q].x = __fmaf_rn(a[p].x, b[q].x, acc[p][q].x);
+          if constexpr (Dt<DT>::cplx) {
+            acc[p][q].x = __fmaf_rn(a[p].y, b[q].y, acc[p][q].x);
+            acc[p][q].y = __fmaf_rn(a[p].y, b[q].x, __fmaf_rn(-a[p].x, b[q].y, acc[p][q].y));
+          }
+        }
     }
     __syncthreads();
+    slot ^= 1;
   }
-  const int64_t I = geo.I;
-  int64_t gi = (int64_t)ti * TI + il;
-  float2* out = partial + (int64_t)split * I * I;
-  for (int q = 0; q < 4; ++q) {
-    int64_t gj = (int64_t)tj * TI + jl + 8 * q;
-    if (gi < I && gj < I) out[gi * I + gj] = acc[q];
+  // group sums in group order, then the tile's rows inside the matrix
+  float2* red = X;
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) red[((size_t)grp * TI + ty + nb * p) * TI + tx + nb * q] = acc[p][q];
+  __syncthreads();
+  float2* out = partial + (int64_t)blockIdx.y * geo.I * geo.I;
+  for (int e = tid; e < TI * TI; e += geo.nthr) {
+    const int r = e / TI, cl = e - r * TI;
+    float2 sum = red[e];
+    for (int gg = 1; gg < ng; ++gg) {
+      const float2 v = red[(size_t)gg * TI * TI + e];
+      sum.x += v.x;
+      sum.y += v.y;
+    }
+    const int64_t gi = (int64_t)ti * TI + r, gj = (int64_t)tj * TI + cl;
+    if (gi < geo.I && gj < geo.I) out[gi * geo.I + gj] = sum;
   }
 }
 
-__global__ void gram_reduce_kernel(const float2* partial, GramGeom geo, double2* gram) {
+// fp64 sum of the split partials: a block takes RC cells, its RS thread rows
+// take interleaved splits, and the RS slices are added in slice order. Lower
+// tiles come from the upper partials, conjugated.
+constexpr int RC = 32, RS = 8;
+__global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* partial, GramGeom geo,
+                                                              double2* gram) {
+  __shared__ double2 part[RS][RC];
   const int64_t I = geo.I;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < I * I;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    int64_t i = e / I, j = e - i * I;
-    bool upper = (i / TI) <= (j / TI);
-    int64_t src = upper ? i * I + j : j * I + i;
-    double sx = 0, sy = 0;
-    for (int s = 0; s < geo.nsplit; ++s) {
-      float2 v = partial[(int64_t)s * I * I + src];
+  const int cl = threadIdx.x % RC, sl = threadIdx.x / RC;
+  const int64_t e = (int64_t)blockIdx.x * RC + cl;
+  double sx = 0, sy = 0;
+  bool upper = true;
+  if (e < I * I) {
+    const int64_t i = e / I, j = e - i * I;
+    upper = (i / geo.TI) <= (j / geo.TI);
+    const int64_t src = upper ? i * I + j : j * I + i;
+#pragma unroll 4
+    for (int s = sl; s < geo.nsplit; s += RS) {
+      const float2 v = partial[(int64_t)s * I * I + src];
       sx += (double)v.x;
       sy += (double)v.y;
     }
-    gram[e] = upper ? make_double2(sx, sy) : make_double2(sx, -sy);
+  }
+  part[sl][cl] = make_double2(sx, sy);
+  __syncthreads();
+  if (sl == 0 && e < I * I) {
+    double tx = 0, ty = 0;
+    for (int q = 0; q < RS; ++q) {
+      tx += part[q][cl].x;
+      ty += part[q][cl].y;
+    }
+    gram[e] = upper ? make_double2(tx, ty) : make_double2(tx, -ty);
   }
 }
 
@@ -327,25 +462,26 @@ cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const
                       int n, float* partial, double* gram, cudaStream_t s) {
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
+  const size_t smem = gram_smem_bytes(geo);
   switch (dt) {
     case TGD_R32:
-      gram_partial_kernel<TGD_R32><<<grid, GT, 0, s>>>(g, bits, geo, (float2*)partial);
+      gram_partial_kernel<TGD_R32><<<grid, geo.nthr, smem, s>>>(g, bits, geo, (float2*)partial);
       break;
     case TGD_C64:
-      gram_partial_kernel<TGD_C64><<<grid, GT, 0, s>>>(g, bits, geo, (float2*)partial);
+      gram_partial_kernel<TGD_C64><<<grid, geo.nthr, smem, s>>>(g, bits, geo, (float2*)partial);
       break;
     case TGD_C32H:
-      gram_partial_kernel<TGD_C32H><<<grid, GT, 0, s>>>(g, bits, geo, (float2*)partial);
+      gram_partial_kernel<TGD_C32H><<<grid, geo.nthr, smem, s>>>(g, bits, geo, (float2*)partial);
       break;
     case TGD_R16:
-      gram_partial_kernel<TGD_R16><<<grid, GT, 0, s>>>(g, bits, geo, (float2*)partial);
+      gram_partial_kernel<TGD_R16><<<grid, geo.nthr, smem, s>>>(g, bits, geo, (float2*)partial);
       break;
     default:
       return cudaErrorInvalidValue;
   }
-  int64_t cells = geo.I * geo.I;
-  int blocks = (int)ceil_div(cells, 256);
-  gram_reduce_kernel<<<blocks, 256, 0, s>>>((const float2*)partial, geo, (double2*)gram);
+  const int64_t cells = geo.I * geo.I;
+  gram_reduce_kernel<<<(int)ceil_div(cells, RC), RC * RS, 0, s>>>((const float2*)partial, geo,
+                                                                   (double2*)gram);
   return cudaGetLastError();
 }
 

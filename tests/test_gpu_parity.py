@@ -44,6 +44,10 @@ CASES = {
     "c64_identity_modes": ((16, 8, 12, 5), (16, 3, 12, 2), (16, 3, 12, 2), "c64", 0.1),
     "c64_rho0": ((16, 12, 8, 9), (4, 3, 2, 3), (4, 3, 2, 3), "c64", 0.0),
     "c64_rho1": ((6, 5, 4, 3), (2, 2, 2, 2), (2, 2, 2, 2), "c64", 1.0),
+    # Gram tiles: pairs of 64-row tiles with a ragged last tile (130, 70, 66),
+    # and tile edges above I_n (9 -> 12, 5 -> 8)
+    "c64_gram_pairs_130x20x9": ((130, 20, 9), (8, 5, 3), (8, 5, 3), "c64", 0.05),
+    "c32h_gram_pairs_70x66x5": ((70, 66, 5), (6, 9, 2), (6, 9, 2), "c32h", 0.05),
 }
 
 
