@@ -65,6 +65,17 @@ def algorithmic_bytes(wl) -> dict:
     return parts
 
 
+def optimizer_state(wl, n_tensors: int, device_bytes: int) -> dict:
+    """Optimizer-state memory of this rank's tensors: the method's count
+    (core and sparse moments, factors, Omega's index; tgd_state_memory) next
+    to AdamW's moments for the same tensors, and the device memory the
+    handles hold (state plus work buffers)."""
+    import rank_sparse_tensor_b200 as rst
+    m = rst.state_memory(wl.shape, wl.ranks, wl.sparse_ratio, wl.dtype, 0)
+    return {"bytes": m["total_bytes"] * n_tensors, "adamw_bytes": m["adamw_bytes"] * n_tensors,
+            "ratio": m["ratio"], "device_bytes": int(device_bytes)}
+
+
 def kernel_algorithmic_bytes(name: str, wl) -> float:
     """Algorithmic bytes of one launch of the named kernel: its share of the
     step's algorithmic bytes (the parts of the step it alone moves)."""
@@ -482,6 +493,8 @@ def main():
         "gpu_launches": int(sum(v[0] for v in prof.values())),  # per K steps (profiled pass)
         "clocks": clocks,
         "e2e": e2e,
+        "optimizer_state": optimizer_state(wl, len(tensors),
+                                           sum(t[0].info["device_bytes"] for t in tensors)),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -155,6 +155,40 @@ typedef struct {
 
 TGD_API tgd_status tgd_query(tgd_handle h, tgd_info* info);
 
+/* Optimizer-state memory of the method for one tensor, next to AdamW's
+ * (host arithmetic only; no handle, no device). The count follows [S3]'s
+ * comparison of matrix and tensor low-rank state (its equations (9) and
+ * (10)): the tensor low-rank branch keeps the core, prod r_n entries, and a
+ * factor U_n of I_n x r_n entries for every projected mode; a mode with
+ * r_n == I_n needs no factor (U_n = I). [S1] section 3 adds the sparse part:
+ * a COO index per entry of Omega and Adam moments on its values, and keeps
+ * all moments in FP32.
+ *
+ * Bytes per element: m = 8 complex / 4 real; v = 4, or 8 for complex tensors
+ * with complex_adam == 1 (two second moments, view-as-real); a factor entry
+ * 8 complex / 4 real; an Omega index 8 (int64). k = floor(sparse_ratio * N).
+ * AdamW's figure is N * (m + v) with the same m and v.
+ *
+ * Arguments are checked as tgd_create checks them (1 <= ranks[n] <= shape[n],
+ * 0 <= sparse_ratio <= 1, N <= 2^40, 1 <= ndim <= TGD_MAX_NDIM, complex_adam 0
+ * or 1); a bad argument returns TGD_ERR_INVALID_ARG and leaves *out untouched.
+ * The caller owns out. */
+typedef struct {
+  int64_t N;              /* elements of the tensor */
+  int64_t k;              /* |Omega| */
+  int64_t core_elems;     /* prod r_n */
+  int64_t factor_elems;   /* sum of I_n r_n over modes with r_n < I_n */
+  int64_t adamw_bytes;    /* N (m + v) */
+  int64_t core_bytes;     /* core_elems (m + v) */
+  int64_t factor_bytes;   /* factor_elems x (8 complex, 4 real) */
+  int64_t sparse_bytes;   /* k (8 + m + v) */
+  int64_t total_bytes;    /* core_bytes + factor_bytes + sparse_bytes */
+} tgd_memory;
+
+TGD_API tgd_status tgd_state_memory(int ndim, const int64_t* shape, const int64_t* ranks,
+                                    double sparse_ratio, tgd_dtype grad_dtype, int complex_adam,
+                                    tgd_memory* out);
+
 /* Host copy of the optimizer state (checkpoint / resume, and teacher-forced
  *  testing). Any pointer may be NULL to skip that part. Layouts:
  *   omega     int64[k], ascending linear indices (complex elements counted once)

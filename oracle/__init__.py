@@ -13,6 +13,7 @@ oracle to facts the pages and mathematics fix live in ``tests/test_oracle_*``.
 from __future__ import annotations
 
 import ctypes as C
+import math
 import os
 import subprocess
 import threading
@@ -280,3 +281,39 @@ class Oracle:
         v = np.ascontiguousarray(v, np.float32).reshape(-1)
         assert v.size == self._msize(which)
         lib().orc_set_moment(self._h, self._MOM[which], _p(v))
+
+
+def state_memory(shape, ranks, sparse_ratio, dtype="c64", complex_adam=0) -> dict:
+    """Optimizer-state bytes of TensorGRaD for one tensor, and AdamW's.
+
+    Low-rank branch: the review's appended paper text counts the tensor
+    low-rank state as the Tucker core (prod r_n entries) plus one factor of
+    I_n x r_n entries per mode (its equation (10), r_max^4 + 2 r_max N +
+    2 r_max M for an N x N x M x M weight at rank r_max in every mode); a mode
+    kept at full rank is the identity and stores nothing. Sparse branch (the
+    nullthought summary, section 3): the COO index of each entry of Omega
+    (int64) and the Adam moments of its value. Moments are FP32: m complex
+    (8 bytes) or real (4); v real (4), or two reals (8) under the view-as-real
+    complex Adam. AdamW keeps m and v for every element.
+    """
+    cplx = dtype in ("c64", "c32h")
+    N = 1
+    for I in shape:
+        N *= int(I)
+    core = 1
+    for r in ranks:
+        core *= int(r)
+    factors = sum(int(I) * int(r) for I, r in zip(shape, ranks) if r < I)
+    k = math.floor(sparse_ratio * N)
+    m_b = 8 if cplx else 4
+    v_b = 8 if (cplx and complex_adam) else 4
+    u_b = 8 if cplx else 4
+    out = {
+        "N": N, "k": k, "core_elems": core, "factor_elems": factors,
+        "adamw_bytes": N * (m_b + v_b),
+        "core_bytes": core * (m_b + v_b),
+        "factor_bytes": factors * u_b,
+        "sparse_bytes": k * (8 + m_b + v_b),
+    }
+    out["total_bytes"] = out["core_bytes"] + out["factor_bytes"] + out["sparse_bytes"]
+    return out

@@ -21,7 +21,7 @@ import numpy as np
 from . import native
 from .native import TgdError, check, lib
 
-__all__ = ["TensorGRaD", "TgdError", "topk_select", "topk_select_static"]
+__all__ = ["TensorGRaD", "TgdError", "state_memory", "topk_select", "topk_select_static"]
 
 
 def _stream_ptr(stream) -> Optional[int]:
@@ -190,6 +190,25 @@ class TensorGRaD:
             if key in state:
                 setattr(v, key, arr(state[key], np.float32, i[key + "_len"]))
         check(lib().tgd_set_state(self._h, C.byref(v), _stream_ptr(stream)), self._h)
+
+
+def state_memory(shape: Sequence[int], ranks: Sequence[int], sparse_ratio: float,
+                 grad_dtype: str = "c64", complex_adam: int = 0) -> dict:
+    """Optimizer-state bytes of the method for one tensor next to AdamW's
+    (tgd_state_memory; host arithmetic, no device needed). Adds "ratio" =
+    total_bytes / adamw_bytes."""
+    d = len(shape)
+    if len(ranks) != d:
+        raise ValueError("shape and ranks differ in length")
+    sh = (C.c_int64 * max(d, 1))(*shape)
+    rk = (C.c_int64 * max(d, 1))(*ranks)
+    m = native.Memory()
+    check(lib().tgd_state_memory(d, C.cast(sh, C.c_void_p), C.cast(rk, C.c_void_p),
+                                 float(sparse_ratio), native.DTYPES[grad_dtype], int(complex_adam),
+                                 C.byref(m)))
+    out = {name: int(getattr(m, name)) for name, _ in native.Memory._fields_}
+    out["ratio"] = out["total_bytes"] / out["adamw_bytes"]
+    return out
 
 
 def topk_select(grad, dtype: str, k: int, stream=None):

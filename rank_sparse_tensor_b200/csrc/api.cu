@@ -576,6 +576,41 @@ tgd_status tgd_query(tgd_handle h, tgd_info* info) {
   return TGD_OK;
 }
 
+tgd_status tgd_state_memory(int ndim, const int64_t* shape, const int64_t* ranks,
+                            double sparse_ratio, tgd_dtype grad_dtype, int complex_adam,
+                            tgd_memory* out) {
+  if (!out || !shape || !ranks) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL argument");
+  if (ndim < 1 || ndim > TGD_MAX_NDIM) return fail(nullptr, TGD_ERR_INVALID_ARG, "bad ndim");
+  if (!(sparse_ratio >= 0.0 && sparse_ratio <= 1.0))
+    return fail(nullptr, TGD_ERR_INVALID_ARG, "sparse_ratio must be in [0, 1]");
+  if (grad_dtype < TGD_R32 || grad_dtype > TGD_R16 || complex_adam < 0 || complex_adam > 1)
+    return fail(nullptr, TGD_ERR_INVALID_ARG, "bad dtype or complex_adam");
+  int64_t N = 1, ncore = 1, nfac = 0;
+  for (int n = 0; n < ndim; ++n) {
+    if (shape[n] < 1 || ranks[n] < 1 || ranks[n] > shape[n])
+      return fail(nullptr, TGD_ERR_INVALID_ARG, "need 1 <= ranks[n] <= shape[n]");
+    if (N > ((int64_t)1 << 40) / shape[n]) return fail(nullptr, TGD_ERR_INVALID_ARG, "tensor too large");
+    N *= shape[n];
+    ncore *= ranks[n];
+    if (ranks[n] < shape[n]) nfac += shape[n] * ranks[n];
+  }
+  const bool cplx = grad_dtype == TGD_C64 || grad_dtype == TGD_C32H;
+  const int64_t mb = cplx ? 8 : 4, vb = cplx && complex_adam ? 8 : 4, ub = cplx ? 8 : 4;
+  const int64_t k = (int64_t)std::floor(sparse_ratio * (double)N);
+  tgd_memory m;
+  m.N = N;
+  m.k = k;
+  m.core_elems = ncore;
+  m.factor_elems = nfac;
+  m.adamw_bytes = N * (mb + vb);
+  m.core_bytes = ncore * (mb + vb);
+  m.factor_bytes = nfac * ub;
+  m.sparse_bytes = k * (8 + mb + vb);
+  m.total_bytes = m.core_bytes + m.factor_bytes + m.sparse_bytes;
+  *out = m;
+  return TGD_OK;
+}
+
 tgd_status tgd_get_state(tgd_handle h, tgd_state_view* out, void* stream) {
   if (!h || !out) return fail(h, TGD_ERR_INVALID_ARG, "NULL argument");
   cudaStream_t s = (cudaStream_t)stream;

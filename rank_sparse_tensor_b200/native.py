@@ -60,7 +60,15 @@ _lock = threading.Lock()
 _lib = None
 
 # name -> (restype, argtypes); the exported symbols of include/tgd.h
+class Memory(C.Structure):
+    _fields_ = [(n, C.c_int64) for n in ("N", "k", "core_elems", "factor_elems", "adamw_bytes",
+                                         "core_bytes", "factor_bytes", "sparse_bytes",
+                                         "total_bytes")]
+
+
 SIGNATURES = {
+    "tgd_state_memory": (C.c_int, [C.c_int, C.c_void_p, C.c_void_p, C.c_double, C.c_int, C.c_int,
+                                   C.POINTER(Memory)]),
     "tgd_default_options": (None, [C.POINTER(Options)]),
     "tgd_create": (C.c_int, [C.POINTER(C.c_void_p), C.c_int, C.c_void_p, C.c_void_p, C.c_double,
                              C.c_int64, C.c_float, C.c_float, C.c_float, C.c_float, C.c_float,
