@@ -33,7 +33,8 @@
  *  - Arguments are checked before any work is enqueued; a bad argument
  *    returns TGD_ERR_INVALID_ARG and changes nothing. Errors found on the
  *    device (a bounded wait that ran out) set an error word in the handle;
- *    the next call or tgd_sync() returns it.
+ *    the calls that synchronise (tgd_sync, tgd_step_host) read it, return
+ *    TGD_ERR_TIMEOUT and clear it. The asynchronous calls do not read it.
  *  - A handle is not thread-safe. It owns all optimizer state (allocated at
  *    tgd_create, freed at tgd_destroy); the caller owns grad and weight.
  */
@@ -125,8 +126,9 @@ TGD_API tgd_status tgd_refresh(tgd_handle h, const void* grad, void* stream);
 
 /* The same step as tgd_step with host buffers: copies grad (host, N elements)
  *  and weight (host, N elements) to the device, steps, copies weight back.
- *  Synchronises the stream before returning. Lazily allocates device staging
- *  for both tensors on first use. */
+ *  Synchronises the stream before returning, then returns any device-side
+ *  error recorded since the last check (TIMEOUT) as tgd_sync does. Lazily
+ *  allocates device staging for both tensors on first use. */
 TGD_API tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host, void* stream);
 
 /* Waits for the handle's work on `stream` and returns any device-side error

@@ -62,7 +62,6 @@ struct tgd_ctx {
   TcPlan tc;
   // errors
   int* d_err = nullptr;
-  int* h_err = nullptr;
   // host-buffer step
   void* stage_g = nullptr;
   void* stage_w = nullptr;
@@ -183,8 +182,6 @@ void free_all(tgd_ctx* h) {
   h->ev_pool.clear();
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
-  if (h->h_err) cudaFreeHost(h->h_err);
-  h->h_err = nullptr;
 }
 
 AdamConst adam_const(const tgd_ctx* h, double scale) {
@@ -536,8 +533,7 @@ tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host,
   tgd_status st = tgd_step(h, h->stage_g, h->stage_w, stream);
   if (st != TGD_OK) return st;
   TGD_CUDA(h, cudaMemcpyAsync(weight_host, h->stage_w, wb, cudaMemcpyDeviceToHost, s));
-  TGD_CUDA(h, cudaStreamSynchronize(s));
-  return TGD_OK;
+  return check_device_error(h, s, true);
 }
 
 tgd_status tgd_sync(tgd_handle h, void* stream) {
