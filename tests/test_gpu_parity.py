@@ -207,3 +207,27 @@ def test_bad_state_rejected(lib):
     with pytest.raises(lib.TgdError) as e:
         g.set_state({"omega": np.arange(k)[::-1].copy()})
     assert e.value.name == "INVALID_ARG"
+
+
+@pytest.mark.parametrize("dtype,shape,ranks", [
+    ("r32", (16, 12, 8, 9), (4, 3, 2, 3)),      # CUDA-core path
+    ("c32h", (4, 8, 64, 33), (2, 4, 16, 8)),    # tensor-core path
+])
+def test_step_host_equals_device_step(lib, dtype, shape, ranks):
+    """tgd_step_host (host buffers, copies inside the call) leaves bit for bit
+    the weights tgd_step leaves from the same state."""
+    from rank_sparse_tensor_b200.synth import GradientStream, weights
+    g = GradientStream(shape, ranks, dtype, 4, outlier_frac=0.02, outlier_scale=10.0).next()
+    w = weights(shape, dtype, 4)
+    a = _gpu(lib, shape, ranks, 0.05, dtype)
+    b = _gpu(lib, shape, ranks, 0.05, dtype)
+    g_dev, w_dev = g.cuda(), w.cuda()
+    a.refresh(g_dev)
+    b.refresh(g_dev)
+    a.step(g_dev, w_dev)
+    a.sync()
+    g_host, w_host = to_np(g).copy(), to_np(w).copy()
+    b.step_host(g_host, w_host)
+    assert np.array_equal(to_np(w_dev).view(np.uint8), w_host.view(np.uint8))
+    assert not np.array_equal(w_host, to_np(w))
+    assert a.get_state()["t"] == b.get_state()["t"] == 1
