@@ -140,9 +140,6 @@ __device__ __forceinline__ float2 adam_elem(float2 g, float* m, float* v, const 
   return make_float2(mr * a.inv_bc1 * inv, mi * a.inv_bc1 * inv);
 }
 
-__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
-  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
-}
 __device__ __forceinline__ float2 cfma(float2 a, float2 b, float2 c) {  // a*b + c
   return make_float2(__fmaf_rn(a.x, b.x, __fmaf_rn(-a.y, b.y, c.x)),
                      __fmaf_rn(a.x, b.y, __fmaf_rn(a.y, b.x, c.y)));
