@@ -14,22 +14,25 @@ import pytest
 import oracle
 
 
-@pytest.mark.parametrize("N,M,r", [(64, 17, 4), (128, 33, 8), (128, 64, 32), (256, 65, 16)])
-def test_oracle_low_rank_count_is_equation_10(N, M, r):
+EQ10_CASES = [(64, 17, 4), (128, 33, 8), (128, 64, 32), (256, 65, 16)]
+
+
+def pin_equation_10(fn):
     """Core plus factors of an N x N x M x M weight at rank r in every mode:
     r^4 + 2 r N + 2 r M entries."""
-    m = oracle.state_memory((N, N, M, M), (r, r, r, r), 0.0, "c64")
-    assert m["core_elems"] + m["factor_elems"] == r ** 4 + 2 * r * N + 2 * r * M
+    for N, M, r in EQ10_CASES:
+        m = fn((N, N, M, M), (r, r, r, r), 0.0, "c64")
+        assert m["core_elems"] + m["factor_elems"] == r ** 4 + 2 * r * N + 2 * r * M
 
 
-def test_oracle_headline_tensor_by_hand():
+def pin_headline_by_hand(fn):
     """(256,256,128,65) complex fp16, ranks (64,64,32,16), rho 0.05:
     N = 545,259,520; k = floor(0.05 N) = 27,262,976;
     core 64*64*32*16 = 2,097,152 entries x (8 + 4) B = 25,165,824 B;
     factors 2*256*64 + 128*32 + 65*16 = 37,904 entries x 8 B = 303,232 B;
     sparse 27,262,976 x (8 + 8 + 4) B = 545,259,520 B;
     AdamW 545,259,520 x 12 B = 6,543,114,240 B."""
-    m = oracle.state_memory((256, 256, 128, 65), (64, 64, 32, 16), 0.05, "c32h")
+    m = fn((256, 256, 128, 65), (64, 64, 32, 16), 0.05, "c32h")
     assert m["N"] == 545_259_520 and m["k"] == 27_262_976
     assert m["core_bytes"] == 25_165_824
     assert m["factor_bytes"] == 303_232
@@ -38,22 +41,63 @@ def test_oracle_headline_tensor_by_hand():
     assert m["adamw_bytes"] == 6_543_114_240
 
 
-def test_oracle_special_cases():
+def pin_special_cases(fn):
     # no sparse part at rho = 0
-    m = oracle.state_memory((16, 12, 8), (4, 3, 2), 0.0, "r32")
+    m = fn((16, 12, 8), (4, 3, 2), 0.0, "r32")
     assert m["k"] == 0 and m["sparse_bytes"] == 0
+    # k = floor(rho N): 0.1 * 21 = 2.1 -> 2
+    assert fn((7, 3), (7, 3), 0.1, "r32")["k"] == 2
     # every mode at full rank: the core is the whole tensor and no factor is kept
-    m = oracle.state_memory((16, 12, 8), (16, 12, 8), 0.0, "c64")
+    m = fn((16, 12, 8), (16, 12, 8), 0.0, "c64")
     assert m["factor_elems"] == 0 and m["core_bytes"] == m["adamw_bytes"]
     # real tensors: 4-byte m and v and factors
-    m = oracle.state_memory((10, 6), (2, 3), 0.5, "r16")
+    m = fn((10, 6), (2, 3), 0.5, "r16")
     assert m["core_bytes"] == 6 * 8 and m["factor_bytes"] == (20 + 18) * 4
     assert m["sparse_bytes"] == 30 * (8 + 8) and m["adamw_bytes"] == 60 * 8
     # view-as-real complex Adam keeps two second moments
-    a = oracle.state_memory((10, 6), (2, 3), 0.5, "c64", complex_adam=0)
-    b = oracle.state_memory((10, 6), (2, 3), 0.5, "c64", complex_adam=1)
+    a = fn((10, 6), (2, 3), 0.5, "c64", complex_adam=0)
+    b = fn((10, 6), (2, 3), 0.5, "c64", complex_adam=1)
     assert b["adamw_bytes"] - a["adamw_bytes"] == 60 * 4
     assert b["sparse_bytes"] - a["sparse_bytes"] == 30 * 4
+
+
+PINS = [pin_equation_10, pin_headline_by_hand, pin_special_cases]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_oracle_pins(pin):
+    pin(oracle.state_memory)
+
+
+# (name, original text, mutated text): plausible slips in the oracle's count
+MUTANTS = [
+    ("factor_for_full_rank_mode", "if r < I)", "if r <= I)"),
+    ("complex_m_as_real", "m_b = 8 if cplx else 4", "m_b = 4"),
+    ("index_4_bytes", "k * (8 + m_b + v_b)", "k * (4 + m_b + v_b)"),
+    ("v_doubled_by_default", "v_b = 8 if (cplx and complex_adam) else 4", "v_b = 8 if cplx else 4"),
+    ("core_m_only", "core * (m_b + v_b)", "core * m_b"),
+    ("k_rounded_up", "math.floor(sparse_ratio * N)", "math.ceil(sparse_ratio * N)"),
+    ("real_factor_8_bytes", "u_b = 8 if cplx else 4", "u_b = 8"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new):
+    """A mutated copy of the oracle's count (the shipped one is untouched)
+    fails at least one pin."""
+    import inspect
+    src = inspect.getsource(oracle.state_memory)
+    assert src.count(old) == 1, name
+    ns = {"math": math}
+    exec(src.replace(old, new), ns)
+    mutant = ns["state_memory"]
+    failed = 0
+    for pin in PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"mutant {name} passed every pin"
 
 
 def test_library_equals_oracle():
