@@ -35,6 +35,22 @@ MUTANTS = [
      "A[p * n + j] = {c * xp.re + s * xq.re, c * xp.im + s * xq.im};"),
     ("mask_not_applied", "X[e] = in_omega[base + e] ? cd{0, 0} : load_elem(g, h.gdt, base + e);",
      "X[e] = load_elem(g, h.gdt, base + e);"),
+    ("bias_correction_step_off_by_one", "const double s = (double)(h.t + 1);",
+     "const double s = (double)(h.t + 2);"),
+    ("decay_applied_after_update",
+     "cd nv = {wv.re * decay - h.lr * X[e].re, wv.im * decay - h.lr * X[e].im};",
+     "cd nv = {(wv.re - h.lr * X[e].re) * decay, (wv.im - h.lr * X[e].im) * decay};"),
+    ("sparse_scale_dropped", "sparse_upd[j] = {h.o.sparse_scale * u.re, h.o.sparse_scale * u.im};",
+     "sparse_upd[j] = {u.re, u.im};"),
+    ("moment_reset_ignored", "if (h.o.moments_on_refresh == 1) {", "if (h.o.moments_on_refresh == 7) {"),
+    ("view_as_real_v_uses_abs2", "v[1] = (float)(b2 * v[1] + (1 - b2) * g.im * g.im);",
+     "v[1] = (float)(b2 * v[1] + (1 - b2) * abs2(g));"),
+    ("refresh_schedule_off_by_one", "if (h.o.auto_refresh && h.T > 0 && h.t % h.T == 0) refresh(h, g);",
+     "if (h.o.auto_refresh && h.T > 0 && (h.t + 1) % h.T == 0) refresh(h, g);"),
+    ("random_draw_ignores_ordinal", "uint64_t s = sm_mix(seed + (ordinal + 1) * SM_GAMMA);",
+     "uint64_t s = sm_mix(seed + SM_GAMMA);"),
+    ("eigenvalues_ascending", "[&](int64_t a, int64_t b) { return A[a * n + a].re > A[b * n + b].re; });",
+     "[&](int64_t a, int64_t b) { return A[a * n + a].re < A[b * n + b].re; });"),
 ]
 
 
