@@ -33,6 +33,9 @@
 //   |g|^2 (mode 0) or re/im treated as separate reals (mode 1); bias
 //   correction with s = t + 1; decoupled weight decay; moments kept across a
 //   refresh unless asked to reset; refresh before the step when t % T == 0.
+//   Low-rank-first order (the ablation of the decomposition order): factors
+//   from the gradient itself, Omega on E = G - L keyed from E rounded to fp32,
+//   sparse values E at Omega with L from the step's pre-Adam core.
 //
 // Everything is computed in fp64. Stored state is rounded to its storage type
 // (moments and factors fp32, weights their own dtype) exactly once.
@@ -405,6 +408,7 @@ struct Opts {
   int complex_adam;        // 0: v = EMA |g|^2; 1: re and im as separate reals
   int moments_on_refresh;  // 0 keep, 1 reset to zero
   int auto_refresh;        // refresh inside step when t % T == 0
+  int order = 0;           // 0 sparse part first; 1 low-rank part first (the ablated order)
 };
 
 struct Orc {
@@ -463,10 +467,41 @@ int64_t n_slabs(const Orc& h) {
   return s;
 }
 
+std::vector<cd> load_all(const void* g, int dt, int64_t N) {
+  std::vector<cd> X(N);
+  parallel_for(N, [&](int64_t lo, int64_t hi) {
+    for (int64_t i = lo; i < hi; ++i) X[i] = load_elem(g, dt, i);
+  });
+  return X;
+}
+
+// U_n for every mode with r_n < I_n: the leading r_n eigenvectors of the
+// mode-n Gram matrix of X (plain HOSVD); all eigenvalues are kept.
+void factors_from(Orc& h, const std::vector<cd>& X) {
+  for (int n = 0; n < h.d; ++n) {
+    int64_t In = h.I[n], rn = h.r[n];
+    if (rn == In) continue;
+    std::vector<cd> Gm(In * In), V(In * In);
+    std::vector<double> w(In);
+    mode_gram(X.data(), h.I, n, Gm.data());
+    jacobi_eigh(Gm.data(), In, w.data(), V.data());
+    h.eigval[n] = w;
+    for (int64_t i = 0; i < In; ++i)
+      for (int64_t j = 0; j < rn; ++j) {
+        h.U[n][2 * (i * rn + j)] = (float)V[i * In + j].re;
+        h.U[n][2 * (i * rn + j) + 1] = (float)V[i * In + j].im;
+      }
+  }
+}
+
+void finish_refresh(Orc& h);
+int refresh_lowrank_first(Orc& h, const void* g);
+
 // Refresh [S1 section 三, S2]: Omega first, then the residual R = G with zeros
 // on Omega, then for each mode with r_n < I_n the leading r_n eigenvectors of
 // the mode-n Gram matrix of R (plain HOSVD).
 int refresh(Orc& h, const void* g) {
+  if (h.o.order == 1) return refresh_lowrank_first(h, g);
   h.omega.assign(h.k, 0);
   if (h.o.omega_mode == 0)
     topk_select(g, h.gdt, h.N, h.k, h.omega.data());
@@ -478,26 +513,15 @@ int refresh(Orc& h, const void* g) {
   for (int n = 0; n < h.d; ++n) need_gram |= h.r[n] < h.I[n];
   h.eigval.assign(h.d, {});
   if (need_gram) {
-    std::vector<cd> R(h.N);
-    parallel_for(h.N, [&](int64_t lo, int64_t hi) {
-      for (int64_t i = lo; i < hi; ++i) R[i] = load_elem(g, h.gdt, i);
-    });
+    std::vector<cd> R = load_all(g, h.gdt, h.N);
     for (int64_t j = 0; j < h.k; ++j) R[h.omega[j]] = {0, 0};
-    for (int n = 0; n < h.d; ++n) {
-      int64_t In = h.I[n], rn = h.r[n];
-      if (rn == In) continue;
-      std::vector<cd> Gm(In * In), V(In * In);
-      std::vector<double> w(In);
-      mode_gram(R.data(), h.I, n, Gm.data());
-      jacobi_eigh(Gm.data(), In, w.data(), V.data());
-      h.eigval[n] = w;
-      for (int64_t i = 0; i < In; ++i)
-        for (int64_t j = 0; j < rn; ++j) {
-          h.U[n][2 * (i * rn + j)] = (float)V[i * In + j].re;
-          h.U[n][2 * (i * rn + j) + 1] = (float)V[i * In + j].im;
-        }
-    }
+    factors_from(h, R);
   }
+  finish_refresh(h);
+  return 0;
+}
+
+void finish_refresh(Orc& h) {
   if (h.o.moments_on_refresh == 1) {
     std::fill(h.core_m.begin(), h.core_m.end(), 0.f);
     std::fill(h.core_v.begin(), h.core_v.end(), 0.f);
@@ -506,6 +530,106 @@ int refresh(Orc& h, const void* g) {
   }
   h.has_subspace = true;
   h.refreshes += 1;
+}
+
+// ------------------------------------------- low-rank-first order (ablation)
+// The decomposition order is a free parameter of the method ([S2]
+// "Assumptions & free parameters": sparse then low-rank is the chosen order;
+// its ablation reverses it, and [S1] section 五 reports that sparse-first
+// wins). Reversed, the low-rank part comes first: the factors are the HOSVD of
+// the gradient itself, L = G x_n U_n U_n^H over the projected modes, and Omega
+// is selected on E = G - L (E rounded to fp32 and keyed like an fp32 gradient
+// of the same kind). A step projects the whole gradient to the core C; the
+// sparse values are E at Omega, with L rebuilt from that step's C before Adam;
+// the update is rebuilt from the Adam core and the sparse update scattered in,
+// as in the sparse-first step.
+
+// X x_n U_n^H (proj) or X x_n U_n over every mode with r_n < I_n, in mode
+// order; dims follows the shape.
+std::vector<cd> products_all(const Orc& h, const std::vector<std::vector<cd>>& Uc,
+                             std::vector<cd> X, std::vector<int64_t>& dims, bool proj) {
+  for (int n = 0; n < h.d; ++n) {
+    if (h.r[n] == h.I[n]) continue;
+    std::vector<int64_t> nd = dims;
+    nd[n] = proj ? h.r[n] : h.I[n];
+    int64_t sz = 1;
+    for (auto v : nd) sz *= v;
+    std::vector<cd> Y(sz);
+    mode_product(X.data(), dims, n, Uc[n].data(), h.I[n], h.r[n], proj, Y.data(), true);
+    X.swap(Y);
+    dims = nd;
+  }
+  return X;
+}
+
+std::vector<std::vector<cd>> all_U(const Orc& h) {
+  std::vector<std::vector<cd>> Uc(h.d);
+  for (int n = 0; n < h.d; ++n) Uc[n] = U_as_cd(h, n);
+  return Uc;
+}
+
+int refresh_lowrank_first(Orc& h, const void* g) {
+  std::vector<cd> G = load_all(g, h.gdt, h.N);
+  h.eigval.assign(h.d, {});
+  factors_from(h, G);
+  const auto Uc = all_U(h);
+  std::vector<int64_t> dims(h.I);
+  std::vector<cd> C = products_all(h, Uc, G, dims, true);
+  std::vector<cd> L = products_all(h, Uc, C, dims, false);
+  const int comps = h.cplx ? 2 : 1;
+  std::vector<float> Ef(h.N * comps);
+  for (int64_t i = 0; i < h.N; ++i) {
+    Ef[i * comps] = (float)(G[i].re - L[i].re);
+    if (h.cplx) Ef[i * comps + 1] = (float)(G[i].im - L[i].im);
+  }
+  h.omega.assign(h.k, 0);
+  if (h.o.omega_mode == 0)
+    topk_select(Ef.data(), h.cplx ? DT_C64 : DT_R32, h.N, h.k, h.omega.data());
+  else
+    random_select(h.o.seed, (uint64_t)h.refreshes, h.N, h.k, h.omega.data());
+  h.omega_val.resize(h.k);
+  for (int64_t j = 0; j < h.k; ++j) {
+    const int64_t i = h.omega[j];
+    h.omega_val[j] = {G[i].re - L[i].re, G[i].im - L[i].im};
+  }
+  finish_refresh(h);
+  return 0;
+}
+
+int step_lowrank_first(Orc& h, const void* g, void* w, int64_t nsel, const int64_t* sel,
+                       double bc1, double bc2) {
+  const int mc = h.mcomp(), vc = h.vcomp();
+  std::vector<cd> G = load_all(g, h.gdt, h.N);
+  const auto Uc = all_U(h);
+  std::vector<int64_t> dims(h.I);
+  std::vector<cd> C = products_all(h, Uc, G, dims, true);
+  const std::vector<int64_t> core_dims = dims;
+  std::vector<cd> L = products_all(h, Uc, C, dims, false);
+  std::vector<cd> sparse_upd(h.k);
+  for (int64_t j = 0; j < h.k; ++j) {
+    const int64_t i = h.omega[j];
+    cd e = {G[i].re - L[i].re, G[i].im - L[i].im};
+    cd u = adam_update(e, &h.sp_m[j * mc], &h.sp_v[j * vc], h, bc1, bc2);
+    sparse_upd[j] = {h.o.sparse_scale * u.re, h.o.sparse_scale * u.im};
+  }
+  for (int64_t j = 0; j < h.ncore; ++j)
+    C[j] = adam_update(C[j], &h.core_m[j * mc], &h.core_v[j * vc], h, bc1, bc2);
+  dims = core_dims;
+  std::vector<cd> D = products_all(h, Uc, C, dims, false);
+  for (int64_t j = 0; j < h.k; ++j) D[h.omega[j]] = D[h.omega[j]] + sparse_upd[j];
+  const int64_t slab = h.I[h.d - 2] * h.I[h.d - 1];
+  const double decay = 1 - h.lr * h.wd;
+  auto update = [&](int64_t e) {
+    cd wv = load_elem(w, h.wdt, e);
+    store_elem(w, h.wdt, e, {wv.re * decay - h.lr * D[e].re, wv.im * decay - h.lr * D[e].im});
+  };
+  if (sel) {
+    for (int64_t q = 0; q < nsel; ++q)
+      for (int64_t e = sel[q] * slab; e < (sel[q] + 1) * slab; ++e) update(e);
+  } else {
+    for (int64_t e = 0; e < h.N; ++e) update(e);
+  }
+  h.t += 1;
   return 0;
 }
 
@@ -518,6 +642,7 @@ int step(Orc& h, const void* g, void* w, int64_t nsel, const int64_t* sel) {
   const int d = h.d;
   const double s = (double)(h.t + 1);
   const double bc1 = 1 - std::pow(h.b1, s), bc2 = 1 - std::pow(h.b2, s);
+  if (h.o.order == 1) return step_lowrank_first(h, g, w, nsel, sel, bc1, bc2);
   const int mc = h.mcomp(), vc = h.vcomp();
   // Sparse part: gather on Omega, Adam on the k values, scale by lambda.
   std::vector<cd> sparse_upd(h.k);
@@ -716,6 +841,12 @@ void* orc_create(int ndim, const int64_t* shape, const int64_t* ranks, double rh
   return h;
 }
 void orc_destroy(void* h) { delete (Orc*)h; }
+// Decomposition order: 0 sparse part first (the method), 1 low-rank part first.
+int orc_set_order(void* h, int order) {
+  if (order < 0 || order > 1) return 1;
+  ((Orc*)h)->o.order = order;
+  return 0;
+}
 
 int orc_refresh(void* h, const void* g) { return refresh(*(Orc*)h, g); }
 int orc_step(void* h, const void* g, void* w, int64_t nsel, const int64_t* sel) {

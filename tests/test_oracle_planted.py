@@ -40,8 +40,11 @@ MUTANTS = [
     ("decay_applied_after_update",
      "cd nv = {wv.re * decay - h.lr * X[e].re, wv.im * decay - h.lr * X[e].im};",
      "cd nv = {(wv.re - h.lr * X[e].re) * decay, (wv.im - h.lr * X[e].im) * decay};"),
-    ("sparse_scale_dropped", "sparse_upd[j] = {h.o.sparse_scale * u.re, h.o.sparse_scale * u.im};",
-     "sparse_upd[j] = {u.re, u.im};"),
+    ("sparse_scale_dropped",
+     "    cd u = adam_update(gj, &h.sp_m[j * mc], &h.sp_v[j * vc], h, bc1, bc2);\n"
+     "    sparse_upd[j] = {h.o.sparse_scale * u.re, h.o.sparse_scale * u.im};",
+     "    cd u = adam_update(gj, &h.sp_m[j * mc], &h.sp_v[j * vc], h, bc1, bc2);\n"
+     "    sparse_upd[j] = {u.re, u.im};"),
     ("moment_reset_ignored", "if (h.o.moments_on_refresh == 1) {", "if (h.o.moments_on_refresh == 7) {"),
     ("view_as_real_v_uses_abs2", "v[1] = (float)(b2 * v[1] + (1 - b2) * g.im * g.im);",
      "v[1] = (float)(b2 * v[1] + (1 - b2) * abs2(g));"),
