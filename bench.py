@@ -115,13 +115,13 @@ class ClockSampler:
     """SM clock and clock-event reasons sampled during the timed region by a
     separate polling process (read-only NVML queries every 2 ms; a thread in
     this process would be starved while it launches). The samples inside the
-    timed region are kept, and written to gpurun_out/."""
+    timed region are kept, and written as clocks_rank<i>.csv to out_dir."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown"}
 
-    def __init__(self, index: int):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+    def __init__(self, index: int, out_dir: str):
+        self.path = os.path.join(out_dir, f"clocks_rank{index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         self.raw = self.path + ".raw"
         self.t0, self.t1 = 0.0, float("inf")
@@ -298,6 +298,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "generic", "tcgen05"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--out-dir", default=os.path.join(ROOT, "bench_out"),
+                    help="directory for the per-rank clock records")
     ap.add_argument("--sequential", action="store_true",
                     help="step the tensors of a multi-tensor workload one after another on one "
                          "stream (default: each on its own stream with an equal share of the SMs)")
@@ -420,7 +422,7 @@ def main():
 
     # the metric: K steps without per-kernel events; then K more with them,
     # for the per-kernel launch times of the roofline
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, args.out_dir)
     time.sleep(1.0)  # the polling process is up before the timed region
     sampler.mark(True)
     total_ms, _ = timed_steps(False)

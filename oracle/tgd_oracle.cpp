@@ -24,7 +24,7 @@
 //   [S4] same review, appended paper text, Appendix K (tensor operations and
 //        notation): mode-k unfolding, mode-k product, Frobenius norm.
 //
-// Readings where the pages are silent (each is listed in the design doc):
+// Readings where the pages are silent:
 //   k = floor(rho * N); top-k key = fp32 |g| (real) or fp32 fma(re,re,im*im)
 //   (complex); ties -> lower linear index; Omega emitted ascending; random
 //   Omega = k smallest splitmix64-derived keys; plain HOSVD (each U_n from the
