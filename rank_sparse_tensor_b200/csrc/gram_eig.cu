@@ -24,8 +24,11 @@
 // r_n eigenvectors, each scaled by a unit phase that makes its largest-
 // magnitude entry (ties to the lowest row) real and positive.
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace tgd {
 namespace {
@@ -280,6 +283,241 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
   }
 }
 
+// ------------------------------------------------ tensor-core Gram (I_n <= 64)
+// The Gram as one tcgen05 GEMM per chunk of 32 unfolding columns. A 128-row
+// K-major tile holds, for each split part, the rows x_i (rows 0..I-1) and
+// J x_i (rows I..2I-1), where J maps each (re, im) pair of a column to
+// (-im, re); the rest are zero. With K = (column, re/im), the product of the
+// tile with its first N = 2I rows gives D[i][j] = Re sum_c x_ic conj(x_jc) and
+// D[i][I + j] = Im sum_c x_ic conj(x_jc). Each fp32 value is split into three
+// bf16 parts h + m + l (each the bf16 rounding of what the earlier parts
+// leave), and the six products hh, hm, mh, hl, lh, mm are accumulated in
+// fp32 in TMEM, which keeps about fp32 accuracy; the products of the two
+// smallest parts (ml, lm, ll, below 2^-24 of the result) are dropped.
+constexpr int TG_THREADS = 128;
+constexpr int TG_COLS = 32;                 // complex columns per chunk: K = 64 bf16 values
+constexpr uint32_t TG_LBO = 2048;           // 128 rows x 16 B between K core matrices
+constexpr uint32_t TG_TILE = 8 * TG_LBO;    // 128 rows x 64 K values of bf16
+constexpr uint64_t TG_WAIT_NS = 2000000000ull;
+
+struct TcGramArgs {
+  const void* g;
+  const uint32_t* bits;
+  int64_t I, B, ncol, cols_per_split;
+  int N;     // MMA N: 2I rounded up to 16
+  int R;     // rows per thread pass: 32 (I <= 32) or 64
+  float* partial;  // [split][I][I] complex, interleaved
+  int* err;
+};
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ float bf16_val(uint16_t b) {
+  return __uint_as_float((uint32_t)b << 16);
+}
+// x = h + m + l (bf16 parts, each the rounding of what the earlier leave)
+__device__ __forceinline__ void split3(float x, uint16_t& h, uint16_t& m, uint16_t& l) {
+  h = bf16_bits(x);
+  const float r1 = x - bf16_val(h);
+  m = bf16_bits(r1);
+  l = bf16_bits(r1 - bf16_val(m));
+}
+
+template <int DT>
+__global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* tiles = smem;                                      // [stage][part] tiles
+  int64_t* colbase = (int64_t*)(smem + 6 * TG_TILE);          // [2][TG_COLS]
+  uint64_t* done = (uint64_t*)(colbase + 2 * TG_COLS);        // [2] MMAs of a stage done
+  uint32_t* tslot = (uint32_t*)(done + 2);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int Q = TG_THREADS / p.R, cpt = TG_COLS / Q;          // column blocks, columns per thread
+  const int i = tid % p.R, q = tid / p.R;
+  const bool row_ok = i < p.I;
+  const int64_t c_begin = (int64_t)blockIdx.y * p.cols_per_split;
+  const int64_t c_end = c_begin + p.cols_per_split < p.ncol ? c_begin + p.cols_per_split : p.ncol;
+  const int nch = (int)((c_end - c_begin + TG_COLS - 1) / TG_COLS);
+  const int64_t IB = p.I * p.B;
+  // zero every tile once: rows 2I..127 stay zero, rows 0..2I-1 are rewritten per chunk
+  for (uint32_t o = tid * 16; o < 6 * TG_TILE; o += TG_THREADS * 16)
+    *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    s_abort = 0;
+    ptx::mbar_init(&done[0], 1);
+    ptx::mbar_init(&done[1], 1);
+    ptx::fence_mbar_init();
+  }
+  auto set_colbase = [&](int slot, int64_t c0) {
+    if (tid < TG_COLS) {
+      const int64_t c = c0 + tid;
+      int64_t off = -1;
+      if (c < c_end) {
+        const int64_t a = c / p.B;
+        off = a * IB + (c - a * p.B);
+      }
+      colbase[slot * TG_COLS + tid] = off;
+    }
+  };
+  set_colbase(0, c_begin);
+  __syncthreads();
+  if (warp == 0) ptx::tmem_alloc(tslot, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t dt_base = *tslot;
+  const uint32_t idesc = ptx::idesc_f16(1, 128, p.N);
+  float2 v[16];
+  auto load = [&](int slot) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      float2 x = make_float2(0.f, 0.f);
+      if (u < cpt && row_ok) {
+        const int64_t cb = colbase[slot * TG_COLS + q * cpt + u];
+        if (cb >= 0) {
+          const int64_t idx = cb + (int64_t)i * p.B;
+          if (!(p.bits && mask_bit(p.bits, idx))) x = load_elem<DT>(p.g, idx);
+        }
+      }
+      v[u] = x;
+    }
+  };
+  // this thread's columns of the chunk -> rows i and I + i of the three tiles of stage s
+  auto store = [&](int s) {
+    if (!row_ok) return;
+#pragma unroll
+    for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
+      if (gq * 4 >= cpt) break;
+      uint32_t xr[3][4], jr[3][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 x = v[gq * 4 + u];
+        uint16_t rh, rm, rl, ih, im, il;
+        split3(x.x, rh, rm, rl);
+        split3(x.y, ih, im, il);
+        // x row: (re, im); J x row: (-im, re); the low half holds the even K
+        xr[0][u] = (uint32_t)rh | ((uint32_t)ih << 16);
+        xr[1][u] = (uint32_t)rm | ((uint32_t)im << 16);
+        xr[2][u] = (uint32_t)rl | ((uint32_t)il << 16);
+        jr[0][u] = (uint32_t)(ih ^ 0x8000u) | ((uint32_t)rh << 16);
+        jr[1][u] = (uint32_t)(im ^ 0x8000u) | ((uint32_t)rm << 16);
+        jr[2][u] = (uint32_t)(il ^ 0x8000u) | ((uint32_t)rl << 16);
+      }
+      const uint32_t kg = (uint32_t)(q * cpt / 4 + gq);
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        uint8_t* t = tiles + (size_t)(s * 3 + part) * TG_TILE + kg * TG_LBO;
+        *(uint4*)(t + (uint32_t)i * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
+        *(uint4*)(t + (uint32_t)(p.I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
+      }
+    }
+  };
+  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
+  load(0);
+  for (int kc = 0; kc < nch; ++kc) {
+    const int s = kc & 1;
+    if (kc >= 2) {
+      if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
+        atomicOr(p.err, DEV_ERR_TIMEOUT);
+        s_abort = 1;
+      }
+      __syncthreads();
+      if (s_abort) break;
+      waited[s]++;
+      ptx::tc_fence_after();
+    }
+    store(s);
+    set_colbase((kc + 1) & 1, c_begin + (int64_t)(kc + 1) * TG_COLS);
+    ptx::fence_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (kc + 1 < nch) load((kc + 1) & 1);
+    if (tid == 0) {
+      const uint32_t base = ptx::smem_u32(tiles + (size_t)s * 3 * TG_TILE);
+      // (A part, B part): hh, hm, mh, hl, lh, mm
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int pr = 0; pr < 6; ++pr) {
+          const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
+          const uint32_t ka = base + pa * TG_TILE + kk * 2 * TG_LBO;
+          const uint32_t kb = base + pb * TG_TILE + kk * 2 * TG_LBO;
+          ptx::mma_f16(dt_base, ptx::sdesc(ka, TG_LBO, 128), ptx::sdesc(kb, TG_LBO, 128), idesc,
+                       (kc > 0 || kk > 0 || pr > 0) ? 1u : 0u);
+        }
+      ptx::mma_commit(&done[s]);
+      issued[s]++;
+    }
+  }
+  __syncthreads();
+  bool ok = !s_abort;
+  if (ok && nch > 0) {
+    const int s = (nch - 1) & 1;
+    if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    ok = !s_abort;
+    ptx::tc_fence_after();
+  }
+  if (ok) {
+    // lane = row of D; columns j < I the real part, I <= j < 2I the imaginary part
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int row = tid;
+    float* out = p.partial + (size_t)blockIdx.y * p.I * p.I * 2;
+    for (int c0 = 0; c0 < p.N; c0 += 16) {
+      float y[16];
+      ptx::tmem_ld16(dt_base + lane_base + c0, y);
+      if (row < p.I) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = c0 + u;
+          if (j < p.I)
+            out[((int64_t)row * p.I + j) * 2] = nch > 0 ? y[u] : 0.f;
+          else if (j < 2 * p.I)
+            out[((int64_t)row * p.I + (j - p.I)) * 2 + 1] = nch > 0 ? y[u] : 0.f;
+        }
+      }
+    }
+  } else if (tid == 0) {
+    // bounded waits for MMAs still in flight
+    for (int st = 0; st < 2; ++st)
+      if (issued[st] > waited[st]) ptx::mbar_wait(&done[st], (issued[st] - 1) & 1u, TG_WAIT_NS / 4);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(dt_base, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+}
+
+size_t tg_smem_bytes() { return 6 * (size_t)TG_TILE + 2 * TG_COLS * 8 + 2 * 8 + 16; }
+
+struct TcGramGeom {
+  int64_t I, B, ncol, cols_per_split;
+  int nsplit, N, R;
+};
+
+TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
+  TcGramGeom g;
+  g.B = 1;
+  int64_t A = 1;
+  for (int q = 0; q < n; ++q) A *= dims[q];
+  for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
+  g.I = dims[n];
+  g.ncol = A * g.B;
+  g.N = (int)((2 * g.I + 15) / 16 * 16);
+  g.R = g.I <= 32 ? 32 : 64;
+  // two CTAs per SM, a few waves; at least four chunks per split; partials under 32 MB
+  int64_t ns = std::min<int64_t>(148 * 2 * 3, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
+  ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
+  g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), TG_COLS) * TG_COLS;
+  g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
+  return g;
+}
+
 // ------------------------------------------------------------- eigensolver
 __device__ __forceinline__ double2 zmul(double2 a, double2 b) {
   return make_double2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
@@ -455,11 +693,67 @@ __global__ void __launch_bounds__(ET) eig_kernel(const EigJob* jobs) {
 
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);
-  return sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
+  size_t b = sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
+  if (g.I <= 64) {
+    TcGramGeom t = tc_gram_geom(nd, dims, n);
+    b = std::max(b, sizeof(float2) * (size_t)t.nsplit * t.I * t.I);
+  }
+  return b;
+}
+
+// Tensor-core Gram for I_n <= 64 (see gram_tc_kernel); the split partials are
+// summed by the same fixed-order fp64 reduction.
+cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
+                         int n, float* partial, double* gram, int* err, cudaStream_t s) {
+  const TcGramGeom t = tc_gram_geom(nd, dims, n);
+  TcGramArgs a;
+  a.g = g;
+  a.bits = bits;
+  a.I = t.I;
+  a.B = t.B;
+  a.ncol = t.ncol;
+  a.cols_per_split = t.cols_per_split;
+  a.N = t.N;
+  a.R = t.R;
+  a.partial = partial;
+  a.err = err;
+  const size_t smem = tg_smem_bytes();
+  const dim3 grid(1, t.nsplit);
+  cudaError_t e = cudaSuccess;
+  switch (dt) {
+    case TGD_R32:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R32><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_C64:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C64><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_C32H:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C32H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C32H><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_R16:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R16><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  GramGeom geo{};
+  geo.I = t.I;
+  geo.TI = 64;  // one tile: every cell is computed directly
+  geo.nsplit = t.nsplit;
+  const int64_t cells = t.I * t.I;
+  gram_reduce_kernel<<<(int)ceil_div(cells, RC), RC * RS, 0, s>>>((const float2*)partial, geo,
+                                                                   (double2*)gram);
+  return cudaGetLastError();
 }
 
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                      int n, float* partial, double* gram, cudaStream_t s) {
+                      int n, float* partial, double* gram, int* err, cudaStream_t s) {
+  if (dims[n] <= 64) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s);
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
   const size_t smem = gram_smem_bytes(geo);
