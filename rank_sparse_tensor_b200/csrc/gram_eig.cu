@@ -689,6 +689,220 @@ __global__ void __launch_bounds__(ET) eig_kernel(const EigJob* jobs) {
   }
 }
 
+// Block form of the same parallel Jacobi for n <= 128: A is Hermitian, so only
+// its upper triangle is kept (packed, in shared memory: 132 KB at n = 128).
+// In a round the n/2 rotations are disjoint; the 2 x 2 block of A at the rows
+// of pair k1 and the columns of pair k2 becomes J1^H B J2 (the column rotation
+// of k2, then the row rotation of k1, as in eig_kernel), and each unordered
+// block (k1 <= k2) is one thread's work, so every stored entry has one writer
+// per round and a round needs two barriers. V is kept transposed (a row per
+// eigenvector): in shared memory for n <= 64, in the job's scratch otherwise.
+constexpr int EB_MAXN = 128;
+
+__device__ __forceinline__ int tri_idx(int i, int j, int n) {  // i <= j
+  return i * n - (i * (i - 1)) / 2 + (j - i);
+}
+
+__global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
+  const EigJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  if (n > EB_MAXN) return;
+  extern __shared__ double2 dyn[];
+  __shared__ int rp[EB_MAXN / 2], rq[EB_MAXN / 2], rrot[EB_MAXN / 2];
+  __shared__ double rcs[EB_MAXN / 2], rsn[EB_MAXN / 2];
+  __shared__ double2 rph[EB_MAXN / 2];
+  __shared__ uint8_t bk1[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2], bk2[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2];
+  __shared__ double red[ET / 32];
+  __shared__ double ev[EB_MAXN];
+  __shared__ int col_of_rank[EB_MAXN];
+  const int ntri = n * (n + 1) / 2;
+  double2* T = dyn;  // packed upper triangle of A
+  double2* Vt = n <= 64 ? dyn + ntri : (double2*)J.work;
+  const double2* G = (const double2*)J.gram;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e - i * n;
+    if (i <= j) T[tri_idx(i, j, n)] = G[e];
+    Vt[e] = make_double2(i == j ? 1.0 : 0.0, 0.0);
+  }
+  const int m = n + (n & 1);
+  const int npairs = m / 2;
+  const int nblk = npairs * (npairs + 1) / 2;
+  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+    int k1 = 0, r = b;
+    while (r >= npairs - k1) {
+      r -= npairs - k1;
+      ++k1;
+    }
+    bk1[b] = (uint8_t)k1;
+    bk2[b] = (uint8_t)(k1 + r);
+  }
+  __syncthreads();
+  auto get = [&](int i, int j) -> double2 {
+    if (i <= j) return T[tri_idx(i, j, n)];
+    const double2 v = T[tri_idx(j, i, n)];
+    return make_double2(v.x, -v.y);
+  };
+  auto put = [&](int i, int j, double2 v) {
+    if (i <= j)
+      T[tri_idx(i, j, n)] = v;
+    else
+      T[tri_idx(j, i, n)] = make_double2(v.x, -v.y);
+  };
+  double part = 0;
+  for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
+    int i = 0, r = e;
+    while (r >= n - i) {
+      r -= n - i;
+      ++i;
+    }
+    part += (r == 0 ? 1.0 : 2.0) * zabs2(T[e]);  // r == 0: the diagonal entry of row i
+  }
+  const double fro = block_sum(part, red);
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    double off_part = 0;
+    for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
+      int i = 0, r = e;
+      while (r >= n - i) {
+        r -= n - i;
+        ++i;
+      }
+      if (r > 0) off_part += zabs2(T[e]);
+    }
+    const double off = block_sum(off_part, red);
+    if (off <= 1e-24 * fro || off == 0.0) break;
+    for (int round = 0; round < m - 1; ++round) {
+      for (int k = threadIdx.x; k < npairs; k += blockDim.x) {
+        int p, q;
+        if (k == 0) {
+          p = round;
+          q = m - 1;
+        } else {
+          p = (round + k) % (m - 1);
+          q = (round - k + (m - 1)) % (m - 1);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        rp[k] = p;
+        rq[k] = q;
+        rrot[k] = 0;
+        if (q < n) {
+          const double2 apq = get(p, q);
+          const double r = sqrt(zabs2(apq));
+          if (r > 0.0) {
+            const double app = get(p, p).x, aqq = get(q, q).x;
+            const double tau = (aqq - app) / (2.0 * r);
+            const double t = (tau >= 0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+            const double c = 1.0 / sqrt(1.0 + t * t);
+            rrot[k] = 1;
+            rcs[k] = c;
+            rsn[k] = t * c;
+            rph[k] = make_double2(apq.x / r, apq.y / r);
+          }
+        }
+      }
+      __syncthreads();
+      for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+        const int k1 = bk1[b], k2 = bk2[b];
+        const int p1 = rp[k1], q1 = rq[k1], p2 = rp[k2], q2 = rq[k2];
+        const bool rot1 = rrot[k1], rot2 = rrot[k2];
+        if (!rot1 && !rot2) continue;
+        const bool h1 = q1 < n, h2 = q2 < n;  // the dummy index of odd n is absent
+        double2 b00 = get(p1, p2), b01 = h2 ? get(p1, q2) : make_double2(0, 0);
+        double2 b10 = h1 ? get(q1, p2) : make_double2(0, 0);
+        double2 b11 = h1 && h2 ? get(q1, q2) : make_double2(0, 0);
+        if (rot2) {  // columns p2, q2: B <- B J2
+          const double c = rcs[k2], s = rsn[k2];
+          const double2 ec = make_double2(rph[k2].x, -rph[k2].y);
+          double2 xp = b00, xq = zmul(b01, ec);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b01 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b10;
+          xq = zmul(b11, ec);
+          b10 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (rot1) {  // rows p1, q1: B <- J1^H B
+          const double c = rcs[k1], s = rsn[k1];
+          const double2 e = rph[k1];
+          double2 xp = b00, xq = zmul(b10, e);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b10 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b01;
+          xq = zmul(b11, e);
+          b01 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (k1 == k2) {
+          // the diagonal block: the rotation zeroes (p, q); the diagonal is real
+          put(p1, p1, make_double2(b00.x, 0.0));
+          if (h1) {
+            put(p1, q1, make_double2(0.0, 0.0));
+            put(q1, q1, make_double2(b11.x, 0.0));
+          }
+        } else {
+          put(p1, p2, b00);
+          if (h2) put(p1, q2, b01);
+          if (h1) put(q1, p2, b10);
+          if (h1 && h2) put(q1, q2, b11);
+        }
+      }
+      // V <- V J on the rows of V^T (no other thread touches them this round)
+      for (int w = threadIdx.x; w < npairs * n; w += blockDim.x) {
+        const int k = w / n, i = w - k * n;
+        if (!rrot[k]) continue;
+        const int p = rp[k], q = rq[k];
+        const double c = rcs[k], s = rsn[k];
+        const double2 ec = make_double2(rph[k].x, -rph[k].y);
+        const double2 xp = Vt[p * n + i], xq = zmul(Vt[q * n + i], ec);
+        Vt[p * n + i] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+        Vt[q * n + i] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) ev[i] = T[tri_idx(i, i, n)].x;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const double li = ev[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += (ev[j] > li) || (ev[j] == li && j < i);
+    col_of_rank[rank] = i;
+    J.evals[rank] = li;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int rr = wid; rr < J.r; rr += nw) {
+    const int c = col_of_rank[rr];
+    double best = -1.0;
+    int bi = 0;
+    for (int row = lane; row < n; row += 32) {
+      const double mg = zabs2(Vt[c * n + row]);
+      if (mg > best) {
+        best = mg;
+        bi = row;
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    const double2 piv = Vt[c * n + bi];
+    const double pm = sqrt(zabs2(piv));
+    const double2 ph = pm > 0 ? make_double2(piv.x / pm, -piv.y / pm) : make_double2(1.0, 0.0);
+    for (int row = lane; row < n; row += 32) {
+      const double2 u = zmul(Vt[c * n + row], ph);
+      ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
+    }
+  }
+}
+
 }  // namespace
 
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
@@ -783,6 +997,26 @@ size_t eig_work_doubles(int n) { return n > 64 ? (size_t)4 * n * n : 0; }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
+  bool all_small = true;
+  size_t bsmem = 16;
+  for (int j = 0; j < njobs; ++j) {
+    const int n = jobs_host[j].n;
+    if (n > EB_MAXN || jobs_host[j].r > n) {
+      all_small = false;
+      break;
+    }
+    const size_t need = sizeof(double2) * ((size_t)n * (n + 1) / 2 + (n <= 64 ? (size_t)n * n : 0));
+    bsmem = std::max(bsmem, need);
+  }
+  if (all_small) {
+    cudaError_t e = cudaFuncSetAttribute(eig_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bsmem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    eig_block_kernel<<<njobs, ET, bsmem, s>>>(jobs_dev);
+    return cudaGetLastError();
+  }
   int smem_n = 0;
   for (int j = 0; j < njobs; ++j) {
     if (jobs_host[j].n > MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;
