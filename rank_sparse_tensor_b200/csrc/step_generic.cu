@@ -164,6 +164,59 @@ __global__ void __launch_bounds__(MT) mode_product_kernel(S src, int64_t A, int6
   }
 }
 
+// Y = X x_n M for coefficient matrices of at most SP_MAXMK entries (the modes
+// of FNO-sized tensors): one thread per column (a, b) of the unfolding reads
+// its K values (stride B: coalesced across threads when B > 1, from cache
+// when B == 1) once per block of SP_J outputs, M is broadcast from shared
+// memory and the outputs stay in registers. The sum over k runs in the same
+// order as in mode_product_kernel, so both give the same bits.
+constexpr int SP_T = 256, SP_J = 16, SP_MAXMK = 4096;
+
+template <class S, bool CPLX>
+__global__ void __launch_bounds__(SP_T) mode_product_small_kernel(S src, int64_t A, int64_t K,
+                                                                  int64_t B, const float* M,
+                                                                  int64_t J, float* Y) {
+  __shared__ float2 Ms[SP_MAXMK];
+  for (int64_t e = threadIdx.x; e < J * K; e += SP_T)
+    Ms[e] = CPLX ? ((const float2*)M)[e] : make_float2(M[e], 0.f);
+  __syncthreads();
+  const int64_t ncol = A * B;
+  for (int64_t c = (int64_t)blockIdx.x * SP_T + threadIdx.x; c < ncol;
+       c += (int64_t)gridDim.x * SP_T) {
+    const int64_t a = c / B, b = c - a * B;
+    const int64_t xb = a * K * B + b, yb = a * J * B + b;
+    for (int64_t j0 = 0; j0 < J; j0 += SP_J) {
+      float2 acc[SP_J];
+#pragma unroll
+      for (int u = 0; u < SP_J; ++u) acc[u] = make_float2(0.f, 0.f);
+      for (int64_t k = 0; k < K; ++k) {
+        const float2 x = src(xb + k * B);
+        const float2* mk = Ms + j0 * K + k;
+#pragma unroll
+        for (int u = 0; u < SP_J; ++u) {
+          if (j0 + u < J) {
+            const float2 m = mk[u * K];
+            if (CPLX)
+              acc[u] = cfma(m, x, acc[u]);
+            else
+              acc[u].x = __fmaf_rn(m.x, x.x, acc[u].x);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < SP_J; ++u) {
+        if (j0 + u < J) {
+          const int64_t o = yb + (j0 + u) * B;
+          if (CPLX)
+            ((float2*)Y)[o] = acc[u];
+          else
+            Y[o] = acc[u].x;
+        }
+      }
+    }
+  }
+}
+
 template <int DT>
 __global__ void masked_copy_kernel(const void* g, const uint32_t* bits, int64_t n, float* out) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -223,11 +276,21 @@ __global__ void coef_kernel(const float2* U, int64_t I, int64_t r, bool cplx, fl
   }
 }
 
+// The small-matrix kernel when M fits its shared memory, else the tiled one.
+template <class S, bool CPLX>
+void launch_product(S src, int64_t A, int64_t K, int64_t B, const float* M, int64_t J, float* Y,
+                    cudaStream_t s, dim3 grid) {
+  if (J * K <= SP_MAXMK)
+    mode_product_small_kernel<S, CPLX><<<grid_for(A * B, SP_T), SP_T, 0, s>>>(src, A, K, B, M, J, Y);
+  else
+    mode_product_kernel<S, CPLX><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
+}
+
 template <int DT>
 cudaError_t launch_first(const void* X, const uint32_t* bits, int64_t A, int64_t K, int64_t B,
                          const float* M, int64_t J, float* Y, cudaStream_t s, dim3 grid) {
   Src<DT, Dt<DT>::cplx> src{X, bits};
-  mode_product_kernel<Src<DT, Dt<DT>::cplx>, Dt<DT>::cplx><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
+  launch_product<Src<DT, Dt<DT>::cplx>, Dt<DT>::cplx>(src, A, K, B, M, J, Y, s, grid);
   return cudaGetLastError();
 }
 
@@ -259,13 +322,10 @@ cudaError_t mode_product(const void* X, int src_dt, const uint32_t* bits, bool c
     default:
       break;
   }
-  if (cplx) {
-    Src<-1, true> src{X, nullptr};
-    mode_product_kernel<Src<-1, true>, true><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
-  } else {
-    Src<-1, false> src{X, nullptr};
-    mode_product_kernel<Src<-1, false>, false><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
-  }
+  if (cplx)
+    launch_product<Src<-1, true>, true>(Src<-1, true>{X, nullptr}, A, K, B, M, J, Y, s, grid);
+  else
+    launch_product<Src<-1, false>, false>(Src<-1, false>{X, nullptr}, A, K, B, M, J, Y, s, grid);
   return cudaGetLastError();
 }
 
