@@ -46,8 +46,12 @@ size_t eig_work_doubles(int n);
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
 
 // ---- step_generic.cu: CUDA-core path of the step
+// L (optional, fp32 like the chain buffers): Adam on G[Omega] - L[Omega].
 cudaError_t sparse_adam(const void* g, int dt, const int64_t* omega, int64_t k, float* m,
-                        float* v, const AdamConst& a, float* upd, cudaStream_t s);
+                        float* v, const AdamConst& a, float* upd, cudaStream_t s,
+                        const float* L = nullptr);
+// L <- G - L over n elements (fp32; float2 for complex dtypes).
+cudaError_t residual_in_place(const void* g, int dt, float* L, int64_t n, cudaStream_t s);
 // Y = X x_n M: X (A, K, B), M (J x K) row-major complex or real, Y (A, J, B).
 // src_dt >= 0: X is the storage-typed gradient, masked by `bits`; src_dt < 0:
 // X is fp32 (float2 when cplx).

@@ -27,13 +27,19 @@ int grid_for(int64_t n, int threads = 256) {
   return (int)(b < 1 ? 1 : (b > cap ? cap : b));
 }
 
+// Adam on the k values at Omega: G[Omega], or G[Omega] - L[Omega] when L (the
+// low-rank part, fp32) is given (the low-rank-first order).
 template <int DT>
-__global__ void sparse_adam_kernel(const void* g, const int64_t* omega, int64_t k, float* m,
-                                   float* v, AdamConst a, float* upd) {
+__global__ void sparse_adam_kernel(const void* g, const float* L, const int64_t* omega, int64_t k,
+                                   float* m, float* v, AdamConst a, float* upd) {
   const int mc = a.cplx ? 2 : 1, vc = (a.cplx && a.cmode == 1) ? 2 : 1;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < k;
        j += (int64_t)gridDim.x * blockDim.x) {
     float2 gv = load_elem<DT>(g, omega[j]);
+    if (L) {
+      const float2 l = a.cplx ? ((const float2*)L)[omega[j]] : make_float2(L[omega[j]], 0.f);
+      gv = make_float2(gv.x - l.x, gv.y - l.y);
+    }
     float mm[2], vv[2];
     for (int c = 0; c < mc; ++c) mm[c] = m[j * mc + c];
     for (int c = 0; c < vc; ++c) vv[c] = v[j * vc + c];
@@ -221,11 +227,26 @@ template <int DT>
 __global__ void masked_copy_kernel(const void* g, const uint32_t* bits, int64_t n, float* out) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    float2 v = mask_bit(bits, i) ? make_float2(0.f, 0.f) : load_elem<DT>(g, i);
+    float2 v = bits && mask_bit(bits, i) ? make_float2(0.f, 0.f) : load_elem<DT>(g, i);
     if (Dt<DT>::cplx)
       ((float2*)out)[i] = v;
     else
       out[i] = v.x;
+  }
+}
+
+// L <- G - L (fp32, in place): the residual after the low-rank part.
+template <int DT>
+__global__ void residual_kernel(const void* g, float* L, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float2 x = load_elem<DT>(g, i);
+    if (Dt<DT>::cplx) {
+      const float2 l = ((const float2*)L)[i];
+      ((float2*)L)[i] = make_float2(x.x - l.x, x.y - l.y);
+    } else {
+      L[i] = x.x - L[i];
+    }
   }
 }
 
@@ -297,14 +318,26 @@ cudaError_t launch_first(const void* X, const uint32_t* bits, int64_t A, int64_t
 }  // namespace
 
 cudaError_t sparse_adam(const void* g, int dt, const int64_t* omega, int64_t k, float* m,
-                        float* v, const AdamConst& a, float* upd, cudaStream_t s) {
+                        float* v, const AdamConst& a, float* upd, cudaStream_t s, const float* L) {
   if (k <= 0) return cudaSuccess;
   int grid = grid_for(k);
   switch (dt) {
-    case TGD_R32: sparse_adam_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_C64: sparse_adam_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_C32H: sparse_adam_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_R16: sparse_adam_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
+    case TGD_R32: sparse_adam_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_C64: sparse_adam_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_C32H: sparse_adam_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_R16: sparse_adam_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t residual_in_place(const void* g, int dt, float* L, int64_t n, cudaStream_t s) {
+  int grid = grid_for(n);
+  switch (dt) {
+    case TGD_R32: residual_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_C64: residual_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_C32H: residual_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_R16: residual_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, L, n); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
