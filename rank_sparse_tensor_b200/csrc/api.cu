@@ -279,7 +279,7 @@ tgd_status do_refresh_lowrank_first(tgd_ctx* h, const void* g, cudaStream_t s) {
   for (int n = 0; n < h->d; ++n) {
     if (!mode_active(h, n)) continue;
     TIMED(h, s, "mode_gram");
-    TGD_CUDA(h, mode_gram(g, h->gdt, nullptr, h->d, h->I, n, h->gram_part, h->gram[n], s));
+    TGD_CUDA(h, mode_gram(g, h->gdt, nullptr, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s));
     EigJob j;
     j.gram = h->gram[n];
     j.work = h->eig_work[n];
