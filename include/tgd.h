@@ -98,6 +98,12 @@ typedef struct {
                              itself, Omega = top-k of E = G - L (L = G x_n U_n U_n^H, E in fp32),
                              each step's sparse values E at Omega with L from that step's core.
                              Order 1 runs on the CUDA-core path. */
+  int basis;              /* factors at a refresh: 0 (default) HOSVD, the leading eigenvectors
+                             of each mode-n Gram [S2]; 1 the r_n columns q_j of the orthonormal
+                             DCT matrix (sqrt(2/n) cos(k (2j+1) pi / 2n), row 0 / sqrt 2) with
+                             the largest alignment q_j^T Gram q_j, ties to the lower column (the
+                             dynamic column selection of the Trion / DCT-AdamW page); no
+                             eigensolver runs */
 } tgd_options;
 
 /* Fills `opt` with the defaults listed above. */

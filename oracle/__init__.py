@@ -55,6 +55,7 @@ def lib():
                                      i32, u64, dbl, i32, i32, i32]
             L.orc_destroy.argtypes = [vp]
             L.orc_set_order.argtypes = [vp, i32]
+            L.orc_set_basis.argtypes = [vp, i32]
             L.orc_refresh.argtypes = [vp, vp]
             L.orc_step.argtypes = [vp, vp, vp, i64, vp]
             L.orc_info.argtypes = [vp, vp]
@@ -191,9 +192,10 @@ class Oracle:
     def __init__(self, shape, ranks, sparse_ratio, T, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
                  wd=0.0, grad_dtype="c64", weight_dtype=None, omega_mode=0, seed=0,
                  sparse_scale=1.0, complex_adam=0, moments_on_refresh=0, auto_refresh=1,
-                 order=0):
+                 order=0, basis=0):
         """order: 0 extracts the sparse part first (the method), 1 the
-        low-rank part first (the ablated order)."""
+        low-rank part first (the ablated order). basis: 0 HOSVD factors (the
+        method), 1 DCT columns chosen by their alignment with the Gram."""
         weight_dtype = weight_dtype or grad_dtype
         self.shape = tuple(int(s) for s in shape)
         self.ranks = tuple(int(r) for r in ranks)
@@ -208,6 +210,8 @@ class Oracle:
             raise ValueError("oracle rejected the configuration")
         if order and lib().orc_set_order(self._h, int(order)) != 0:
             raise ValueError("unknown decomposition order")
+        if basis and lib().orc_set_basis(self._h, int(basis)) != 0:
+            raise ValueError("unknown factor basis")
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -409,6 +409,7 @@ struct Opts {
   int moments_on_refresh;  // 0 keep, 1 reset to zero
   int auto_refresh;        // refresh inside step when t % T == 0
   int order = 0;           // 0 sparse part first; 1 low-rank part first (the ablated order)
+  int basis = 0;           // 0 HOSVD eigenvectors; 1 DCT columns chosen by alignment
 };
 
 struct Orc {
@@ -475,8 +476,43 @@ std::vector<cd> load_all(const void* g, int dt, int64_t N) {
   return X;
 }
 
+// Entry (k, j) of the orthonormal n x n DCT matrix of the dynamic column
+// selection (the Trion / DCT-AdamW page, "dynamic column selection"):
+// sqrt(2 / n) cos(k (2j + 1) pi / (2n)), row k = 0 divided by sqrt(2).
+double dct_entry(int64_t k, int64_t j, int64_t n) {
+  const double v = std::sqrt(2.0 / (double)n) * std::cos((double)k * (2.0 * j + 1.0) * M_PI / (2.0 * n));
+  return k == 0 ? v / std::sqrt(2.0) : v;
+}
+
+// DCT basis for mode n: the r_n columns q_j of the DCT matrix with the largest
+// alignment q_j^T Gram q_j (the squared l2 norm of the unfolding's components
+// along q_j), ties to the lower column, listed by descending alignment; the
+// sorted alignments stand where the eigenvalues would.
+void dct_factor(Orc& h, int n, const std::vector<cd>& Gm) {
+  const int64_t In = h.I[n], rn = h.r[n];
+  std::vector<double> score(In);
+  for (int64_t j = 0; j < In; ++j) {
+    double sc = 0;
+    for (int64_t a = 0; a < In; ++a)
+      for (int64_t b = 0; b < In; ++b) sc += dct_entry(a, j, In) * Gm[a * In + b].re * dct_entry(b, j, In);
+    score[j] = sc;
+  }
+  std::vector<int64_t> ord(In);
+  for (int64_t j = 0; j < In; ++j) ord[j] = j;
+  std::stable_sort(ord.begin(), ord.end(), [&](int64_t a, int64_t b) { return score[a] > score[b]; });
+  std::vector<double> w(In);
+  for (int64_t c = 0; c < In; ++c) w[c] = score[ord[c]];
+  h.eigval[n] = w;
+  for (int64_t i = 0; i < In; ++i)
+    for (int64_t c = 0; c < rn; ++c) {
+      h.U[n][2 * (i * rn + c)] = (float)dct_entry(i, ord[c], In);
+      h.U[n][2 * (i * rn + c) + 1] = 0.f;
+    }
+}
+
 // U_n for every mode with r_n < I_n: the leading r_n eigenvectors of the
-// mode-n Gram matrix of X (plain HOSVD); all eigenvalues are kept.
+// mode-n Gram matrix of X (plain HOSVD), or the DCT columns most aligned with
+// it; all eigenvalues (alignments) are kept.
 void factors_from(Orc& h, const std::vector<cd>& X) {
   for (int n = 0; n < h.d; ++n) {
     int64_t In = h.I[n], rn = h.r[n];
@@ -484,6 +520,10 @@ void factors_from(Orc& h, const std::vector<cd>& X) {
     std::vector<cd> Gm(In * In), V(In * In);
     std::vector<double> w(In);
     mode_gram(X.data(), h.I, n, Gm.data());
+    if (h.o.basis == 1) {
+      dct_factor(h, n, Gm);
+      continue;
+    }
     jacobi_eigh(Gm.data(), In, w.data(), V.data());
     h.eigval[n] = w;
     for (int64_t i = 0; i < In; ++i)
@@ -841,6 +881,12 @@ void* orc_create(int ndim, const int64_t* shape, const int64_t* ranks, double rh
   return h;
 }
 void orc_destroy(void* h) { delete (Orc*)h; }
+// Factor basis: 0 HOSVD eigenvectors (the method), 1 DCT column selection.
+int orc_set_basis(void* h, int basis) {
+  if (basis < 0 || basis > 1) return 1;
+  ((Orc*)h)->o.basis = basis;
+  return 0;
+}
 // Decomposition order: 0 sparse part first (the method), 1 low-rank part first.
 int orc_set_order(void* h, int order) {
   if (order < 0 || order > 1) return 1;

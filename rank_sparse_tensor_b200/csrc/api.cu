@@ -386,7 +386,10 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
   }
-  {
+  if (h->opt.basis == 1) {
+    TIMED(h, s, "dct_select");
+    TGD_CUDA(h, batched_dct_select(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+  } else {
     TIMED(h, s, "eigh");
     TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
   }
@@ -494,6 +497,7 @@ void tgd_default_options(tgd_options* opt) {
   opt->path = TGD_PATH_AUTO;
   opt->sm_budget = 0;
   opt->order = 0;
+  opt->basis = 0;
 }
 
 tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int64_t* ranks,
@@ -519,7 +523,8 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (opt) o = *opt;
   if (o.omega_mode < 0 || o.omega_mode > 1 || o.complex_adam < 0 || o.complex_adam > 1 ||
       o.moments_on_refresh < 0 || o.moments_on_refresh > 1 || o.path < 0 || o.path > 2 ||
-      o.sm_budget < 0 || !std::isfinite(o.sparse_scale) || o.order < 0 || o.order > 1)
+      o.sm_budget < 0 || !std::isfinite(o.sparse_scale) || o.order < 0 || o.order > 1 ||
+      o.basis < 0 || o.basis > 1)
     return fail(nullptr, TGD_ERR_INVALID_ARG, "bad option value");
   if (o.order == 1 && o.path == TGD_PATH_TCGEN05)
     return fail(nullptr, TGD_ERR_UNSUPPORTED, "the low-rank-first order runs on the CUDA-core path");

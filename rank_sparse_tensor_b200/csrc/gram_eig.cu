@@ -903,7 +903,61 @@ __global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
   }
 }
 
+// ------------------------------------------------------- DCT column selection
+// The dynamic column selection of the Trion / DCT-AdamW page as a factor
+// basis: thread j holds column q_j of the orthonormal DCT matrix (entry (k, j)
+// = sqrt(2/n) cos(k (2j+1) pi / (2n)), row 0 divided by sqrt 2) and forms its
+// alignment q_j^T Re(Gram) q_j in fp64; the columns are ranked by descending
+// alignment (ties to the lower column) and the first r written to U.
+constexpr int DCT_MAXN = 256;
+
+__global__ void __launch_bounds__(DCT_MAXN) dct_select_kernel(const EigJob* jobs) {
+  const EigJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  __shared__ double score[DCT_MAXN];
+  __shared__ int col_of_rank[DCT_MAXN];
+  const int j = threadIdx.x;
+  const double2* G = (const double2*)J.gram;
+  if (j < n) {
+    double q[DCT_MAXN];
+    const double theta = (2.0 * j + 1.0) * M_PI / (2.0 * n);
+    for (int k = 0; k < n; ++k) q[k] = sqrt((k == 0 ? 1.0 : 2.0) / n) * cos(k * theta);
+    double sc = 0;
+    for (int a = 0; a < n; ++a) {
+      double t = 0;
+      for (int b = 0; b < n; ++b) t += G[(int64_t)a * n + b].x * q[b];
+      sc += q[a] * t;
+    }
+    score[j] = sc;
+  }
+  __syncthreads();
+  if (j < n) {
+    const double sj = score[j];
+    int rank = 0;
+    for (int i = 0; i < n; ++i) rank += (score[i] > sj) || (score[i] == sj && i < j);
+    col_of_rank[rank] = j;
+    J.evals[rank] = sj;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * J.r; e += blockDim.x) {
+    const int row = e / J.r, c = e - row * J.r;
+    const int col = col_of_rank[c];
+    const double v = sqrt((row == 0 ? 1.0 : 2.0) / n) * cos(row * (2.0 * col + 1.0) * M_PI / (2.0 * n));
+    ((float2*)J.U)[e] = make_float2((float)v, 0.f);
+  }
+}
+
 }  // namespace
+
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
+  if (njobs <= 0) return cudaSuccess;
+  for (int j = 0; j < njobs; ++j)
+    if (jobs_host[j].n > DCT_MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  dct_select_kernel<<<njobs, DCT_MAXN, 0, s>>>(jobs_dev);
+  return cudaGetLastError();
+}
 
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);

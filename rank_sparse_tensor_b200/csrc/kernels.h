@@ -44,6 +44,9 @@ struct EigJob {
 };
 size_t eig_work_doubles(int n);
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
+// DCT basis instead of eigenvectors: U = the r columns of the orthonormal DCT
+// matrix most aligned with the Gram (evals: the alignments, descending).
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
 
 // ---- step_generic.cu: CUDA-core path of the step
 // L (optional, fp32 like the chain buffers): Adam on G[Omega] - L[Omega].
