@@ -92,6 +92,18 @@ typedef struct {
   int sm_budget;          /* 0 (default): the stream kernels spread over every SM; n > 0: over at
                              most n SMs, so that several tensors stepped on separate streams run
                              side by side (tensor-core path; results do not change) */
+  int order;              /* decomposition order, a free parameter of the method [S2]:
+                             0 (default) sparse part first, the low-rank part on the residual;
+                             1 low-rank part first (the ablated order): U_n from the Gram of G
+                             itself, Omega = top-k of E = G - L (L = G x_n U_n U_n^H, E in fp32),
+                             each step's sparse values E at Omega with L from that step's core.
+                             Order 1 runs on the CUDA-core path. */
+  int basis;              /* factors at a refresh: 0 (default) HOSVD, the leading eigenvectors
+                             of each mode-n Gram [S2]; 1 the r_n columns q_j of the orthonormal
+                             DCT matrix (sqrt(2/n) cos(k (2j+1) pi / 2n), row 0 / sqrt 2) with
+                             the largest alignment q_j^T Gram q_j, ties to the lower column (the
+                             dynamic column selection of the Trion / DCT-AdamW page); no
+                             eigensolver runs */
 } tgd_options;
 
 /* Fills `opt` with the defaults listed above. */

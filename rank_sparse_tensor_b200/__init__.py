@@ -54,7 +54,7 @@ class TensorGRaD:
                  grad_dtype: str = "c64", weight_dtype: Optional[str] = None,
                  omega_mode: int = 0, seed: int = 0, sparse_scale: float = 1.0,
                  complex_adam: int = 0, moments_on_refresh: int = 0, auto_refresh: int = 1,
-                 path: str = "auto", sm_budget: int = 0):
+                 path: str = "auto", sm_budget: int = 0, order: int = 0, basis: int = 0):
         weight_dtype = weight_dtype or grad_dtype
         self.shape = tuple(int(s) for s in shape)
         self.ranks = tuple(int(r) for r in ranks)
@@ -66,6 +66,8 @@ class TensorGRaD:
         opt.complex_adam, opt.moments_on_refresh = complex_adam, moments_on_refresh
         opt.auto_refresh, opt.path = auto_refresh, native.PATHS[path]
         opt.sm_budget = sm_budget
+        opt.order = order
+        opt.basis = basis
         sh = (C.c_int64 * len(self.shape))(*self.shape)
         rk = (C.c_int64 * len(self.ranks))(*self.ranks)
         h = C.c_void_p()

@@ -58,6 +58,7 @@ struct tgd_ctx {
   float* bufA = nullptr;
   float* bufB = nullptr;
   float* sp_upd = nullptr;
+  float* core_buf = nullptr;  // low-rank-first order: the core kept across the L rebuild
   // tensor-core path
   TcPlan tc;
   // errors
@@ -216,7 +217,152 @@ tgd_status rebuild_derived(tgd_ctx* h, cudaStream_t s) {
   return TGD_OK;
 }
 
+// ------------------------------------------------ low-rank-first order
+// The decomposition order reversed (the method's free parameter "decomposition
+// order" in the Pith review; sparse-first is the chosen order): the low-rank
+// part of the whole gradient comes first and Omega is selected on what it
+// leaves. CUDA-core kernels only.
+
+float* other_buf(tgd_ctx* h, const float* c) { return c == h->bufA ? h->bufB : h->bufA; }
+
+// C = G x_n U_n^H over the projected modes (last mode first), read from the
+// storage-typed gradient without a mask; *out is the buffer holding C (G
+// itself, copied to fp32, when no mode is projected). dims follows the shape.
+tgd_status project_all(tgd_ctx* h, const void* g, int64_t* dims, float** out, cudaStream_t s) {
+  float* cur = nullptr;
+  for (int n = h->d - 1; n >= 0; --n) {
+    if (!mode_active(h, n)) continue;
+    int64_t A = 1, B = 1;
+    for (int q = 0; q < n; ++q) A *= dims[q];
+    for (int q = n + 1; q < h->d; ++q) B *= dims[q];
+    float* o = other_buf(h, cur);
+    TIMED(h, s, "mode_product");
+    if (cur == nullptr)
+      TGD_CUDA(h, mode_product(g, h->gdt, nullptr, h->cplx, A, dims[n], B, h->P[n], h->r[n], o, s));
+    else
+      TGD_CUDA(h, mode_product(cur, -1, nullptr, h->cplx, A, dims[n], B, h->P[n], h->r[n], o, s));
+    cur = o;
+    dims[n] = h->r[n];
+  }
+  if (cur == nullptr) {
+    TIMED(h, s, "masked_copy");
+    TGD_CUDA(h, masked_copy(g, h->gdt, nullptr, h->N, h->bufA, s));
+    cur = h->bufA;
+  }
+  *out = cur;
+  return TGD_OK;
+}
+
+// X x_n U_n over the projected modes, from src (never written); *out holds the
+// result (src itself when no mode is projected).
+tgd_status expand_all(tgd_ctx* h, float* src, int64_t* dims, float** out, cudaStream_t s) {
+  float* cur = src;
+  for (int n = 0; n < h->d; ++n) {
+    if (!mode_active(h, n)) continue;
+    int64_t A = 1, B = 1;
+    for (int q = 0; q < n; ++q) A *= dims[q];
+    for (int q = n + 1; q < h->d; ++q) B *= dims[q];
+    float* o = other_buf(h, cur);
+    TIMED(h, s, "mode_product");
+    TGD_CUDA(h, mode_product(cur, -1, nullptr, h->cplx, A, dims[n], B, h->E[n], h->I[n], o, s));
+    cur = o;
+    dims[n] = h->I[n];
+  }
+  *out = cur;
+  return TGD_OK;
+}
+
+// Refresh: U_n from the Grams of G itself, L = G x_n U_n U_n^H, Omega = top-k
+// (or the random draw) of E = G - L in fp32; Omega's values are E there.
+tgd_status do_refresh_lowrank_first(tgd_ctx* h, const void* g, cudaStream_t s) {
+  h->jobs.clear();
+  for (int n = 0; n < h->d; ++n) {
+    if (!mode_active(h, n)) continue;
+    TIMED(h, s, "mode_gram");
+    TGD_CUDA(h, mode_gram(g, h->gdt, nullptr, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s));
+    EigJob j;
+    j.gram = h->gram[n];
+    j.work = h->eig_work[n];
+    j.U = h->U[n];
+    j.evals = h->evals[n];
+    j.n = (int)h->I[n];
+    j.r = (int)h->r[n];
+    h->jobs.push_back(j);
+  }
+  {
+    TIMED(h, s, "eigh");
+    TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+  }
+  for (int n = 0; n < h->d; ++n)
+    if (mode_active(h, n)) TGD_CUDA(h, coef_matrices(h->U[n], h->I[n], h->r[n], h->cplx, h->P[n], h->E[n], s));
+  int64_t dims[TGD_MAX_NDIM];
+  for (int n = 0; n < h->d; ++n) dims[n] = h->I[n];
+  float *C = nullptr, *L = nullptr;
+  tgd_status st = project_all(h, g, dims, &C, s);
+  if (st != TGD_OK) return st;
+  st = expand_all(h, C, dims, &L, s);
+  if (st != TGD_OK) return st;
+  TGD_CUDA(h, residual_in_place(g, h->gdt, L, h->N, s));
+  const int edt = h->cplx ? TGD_C64 : TGD_R32;
+  if (h->k > 0) {
+    KTimer kt(h, s, "select");
+    if (h->opt.omega_mode == 0)
+      TGD_CUDA(h, select_topk(L, edt, h->N, h->k, h->omega, h->omega_val, h->sel_ws, s));
+    else
+      TGD_CUDA(h, select_random(h->opt.seed, (uint64_t)h->refreshes, L, edt, h->N, h->k, h->omega,
+                                h->omega_val, h->sel_ws, s));
+  }
+  st = rebuild_derived(h, s);
+  if (st != TGD_OK) return st;
+  if (h->opt.moments_on_refresh == 1) {
+    TGD_CUDA(h, cudaMemsetAsync(h->core_m, 0, sizeof(float) * h->ncore * h->mc, s));
+    TGD_CUDA(h, cudaMemsetAsync(h->core_v, 0, sizeof(float) * h->ncore * h->vc, s));
+    TGD_CUDA(h, cudaMemsetAsync(h->sp_m, 0, sizeof(float) * h->k * h->mc, s));
+    TGD_CUDA(h, cudaMemsetAsync(h->sp_v, 0, sizeof(float) * h->k * h->vc, s));
+  }
+  h->has_subspace = true;
+  h->refreshes += 1;
+  return TGD_OK;
+}
+
+// Step: C = G x_n U_n^H (the whole gradient), L = C x_n U_n from the pre-Adam
+// core, sparse Adam on E[Omega] = G[Omega] - L[Omega], core Adam, Delta =
+// C~ x_n U_n with lambda S~ scattered in, the AdamW weight update.
+tgd_status step_lowrank_first(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
+  AdamConst asp = adam_const(h, h->opt.sparse_scale);
+  AdamConst acore = adam_const(h, 1.0);
+  int64_t dims[TGD_MAX_NDIM], ldims[TGD_MAX_NDIM];
+  for (int n = 0; n < h->d; ++n) dims[n] = h->I[n];
+  float *C = nullptr, *L = nullptr, *D = nullptr;
+  tgd_status st = project_all(h, g, dims, &C, s);
+  if (st != TGD_OK) return st;
+  TGD_CUDA(h, cudaMemcpyAsync(h->core_buf, C, sizeof(float) * h->ncore * h->mc,
+                              cudaMemcpyDeviceToDevice, s));
+  for (int n = 0; n < h->d; ++n) ldims[n] = dims[n];
+  st = expand_all(h, C, ldims, &L, s);
+  if (st != TGD_OK) return st;
+  {
+    TIMED(h, s, "sparse_adam");
+    TGD_CUDA(h, sparse_adam(g, h->gdt, h->omega, h->k, h->sp_m, h->sp_v, asp, h->sp_upd, s, L));
+  }
+  {
+    TIMED(h, s, "core_adam");
+    TGD_CUDA(h, core_adam(h->core_buf, h->ncore, h->core_m, h->core_v, acore, s));
+  }
+  st = expand_all(h, h->core_buf, dims, &D, s);
+  if (st != TGD_OK) return st;
+  {
+    TIMED(h, s, "scatter_add");
+    TGD_CUDA(h, scatter_add(D, h->cplx, h->omega, h->k, h->sp_upd, s));
+  }
+  float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
+  TIMED(h, s, "weight_update");
+  TGD_CUDA(h, weight_update(w, h->wdt, D, h->N, decay, h->lr, s));
+  return TGD_OK;
+}
+
 tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
+  if (h->opt.order == 1) return do_refresh_lowrank_first(h, g, s);
   if (h->k > 0) {
     KTimer kt(h, s, "select");
     if (h->opt.omega_mode == 0)
@@ -230,7 +376,7 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
   for (int n = 0; n < h->d; ++n) {
     if (!mode_active(h, n)) continue;
     TIMED(h, s, "mode_gram");
-    TGD_CUDA(h, mode_gram(g, h->gdt, h->bits, h->d, h->I, n, h->gram_part, h->gram[n], s));
+    TGD_CUDA(h, mode_gram(g, h->gdt, h->bits, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s));
     EigJob j;
     j.gram = h->gram[n];
     j.work = h->eig_work[n];
@@ -240,7 +386,10 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
   }
-  {
+  if (h->opt.basis == 1) {
+    TIMED(h, s, "dct_select");
+    TGD_CUDA(h, batched_dct_select(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+  } else {
     TIMED(h, s, "eigh");
     TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
   }
@@ -347,6 +496,8 @@ void tgd_default_options(tgd_options* opt) {
   opt->auto_refresh = 1;
   opt->path = TGD_PATH_AUTO;
   opt->sm_budget = 0;
+  opt->order = 0;
+  opt->basis = 0;
 }
 
 tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int64_t* ranks,
@@ -372,8 +523,11 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (opt) o = *opt;
   if (o.omega_mode < 0 || o.omega_mode > 1 || o.complex_adam < 0 || o.complex_adam > 1 ||
       o.moments_on_refresh < 0 || o.moments_on_refresh > 1 || o.path < 0 || o.path > 2 ||
-      o.sm_budget < 0 || !std::isfinite(o.sparse_scale))
+      o.sm_budget < 0 || !std::isfinite(o.sparse_scale) || o.order < 0 || o.order > 1 ||
+      o.basis < 0 || o.basis > 1)
     return fail(nullptr, TGD_ERR_INVALID_ARG, "bad option value");
+  if (o.order == 1 && o.path == TGD_PATH_TCGEN05)
+    return fail(nullptr, TGD_ERR_UNSUPPORTED, "the low-rank-first order runs on the CUDA-core path");
   int64_t N = 1, ncore = 1;
   for (int n = 0; n < ndim; ++n) {
     if (shape[n] < 1 || ranks[n] < 1 || ranks[n] > shape[n])
@@ -415,7 +569,8 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
     return fail(nullptr, TGD_ERR_UNSUPPORTED, "tensor-core path: needs complex fp16 gradients, d >= 3, "
                                               "a power-of-two I_{d-1} <= 128, I_d <= 120 and ranks below the modes");
   }
-  h->path = (o.path == TGD_PATH_GENERIC || !tc_ok) ? TGD_PATH_GENERIC : TGD_PATH_TCGEN05;
+  h->path = (o.path == TGD_PATH_GENERIC || !tc_ok || o.order == 1) ? TGD_PATH_GENERIC
+                                                                    : TGD_PATH_TCGEN05;
   cudaError_t ce = cudaGetDevice(&h->device);
   if (ce != cudaSuccess) {
     delete h;
@@ -452,6 +607,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
     ok &= dalloc_t(h, &h->bufA, (size_t)N * h->mc);
     ok &= dalloc_t(h, &h->bufB, (size_t)N * h->mc);
     ok &= dalloc_t(h, &h->sp_upd, std::max<int64_t>(h->k, 1) * h->mc);
+    if (o.order == 1) ok &= dalloc_t(h, &h->core_buf, ncore * h->mc);
   }
   if (ok && h->path == TGD_PATH_TCGEN05) {
     auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
@@ -507,7 +663,7 @@ tgd_status tgd_step(tgd_handle h, const void* grad, void* weight, void* stream) 
   if (!h->has_subspace) return fail(h, TGD_ERR_STATE, "no refresh has run: call tgd_refresh first");
   tgd_status st;
   if (h->path == TGD_PATH_GENERIC) {
-    st = step_generic(h, grad, weight, s);
+    st = h->opt.order == 1 ? step_lowrank_first(h, grad, weight, s) : step_generic(h, grad, weight, s);
   } else {
     AdamConst asp = adam_const(h, h->opt.sparse_scale);
     AdamConst acore = adam_const(h, 1.0);

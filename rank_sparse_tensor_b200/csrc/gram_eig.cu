@@ -24,8 +24,11 @@
 // r_n eigenvectors, each scaled by a unit phase that makes its largest-
 // magnitude entry (ties to the lowest row) real and positive.
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace tgd {
 namespace {
@@ -280,6 +283,241 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
   }
 }
 
+// ------------------------------------------------ tensor-core Gram (I_n <= 64)
+// The Gram as one tcgen05 GEMM per chunk of 32 unfolding columns. A 128-row
+// K-major tile holds, for each split part, the rows x_i (rows 0..I-1) and
+// J x_i (rows I..2I-1), where J maps each (re, im) pair of a column to
+// (-im, re); the rest are zero. With K = (column, re/im), the product of the
+// tile with its first N = 2I rows gives D[i][j] = Re sum_c x_ic conj(x_jc) and
+// D[i][I + j] = Im sum_c x_ic conj(x_jc). Each fp32 value is split into three
+// bf16 parts h + m + l (each the bf16 rounding of what the earlier parts
+// leave), and the six products hh, hm, mh, hl, lh, mm are accumulated in
+// fp32 in TMEM, which keeps about fp32 accuracy; the products of the two
+// smallest parts (ml, lm, ll, below 2^-24 of the result) are dropped.
+constexpr int TG_THREADS = 128;
+constexpr int TG_COLS = 32;                 // complex columns per chunk: K = 64 bf16 values
+constexpr uint32_t TG_LBO = 2048;           // 128 rows x 16 B between K core matrices
+constexpr uint32_t TG_TILE = 8 * TG_LBO;    // 128 rows x 64 K values of bf16
+constexpr uint64_t TG_WAIT_NS = 2000000000ull;
+
+struct TcGramArgs {
+  const void* g;
+  const uint32_t* bits;
+  int64_t I, B, ncol, cols_per_split;
+  int N;     // MMA N: 2I rounded up to 16
+  int R;     // rows per thread pass: 32 (I <= 32) or 64
+  float* partial;  // [split][I][I] complex, interleaved
+  int* err;
+};
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ float bf16_val(uint16_t b) {
+  return __uint_as_float((uint32_t)b << 16);
+}
+// x = h + m + l (bf16 parts, each the rounding of what the earlier leave)
+__device__ __forceinline__ void split3(float x, uint16_t& h, uint16_t& m, uint16_t& l) {
+  h = bf16_bits(x);
+  const float r1 = x - bf16_val(h);
+  m = bf16_bits(r1);
+  l = bf16_bits(r1 - bf16_val(m));
+}
+
+template <int DT>
+__global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* tiles = smem;                                      // [stage][part] tiles
+  int64_t* colbase = (int64_t*)(smem + 6 * TG_TILE);          // [2][TG_COLS]
+  uint64_t* done = (uint64_t*)(colbase + 2 * TG_COLS);        // [2] MMAs of a stage done
+  uint32_t* tslot = (uint32_t*)(done + 2);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int Q = TG_THREADS / p.R, cpt = TG_COLS / Q;          // column blocks, columns per thread
+  const int i = tid % p.R, q = tid / p.R;
+  const bool row_ok = i < p.I;
+  const int64_t c_begin = (int64_t)blockIdx.y * p.cols_per_split;
+  const int64_t c_end = c_begin + p.cols_per_split < p.ncol ? c_begin + p.cols_per_split : p.ncol;
+  const int nch = (int)((c_end - c_begin + TG_COLS - 1) / TG_COLS);
+  const int64_t IB = p.I * p.B;
+  // zero every tile once: rows 2I..127 stay zero, rows 0..2I-1 are rewritten per chunk
+  for (uint32_t o = tid * 16; o < 6 * TG_TILE; o += TG_THREADS * 16)
+    *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    s_abort = 0;
+    ptx::mbar_init(&done[0], 1);
+    ptx::mbar_init(&done[1], 1);
+    ptx::fence_mbar_init();
+  }
+  auto set_colbase = [&](int slot, int64_t c0) {
+    if (tid < TG_COLS) {
+      const int64_t c = c0 + tid;
+      int64_t off = -1;
+      if (c < c_end) {
+        const int64_t a = c / p.B;
+        off = a * IB + (c - a * p.B);
+      }
+      colbase[slot * TG_COLS + tid] = off;
+    }
+  };
+  set_colbase(0, c_begin);
+  __syncthreads();
+  if (warp == 0) ptx::tmem_alloc(tslot, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t dt_base = *tslot;
+  const uint32_t idesc = ptx::idesc_f16(1, 128, p.N);
+  float2 v[16];
+  auto load = [&](int slot) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      float2 x = make_float2(0.f, 0.f);
+      if (u < cpt && row_ok) {
+        const int64_t cb = colbase[slot * TG_COLS + q * cpt + u];
+        if (cb >= 0) {
+          const int64_t idx = cb + (int64_t)i * p.B;
+          if (!(p.bits && mask_bit(p.bits, idx))) x = load_elem<DT>(p.g, idx);
+        }
+      }
+      v[u] = x;
+    }
+  };
+  // this thread's columns of the chunk -> rows i and I + i of the three tiles of stage s
+  auto store = [&](int s) {
+    if (!row_ok) return;
+#pragma unroll
+    for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
+      if (gq * 4 >= cpt) break;
+      uint32_t xr[3][4], jr[3][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 x = v[gq * 4 + u];
+        uint16_t rh, rm, rl, ih, im, il;
+        split3(x.x, rh, rm, rl);
+        split3(x.y, ih, im, il);
+        // x row: (re, im); J x row: (-im, re); the low half holds the even K
+        xr[0][u] = (uint32_t)rh | ((uint32_t)ih << 16);
+        xr[1][u] = (uint32_t)rm | ((uint32_t)im << 16);
+        xr[2][u] = (uint32_t)rl | ((uint32_t)il << 16);
+        jr[0][u] = (uint32_t)(ih ^ 0x8000u) | ((uint32_t)rh << 16);
+        jr[1][u] = (uint32_t)(im ^ 0x8000u) | ((uint32_t)rm << 16);
+        jr[2][u] = (uint32_t)(il ^ 0x8000u) | ((uint32_t)rl << 16);
+      }
+      const uint32_t kg = (uint32_t)(q * cpt / 4 + gq);
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        uint8_t* t = tiles + (size_t)(s * 3 + part) * TG_TILE + kg * TG_LBO;
+        *(uint4*)(t + (uint32_t)i * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
+        *(uint4*)(t + (uint32_t)(p.I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
+      }
+    }
+  };
+  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
+  load(0);
+  for (int kc = 0; kc < nch; ++kc) {
+    const int s = kc & 1;
+    if (kc >= 2) {
+      if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
+        atomicOr(p.err, DEV_ERR_TIMEOUT);
+        s_abort = 1;
+      }
+      __syncthreads();
+      if (s_abort) break;
+      waited[s]++;
+      ptx::tc_fence_after();
+    }
+    store(s);
+    set_colbase((kc + 1) & 1, c_begin + (int64_t)(kc + 1) * TG_COLS);
+    ptx::fence_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (kc + 1 < nch) load((kc + 1) & 1);
+    if (tid == 0) {
+      const uint32_t base = ptx::smem_u32(tiles + (size_t)s * 3 * TG_TILE);
+      // (A part, B part): hh, hm, mh, hl, lh, mm
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int pr = 0; pr < 6; ++pr) {
+          const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
+          const uint32_t ka = base + pa * TG_TILE + kk * 2 * TG_LBO;
+          const uint32_t kb = base + pb * TG_TILE + kk * 2 * TG_LBO;
+          ptx::mma_f16(dt_base, ptx::sdesc(ka, TG_LBO, 128), ptx::sdesc(kb, TG_LBO, 128), idesc,
+                       (kc > 0 || kk > 0 || pr > 0) ? 1u : 0u);
+        }
+      ptx::mma_commit(&done[s]);
+      issued[s]++;
+    }
+  }
+  __syncthreads();
+  bool ok = !s_abort;
+  if (ok && nch > 0) {
+    const int s = (nch - 1) & 1;
+    if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    ok = !s_abort;
+    ptx::tc_fence_after();
+  }
+  if (ok) {
+    // lane = row of D; columns j < I the real part, I <= j < 2I the imaginary part
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int row = tid;
+    float* out = p.partial + (size_t)blockIdx.y * p.I * p.I * 2;
+    for (int c0 = 0; c0 < p.N; c0 += 16) {
+      float y[16];
+      ptx::tmem_ld16(dt_base + lane_base + c0, y);
+      if (row < p.I) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = c0 + u;
+          if (j < p.I)
+            out[((int64_t)row * p.I + j) * 2] = nch > 0 ? y[u] : 0.f;
+          else if (j < 2 * p.I)
+            out[((int64_t)row * p.I + (j - p.I)) * 2 + 1] = nch > 0 ? y[u] : 0.f;
+        }
+      }
+    }
+  } else if (tid == 0) {
+    // bounded waits for MMAs still in flight
+    for (int st = 0; st < 2; ++st)
+      if (issued[st] > waited[st]) ptx::mbar_wait(&done[st], (issued[st] - 1) & 1u, TG_WAIT_NS / 4);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(dt_base, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+}
+
+size_t tg_smem_bytes() { return 6 * (size_t)TG_TILE + 2 * TG_COLS * 8 + 2 * 8 + 16; }
+
+struct TcGramGeom {
+  int64_t I, B, ncol, cols_per_split;
+  int nsplit, N, R;
+};
+
+TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
+  TcGramGeom g;
+  g.B = 1;
+  int64_t A = 1;
+  for (int q = 0; q < n; ++q) A *= dims[q];
+  for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
+  g.I = dims[n];
+  g.ncol = A * g.B;
+  g.N = (int)((2 * g.I + 15) / 16 * 16);
+  g.R = g.I <= 32 ? 32 : 64;
+  // two CTAs per SM, a few waves; at least four chunks per split; partials under 32 MB
+  int64_t ns = std::min<int64_t>(148 * 2 * 3, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
+  ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
+  g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), TG_COLS) * TG_COLS;
+  g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
+  return g;
+}
+
 // ------------------------------------------------------------- eigensolver
 __device__ __forceinline__ double2 zmul(double2 a, double2 b) {
   return make_double2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
@@ -451,15 +689,339 @@ __global__ void __launch_bounds__(ET) eig_kernel(const EigJob* jobs) {
   }
 }
 
+// Block form of the same parallel Jacobi for n <= 128: A is Hermitian, so only
+// its upper triangle is kept (packed, in shared memory: 132 KB at n = 128).
+// In a round the n/2 rotations are disjoint; the 2 x 2 block of A at the rows
+// of pair k1 and the columns of pair k2 becomes J1^H B J2 (the column rotation
+// of k2, then the row rotation of k1, as in eig_kernel), and each unordered
+// block (k1 <= k2) is one thread's work, so every stored entry has one writer
+// per round and a round needs two barriers. V is kept transposed (a row per
+// eigenvector): in shared memory for n <= 64, in the job's scratch otherwise.
+constexpr int EB_MAXN = 128;
+
+__device__ __forceinline__ int tri_idx(int i, int j, int n) {  // i <= j
+  return i * n - (i * (i - 1)) / 2 + (j - i);
+}
+
+__global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
+  const EigJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  if (n > EB_MAXN) return;
+  extern __shared__ double2 dyn[];
+  __shared__ int rp[EB_MAXN / 2], rq[EB_MAXN / 2], rrot[EB_MAXN / 2];
+  __shared__ double rcs[EB_MAXN / 2], rsn[EB_MAXN / 2];
+  __shared__ double2 rph[EB_MAXN / 2];
+  __shared__ uint8_t bk1[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2], bk2[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2];
+  __shared__ double red[ET / 32];
+  __shared__ double ev[EB_MAXN];
+  __shared__ int col_of_rank[EB_MAXN];
+  const int ntri = n * (n + 1) / 2;
+  double2* T = dyn;  // packed upper triangle of A
+  double2* Vt = n <= 64 ? dyn + ntri : (double2*)J.work;
+  const double2* G = (const double2*)J.gram;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e - i * n;
+    if (i <= j) T[tri_idx(i, j, n)] = G[e];
+    Vt[e] = make_double2(i == j ? 1.0 : 0.0, 0.0);
+  }
+  const int m = n + (n & 1);
+  const int npairs = m / 2;
+  const int nblk = npairs * (npairs + 1) / 2;
+  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+    int k1 = 0, r = b;
+    while (r >= npairs - k1) {
+      r -= npairs - k1;
+      ++k1;
+    }
+    bk1[b] = (uint8_t)k1;
+    bk2[b] = (uint8_t)(k1 + r);
+  }
+  __syncthreads();
+  auto get = [&](int i, int j) -> double2 {
+    if (i <= j) return T[tri_idx(i, j, n)];
+    const double2 v = T[tri_idx(j, i, n)];
+    return make_double2(v.x, -v.y);
+  };
+  auto put = [&](int i, int j, double2 v) {
+    if (i <= j)
+      T[tri_idx(i, j, n)] = v;
+    else
+      T[tri_idx(j, i, n)] = make_double2(v.x, -v.y);
+  };
+  double part = 0;
+  for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
+    int i = 0, r = e;
+    while (r >= n - i) {
+      r -= n - i;
+      ++i;
+    }
+    part += (r == 0 ? 1.0 : 2.0) * zabs2(T[e]);  // r == 0: the diagonal entry of row i
+  }
+  const double fro = block_sum(part, red);
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    double off_part = 0;
+    for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
+      int i = 0, r = e;
+      while (r >= n - i) {
+        r -= n - i;
+        ++i;
+      }
+      if (r > 0) off_part += zabs2(T[e]);
+    }
+    const double off = block_sum(off_part, red);
+    if (off <= 1e-24 * fro || off == 0.0) break;
+    for (int round = 0; round < m - 1; ++round) {
+      for (int k = threadIdx.x; k < npairs; k += blockDim.x) {
+        int p, q;
+        if (k == 0) {
+          p = round;
+          q = m - 1;
+        } else {
+          p = (round + k) % (m - 1);
+          q = (round - k + (m - 1)) % (m - 1);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        rp[k] = p;
+        rq[k] = q;
+        rrot[k] = 0;
+        if (q < n) {
+          const double2 apq = get(p, q);
+          const double r = sqrt(zabs2(apq));
+          if (r > 0.0) {
+            const double app = get(p, p).x, aqq = get(q, q).x;
+            const double tau = (aqq - app) / (2.0 * r);
+            const double t = (tau >= 0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+            const double c = 1.0 / sqrt(1.0 + t * t);
+            rrot[k] = 1;
+            rcs[k] = c;
+            rsn[k] = t * c;
+            rph[k] = make_double2(apq.x / r, apq.y / r);
+          }
+        }
+      }
+      __syncthreads();
+      for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+        const int k1 = bk1[b], k2 = bk2[b];
+        const int p1 = rp[k1], q1 = rq[k1], p2 = rp[k2], q2 = rq[k2];
+        const bool rot1 = rrot[k1], rot2 = rrot[k2];
+        if (!rot1 && !rot2) continue;
+        const bool h1 = q1 < n, h2 = q2 < n;  // the dummy index of odd n is absent
+        double2 b00 = get(p1, p2), b01 = h2 ? get(p1, q2) : make_double2(0, 0);
+        double2 b10 = h1 ? get(q1, p2) : make_double2(0, 0);
+        double2 b11 = h1 && h2 ? get(q1, q2) : make_double2(0, 0);
+        if (rot2) {  // columns p2, q2: B <- B J2
+          const double c = rcs[k2], s = rsn[k2];
+          const double2 ec = make_double2(rph[k2].x, -rph[k2].y);
+          double2 xp = b00, xq = zmul(b01, ec);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b01 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b10;
+          xq = zmul(b11, ec);
+          b10 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (rot1) {  // rows p1, q1: B <- J1^H B
+          const double c = rcs[k1], s = rsn[k1];
+          const double2 e = rph[k1];
+          double2 xp = b00, xq = zmul(b10, e);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b10 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b01;
+          xq = zmul(b11, e);
+          b01 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (k1 == k2) {
+          // the diagonal block: the rotation zeroes (p, q); the diagonal is real
+          put(p1, p1, make_double2(b00.x, 0.0));
+          if (h1) {
+            put(p1, q1, make_double2(0.0, 0.0));
+            put(q1, q1, make_double2(b11.x, 0.0));
+          }
+        } else {
+          put(p1, p2, b00);
+          if (h2) put(p1, q2, b01);
+          if (h1) put(q1, p2, b10);
+          if (h1 && h2) put(q1, q2, b11);
+        }
+      }
+      // V <- V J on the rows of V^T (no other thread touches them this round)
+      for (int w = threadIdx.x; w < npairs * n; w += blockDim.x) {
+        const int k = w / n, i = w - k * n;
+        if (!rrot[k]) continue;
+        const int p = rp[k], q = rq[k];
+        const double c = rcs[k], s = rsn[k];
+        const double2 ec = make_double2(rph[k].x, -rph[k].y);
+        const double2 xp = Vt[p * n + i], xq = zmul(Vt[q * n + i], ec);
+        Vt[p * n + i] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+        Vt[q * n + i] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) ev[i] = T[tri_idx(i, i, n)].x;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const double li = ev[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += (ev[j] > li) || (ev[j] == li && j < i);
+    col_of_rank[rank] = i;
+    J.evals[rank] = li;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int rr = wid; rr < J.r; rr += nw) {
+    const int c = col_of_rank[rr];
+    double best = -1.0;
+    int bi = 0;
+    for (int row = lane; row < n; row += 32) {
+      const double mg = zabs2(Vt[c * n + row]);
+      if (mg > best) {
+        best = mg;
+        bi = row;
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    const double2 piv = Vt[c * n + bi];
+    const double pm = sqrt(zabs2(piv));
+    const double2 ph = pm > 0 ? make_double2(piv.x / pm, -piv.y / pm) : make_double2(1.0, 0.0);
+    for (int row = lane; row < n; row += 32) {
+      const double2 u = zmul(Vt[c * n + row], ph);
+      ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
+    }
+  }
+}
+
+// ------------------------------------------------------- DCT column selection
+// The dynamic column selection of the Trion / DCT-AdamW page as a factor
+// basis: thread j holds column q_j of the orthonormal DCT matrix (entry (k, j)
+// = sqrt(2/n) cos(k (2j+1) pi / (2n)), row 0 divided by sqrt 2) and forms its
+// alignment q_j^T Re(Gram) q_j in fp64; the columns are ranked by descending
+// alignment (ties to the lower column) and the first r written to U.
+constexpr int DCT_MAXN = 256;
+
+__global__ void __launch_bounds__(DCT_MAXN) dct_select_kernel(const EigJob* jobs) {
+  const EigJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  __shared__ double score[DCT_MAXN];
+  __shared__ int col_of_rank[DCT_MAXN];
+  const int j = threadIdx.x;
+  const double2* G = (const double2*)J.gram;
+  if (j < n) {
+    double q[DCT_MAXN];
+    const double theta = (2.0 * j + 1.0) * M_PI / (2.0 * n);
+    for (int k = 0; k < n; ++k) q[k] = sqrt((k == 0 ? 1.0 : 2.0) / n) * cos(k * theta);
+    double sc = 0;
+    for (int a = 0; a < n; ++a) {
+      double t = 0;
+      for (int b = 0; b < n; ++b) t += G[(int64_t)a * n + b].x * q[b];
+      sc += q[a] * t;
+    }
+    score[j] = sc;
+  }
+  __syncthreads();
+  if (j < n) {
+    const double sj = score[j];
+    int rank = 0;
+    for (int i = 0; i < n; ++i) rank += (score[i] > sj) || (score[i] == sj && i < j);
+    col_of_rank[rank] = j;
+    J.evals[rank] = sj;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * J.r; e += blockDim.x) {
+    const int row = e / J.r, c = e - row * J.r;
+    const int col = col_of_rank[c];
+    const double v = sqrt((row == 0 ? 1.0 : 2.0) / n) * cos(row * (2.0 * col + 1.0) * M_PI / (2.0 * n));
+    ((float2*)J.U)[e] = make_float2((float)v, 0.f);
+  }
+}
+
 }  // namespace
+
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
+  if (njobs <= 0) return cudaSuccess;
+  for (int j = 0; j < njobs; ++j)
+    if (jobs_host[j].n > DCT_MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  dct_select_kernel<<<njobs, DCT_MAXN, 0, s>>>(jobs_dev);
+  return cudaGetLastError();
+}
 
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);
-  return sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
+  size_t b = sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
+  if (g.I <= 64) {
+    TcGramGeom t = tc_gram_geom(nd, dims, n);
+    b = std::max(b, sizeof(float2) * (size_t)t.nsplit * t.I * t.I);
+  }
+  return b;
+}
+
+// Tensor-core Gram for I_n <= 64 (see gram_tc_kernel); the split partials are
+// summed by the same fixed-order fp64 reduction.
+cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
+                         int n, float* partial, double* gram, int* err, cudaStream_t s) {
+  const TcGramGeom t = tc_gram_geom(nd, dims, n);
+  TcGramArgs a;
+  a.g = g;
+  a.bits = bits;
+  a.I = t.I;
+  a.B = t.B;
+  a.ncol = t.ncol;
+  a.cols_per_split = t.cols_per_split;
+  a.N = t.N;
+  a.R = t.R;
+  a.partial = partial;
+  a.err = err;
+  const size_t smem = tg_smem_bytes();
+  const dim3 grid(1, t.nsplit);
+  cudaError_t e = cudaSuccess;
+  switch (dt) {
+    case TGD_R32:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R32><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_C64:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C64><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_C32H:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C32H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C32H><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    case TGD_R16:
+      e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R16><<<grid, TG_THREADS, smem, s>>>(a);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  GramGeom geo{};
+  geo.I = t.I;
+  geo.TI = 64;  // one tile: every cell is computed directly
+  geo.nsplit = t.nsplit;
+  const int64_t cells = t.I * t.I;
+  gram_reduce_kernel<<<(int)ceil_div(cells, RC), RC * RS, 0, s>>>((const float2*)partial, geo,
+                                                                   (double2*)gram);
+  return cudaGetLastError();
 }
 
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                      int n, float* partial, double* gram, cudaStream_t s) {
+                      int n, float* partial, double* gram, int* err, cudaStream_t s) {
+  if (dims[n] <= 64) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s);
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
   const size_t smem = gram_smem_bytes(geo);
@@ -489,6 +1051,26 @@ size_t eig_work_doubles(int n) { return n > 64 ? (size_t)4 * n * n : 0; }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
+  bool all_small = true;
+  size_t bsmem = 16;
+  for (int j = 0; j < njobs; ++j) {
+    const int n = jobs_host[j].n;
+    if (n > EB_MAXN || jobs_host[j].r > n) {
+      all_small = false;
+      break;
+    }
+    const size_t need = sizeof(double2) * ((size_t)n * (n + 1) / 2 + (n <= 64 ? (size_t)n * n : 0));
+    bsmem = std::max(bsmem, need);
+  }
+  if (all_small) {
+    cudaError_t e = cudaFuncSetAttribute(eig_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bsmem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    eig_block_kernel<<<njobs, ET, bsmem, s>>>(jobs_dev);
+    return cudaGetLastError();
+  }
   int smem_n = 0;
   for (int j = 0; j < njobs; ++j) {
     if (jobs_host[j].n > MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;

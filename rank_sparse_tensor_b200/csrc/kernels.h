@@ -30,8 +30,10 @@ cudaError_t build_tile_index(const int64_t* omega, int64_t k, int64_t tile_elems
 // Omega bitmask `bits`), accumulated in fp32 partials and summed in fp64
 // into gram (I_n x I_n complex, interleaved doubles).
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n);
+// Modes with I_n <= 64 run on the tensor cores; err is the device error word
+// a bounded wait sets when it gives up.
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                      int n, float* partial, double* gram, cudaStream_t s);
+                      int n, float* partial, double* gram, int* err, cudaStream_t s);
 
 struct EigJob {
   const double* gram;  // n x n complex (interleaved doubles)
@@ -42,10 +44,17 @@ struct EigJob {
 };
 size_t eig_work_doubles(int n);
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
+// DCT basis instead of eigenvectors: U = the r columns of the orthonormal DCT
+// matrix most aligned with the Gram (evals: the alignments, descending).
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
 
 // ---- step_generic.cu: CUDA-core path of the step
+// L (optional, fp32 like the chain buffers): Adam on G[Omega] - L[Omega].
 cudaError_t sparse_adam(const void* g, int dt, const int64_t* omega, int64_t k, float* m,
-                        float* v, const AdamConst& a, float* upd, cudaStream_t s);
+                        float* v, const AdamConst& a, float* upd, cudaStream_t s,
+                        const float* L = nullptr);
+// L <- G - L over n elements (fp32; float2 for complex dtypes).
+cudaError_t residual_in_place(const void* g, int dt, float* L, int64_t n, cudaStream_t s);
 // Y = X x_n M: X (A, K, B), M (J x K) row-major complex or real, Y (A, J, B).
 // src_dt >= 0: X is the storage-typed gradient, masked by `bits`; src_dt < 0:
 // X is fp32 (float2 when cplx).

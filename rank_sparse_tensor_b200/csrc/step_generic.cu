@@ -27,13 +27,19 @@ int grid_for(int64_t n, int threads = 256) {
   return (int)(b < 1 ? 1 : (b > cap ? cap : b));
 }
 
+// Adam on the k values at Omega: G[Omega], or G[Omega] - L[Omega] when L (the
+// low-rank part, fp32) is given (the low-rank-first order).
 template <int DT>
-__global__ void sparse_adam_kernel(const void* g, const int64_t* omega, int64_t k, float* m,
-                                   float* v, AdamConst a, float* upd) {
+__global__ void sparse_adam_kernel(const void* g, const float* L, const int64_t* omega, int64_t k,
+                                   float* m, float* v, AdamConst a, float* upd) {
   const int mc = a.cplx ? 2 : 1, vc = (a.cplx && a.cmode == 1) ? 2 : 1;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < k;
        j += (int64_t)gridDim.x * blockDim.x) {
     float2 gv = load_elem<DT>(g, omega[j]);
+    if (L) {
+      const float2 l = a.cplx ? ((const float2*)L)[omega[j]] : make_float2(L[omega[j]], 0.f);
+      gv = make_float2(gv.x - l.x, gv.y - l.y);
+    }
     float mm[2], vv[2];
     for (int c = 0; c < mc; ++c) mm[c] = m[j * mc + c];
     for (int c = 0; c < vc; ++c) vv[c] = v[j * vc + c];
@@ -164,15 +170,83 @@ __global__ void __launch_bounds__(MT) mode_product_kernel(S src, int64_t A, int6
   }
 }
 
+// Y = X x_n M for coefficient matrices of at most SP_MAXMK entries (the modes
+// of FNO-sized tensors): one thread per column (a, b) of the unfolding reads
+// its K values (stride B: coalesced across threads when B > 1, from cache
+// when B == 1) once per block of SP_J outputs, M is broadcast from shared
+// memory and the outputs stay in registers. The sum over k runs in the same
+// order as in mode_product_kernel, so both give the same bits.
+constexpr int SP_T = 256, SP_J = 16, SP_MAXMK = 4096;
+
+template <class S, bool CPLX>
+__global__ void __launch_bounds__(SP_T) mode_product_small_kernel(S src, int64_t A, int64_t K,
+                                                                  int64_t B, const float* M,
+                                                                  int64_t J, float* Y) {
+  __shared__ float2 Ms[SP_MAXMK];
+  for (int64_t e = threadIdx.x; e < J * K; e += SP_T)
+    Ms[e] = CPLX ? ((const float2*)M)[e] : make_float2(M[e], 0.f);
+  __syncthreads();
+  const int64_t ncol = A * B;
+  for (int64_t c = (int64_t)blockIdx.x * SP_T + threadIdx.x; c < ncol;
+       c += (int64_t)gridDim.x * SP_T) {
+    const int64_t a = c / B, b = c - a * B;
+    const int64_t xb = a * K * B + b, yb = a * J * B + b;
+    for (int64_t j0 = 0; j0 < J; j0 += SP_J) {
+      float2 acc[SP_J];
+#pragma unroll
+      for (int u = 0; u < SP_J; ++u) acc[u] = make_float2(0.f, 0.f);
+      for (int64_t k = 0; k < K; ++k) {
+        const float2 x = src(xb + k * B);
+        const float2* mk = Ms + j0 * K + k;
+#pragma unroll
+        for (int u = 0; u < SP_J; ++u) {
+          if (j0 + u < J) {
+            const float2 m = mk[u * K];
+            if (CPLX)
+              acc[u] = cfma(m, x, acc[u]);
+            else
+              acc[u].x = __fmaf_rn(m.x, x.x, acc[u].x);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < SP_J; ++u) {
+        if (j0 + u < J) {
+          const int64_t o = yb + (j0 + u) * B;
+          if (CPLX)
+            ((float2*)Y)[o] = acc[u];
+          else
+            Y[o] = acc[u].x;
+        }
+      }
+    }
+  }
+}
+
 template <int DT>
 __global__ void masked_copy_kernel(const void* g, const uint32_t* bits, int64_t n, float* out) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    float2 v = mask_bit(bits, i) ? make_float2(0.f, 0.f) : load_elem<DT>(g, i);
+    float2 v = bits && mask_bit(bits, i) ? make_float2(0.f, 0.f) : load_elem<DT>(g, i);
     if (Dt<DT>::cplx)
       ((float2*)out)[i] = v;
     else
       out[i] = v.x;
+  }
+}
+
+// L <- G - L (fp32, in place): the residual after the low-rank part.
+template <int DT>
+__global__ void residual_kernel(const void* g, float* L, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float2 x = load_elem<DT>(g, i);
+    if (Dt<DT>::cplx) {
+      const float2 l = ((const float2*)L)[i];
+      ((float2*)L)[i] = make_float2(x.x - l.x, x.y - l.y);
+    } else {
+      L[i] = x.x - L[i];
+    }
   }
 }
 
@@ -223,25 +297,47 @@ __global__ void coef_kernel(const float2* U, int64_t I, int64_t r, bool cplx, fl
   }
 }
 
+// The small-matrix kernel when M fits its shared memory, else the tiled one.
+template <class S, bool CPLX>
+void launch_product(S src, int64_t A, int64_t K, int64_t B, const float* M, int64_t J, float* Y,
+                    cudaStream_t s, dim3 grid) {
+  if (J * K <= SP_MAXMK)
+    mode_product_small_kernel<S, CPLX><<<grid_for(A * B, SP_T), SP_T, 0, s>>>(src, A, K, B, M, J, Y);
+  else
+    mode_product_kernel<S, CPLX><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
+}
+
 template <int DT>
 cudaError_t launch_first(const void* X, const uint32_t* bits, int64_t A, int64_t K, int64_t B,
                          const float* M, int64_t J, float* Y, cudaStream_t s, dim3 grid) {
   Src<DT, Dt<DT>::cplx> src{X, bits};
-  mode_product_kernel<Src<DT, Dt<DT>::cplx>, Dt<DT>::cplx><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
+  launch_product<Src<DT, Dt<DT>::cplx>, Dt<DT>::cplx>(src, A, K, B, M, J, Y, s, grid);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t sparse_adam(const void* g, int dt, const int64_t* omega, int64_t k, float* m,
-                        float* v, const AdamConst& a, float* upd, cudaStream_t s) {
+                        float* v, const AdamConst& a, float* upd, cudaStream_t s, const float* L) {
   if (k <= 0) return cudaSuccess;
   int grid = grid_for(k);
   switch (dt) {
-    case TGD_R32: sparse_adam_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_C64: sparse_adam_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_C32H: sparse_adam_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
-    case TGD_R16: sparse_adam_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, omega, k, m, v, a, upd); break;
+    case TGD_R32: sparse_adam_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_C64: sparse_adam_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_C32H: sparse_adam_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    case TGD_R16: sparse_adam_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, L, omega, k, m, v, a, upd); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t residual_in_place(const void* g, int dt, float* L, int64_t n, cudaStream_t s) {
+  int grid = grid_for(n);
+  switch (dt) {
+    case TGD_R32: residual_kernel<TGD_R32><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_C64: residual_kernel<TGD_C64><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_C32H: residual_kernel<TGD_C32H><<<grid, 256, 0, s>>>(g, L, n); break;
+    case TGD_R16: residual_kernel<TGD_R16><<<grid, 256, 0, s>>>(g, L, n); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -259,13 +355,10 @@ cudaError_t mode_product(const void* X, int src_dt, const uint32_t* bits, bool c
     default:
       break;
   }
-  if (cplx) {
-    Src<-1, true> src{X, nullptr};
-    mode_product_kernel<Src<-1, true>, true><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
-  } else {
-    Src<-1, false> src{X, nullptr};
-    mode_product_kernel<Src<-1, false>, false><<<grid, MT, 0, s>>>(src, A, K, B, M, J, Y);
-  }
+  if (cplx)
+    launch_product<Src<-1, true>, true>(Src<-1, true>{X, nullptr}, A, K, B, M, J, Y, s, grid);
+  else
+    launch_product<Src<-1, false>, false>(Src<-1, false>{X, nullptr}, A, K, B, M, J, Y, s, grid);
   return cudaGetLastError();
 }
 

@@ -91,7 +91,27 @@ def test_default_options(tgd):
     o = tgd.Options()
     tgd.lib().tgd_default_options(C.byref(o))
     assert (o.omega_mode, o.sparse_scale, o.complex_adam, o.moments_on_refresh, o.auto_refresh,
-            o.path, o.sm_budget) == (0, 1.0, 0, 0, 1, 0, 0)
+            o.path, o.sm_budget, o.order, o.basis) == (0, 1.0, 0, 0, 1, 0, 0, 0, 0)
+
+
+@pytest.mark.parametrize("order,path,status", [(2, 0, 1), (-1, 0, 1), (1, 2, 2)])
+def test_bad_decomposition_order(tgd, order, path, status):
+    """Orders other than 0 and 1 are invalid; the low-rank-first order on
+    the forced tensor-core path is unsupported. Both fail before the device."""
+    o = tgd.Options()
+    tgd.lib().tgd_default_options(C.byref(o))
+    o.order, o.path = order, path
+    st, h = _create(tgd, (4, 8, 16), (2, 4, 8), opt=C.byref(o))
+    assert st == status and not h.value
+
+
+@pytest.mark.parametrize("basis", [-1, 2])
+def test_bad_factor_basis(tgd, basis):
+    o = tgd.Options()
+    tgd.lib().tgd_default_options(C.byref(o))
+    o.basis = basis
+    st, h = _create(tgd, (4, 8, 16), (2, 4, 8), opt=C.byref(o))
+    assert st == 1 and not h.value
 
 
 def test_create_without_device_fails_cleanly(tgd):
