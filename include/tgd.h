@@ -77,8 +77,11 @@ typedef enum {
   TGD_R16 = 3    /* real fp16 */
 } tgd_dtype;
 
-/* Kernel path. AUTO picks TCGEN05 for complex fp16 gradients whose trailing
- * modes fit its tiles, and GENERIC otherwise. */
+/* Kernel path. AUTO picks TCGEN05 where the tensor-core kernels apply, GENERIC
+ * (CUDA cores) otherwise. TCGEN05 covers complex fp16 gradients whose trailing
+ * modes fit its streaming tiles (fp16 or fp32 weights), and fp32 gradients
+ * with fp32 weights (real or complex) whose projected modes have at most 256
+ * entries. */
 typedef enum { TGD_PATH_AUTO = 0, TGD_PATH_GENERIC = 1, TGD_PATH_TCGEN05 = 2 } tgd_path;
 
 typedef struct {
@@ -104,6 +107,15 @@ typedef struct {
                              the largest alignment q_j^T Gram q_j, ties to the lower column (the
                              dynamic column selection of the Trion / DCT-AdamW page); no
                              eigensolver runs */
+  int wait_limit_ms;      /* limit of each bounded wait inside the projection kernel of the
+                             tensor-core path, in milliseconds; 0 (default) = 2000. A wait that
+                             runs out makes the kernel stop its work and return, and the next
+                             synchronising call (tgd_sync, tgd_step_host) reports
+                             TGD_ERR_TIMEOUT */
+  int test_stall;         /* test hook, 0 (default) = off. 1: in every step, the projection
+                             kernel's first CTA skips the load of its first tile, so one of its
+                             bounded waits runs out after wait_limit_ms (failure detection
+                             without a fault); the step's results are then undefined */
 } tgd_options;
 
 /* Fills `opt` with the defaults listed above. */
@@ -258,7 +270,10 @@ TGD_API tgd_status tgd_topk_select(const void* grad, tgd_dtype dtype, int64_t n,
  *    that loads the library and stays allocated until the process exits.
  *  - The first call on each device looks up the array's device address on
  *    that device (the current device); make that first call before any
- *    stream capture.
+ *    stream capture. This note is about that set-up only.
+ *  - The address is looked up once per device and kept until the process
+ *    exits: after cudaDeviceReset on a device, this entry point must not be
+ *    called on that device again in the same process.
  *  - All calls share the array: calls whose work overlaps on the GPU (on
  *    different streams, or from different threads) race and give wrong
  *    results. Calls in one stream are ordered and safe; the array keeps the

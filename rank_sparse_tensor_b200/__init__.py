@@ -54,7 +54,8 @@ class TensorGRaD:
                  grad_dtype: str = "c64", weight_dtype: Optional[str] = None,
                  omega_mode: int = 0, seed: int = 0, sparse_scale: float = 1.0,
                  complex_adam: int = 0, moments_on_refresh: int = 0, auto_refresh: int = 1,
-                 path: str = "auto", sm_budget: int = 0, order: int = 0, basis: int = 0):
+                 path: str = "auto", sm_budget: int = 0, order: int = 0, basis: int = 0,
+                 wait_limit_ms: int = 0, test_stall: int = 0):
         weight_dtype = weight_dtype or grad_dtype
         self.shape = tuple(int(s) for s in shape)
         self.ranks = tuple(int(r) for r in ranks)
@@ -68,6 +69,8 @@ class TensorGRaD:
         opt.sm_budget = sm_budget
         opt.order = order
         opt.basis = basis
+        opt.wait_limit_ms = wait_limit_ms
+        opt.test_stall = test_stall
         sh = (C.c_int64 * len(self.shape))(*self.shape)
         rk = (C.c_int64 * len(self.ranks))(*self.ranks)
         h = C.c_void_p()

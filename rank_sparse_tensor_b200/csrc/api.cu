@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "step_tc.h"
+#include "step_tc32.h"
 
 using namespace tgd;
 
@@ -59,8 +60,10 @@ struct tgd_ctx {
   float* bufB = nullptr;
   float* sp_upd = nullptr;
   float* core_buf = nullptr;  // low-rank-first order: the core kept across the L rebuild
-  // tensor-core path
+  // tensor-core paths: complex fp16 gradients (tc), fp32 gradients (tc32)
   TcPlan tc;
+  Tc32Plan tc32;
+  bool use_tc32 = false;
   // errors
   int* d_err = nullptr;
   // host-buffer step
@@ -179,6 +182,7 @@ bool dalloc_t(tgd_ctx* h, T** p, size_t count) {
 
 void free_all(tgd_ctx* h) {
   tc_release(h->tc);
+  tc32_release(h->tc32);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   h->ev_pool.clear();
   for (void* p : h->allocs) cudaFree(p);
@@ -211,9 +215,31 @@ tgd_status rebuild_derived(tgd_ctx* h, cudaStream_t s) {
   if (h->path == TGD_PATH_GENERIC) {
     for (int n = 0; n < h->d; ++n)
       if (mode_active(h, n)) TGD_CUDA(h, coef_matrices(h->U[n], h->I[n], h->r[n], h->cplx, h->P[n], h->E[n], s));
+  } else if (h->use_tc32) {
+    TGD_CUDA(h, tc32_rebuild(h->tc32, h->omega, h->k, (const float* const*)h->U, s));
   } else {
     TGD_CUDA(h, tc_rebuild(h->tc, h->omega, h->k, (const float* const*)h->U, s));
   }
+  return TGD_OK;
+}
+
+// The fp32 tensor-core step: sparse AdamW into lambda S~, the projection
+// chain into the core, core AdamW in place, the expansion chain whose last
+// product updates the weights with lambda S~ added on Omega.
+tgd_status step_tc32(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
+  AdamConst asp = adam_const(h, h->opt.sparse_scale);
+  AdamConst acore = adam_const(h, 1.0);
+  {
+    TIMED(h, s, "sparse_adam");
+    TGD_CUDA(h, sparse_adam(g, h->gdt, h->omega, h->k, h->sp_m, h->sp_v, asp, tc32_sparse_update(h->tc32), s));
+  }
+  TGD_CUDA(h, tc32_project(h->tc32, g, h->bits, h->d_err, s, timer_hook, h));
+  {
+    TIMED(h, s, "core_adam");
+    TGD_CUDA(h, core_adam(tc32_core(h->tc32), h->ncore, h->core_m, h->core_v, acore, s));
+  }
+  const float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
+  TGD_CUDA(h, tc32_expand_update(h->tc32, w, h->bits, decay, h->lr, h->d_err, s, timer_hook, h));
   return TGD_OK;
 }
 
@@ -498,6 +524,8 @@ void tgd_default_options(tgd_options* opt) {
   opt->sm_budget = 0;
   opt->order = 0;
   opt->basis = 0;
+  opt->wait_limit_ms = 0;
+  opt->test_stall = 0;
 }
 
 tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int64_t* ranks,
@@ -524,7 +552,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (o.omega_mode < 0 || o.omega_mode > 1 || o.complex_adam < 0 || o.complex_adam > 1 ||
       o.moments_on_refresh < 0 || o.moments_on_refresh > 1 || o.path < 0 || o.path > 2 ||
       o.sm_budget < 0 || !std::isfinite(o.sparse_scale) || o.order < 0 || o.order > 1 ||
-      o.basis < 0 || o.basis > 1)
+      o.basis < 0 || o.basis > 1 || o.wait_limit_ms < 0 || o.test_stall < 0 || o.test_stall > 1)
     return fail(nullptr, TGD_ERR_INVALID_ARG, "bad option value");
   if (o.order == 1 && o.path == TGD_PATH_TCGEN05)
     return fail(nullptr, TGD_ERR_UNSUPPORTED, "the low-rank-first order runs on the CUDA-core path");
@@ -563,14 +591,19 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   h->vc = (h->cplx && o.complex_adam == 1) ? 2 : 1;
   // Path: the tensor-core kernels need complex fp16 gradients and tiles that
   // fit the trailing two modes.
-  bool tc_ok = tc_supported(ndim, shape, ranks, grad_dtype, weight_dtype);
+  const bool tc16_ok = tc_supported(ndim, shape, ranks, grad_dtype, weight_dtype);
+  const bool tc32_ok = tc32_supported(ndim, shape, ranks, grad_dtype, weight_dtype);
+  const bool tc_ok = tc16_ok || tc32_ok;
   if (o.path == TGD_PATH_TCGEN05 && !tc_ok) {
     delete h;
-    return fail(nullptr, TGD_ERR_UNSUPPORTED, "tensor-core path: needs complex fp16 gradients, d >= 3, "
-                                              "a power-of-two I_{d-1} <= 128, I_d <= 120 and ranks below the modes");
+    return fail(nullptr, TGD_ERR_UNSUPPORTED, "tensor-core path: needs complex fp16 gradients with d >= 3, "
+                                              "a power-of-two I_{d-1} <= 128, I_d <= 120 and ranks below the "
+                                              "modes; or fp32 gradients and weights of one kind with a "
+                                              "projected mode");
   }
   h->path = (o.path == TGD_PATH_GENERIC || !tc_ok || o.order == 1) ? TGD_PATH_GENERIC
                                                                     : TGD_PATH_TCGEN05;
+  h->use_tc32 = h->path == TGD_PATH_TCGEN05 && !tc16_ok;
   cudaError_t ce = cudaGetDevice(&h->device);
   if (ce != cudaSuccess) {
     delete h;
@@ -609,9 +642,15 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
     ok &= dalloc_t(h, &h->sp_upd, std::max<int64_t>(h->k, 1) * h->mc);
     if (o.order == 1) ok &= dalloc_t(h, &h->core_buf, ncore * h->mc);
   }
-  if (ok && h->path == TGD_PATH_TCGEN05) {
+  if (ok && h->use_tc32) {
+    auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
+    ok &= tc32_plan(h->tc32, ndim, shape, ranks, h->k, grad_dtype, alloc_fn, h);
+  }
+  if (ok && h->path == TGD_PATH_TCGEN05 && !h->use_tc32) {
     auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
     h->tc.sm_budget = o.sm_budget;
+    h->tc.wait_ns = (uint64_t)o.wait_limit_ms * 1000000ull;
+    h->tc.skip_first_copy = o.test_stall;
     ok &= tc_plan(h->tc, ndim, shape, ranks, h->k, grad_dtype, weight_dtype, alloc_fn, h);
   }
   if (!ok) {
@@ -664,6 +703,8 @@ tgd_status tgd_step(tgd_handle h, const void* grad, void* weight, void* stream) 
   tgd_status st;
   if (h->path == TGD_PATH_GENERIC) {
     st = h->opt.order == 1 ? step_lowrank_first(h, grad, weight, s) : step_generic(h, grad, weight, s);
+  } else if (h->use_tc32) {
+    st = step_tc32(h, grad, weight, s);
   } else {
     AdamConst asp = adam_const(h, h->opt.sparse_scale);
     AdamConst acore = adam_const(h, 1.0);
@@ -777,7 +818,7 @@ tgd_status tgd_get_state(tgd_handle h, tgd_state_view* out, void* stream) {
   for (int n = 0; n < h->d; ++n)
     if (out->U[n])
       TGD_CUDA(h, cudaMemcpy(out->U[n], h->U[n], sizeof(float) * 2 * h->I[n] * h->r[n], cudaMemcpyDeviceToHost));
-  if (h->path == TGD_PATH_TCGEN05) {
+  if (h->path == TGD_PATH_TCGEN05 && !h->use_tc32) {
     if (out->core_m) TGD_CUDA(h, tc_core_to_canonical(h->tc, h->core_m, h->mc, out->core_m));
     if (out->core_v) TGD_CUDA(h, tc_core_to_canonical(h->tc, h->core_v, h->vc, out->core_v));
   } else {
@@ -811,7 +852,7 @@ tgd_status tgd_set_state(tgd_handle h, const tgd_state_view* in, void* stream) {
   for (int n = 0; n < h->d; ++n)
     if (in->U[n])
       TGD_CUDA(h, cudaMemcpy(h->U[n], in->U[n], sizeof(float) * 2 * h->I[n] * h->r[n], cudaMemcpyHostToDevice));
-  if (h->path == TGD_PATH_TCGEN05) {
+  if (h->path == TGD_PATH_TCGEN05 && !h->use_tc32) {
     if (in->core_m) TGD_CUDA(h, tc_core_from_canonical(h->tc, in->core_m, h->mc, h->core_m));
     if (in->core_v) TGD_CUDA(h, tc_core_from_canonical(h->tc, in->core_v, h->vc, h->core_v));
   } else {

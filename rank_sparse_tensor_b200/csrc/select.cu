@@ -239,6 +239,14 @@ __global__ void __launch_bounds__(CT) write_kernel(KeyF kf, const void* g, int64
   }
 }
 
+// Selection state before the first digit pass: no prefix fixed, k to find.
+__global__ void init_state_kernel(SelState* st, long long k) {
+  st->prefix = 0ull;
+  st->mask = 0ull;
+  st->need = k;
+  st->pad = 0;
+}
+
 template <int DT>
 __global__ void iota_kernel(const void* g, int64_t n, int64_t* out_idx, float* out_val) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -334,11 +342,8 @@ cudaError_t run_select(KeyF kf, int key_bits, const void* g, int64_t n, int64_t 
   WsLayout L = carve(ws, n);
   cudaError_t e = cudaMemsetAsync(L.hist, 0, sizeof(unsigned long long) * BINS * MAX_PASSES, s);
   if (e != cudaSuccess) return e;
-  SelState init{0ull, 0ull, (long long)k, 0};
-  e = cudaMemcpyAsync(L.st, &init, sizeof(SelState), cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return e;
-  // The host copy above reads `init` asynchronously only for pinned memory;
-  // pageable memory is staged before the call returns, so a stack value is safe.
+  // the selection state is set on the device: nothing is copied from the host
+  init_state_kernel<<<1, 1, 0, s>>>(L.st, (long long)k);
   int pass = 0;
   for (int hi = key_bits; hi > 0; ++pass) {
     int width = hi >= DIGIT ? DIGIT : hi;

@@ -78,13 +78,14 @@ constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 // ----------------------------------------------------------- projection
 // Bounded wait for one thread. Gives up when another role has aborted or
 // after WAIT_NS, setting the CTA's abort flag and the device error word.
-__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                      uint64_t limit_ns = WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   // sleep in the barrier (no issue slots) until the phase completes
   while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
     if (*abort) return false;
-    if (global_ns() - t0 > WAIT_NS) {
+    if (global_ns() - t0 > limit_ns) {
       *abort = 1;
       atomicOr(err, DEV_ERR_TIMEOUT);
       return false;
@@ -93,9 +94,10 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile i
   return true;
 }
 // The same for a whole warp: lane 0 polls, the warp re-converges after.
-__device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+__device__ __forceinline__ bool waitw(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                      uint64_t limit_ns = WAIT_NS) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = wait1(bar, parity, abort, err) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = wait1(bar, parity, abort, err, limit_ns) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;
@@ -129,6 +131,8 @@ struct P1Args {
   int* err;
   int nstage;  // load stages
   uint32_t stage_bytes, off_stage, off_A2, off_B1, off_B2, off_bar;
+  uint64_t wait_ns;     // limit of each wait (normally WAIT_NS)
+  int skip_first_copy;  // test only: CTA 0 never loads its first tile, so a wait runs out
 };
 
 // Position in this CTA's tile sequence: groups blockIdx.x, +gridDim.x, ...,
@@ -233,13 +237,16 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
+      const bool skip0 = p.skip_first_copy && blockIdx.x == 0;
       for (int64_t it = 0; it < n_it; ++it) {
-        if (!wait1(&sempty[s], ph ^ 1u, s_abort, p.err)) break;
+        if (!wait1(&sempty[s], ph ^ 1u, s_abort, p.err, p.wait_ns)) break;
         const int64_t t = c.tile(q);
         const int64_t rem = p.N - t * p.tile_elems;
         const uint32_t nb = (uint32_t)((rem < p.tile_elems ? rem : p.tile_elems) * 4);
-        mbar_expect_tx(&full[s], nb);
-        bulk_g2s(stage(s), p.G + t * p.tile_elems, nb, &full[s]);
+        if (!(skip0 && it == 0)) {
+          mbar_expect_tx(&full[s], nb);
+          bulk_g2s(stage(s), p.G + t * p.tile_elems, nb, &full[s]);
+        }
         ++issued;
         c.next(q);
         if (++s == ns) {
@@ -248,10 +255,12 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
         }
       }
       // wait (bounded) for the operand copies and for tile copies still in
-      // flight before the CTA exits
+      // flight before the CTA exits: the last copy into each stage (earlier
+      // phases of a stage's barrier have completed before it was reused)
       mbar_wait(opnd, 0, WAIT_NS / 4);
-      if (*s_abort) {
-        for (int64_t it = 0; it < issued; ++it) mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
+      for (int64_t it = issued > ns ? issued - ns : 0; it < issued; ++it) {
+        if (skip0 && it == 0) continue;
+        mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
       }
     }
   } else if (warp == 1) {
@@ -260,14 +269,14 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       const uint32_t lbo_b1 = (uint32_t)(p.N1 / 8) * 128, lbo_b2 = (uint32_t)(p.N2 / 8) * 128;
       const uint32_t id1 = idesc_f16(0, 128, p.N1), id2 = idesc_f16(1, 128, p.N2);
       const uint32_t sB1 = smem_u32(B1), sB2 = smem_u32(B2);
-      bool ok = wait1(opnd, 0, s_abort, p.err);
+      bool ok = wait1(opnd, 0, s_abort, p.err, p.wait_ns);
       TileCursor c{(int64_t)blockIdx.x, 0};
       int64_t it = 0, g2_issued = 0;
       bool pending = false;  // a group whose GEMM1s are all issued awaits its GEMM2
       auto gemm2 = [&]() -> bool {
         const int gb = (int)(g2_issued & 1);
         const uint32_t gpar = (uint32_t)((g2_issued >> 1) & 1);
-        if (!wait1(&a2full[gb], gpar, s_abort, p.err) || !wait1(&d2empty[gb], gpar ^ 1u, s_abort, p.err))
+        if (!wait1(&a2full[gb], gpar, s_abort, p.err, p.wait_ns) || !wait1(&d2empty[gb], gpar ^ 1u, s_abort, p.err, p.wait_ns))
           return false;
         tc_fence_after();
         const uint32_t sA2 = smem_u32(A2b(gb));
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       for (; ok && it < n_it; ++it) {
         const int b = (int)(it & 1);
         const uint32_t par = (uint32_t)((it >> 1) & 1);
-        if (!wait1(&a1full[b], par, s_abort, p.err) || !wait1(&d1empty[b], par ^ 1u, s_abort, p.err)) {
+        if (!wait1(&a1full[b], par, s_abort, p.err, p.wait_ns) || !wait1(&d1empty[b], par ^ 1u, s_abort, p.err, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
         nn_e0 = p.tile_off[t2];
         nn_e1 = p.tile_off[t2 + 1];
       }
-      if (!waitw(&full[s], ph, s_abort, p.err)) {
+      if (!waitw(&full[s], ph, s_abort, p.err, p.wait_ns)) {
         named_sync(1, 256);
         dead_from = it + 1;
         continue;
@@ -402,7 +411,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       nx_e0 = nn_e0;
       nx_e1 = nn_e1;
       named_sync(1, 256);  // every zeroed entry is in place before conversion
-      if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err)) {
+      if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err, p.wait_ns)) {
         dead_from = it + 1;
         continue;
       }
@@ -450,7 +459,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     // Y of one group from D2[gi & 1] (row = (slab in group, j_b)), j_a contiguous
     auto write_y = [&](int64_t gi, int64_t gabs) -> bool {
       const int gb = (int)(gi & 1);
-      if (!waitw(&d2full[gb], (uint32_t)((gi >> 1) & 1), s_abort, p.err)) return false;
+      if (!waitw(&d2full[gb], (uint32_t)((gi >> 1) & 1), s_abort, p.err, p.wait_ns)) return false;
       tc_fence_after();
       const int sb = row / p.rb, jb = row - sb * p.rb;
       const int64_t slab = gabs * p.sg + sb;
@@ -499,7 +508,7 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       const int b = (int)(it & 1);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
       const int64_t t = c.tile(q);
-      if (!waitw(&d1full[b], par, s_abort, p.err)) {
+      if (!waitw(&d1full[b], par, s_abort, p.err, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -904,10 +913,10 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
           ph ^= 1u;
         }
       }
-      if (*s_abort) {
-        // wait (bounded) for loads still in flight before the CTA exits
-        for (int64_t it = 0; it < loaded; ++it) mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
-      }
+      // wait (bounded) for loads still in flight before the CTA exits: the
+      // last load into each stage (earlier phases completed before reuse)
+      for (int64_t it = loaded > ns ? loaded - ns : 0; it < loaded; ++it)
+        mbar_wait(&full[it % ns], (uint32_t)((it / ns) & 1), WAIT_NS / 4);
       bulk_wait_all0();
     }
   } else if (warp == 1) {
@@ -1611,6 +1620,8 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
   a.y_f32 = no_inner ? 1 : 0;
   a.y_vec = a.y_f32 ? (g->ra % 2 == 0) : (g->ra % 4 == 0);
   a.err = d_err;
+  a.wait_ns = p.wait_ns ? p.wait_ns : WAIT_NS;
+  a.skip_first_copy = p.skip_first_copy;
   // At least half the shared memory of an SM, so one CTA (and its 512 TMEM
   // columns) per SM.
   const size_t p1_launch_smem = std::max(g->p1_smem, ONE_CTA_SMEM);

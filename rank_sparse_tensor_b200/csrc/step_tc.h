@@ -19,6 +19,8 @@ struct TcPlan {
   int64_t N = 0, k = 0, ncore = 0;
   int gdt = 0, wdt = 0;
   int sm_budget = 0;  // > 0: the persistent kernels use at most this many CTAs
+  uint64_t wait_ns = 0;      // limit of each projection wait; 0: the default (2 s)
+  int skip_first_copy = 0;   // test only: the projection's CTA 0 skips its first tile copy
   bool ready = false;
   void* impl = nullptr;  // owned by step_tc.cu (host-side description)
 };

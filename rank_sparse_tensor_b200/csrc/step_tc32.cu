@@ -1,0 +1,571 @@
+// Tensor-core (tcgen05, sm_100a) path of the TensorGRaD step for fp32
+// gradients and weights (real fp32 and complex64).
+//
+// The step is the one of the nullthought.net TensorGRaD summary (section 三:
+// sparse part first, Tucker part on the residual, separate Adam updates, the
+// sparse update scatter-added in place into the rebuilt tensor) and of
+// Theorem 2 in the paper text appended to the Pith review (project with the
+// conjugate-transposed factors, Adam on the core, project back):
+//
+//   sparse_adam   S~ = lambda Adam(G[Omega]) (CUDA cores, in Omega order)
+//   mode_gemm32   C = R x_n U_n^H for every projected mode, last mode first;
+//                 the first contraction reads G itself with Omega zeroed
+//                 through the index set's bit mask (R is never stored)
+//   core_adam     C~ = Adam(C) in place
+//   mode_gemm32   C~ x_n U_n for every projected mode, first mode first; the
+//                 last one does not store Delta: its epilogue adds lambda S~
+//                 where the output index is in Omega and writes
+//                 W <- W (1 - lr wd) - lr (Delta + lambda S~), one rounding
+//
+// Every mode product is one tcgen05 GEMM per 128 unfolding rows (a, b) of
+// the tensor X[a][k][b]: A = the rows' K values gathered by the threads
+// (coalesced across threads when b varies fastest), B = the factor's
+// embedding (complex products as real 2 x 2 blocks, as in step_tc.cu),
+// accumulators in TMEM. fp32 operands are split into two bf16 parts, x = h +
+// l with h = bf16(x) and l = bf16(x - h), and three products h.h + l.h + h.l
+// are accumulated in fp32: the dropped l.l term and the rounding of l leave a
+// relative error near 2^-16 per product, against 2^-9 for one bf16 operand.
+// Every wait is bounded and reports TGD_ERR_TIMEOUT.
+
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "step_tc32.h"
+#include "tc_ptx.cuh"
+
+namespace tgd {
+namespace {
+
+using namespace ptx;
+
+constexpr int G32T = 128;                    // threads = GEMM rows per CTA
+constexpr uint32_t G32_LBO = 2048;           // A tile: 128 rows x 16 B between K core matrices
+constexpr uint32_t G32_ATILE = 8 * G32_LBO;  // 128 rows x 64 bf16
+constexpr uint64_t G32_WAIT_NS = 2000000000ull;
+
+__host__ __device__ __forceinline__ uint32_t kmaj(uint32_t row, uint32_t k, uint32_t lbo) {
+  return (row & 7u) * 16u + (row >> 3) * 128u + (k >> 3) * lbo + (k & 7u) * 2u;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+// x = h + l (+ a remainder below 2^-16 |x|): the two bf16 parts, packed with
+// the neighbouring K value (lo half = even K)
+__device__ __forceinline__ void split2(float x, float y, uint32_t& h, uint32_t& l) {
+  const uint16_t hx = bf16_bits(x), hy = bf16_bits(y);
+  const uint16_t lx = bf16_bits(x - bf16_val(hx)), ly = bf16_bits(y - bf16_val(hy));
+  h = (uint32_t)hx | ((uint32_t)hy << 16);
+  l = (uint32_t)lx | ((uint32_t)ly << 16);
+}
+
+struct MG32Args {
+  const float* X;         // [a][k][b] fp32 values (re, im interleaved when complex)
+  const uint32_t* bits;   // Omega's bit mask when X is the gradient (zeros there), else null
+  int64_t rows, K, B;     // rows = A * B unfolding rows; K entries along the mode
+  float* Y;               // [a][j][b] output (unused when the epilogue updates W)
+  int64_t J;
+  const uint8_t* img;     // B operand blocks [n block][k chunk][hi, lo], NT x 64 bf16 each
+  int NT, nkc;
+  uint32_t tmem_cols;
+  // epilogue of the last expansion: the weight update
+  float* W;               // the weights, the full tensor (Y's layout)
+  const float* S;         // lambda S~ in Omega order
+  const int64_t* wrank;   // Omega entries before each 32-element word of the mask
+  const uint32_t* wbits;  // Omega's bit mask for the update
+  float decay, lr;
+  int* err;
+};
+
+// Y[a][j][b] = sum_k X[a][k][b] M[k][j] over one 128-row block of the
+// unfolding and one NT-wide block of (j, re/im) columns. K advances in chunks
+// of 32 complex (64 real) values, two stages: the chunk's operand image
+// arrives by bulk copy while the threads split and store their rows' values,
+// and the next chunk's values are loaded while its MMAs run.
+// WUPD: instead of storing Y, W[o] <- W[o] decay - lr (Y[o] + S~[o in Omega]).
+template <bool CPLX, bool WUPD>
+__global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t b_bytes = (uint32_t)p.NT * 64 * 2;
+  // stage s: A hi, A lo, B hi, B lo
+  auto Ah = [&](int s) { return smem + (uint32_t)s * 2 * G32_ATILE; };
+  auto Al = [&](int s) { return smem + (uint32_t)s * 2 * G32_ATILE + G32_ATILE; };
+  auto Bh = [&](int s) { return smem + 4 * G32_ATILE + (uint32_t)s * 2 * b_bytes; };
+  uint64_t* bars = (uint64_t*)(smem + 4 * G32_ATILE + 4 * b_bytes);  // [0,1] MMAs done, [2,3] B landed
+  uint32_t* tslot = (uint32_t*)(bars + 4);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int64_t rho = (int64_t)blockIdx.x * G32T + tid;
+  const bool valid = rho < p.rows;
+  const int64_t a = valid ? rho / p.B : 0, b = valid ? rho - a * p.B : 0;
+  const int64_t xbase = a * p.K * p.B + b;  // element index of (a, k = 0, b)
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) tmem_alloc(tslot, p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t dt = *tslot;
+  const uint32_t lbo_b = (uint32_t)(p.NT / 8) * 128;
+  const uint32_t idesc = idesc_f16(1, 128, p.NT);
+  const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * 2 * b_bytes;
+  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0}, bloaded[2] = {0, 0};
+  constexpr int KE = CPLX ? 32 : 64;  // entries per chunk
+  constexpr int NV = 64;              // fp32 values per chunk and row
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (tid == 0 && !mbar_wait(bar, parity, G32_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    return s_abort == 0;
+  };
+  float v[NV];
+  auto load_x = [&](int kc) {
+#pragma unroll
+    for (int i = 0; i < KE; ++i) {
+      const int64_t k = (int64_t)kc * KE + i;
+      float2 x = make_float2(0.f, 0.f);
+      if (valid && k < p.K) {
+        const int64_t idx = xbase + k * p.B;
+        if (!(p.bits && ((__ldg(p.bits + (idx >> 5)) >> (idx & 31)) & 1u))) {
+          if (CPLX)
+            x = __ldg((const float2*)p.X + idx);
+          else
+            x.x = __ldg(p.X + idx);
+        }
+      }
+      if (CPLX) {
+        v[2 * i] = x.x;
+        v[2 * i + 1] = x.y;
+      } else {
+        v[i] = x.x;
+      }
+    }
+  };
+  load_x(0);
+  for (int kc = 0; kc < p.nkc; ++kc) {
+    const int s = kc & 1;
+    if (kc >= 2) {
+      const bool ok = wait_all(&bars[s], waited[s] & 1u);
+      waited[s]++;
+      if (!ok) break;
+      tc_fence_after();
+    }
+    if (tid == 0) {
+      mbar_expect_tx(&bars[2 + s], 2 * b_bytes);
+      bulk_g2s(Bh(s), img + (int64_t)kc * 2 * b_bytes, 2 * b_bytes, &bars[2 + s]);
+      bloaded[s]++;
+    }
+    // this row's 64 K values -> the hi and lo A tiles (8 core matrices each)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t h[4], l[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) split2(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], h[u], l[u]);
+      *(uint4*)(Ah(s) + q * G32_LBO + tid * 16) = make_uint4(h[0], h[1], h[2], h[3]);
+      *(uint4*)(Al(s) + q * G32_LBO + tid * 16) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+    if (kc + 1 < p.nkc) load_x(kc + 1);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (s_abort) break;
+    if (tid == 0) {
+      if (!mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, G32_WAIT_NS)) {
+        atomicOr(p.err, DEV_ERR_TIMEOUT);
+        s_abort = 1;
+      } else {
+        const uint32_t ah = smem_u32(Ah(s)), al = smem_u32(Al(s));
+        const uint32_t bh = smem_u32(Bh(s)), bl = bh + b_bytes;
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t dah = sdesc(ah + kk * 2 * G32_LBO, G32_LBO, 128);
+          const uint64_t dal = sdesc(al + kk * 2 * G32_LBO, G32_LBO, 128);
+          const uint64_t dbh = sdesc(bh + kk * 2 * lbo_b, lbo_b, 128);
+          const uint64_t dbl = sdesc(bl + kk * 2 * lbo_b, lbo_b, 128);
+          mma_f16(dt, dah, dbh, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          mma_f16(dt, dal, dbh, idesc, 1u);
+          mma_f16(dt, dah, dbl, idesc, 1u);
+        }
+        mma_commit(&bars[s]);
+        issued[s]++;
+      }
+    }
+  }
+  __syncthreads();
+  if (!s_abort) {
+    const int s = (p.nkc - 1) & 1;
+    wait_all(&bars[s], waited[s] & 1u);
+    waited[s]++;
+    tc_fence_after();
+  }
+  if (!s_abort) {
+    const int64_t j0 = (int64_t)blockIdx.y * (CPLX ? p.NT / 2 : p.NT);
+    for (int c0 = 0; c0 < p.NT; c0 += 16) {
+      float y[16];
+      tmem_ld16(dt + lane_base + c0, y);
+      constexpr int PER = CPLX ? 8 : 16;  // outputs per 16 columns
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int64_t j = j0 + (CPLX ? c0 / 2 : c0) + u;
+        if (!valid || j >= p.J) continue;
+        const int64_t o = (a * p.J + j) * p.B + b;
+        float dr = CPLX ? y[2 * u] : y[u], di = CPLX ? y[2 * u + 1] : 0.f;
+        if (!WUPD) {
+          if (CPLX)
+            ((float2*)p.Y)[o] = make_float2(dr, di);
+          else
+            p.Y[o] = dr;
+        } else {
+          const uint32_t word = __ldg(p.wbits + (o >> 5));
+          const uint32_t bit = (uint32_t)(o & 31);
+          if ((word >> bit) & 1u) {
+            const int64_t e = __ldg(p.wrank + (o >> 5)) + __popc(word & ((1u << bit) - 1u));
+            if (CPLX) {
+              const float2 sv = __ldg((const float2*)p.S + e);
+              dr += sv.x;
+              di += sv.y;
+            } else {
+              dr += __ldg(p.S + e);
+            }
+          }
+          if (CPLX) {
+            float2* wp = (float2*)p.W + o;
+            const float2 w = *wp;
+            *wp = make_float2(__fmaf_rn(-p.lr, dr, w.x * p.decay), __fmaf_rn(-p.lr, di, w.y * p.decay));
+          } else {
+            float* wp = p.W + o;
+            *wp = __fmaf_rn(-p.lr, dr, *wp * p.decay);
+          }
+        }
+      }
+    }
+  } else if (tid == 0) {
+    // bounded waits for the copies and MMAs still in flight
+    for (int s = 0; s < 2; ++s) {
+      if (issued[s] > waited[s]) mbar_wait(&bars[s], (issued[s] - 1) & 1u, G32_WAIT_NS / 4);
+      if (bloaded[s] > 0) mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, G32_WAIT_NS / 4);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(dt, p.tmem_cols);
+}
+
+// B operand of y = x M for one mode, M from U (I x r, complex fp32 pairs; the
+// real part only for real tensors): kind 0 projection M = conj(U) (Kc = I,
+// Jc = r), kind 1 expansion M = U^T (Kc = r, Jc = I). Complex M as the real
+// embedding E[(kk,0)][(j,0)] = Mr, E[(kk,1)][(j,0)] = -Mi, E[(kk,0)][(j,1)] =
+// Mi, E[(kk,1)][(j,1)] = Mr; real M as itself. Zero padded to Np x Kp, stored
+// as [n block][k chunk][hi, lo] blocks of NT x 64, each K-major no-swizzle
+// with 8-row groups 128 B apart and K core matrices NT / 8 * 128 B apart.
+__global__ void embed32_kernel(const float2* U, int I, int r, int kind, int cplx, int Np, int Kp, int NT,
+                               uint16_t* img) {
+  const int nkb = Kp / 64;
+  const int Kc = kind == 0 ? I : r, Jc = kind == 0 ? r : I;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)Np * Kp;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int n = (int)(e / Kp), k = (int)(e - (int64_t)n * Kp);
+    float val = 0.f;
+    if (cplx) {
+      const int j = n >> 1, cp = n & 1, kk = k >> 1, c = k & 1;
+      if (j < Jc && kk < Kc) {
+        const float2 u = kind == 0 ? U[(int64_t)kk * r + j] : U[(int64_t)j * r + kk];
+        const float mr = u.x, mi = kind == 0 ? -u.y : u.y;
+        val = (c == 0) ? (cp == 0 ? mr : mi) : (cp == 0 ? -mi : mr);
+      }
+    } else if (n < Jc && k < Kc) {
+      val = kind == 0 ? U[(int64_t)k * r + n].x : U[(int64_t)n * r + k].x;
+    }
+    const uint16_t h = bf16_bits(val), l = bf16_bits(val - bf16_val(h));
+    const int nb = n / NT, nl = n - nb * NT, kb = k / 64, kl = k - kb * 64;
+    const int64_t base = ((int64_t)nb * nkb + kb) * 2 * NT * 64;
+    const uint32_t off = kmaj((uint32_t)nl, (uint32_t)kl, (uint32_t)(NT / 8) * 128u) / 2;
+    img[base + off] = h;
+    img[base + (int64_t)NT * 64 + off] = l;
+  }
+}
+
+// wrank[w] = number of Omega entries below 32 w (Omega ascending).
+__global__ void word_rank_kernel(const int64_t* omega, int64_t k, int64_t nwords, int64_t* wrank) {
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t target = w * 32;
+    int64_t lo = 0, hi = k;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi) >> 1;
+      if (omega[mid] < target)
+        lo = mid + 1;
+      else
+        hi = mid;
+    }
+    wrank[w] = lo;
+  }
+}
+
+struct Mode32 {
+  int n = 0;
+  int64_t I = 0, r = 0;
+  bool active = false;
+  uint16_t* img_p = nullptr;  // projection image
+  uint16_t* img_e = nullptr;  // expansion image
+  int NTp = 0, nntp = 0, nkcp = 0, NTe = 0, nnte = 0, nkce = 0;
+};
+
+struct Tc32Impl {
+  int d = 0;
+  bool cplx = false;
+  int64_t N = 0, k = 0, ncore = 0, nwords = 0;
+  std::vector<Mode32> modes;
+  float* X0 = nullptr;
+  float* X1 = nullptr;
+  float* C = nullptr;
+  float* S = nullptr;     // lambda S~, Omega order
+  int64_t* wrank = nullptr;
+  int num_sms = 148;
+};
+
+int r16i(int x) { return (x + 15) / 16 * 16; }
+int pow2_cols32(int n) {
+  int c = 32;
+  while (c < n) c <<= 1;
+  return c;
+}
+size_t g32_smem(int NT) { return 4 * (size_t)G32_ATILE + 4 * (size_t)NT * 64 * 2 + 64; }
+
+Tc32Impl* impl32(Tc32Plan& p) { return (Tc32Impl*)p.impl; }
+
+// Geometry of one mode's GEMM: N = 2 Jc (complex) or Jc columns in blocks of
+// at most 256; K chunks of 64 real values (32 complex).
+void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc) {
+  const int Np = r16i((int)(cplx ? 2 * Jc : Jc));
+  NT = Np <= 256 ? Np : 256;
+  nnt = (int)ceil_div(Np, NT);
+  nkc = (int)ceil_div(cplx ? 2 * Kc : Kc, 64);
+}
+
+template <bool CPLX, bool WUPD>
+cudaError_t launch32(const MG32Args& a, int nnt, cudaStream_t s) {
+  const size_t sm = g32_smem(a.NT);
+  cudaError_t e = cudaFuncSetAttribute(mode_gemm32_kernel<CPLX, WUPD>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)ceil_div(a.rows, G32T), (unsigned)nnt);
+  mode_gemm32_kernel<CPLX, WUPD><<<grid, G32T, sm, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mode32(bool cplx, bool wupd, const MG32Args& a, int nnt, cudaStream_t s) {
+  if (cplx) return wupd ? launch32<true, true>(a, nnt, s) : launch32<true, false>(a, nnt, s);
+  return wupd ? launch32<false, true>(a, nnt, s) : launch32<false, false>(a, nnt, s);
+}
+
+}  // namespace
+
+bool tc32_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt) {
+  if (!((gdt == TGD_C64 && wdt == TGD_C64) || (gdt == TGD_R32 && wdt == TGD_R32))) return false;
+  bool any = false;
+  for (int n = 0; n < nd; ++n) {
+    if (ranks[n] < shape[n]) {
+      any = true;
+      if (shape[n] > 256) return false;
+    }
+  }
+  return any;
+}
+
+bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
+               AllocFn alloc, void* ctx) {
+  Tc32Impl* g = new Tc32Impl;
+  p.impl = g;
+  g->d = nd;
+  g->cplx = gdt == TGD_C64;
+  g->N = 1;
+  g->ncore = 1;
+  for (int n = 0; n < nd; ++n) {
+    g->N *= shape[n];
+    g->ncore *= ranks[n];
+  }
+  g->k = k;
+  g->nwords = ceil_div(g->N, 32);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&g->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const int comps = g->cplx ? 2 : 1;
+  auto A = [&](void** ptr, size_t bytes) { return alloc(ctx, ptr, bytes); };
+  bool ok = true;
+  // intermediates: the largest tensor of either chain short of the full one
+  // (the expansion chain passes through the same sizes in reverse)
+  int64_t maxe = 1, cur = g->N;
+  int first = -1;
+  for (int n = nd - 1; n >= 0; --n) {
+    if (ranks[n] == shape[n]) continue;
+    if (first < 0) first = n;
+    cur = cur / shape[n] * ranks[n];
+    maxe = std::max(maxe, cur);
+  }
+  g->modes.clear();
+  for (int n = 0; n < nd; ++n) {
+    Mode32 m;
+    m.n = n;
+    m.I = shape[n];
+    m.r = ranks[n];
+    m.active = ranks[n] < shape[n];
+    if (m.active) {
+      mode_geom(m.I, m.r, g->cplx, m.NTp, m.nntp, m.nkcp);
+      mode_geom(m.r, m.I, g->cplx, m.NTe, m.nnte, m.nkce);
+      ok &= A((void**)&m.img_p, (size_t)m.nntp * m.nkcp * 2 * m.NTp * 64 * 2);
+      ok &= A((void**)&m.img_e, (size_t)m.nnte * m.nkce * 2 * m.NTe * 64 * 2);
+    }
+    g->modes.push_back(m);
+  }
+  ok &= A((void**)&g->X0, sizeof(float) * comps * maxe);
+  ok &= A((void**)&g->X1, sizeof(float) * comps * maxe);
+  ok &= A((void**)&g->C, sizeof(float) * comps * g->ncore);
+  ok &= A((void**)&g->S, sizeof(float) * comps * std::max<int64_t>(k, 1));
+  ok &= A((void**)&g->wrank, sizeof(int64_t) * (g->nwords + 1));
+  p.ready = ok;
+  return ok;
+}
+
+void tc32_release(Tc32Plan& p) {
+  delete impl32(p);
+  p.impl = nullptr;
+  p.ready = false;
+}
+
+float* tc32_core(Tc32Plan& p) { return impl32(p) ? impl32(p)->C : nullptr; }
+float* tc32_sparse_update(Tc32Plan& p) { return impl32(p) ? impl32(p)->S : nullptr; }
+
+cudaError_t tc32_rebuild(Tc32Plan& p, const int64_t* omega, int64_t k, const float* const* U,
+                         cudaStream_t s) {
+  Tc32Impl* g = impl32(p);
+  if (!g) return cudaErrorNotReady;
+  auto blocks = [](int64_t n) { return (unsigned)std::min<int64_t>(ceil_div(n, 256), 4096); };
+  word_rank_kernel<<<blocks(g->nwords), 256, 0, s>>>(omega, k, g->nwords, g->wrank);
+  for (auto& m : g->modes) {
+    if (!m.active) continue;
+    const float2* Un = (const float2*)U[m.n];
+    int Np = m.nntp * m.NTp, Kp = m.nkcp * 64;
+    embed32_kernel<<<blocks((int64_t)Np * Kp), 256, 0, s>>>(Un, (int)m.I, (int)m.r, 0, g->cplx ? 1 : 0, Np, Kp,
+                                                            m.NTp, m.img_p);
+    Np = m.nnte * m.NTe;
+    Kp = m.nkce * 64;
+    embed32_kernel<<<blocks((int64_t)Np * Kp), 256, 0, s>>>(Un, (int)m.I, (int)m.r, 1, g->cplx ? 1 : 0, Np, Kp,
+                                                            m.NTe, m.img_e);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t tc32_project(Tc32Plan& p, const void* grad, const uint32_t* bits, int* d_err, cudaStream_t s,
+                         TimerHook hook, void* hook_ctx) {
+  Tc32Impl* g = impl32(p);
+  if (!g) return cudaErrorNotReady;
+  const int d = g->d;
+  int64_t dims[TGD_MAX_NDIM];
+  for (int n = 0; n < d; ++n) dims[n] = g->modes[n].I;
+  int first_active = -1;
+  for (int n = 0; n < d; ++n)
+    if (g->modes[n].active) {
+      first_active = n;
+      break;
+    }
+  const float* cur = (const float*)grad;
+  bool from_grad = true;
+  float* bufs[2] = {g->X0, g->X1};
+  int which = 0;
+  for (int n = d - 1; n >= 0; --n) {
+    Mode32& m = g->modes[n];
+    if (!m.active) continue;
+    int64_t A = 1, B = 1;
+    for (int q = 0; q < n; ++q) A *= dims[q];
+    for (int q = n + 1; q < d; ++q) B *= dims[q];
+    float* out = n == first_active ? g->C : bufs[which];
+    MG32Args a{};
+    a.X = cur;
+    a.bits = from_grad ? bits : nullptr;
+    a.rows = A * B;
+    a.K = m.I;
+    a.B = B;
+    a.Y = out;
+    a.J = m.r;
+    a.img = (const uint8_t*)m.img_p;
+    a.NT = m.NTp;
+    a.nkc = m.nkcp;
+    a.tmem_cols = (uint32_t)pow2_cols32(m.NTp);
+    a.err = d_err;
+    if (hook) hook(hook_ctx, 0, "mode_gemm32", s);
+    cudaError_t e = launch_mode32(g->cplx, false, a, m.nntp, s);
+    if (hook) hook(hook_ctx, 1, "mode_gemm32", s);
+    if (e != cudaSuccess) return e;
+    dims[n] = m.r;
+    cur = out;
+    from_grad = false;
+    which ^= 1;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t tc32_expand_update(Tc32Plan& p, void* w, const uint32_t* bits, float decay, float lr, int* d_err,
+                               cudaStream_t s, TimerHook hook, void* hook_ctx) {
+  Tc32Impl* g = impl32(p);
+  if (!g) return cudaErrorNotReady;
+  const int d = g->d;
+  int64_t dims[TGD_MAX_NDIM];
+  for (int n = 0; n < d; ++n) dims[n] = g->modes[n].r;
+  int last_active = -1;
+  for (int n = 0; n < d; ++n)
+    if (g->modes[n].active) last_active = n;
+  const float* cur = g->C;
+  float* bufs[2] = {g->X0, g->X1};
+  int which = 0;
+  for (int n = 0; n < d; ++n) {
+    Mode32& m = g->modes[n];
+    if (!m.active) continue;
+    int64_t A = 1, B = 1;
+    for (int q = 0; q < n; ++q) A *= dims[q];
+    for (int q = n + 1; q < d; ++q) B *= dims[q];
+    const bool last = n == last_active;
+    MG32Args a{};
+    a.X = cur;
+    a.bits = nullptr;
+    a.rows = A * B;
+    a.K = m.r;
+    a.B = B;
+    a.Y = last ? nullptr : bufs[which];
+    a.J = m.I;
+    a.img = (const uint8_t*)m.img_e;
+    a.NT = m.NTe;
+    a.nkc = m.nkce;
+    a.tmem_cols = (uint32_t)pow2_cols32(m.NTe);
+    a.W = (float*)w;
+    a.S = g->S;
+    a.wrank = g->wrank;
+    a.wbits = bits;
+    a.decay = decay;
+    a.lr = lr;
+    a.err = d_err;
+    if (hook) hook(hook_ctx, 0, last ? "expand_update32" : "mode_gemm32", s);
+    cudaError_t e = launch_mode32(g->cplx, last, a, m.nnte, s);
+    if (hook) hook(hook_ctx, 1, last ? "expand_update32" : "mode_gemm32", s);
+    if (e != cudaSuccess) return e;
+    dims[n] = m.I;
+    if (!last) {
+      cur = bufs[which];
+      which ^= 1;
+    }
+  }
+  return cudaSuccess;
+}
+
+}  // namespace tgd

@@ -34,7 +34,8 @@ class Options(C.Structure):
     _fields_ = [("omega_mode", C.c_int), ("seed", C.c_uint64), ("sparse_scale", C.c_float),
                 ("complex_adam", C.c_int), ("moments_on_refresh", C.c_int),
                 ("auto_refresh", C.c_int), ("path", C.c_int), ("sm_budget", C.c_int),
-                ("order", C.c_int), ("basis", C.c_int)]
+                ("order", C.c_int), ("basis", C.c_int), ("wait_limit_ms", C.c_int),
+                ("test_stall", C.c_int)]
 
 
 class Info(C.Structure):

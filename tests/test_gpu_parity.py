@@ -209,18 +209,19 @@ def test_bad_state_rejected(lib):
     assert e.value.name == "INVALID_ARG"
 
 
-@pytest.mark.parametrize("dtype,shape,ranks", [
-    ("r32", (16, 12, 8, 9), (4, 3, 2, 3)),      # CUDA-core path
-    ("c32h", (4, 8, 64, 33), (2, 4, 16, 8)),    # tensor-core path
+@pytest.mark.parametrize("dtype,shape,ranks,path", [
+    ("r32", (16, 12, 8, 9), (4, 3, 2, 3), "generic"),     # CUDA-core path
+    ("c32h", (4, 8, 64, 33), (2, 4, 16, 8), "tcgen05"),   # tensor-core path, fp16
+    ("c64", (16, 12, 8, 9), (4, 3, 2, 3), "tcgen05"),     # tensor-core path, fp32
 ])
-def test_step_host_equals_device_step(lib, dtype, shape, ranks):
+def test_step_host_equals_device_step(lib, dtype, shape, ranks, path):
     """tgd_step_host (host buffers, copies inside the call) leaves bit for bit
     the weights tgd_step leaves from the same state."""
     from rank_sparse_tensor_b200.synth import GradientStream, weights
     g = GradientStream(shape, ranks, dtype, 4, outlier_frac=0.02, outlier_scale=10.0).next()
     w = weights(shape, dtype, 4)
-    a = _gpu(lib, shape, ranks, 0.05, dtype)
-    b = _gpu(lib, shape, ranks, 0.05, dtype)
+    a = _gpu(lib, shape, ranks, 0.05, dtype, path=path)
+    b = _gpu(lib, shape, ranks, 0.05, dtype, path=path)
     g_dev, w_dev = g.cuda(), w.cuda()
     a.refresh(g_dev)
     b.refresh(g_dev)

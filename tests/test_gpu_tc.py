@@ -136,7 +136,9 @@ def test_tc_selected_automatically(lib):
     g = lib.TensorGRaD((8, 8, 64, 33), (4, 4, 16, 8), 0.05, 0, grad_dtype="c32h")
     assert g.info["path"] == "tcgen05"
     h = lib.TensorGRaD((8, 8, 64, 33), (4, 4, 16, 8), 0.05, 0, grad_dtype="c64")
-    assert h.info["path"] == "generic"
+    assert h.info["path"] == "tcgen05"     # the fp32 tensor-core path
+    f = lib.TensorGRaD((8, 8, 64, 33), (8, 8, 64, 33), 0.05, 0, grad_dtype="c64")
+    assert f.info["path"] == "generic"     # no projected mode: plain sparse + AdamW
     with pytest.raises(lib.TgdError) as e:
         lib.TensorGRaD((8, 8, 6, 33), (4, 4, 3, 8), 0.05, 0, grad_dtype="c32h", path="tcgen05")
     assert e.value.name == "UNSUPPORTED"

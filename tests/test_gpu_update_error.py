@@ -1,0 +1,156 @@
+"""GPU parity of the update itself, and of the factors at full size.
+
+The weight gate (max |W_gpu - W_ref| / max |W_ref|) sees an error in the
+update only scaled by lr |Delta| / |W|, about 5% at these settings. Here the
+weights' change over one teacher-forced step is compared directly,
+max |dW_gpu - dW_ref| / max |dW_ref|, with fp32 weights so that storage
+rounding does not hide it. The bound for each kernel path follows from its
+arithmetic (see UPDATE_TOL).
+
+The factors of a device refresh are compared with the oracle's on the full
+tensors of the 4-tensor workload and of the 5-way refresh workload, by
+projector distance where the eigengap is open (eigenvectors are unique only
+up to phase, and only when the gap is open).
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from tests.helpers import eigengap, projector_distance, random_moments, to_np
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+# Bound on max |dW_gpu - dW_ref| / max |dW_ref| for one step:
+# - generic path: fp32 FFMA chains, a few hundred terms per sum: ~1e-6, bound 1e-4;
+# - tensor-core path, fp16 gradients: the gradient and U_b are exact or
+#   rounded once to fp16 (2^-11); the intermediates between the GEMMs are
+#   16-bit (Y, Y', C~ and P': four roundings of 2^-9 each for bf16) and the
+#   factor images U_a, U_n are 16-bit too. Four to six roundings of 2^-9 add
+#   to about 1e-2 in the worst case; the bound keeps a factor 2 for the
+#   element where the max is taken.
+# - tensor-core path, fp32 gradients: every operand is split into two bf16
+#   parts and three products are kept (relative error near 2^-16 per
+#   product); about eight GEMMs in the chain: ~1e-4 worst case, bound 1e-4.
+UPDATE_TOL = {("generic", "c32h"): 1e-4, ("generic", "c64"): 1e-4, ("generic", "r32"): 1e-4,
+              ("tcgen05", "c32h"): 2e-2, ("tcgen05", "c64"): 1e-4, ("tcgen05", "r32"): 1e-4}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import rank_sparse_tensor_b200 as rst
+    return rst
+
+
+@pytest.fixture(scope="module")
+def orc():
+    import oracle
+    oracle.build()
+    return oracle
+
+
+def update_error(w1, w_ref, w0):
+    a = w1.astype(np.complex128) - w0.astype(np.complex128)
+    b = w_ref.astype(np.complex128) - w0.astype(np.complex128)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
+
+
+def _complexify(a, dtype):
+    if dtype == "c32h":
+        return a[..., 0].astype(np.float64) + 1j * a[..., 1].astype(np.float64)
+    return a.astype(np.complex128)
+
+
+def _step(lib, orc, shape, ranks, rho, gdt, wdt, path, seed=3, wd=0.01, lr=1e-3):
+    from rank_sparse_tensor_b200.synth import GradientStream, weights
+    gs = GradientStream(shape, ranks, gdt, seed, outlier_frac=0.02, outlier_scale=10.0)
+    g0, g1 = to_np(gs.next()), to_np(gs.next())
+    w0 = to_np(weights(shape, wdt, seed))
+    o = orc.Oracle(shape, ranks, rho, 0, lr=lr, wd=wd, grad_dtype=gdt, weight_dtype=wdt,
+                   auto_refresh=0)
+    o.refresh(g0)
+    g = lib.TensorGRaD(shape, ranks, rho, 0, lr=lr, wd=wd, grad_dtype=gdt, weight_dtype=wdt,
+                       auto_refresh=0, path=path)
+    assert g.info["path"] == path
+    mom = random_moments(np.random.default_rng(seed + 4), g.info, True)
+    for key, v in mom.items():
+        o.set_moment(key, v)
+    o.set_counters(2, 1, True)
+    g.set_state(dict(mom, omega=o.omega, U=[o.get_U(n) for n in range(len(shape))], t=2,
+                     refreshes=1, has_subspace=True))
+    w_ref = w0.copy()
+    assert o.step(g1, w_ref) == 0
+    w_dev = torch.from_numpy(w0.copy()).cuda()
+    g.step(torch.from_numpy(g1).cuda(), w_dev)
+    g.sync()
+    return to_np(w_dev), w_ref, w0
+
+
+UPDATE_CASES = {
+    # fp16 gradients, fp32 weights (the tensor-core path and the generic one)
+    "c32h_4way_spb4": ((16, 8, 32, 17), (4, 2, 8, 5), 0.05, "c32h", "c64"),
+    "c32h_4way_spb2": ((24, 16, 64, 33), (6, 4, 13, 7), 0.05, "c32h", "c64"),
+    "c32h_5way": ((4, 6, 8, 32, 17), (2, 3, 4, 8, 5), 0.05, "c32h", "c64"),
+    # fp32 gradients and weights
+    "c64_64x64x32x17": ((64, 64, 32, 17), (16, 16, 8, 5), 0.05, "c64", "c64"),
+    "r32_16x16x8x8": ((16, 16, 8, 8), (4, 4, 2, 2), 0.05, "r32", "r32"),
+}
+
+
+def _paths(lib, shape, ranks, gdt, wdt):
+    out = ["generic"]
+    g = lib.TensorGRaD(shape, ranks, 0.05, 0, grad_dtype=gdt, weight_dtype=wdt)
+    if g.info["path"] != "generic":
+        out.append(g.info["path"])
+    return out
+
+
+@pytest.mark.parametrize("name", list(UPDATE_CASES))
+def test_update_error(lib, orc, name, capsys):
+    shape, ranks, rho, gdt, wdt = UPDATE_CASES[name]
+    for path in _paths(lib, shape, ranks, gdt, wdt):
+        w, w_ref, w0 = _step(lib, orc, shape, ranks, rho, gdt, wdt, path)
+        e = update_error(w, w_ref, w0)
+        tol = UPDATE_TOL[(path, gdt)]
+        with capsys.disabled():
+            print(f"\n[update error] {name} {path}: {e:.3e} (bound {tol:.0e})")
+        assert e <= tol, (path, e)
+
+
+@pytest.mark.parametrize("wl_name,omega_mode", [
+    ("fno4_c32h_128x128x64x33", 0),
+    ("refresh_c64_64x64x32x32x17", 0),
+    ("refresh_c64_64x64x32x32x17", 1),
+])
+def test_full_size_factor_parity(lib, orc, wl_name, omega_mode):
+    """Factors of one device refresh against the oracle's on the full tensor."""
+    from rank_sparse_tensor_b200.synth import WORKLOADS, GradientStream
+    wl = WORKLOADS[wl_name]
+    gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, 6, outlier_frac=wl.outlier_frac,
+                        outlier_scale=wl.outlier_scale, device="cuda")
+    g_dev = gs.next()
+    gpu = lib.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, 0, grad_dtype=wl.dtype,
+                         weight_dtype=wl.weight_dtype, omega_mode=omega_mode, seed=9,
+                         auto_refresh=0)
+    gpu.refresh(g_dev)
+    st = gpu.get_state()
+    o = orc.Oracle(wl.shape, wl.ranks, wl.sparse_ratio, 0, grad_dtype=wl.dtype,
+                   weight_dtype=wl.weight_dtype, omega_mode=omega_mode, seed=9, auto_refresh=0)
+    o.refresh(to_np(g_dev))
+    assert np.array_equal(st["omega"], o.omega)
+    checked = 0
+    for n, (I, r) in enumerate(zip(wl.shape, wl.ranks)):
+        if r == I:
+            continue
+        Uo = o.get_U(n)
+        gap = eigengap(o.eigvals(n), r)
+        d = projector_distance(st["U"][n], Uo)
+        assert np.allclose(st["U"][n].conj().T @ st["U"][n], np.eye(r), atol=1e-5)
+        if gap > 1e-3:
+            assert d <= 1e-3, (n, d, gap)
+            checked += 1
+    assert checked >= 1
