@@ -116,6 +116,18 @@ typedef struct {
                              kernel's first CTA skips the load of its first tile, so one of its
                              bounded waits runs out after wait_limit_ms (failure detection
                              without a fault); the step's results are then undefined */
+  int64_t sparse_k;       /* -1 (default): k = floor(sparse_ratio * N) entries in Omega [S1
+                             section 三]; >= 0: exactly this many (a block of a split tensor
+                             holds its share of the whole tensor's index set) */
+  int64_t mode0_total;    /* 0 (default): the handle holds a whole tensor. > 0: it holds a
+                             contiguous block of rows of mode 0 of a tensor whose mode 0 has
+                             mode0_total entries (shape[0] = the block's rows; ranks[0] may
+                             exceed shape[0]). Mode 0 is projected when ranks[0] < mode0_total,
+                             with U_0 = this block's rows of the whole factor (shape[0] x
+                             ranks[0]). Such a handle steps only through tgd_step_begin /
+                             tgd_step_end with the blocks' partial cores summed in between, and
+                             takes its factors and index set from tgd_set_state (no refresh of
+                             its own: T = 0 or auto_refresh = 0) */
 } tgd_options;
 
 /* Fills `opt` with the defaults listed above. */
@@ -235,6 +247,27 @@ typedef struct {
   float* sparse_m;
   float* sparse_v;
 } tgd_state_view;
+
+/* The step in two halves, for one tensor split across GPUs along mode 0
+ *  (each GPU holds a block of rows; see tgd_options.mode0_total). The mode-0
+ *  product of the projection is a sum over mode 0's rows [S2 Appendix K: the
+ *  mode-n product sums over i_n], so each block's projection is a partial
+ *  core and the whole core is their sum; the core AdamW, the expansion with
+ *  the block's rows of U_0, the sparse part and the weight update are local.
+ *  - tgd_step_begin: refresh when due (whole tensors only), the sparse AdamW
+ *    and the projection of this block into the handle's core buffer.
+ *  - tgd_core_buffer: the core buffer's device address and its length in
+ *    floats (fp32; (re, im) pairs for complex tensors, in the kernel path's
+ *    own element order, the same on every block of one configuration). The
+ *    caller sums the blocks' buffers elementwise in place on every block
+ *    (for example with an all-reduce over the GPUs, ordered on `stream`).
+ *  - tgd_step_end: the core AdamW on the summed core, the expansion, the
+ *    scatter-add of the sparse update and the weight update; t advances.
+ *  tgd_step equals begin + end on a whole tensor. Out of order calls return
+ *  TGD_ERR_STATE; the low-rank-first order has no split (UNSUPPORTED). */
+TGD_API tgd_status tgd_step_begin(tgd_handle h, const void* grad, void* stream);
+TGD_API tgd_status tgd_core_buffer(tgd_handle h, float** core, int64_t* count);
+TGD_API tgd_status tgd_step_end(tgd_handle h, void* weight, void* stream);
 
 /* Copies the state to host buffers. Synchronises `stream`. */
 TGD_API tgd_status tgd_get_state(tgd_handle h, tgd_state_view* out, void* stream);

@@ -31,6 +31,20 @@ def _stream_ptr(stream) -> Optional[int]:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+class _DeviceMemory:
+    """A float32 device buffer described for torch.as_tensor (no copy)."""
+
+    def __init__(self, ptr: int, count: int):
+        self.__cuda_array_interface__ = {"shape": (count,), "typestr": "<f4",
+                                         "data": (ptr, False), "version": 2}
+
+
+def _device_view(ptr: int, count: int, dtype):
+    import torch
+    assert dtype == torch.float32
+    return torch.as_tensor(_DeviceMemory(ptr, count), device="cuda")
+
+
 def _check_tensor(t, dtype: str, n: int, what: str):
     import torch
     if not isinstance(t, torch.Tensor):
@@ -55,7 +69,8 @@ class TensorGRaD:
                  omega_mode: int = 0, seed: int = 0, sparse_scale: float = 1.0,
                  complex_adam: int = 0, moments_on_refresh: int = 0, auto_refresh: int = 1,
                  path: str = "auto", sm_budget: int = 0, order: int = 0, basis: int = 0,
-                 wait_limit_ms: int = 0, test_stall: int = 0):
+                 wait_limit_ms: int = 0, test_stall: int = 0, sparse_k: int = -1,
+                 mode0_total: int = 0):
         weight_dtype = weight_dtype or grad_dtype
         self.shape = tuple(int(s) for s in shape)
         self.ranks = tuple(int(r) for r in ranks)
@@ -71,6 +86,8 @@ class TensorGRaD:
         opt.basis = basis
         opt.wait_limit_ms = wait_limit_ms
         opt.test_stall = test_stall
+        opt.sparse_k = sparse_k
+        opt.mode0_total = mode0_total
         sh = (C.c_int64 * len(self.shape))(*self.shape)
         rk = (C.c_int64 * len(self.ranks))(*self.ranks)
         h = C.c_void_p()
@@ -101,6 +118,30 @@ class TensorGRaD:
     def refresh(self, grad, stream=None):
         _check_tensor(grad, self.grad_dtype, self.N, "grad")
         check(lib().tgd_refresh(self._h, grad.data_ptr(), _stream_ptr(stream)), self._h)
+
+    # -------------------------------------------- the step in two halves
+    def step_begin(self, grad, stream=None):
+        """Sparse AdamW and the projection into the core buffer."""
+        _check_tensor(grad, self.grad_dtype, self.N, "grad")
+        check(lib().tgd_step_begin(self._h, grad.data_ptr(), _stream_ptr(stream)), self._h)
+
+    def core_buffer(self):
+        """(device address, float count) of the core between the halves."""
+        ptr, cnt = C.c_void_p(), C.c_int64()
+        check(lib().tgd_core_buffer(self._h, C.byref(ptr), C.byref(cnt)), self._h)
+        return int(ptr.value or 0), int(cnt.value)
+
+    def core_tensor(self):
+        """The core buffer as a torch float32 tensor viewing the device
+        memory (valid until step_end), for summing partial cores."""
+        import torch
+        ptr, cnt = self.core_buffer()
+        return _device_view(ptr, cnt, torch.float32)
+
+    def step_end(self, weight, stream=None):
+        """Core AdamW on the (summed) core, expansion and weight update."""
+        _check_tensor(weight, self.weight_dtype, self.N, "weight")
+        check(lib().tgd_step_end(self._h, weight.data_ptr(), _stream_ptr(stream)), self._h)
 
     def step_host(self, grad_host: np.ndarray, weight_host: np.ndarray, stream=None):
         """Host buffers in, host weights out (copies inside the call)."""

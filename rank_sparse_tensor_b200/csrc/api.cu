@@ -33,6 +33,10 @@ struct tgd_ctx {
   int64_t T = 0;
   tgd_options opt{};
   int path = TGD_PATH_GENERIC;
+  uint32_t proj = 0;          // bit n: mode n is projected
+  int64_t mode0_total = 0;    // > 0: this handle holds a block of rows of mode 0
+  bool pending = false;       // tgd_step_begin has run, tgd_step_end has not
+  float* core_ptr = nullptr;  // the core buffer of the step in progress (generic path)
   int64_t t = 0, refreshes = 0;
   bool has_subspace = false;
   int device = 0;
@@ -206,7 +210,7 @@ AdamConst adam_const(const tgd_ctx* h, double scale) {
   return a;
 }
 
-bool mode_active(const tgd_ctx* h, int n) { return h->r[n] < h->I[n]; }
+bool mode_active(const tgd_ctx* h, int n) { return ((h->proj >> n) & 1u) != 0; }
 
 // Derived device data that depends on Omega and U: the Omega bitmask, the
 // coefficient matrices of the generic path and the tensor-core operands.
@@ -226,14 +230,18 @@ tgd_status rebuild_derived(tgd_ctx* h, cudaStream_t s) {
 // The fp32 tensor-core step: sparse AdamW into lambda S~, the projection
 // chain into the core, core AdamW in place, the expansion chain whose last
 // product updates the weights with lambda S~ added on Omega.
-tgd_status step_tc32(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
+tgd_status tc32_begin(tgd_ctx* h, const void* g, cudaStream_t s) {
   AdamConst asp = adam_const(h, h->opt.sparse_scale);
-  AdamConst acore = adam_const(h, 1.0);
   {
     TIMED(h, s, "sparse_adam");
     TGD_CUDA(h, sparse_adam(g, h->gdt, h->omega, h->k, h->sp_m, h->sp_v, asp, tc32_sparse_update(h->tc32), s));
   }
   TGD_CUDA(h, tc32_project(h->tc32, g, h->bits, h->d_err, s, timer_hook, h));
+  return TGD_OK;
+}
+
+tgd_status tc32_end(tgd_ctx* h, void* w, cudaStream_t s) {
+  AdamConst acore = adam_const(h, 1.0);
   {
     TIMED(h, s, "core_adam");
     TGD_CUDA(h, core_adam(tc32_core(h->tc32), h->ncore, h->core_m, h->core_v, acore, s));
@@ -432,9 +440,10 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
   return TGD_OK;
 }
 
-tgd_status step_generic(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
+// The generic step, first half: sparse AdamW, then the projection chain; the
+// core is left in h->core_ptr.
+tgd_status generic_begin(tgd_ctx* h, const void* g, cudaStream_t s) {
   AdamConst asp = adam_const(h, h->opt.sparse_scale);
-  AdamConst acore = adam_const(h, 1.0);
   {
     TIMED(h, s, "sparse_adam");
     TGD_CUDA(h, sparse_adam(g, h->gdt, h->omega, h->k, h->sp_m, h->sp_v, asp, h->sp_upd, s));
@@ -462,10 +471,22 @@ tgd_status step_generic(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
     TGD_CUDA(h, masked_copy(g, h->gdt, h->bits, h->N, h->bufA, s));
     cur = h->bufA;
   }
+  h->core_ptr = cur;
+  return TGD_OK;
+}
+
+// Second half: core AdamW, the expansion chain, the scatter of lambda S~ and
+// the weight update.
+tgd_status generic_end(tgd_ctx* h, void* w, cudaStream_t s) {
+  AdamConst acore = adam_const(h, 1.0);
+  float* cur = h->core_ptr;
+  auto other = [&](float* c) { return c == h->bufA ? h->bufB : h->bufA; };
   {
     TIMED(h, s, "core_adam");
     TGD_CUDA(h, core_adam(cur, h->ncore, h->core_m, h->core_v, acore, s));
   }
+  int64_t dims[TGD_MAX_NDIM];
+  for (int n = 0; n < h->d; ++n) dims[n] = mode_active(h, n) ? h->r[n] : h->I[n];
   for (int n = 0; n < h->d; ++n) {
     if (!mode_active(h, n)) continue;
     int64_t A = 1, B = 1;
@@ -485,6 +506,46 @@ tgd_status step_generic(tgd_ctx* h, const void* g, void* w, cudaStream_t s) {
   TIMED(h, s, "weight_update");
   TGD_CUDA(h, weight_update(w, h->wdt, cur, h->N, decay, h->lr, s));
   return TGD_OK;
+}
+
+// The two halves on the handle's kernel path.
+tgd_status step_begin(tgd_ctx* h, const void* g, cudaStream_t s) {
+  tgd_status st = TGD_OK;
+  if (h->path == TGD_PATH_GENERIC) {
+    st = generic_begin(h, g, s);
+  } else if (h->use_tc32) {
+    st = tc32_begin(h, g, s);
+  } else {
+    AdamConst asp = adam_const(h, h->opt.sparse_scale);
+    cudaError_t e = tc_step_project(h->tc, g, h->sp_m, h->sp_v, asp, h->d_err, s, timer_hook, h);
+    if (e != cudaSuccess) st = cuda_fail(h, e, "tensor-core projection");
+  }
+  if (st == TGD_OK) h->pending = true;
+  return st;
+}
+
+tgd_status step_end(tgd_ctx* h, void* w, cudaStream_t s) {
+  tgd_status st = TGD_OK;
+  if (h->path == TGD_PATH_GENERIC) {
+    st = generic_end(h, w, s);
+  } else if (h->use_tc32) {
+    st = tc32_end(h, w, s);
+  } else {
+    AdamConst acore = adam_const(h, 1.0);
+    float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
+    cudaError_t e = tc_step_finish(h->tc, w, h->core_m, h->core_v, acore, decay, h->lr, h->d_err, s, timer_hook, h);
+    if (e != cudaSuccess) st = cuda_fail(h, e, "tensor-core reconstruction");
+  }
+  if (st != TGD_OK) return st;
+  h->pending = false;
+  h->t += 1;
+  return TGD_OK;
+}
+
+// The core buffer between the halves: device pointer and float count.
+float* core_buffer(tgd_ctx* h) {
+  if (h->path == TGD_PATH_GENERIC) return h->core_ptr;
+  return h->use_tc32 ? tc32_core(h->tc32) : tc_core(h->tc);
 }
 
 tgd_status check_device_error(tgd_ctx* h, cudaStream_t s, bool wait) {
@@ -526,6 +587,8 @@ void tgd_default_options(tgd_options* opt) {
   opt->basis = 0;
   opt->wait_limit_ms = 0;
   opt->test_stall = 0;
+  opt->sparse_k = -1;
+  opt->mode0_total = 0;
 }
 
 tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int64_t* ranks,
@@ -552,20 +615,31 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (o.omega_mode < 0 || o.omega_mode > 1 || o.complex_adam < 0 || o.complex_adam > 1 ||
       o.moments_on_refresh < 0 || o.moments_on_refresh > 1 || o.path < 0 || o.path > 2 ||
       o.sm_budget < 0 || !std::isfinite(o.sparse_scale) || o.order < 0 || o.order > 1 ||
-      o.basis < 0 || o.basis > 1 || o.wait_limit_ms < 0 || o.test_stall < 0 || o.test_stall > 1)
+      o.basis < 0 || o.basis > 1 || o.wait_limit_ms < 0 || o.test_stall < 0 || o.test_stall > 1 ||
+      o.sparse_k < -1 || o.mode0_total < 0)
     return fail(nullptr, TGD_ERR_INVALID_ARG, "bad option value");
+  if (o.mode0_total > 0 && (o.order != 0 || (o.auto_refresh && T > 0)))
+    return fail(nullptr, TGD_ERR_INVALID_ARG,
+                "a block of mode-0 rows takes its factors and index set from tgd_set_state: "
+                "set T = 0 or auto_refresh = 0, and the sparse-first order");
   if (o.order == 1 && o.path == TGD_PATH_TCGEN05)
     return fail(nullptr, TGD_ERR_UNSUPPORTED, "the low-rank-first order runs on the CUDA-core path");
   int64_t N = 1, ncore = 1;
+  uint32_t proj = 0;
   for (int n = 0; n < ndim; ++n) {
-    if (shape[n] < 1 || ranks[n] < 1 || ranks[n] > shape[n])
-      return fail(nullptr, TGD_ERR_INVALID_ARG, "need 1 <= ranks[n] <= shape[n]");
-    if (shape[n] > 256 && ranks[n] < shape[n])
+    // a block of mode-0 rows: the mode's full size is mode0_total
+    const int64_t full = (n == 0 && o.mode0_total > 0) ? o.mode0_total : shape[n];
+    if (shape[n] < 1 || ranks[n] < 1 || ranks[n] > full || shape[n] > full)
+      return fail(nullptr, TGD_ERR_INVALID_ARG, "need 1 <= ranks[n] <= shape[n] (mode 0 of a block: "
+                                                "ranks[0], shape[0] <= mode0_total)");
+    if (full > 256 && ranks[n] < full)
       return fail(nullptr, TGD_ERR_UNSUPPORTED, "projected modes are limited to 256 entries");
     if (N > ((int64_t)1 << 40) / shape[n]) return fail(nullptr, TGD_ERR_INVALID_ARG, "tensor too large");
+    if (ranks[n] < full) proj |= 1u << n;
     N *= shape[n];
     ncore *= ranks[n];
   }
+  if (o.sparse_k > N) return fail(nullptr, TGD_ERR_INVALID_ARG, "sparse_k exceeds the element count");
   tgd_ctx* h = new (std::nothrow) tgd_ctx;
   if (!h) return fail(nullptr, TGD_ERR_OOM, "host allocation failed");
   h->d = ndim;
@@ -576,7 +650,9 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   h->N = N;
   h->ncore = ncore;
   h->rho = sparse_ratio;
-  h->k = (int64_t)std::floor(sparse_ratio * (double)N);
+  h->k = o.sparse_k >= 0 ? o.sparse_k : (int64_t)std::floor(sparse_ratio * (double)N);
+  h->proj = proj;
+  h->mode0_total = o.mode0_total;
   h->T = T;
   h->lr = lr;
   h->b1 = beta1;
@@ -591,8 +667,8 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   h->vc = (h->cplx && o.complex_adam == 1) ? 2 : 1;
   // Path: the tensor-core kernels need complex fp16 gradients and tiles that
   // fit the trailing two modes.
-  const bool tc16_ok = tc_supported(ndim, shape, ranks, grad_dtype, weight_dtype);
-  const bool tc32_ok = tc32_supported(ndim, shape, ranks, grad_dtype, weight_dtype);
+  const bool tc16_ok = tc_supported(ndim, shape, ranks, proj, grad_dtype, weight_dtype);
+  const bool tc32_ok = tc32_supported(ndim, shape, ranks, proj, grad_dtype, weight_dtype);
   const bool tc_ok = tc16_ok || tc32_ok;
   if (o.path == TGD_PATH_TCGEN05 && !tc_ok) {
     delete h;
@@ -622,7 +698,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   ok &= dalloc(h, &h->sel_ws, select_workspace_bytes(N));
   size_t gp = 0;
   for (int n = 0; n < ndim; ++n)
-    if (ranks[n] < shape[n]) {
+    if (ranks[n] < shape[n] && o.mode0_total == 0) {
       gp = std::max(gp, gram_partial_bytes(ndim, shape, n));
       ok &= dalloc_t(h, &h->gram[n], (size_t)shape[n] * shape[n] * 2);
       ok &= dalloc_t(h, &h->evals[n], (size_t)shape[n]);
@@ -633,7 +709,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   ok &= dalloc_t(h, &h->d_err, 1);
   if (ok && h->path == TGD_PATH_GENERIC) {
     for (int n = 0; n < ndim; ++n)
-      if (ranks[n] < shape[n]) {
+      if ((proj >> n) & 1u) {
         ok &= dalloc_t(h, &h->P[n], (size_t)shape[n] * ranks[n] * h->mc);
         ok &= dalloc_t(h, &h->E[n], (size_t)shape[n] * ranks[n] * h->mc);
       }
@@ -644,14 +720,14 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   }
   if (ok && h->use_tc32) {
     auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
-    ok &= tc32_plan(h->tc32, ndim, shape, ranks, h->k, grad_dtype, alloc_fn, h);
+    ok &= tc32_plan(h->tc32, ndim, shape, ranks, proj, h->k, grad_dtype, alloc_fn, h);
   }
   if (ok && h->path == TGD_PATH_TCGEN05 && !h->use_tc32) {
     auto alloc_fn = [](void* ctx, void** p, size_t b) { return dalloc((tgd_ctx*)ctx, p, b); };
     h->tc.sm_budget = o.sm_budget;
     h->tc.wait_ns = (uint64_t)o.wait_limit_ms * 1000000ull;
     h->tc.skip_first_copy = o.test_stall;
-    ok &= tc_plan(h->tc, ndim, shape, ranks, h->k, grad_dtype, weight_dtype, alloc_fn, h);
+    ok &= tc_plan(h->tc, ndim, shape, ranks, proj, h->k, grad_dtype, weight_dtype, alloc_fn, h);
   }
   if (!ok) {
     free_all(h);
@@ -667,7 +743,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
   if (e == cudaSuccess) e = cudaMemsetAsync(h->omega, 0, sizeof(int64_t) * std::max<int64_t>(h->k, 1), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->d_err, 0, sizeof(int), s);
   for (int n = 0; n < ndim && e == cudaSuccess; ++n) {
-    if (ranks[n] == shape[n]) {
+    if (!((proj >> n) & 1u)) {
       identity_kernel<<<(unsigned)std::min<int64_t>(ceil_div(shape[n] * shape[n], 256), 1024), 256, 0, s>>>(
           (float2*)h->U[n], shape[n]);
       e = cudaGetLastError();
@@ -688,6 +764,10 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
 tgd_status tgd_refresh(tgd_handle h, const void* grad, void* stream) {
   if (!h) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL handle");
   if (!grad) return fail(h, TGD_ERR_INVALID_ARG, "grad is NULL");
+  if (h->mode0_total > 0)
+    return fail(h, TGD_ERR_UNSUPPORTED, "a block of mode-0 rows is not refreshed on its own: set its "
+                                        "factors and index set with tgd_set_state");
+  if (h->pending) return fail(h, TGD_ERR_STATE, "tgd_step_begin is waiting for tgd_step_end");
   return do_refresh(h, grad, (cudaStream_t)stream);
 }
 
@@ -695,27 +775,54 @@ tgd_status tgd_step(tgd_handle h, const void* grad, void* weight, void* stream) 
   if (!h) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL handle");
   if (!grad || !weight) return fail(h, TGD_ERR_INVALID_ARG, "grad or weight is NULL");
   cudaStream_t s = (cudaStream_t)stream;
+  if (h->pending) return fail(h, TGD_ERR_STATE, "tgd_step_begin is waiting for tgd_step_end");
+  if (h->mode0_total > 0)
+    return fail(h, TGD_ERR_STATE, "a block of mode-0 rows steps with tgd_step_begin, a sum of the "
+                                  "blocks' cores, and tgd_step_end");
   if (h->opt.auto_refresh && h->T > 0 && h->t % h->T == 0) {
     tgd_status st = do_refresh(h, grad, s);
     if (st != TGD_OK) return st;
   }
   if (!h->has_subspace) return fail(h, TGD_ERR_STATE, "no refresh has run: call tgd_refresh first");
-  tgd_status st;
-  if (h->path == TGD_PATH_GENERIC) {
-    st = h->opt.order == 1 ? step_lowrank_first(h, grad, weight, s) : step_generic(h, grad, weight, s);
-  } else if (h->use_tc32) {
-    st = step_tc32(h, grad, weight, s);
-  } else {
-    AdamConst asp = adam_const(h, h->opt.sparse_scale);
-    AdamConst acore = adam_const(h, 1.0);
-    float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
-    cudaError_t e = tc_step(h->tc, grad, weight, h->sp_m, h->sp_v, h->core_m, h->core_v, asp, acore,
-                            decay, h->lr, h->d_err, s, timer_hook, h);
-    st = e == cudaSuccess ? TGD_OK : cuda_fail(h, e, "tensor-core step");
+  if (h->opt.order == 1) {
+    tgd_status st = step_lowrank_first(h, grad, weight, s);
+    if (st != TGD_OK) return st;
+    h->t += 1;
+    return TGD_OK;
   }
+  tgd_status st = step_begin(h, grad, s);
   if (st != TGD_OK) return st;
-  h->t += 1;
+  return step_end(h, weight, s);
+}
+
+tgd_status tgd_step_begin(tgd_handle h, const void* grad, void* stream) {
+  if (!h) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL handle");
+  if (!grad) return fail(h, TGD_ERR_INVALID_ARG, "grad is NULL");
+  if (h->pending) return fail(h, TGD_ERR_STATE, "tgd_step_begin is waiting for tgd_step_end");
+  if (h->opt.order == 1)
+    return fail(h, TGD_ERR_UNSUPPORTED, "the low-rank-first order has no split step");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (h->mode0_total == 0 && h->opt.auto_refresh && h->T > 0 && h->t % h->T == 0) {
+    tgd_status st = do_refresh(h, grad, s);
+    if (st != TGD_OK) return st;
+  }
+  if (!h->has_subspace) return fail(h, TGD_ERR_STATE, "no refresh has run: call tgd_refresh first");
+  return step_begin(h, grad, s);
+}
+
+tgd_status tgd_core_buffer(tgd_handle h, float** core, int64_t* count) {
+  if (!h || !core || !count) return fail(h, TGD_ERR_INVALID_ARG, "NULL argument");
+  if (!h->pending) return fail(h, TGD_ERR_STATE, "no tgd_step_begin is waiting for tgd_step_end");
+  *core = core_buffer(h);
+  *count = h->ncore * h->mc;
   return TGD_OK;
+}
+
+tgd_status tgd_step_end(tgd_handle h, void* weight, void* stream) {
+  if (!h) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL handle");
+  if (!weight) return fail(h, TGD_ERR_INVALID_ARG, "weight is NULL");
+  if (!h->pending) return fail(h, TGD_ERR_STATE, "tgd_step_end without tgd_step_begin");
+  return step_end(h, weight, (cudaStream_t)stream);
 }
 
 tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host, void* stream) {

@@ -1339,7 +1339,7 @@ size_t r3_smem_bytes(int Ib, int spb, int64_t yp_bs, int wbytes, int nstage, int
 constexpr size_t SMEM_LIMIT = 227 * 1024 - 1024;
 constexpr size_t ONE_CTA_SMEM = 120 * 1024;
 
-bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int wdt) {
+bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int wdt) {
   if (nd < 3) return false;
   g.d = nd;
   g.Ia = (int)shape[nd - 2];
@@ -1405,7 +1405,7 @@ bool geometry(TcImpl& g, int nd, const int64_t* shape, const int64_t* ranks, int
     m.n = n;
     m.I = shape[n];
     m.r = ranks[n];
-    m.active = ranks[n] < shape[n];
+    m.active = ((proj_mask >> n) & 1u) != 0;
     int Np = r16(2 * (int)m.r), Kp = (int)ceil_div(2 * m.I, 64) * 64;
     m.NTp = Np <= 256 ? Np : 256;
     m.nntp = (int)ceil_div(Np, m.NTp);
@@ -1458,16 +1458,16 @@ cudaError_t launch_mode_gemm(const uint32_t* X, int64_t A, int64_t K, int64_t B,
 
 }  // namespace
 
-bool tc_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt) {
+bool tc_supported(int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int gdt, int wdt) {
   if (gdt != TGD_C32H || (wdt != TGD_C32H && wdt != TGD_C64)) return false;
   TcImpl g;
-  return geometry(g, nd, shape, ranks, wdt);
+  return geometry(g, nd, shape, ranks, proj_mask, wdt);
 }
 
-bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
-             int wdt, AllocFn alloc, void* ctx) {
+bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int64_t k,
+             int gdt, int wdt, AllocFn alloc, void* ctx) {
   TcImpl* g = new TcImpl;
-  if (!geometry(*g, nd, shape, ranks, wdt)) {
+  if (!geometry(*g, nd, shape, ranks, proj_mask, wdt)) {
     delete g;
     return false;
   }
@@ -1563,21 +1563,30 @@ cudaError_t tc_rebuild(TcPlan& p, const int64_t* omega, int64_t k, const float* 
   return cudaGetLastError();
 }
 
+float* tc_core(TcPlan& p) {
+  TcImpl* g = impl_of(p);
+  return g ? g->C : nullptr;
+}
+
 cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp_v, float* core_m,
                     float* core_v, const AdamConst& asp, const AdamConst& acore, float decay, float lr,
                     int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx) {
+  cudaError_t e = tc_step_project(p, grad, sp_m, sp_v, asp, d_err, s, hook, hook_ctx);
+  if (e != cudaSuccess) return e;
+  return tc_step_finish(p, w, core_m, core_v, acore, decay, lr, d_err, s, hook, hook_ctx);
+}
+
+cudaError_t tc_step_project(TcPlan& p, const void* grad, float* sp_m, float* sp_v, const AdamConst& asp,
+                            int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx) {
   TcImpl* g = impl_of(p);
   if (!g) return cudaErrorNotReady;
   auto H = [&](int ph, const char* name) {
     if (hook) hook(hook_ctx, ph, name, s);
   };
   const int d = p.d;
-  int last_active = -1, first_active = -1;
+  int first_active = -1;
   for (int n = 0; n < d - 2; ++n)
-    if (g->inner[n].active) {
-      if (first_active < 0) first_active = n;
-      last_active = n;
-    }
+    if (g->inner[n].active && first_active < 0) first_active = n;
   // ---- projection stream over G
   P1Args& a = g->p1;
   p1_smem_bytes(g->Ib, g->p1_nstage, g->K2, g->K1, g->N1, g->N2, (uint32_t)(g->a2_rows / 8) * 128 + 16, &a);
@@ -1664,6 +1673,31 @@ cudaError_t tc_step(TcPlan& p, const void* grad, void* w, float* sp_m, float* sp
       which ^= 1;
     }
   }
+  return cudaSuccess;
+}
+
+cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, const AdamConst& acore,
+                           float decay, float lr, int* d_err, cudaStream_t s, TimerHook hook,
+                           void* hook_ctx) {
+  TcImpl* g = impl_of(p);
+  if (!g) return cudaErrorNotReady;
+  auto H = [&](int ph, const char* name) {
+    if (hook) hook(hook_ctx, ph, name, s);
+  };
+  const int d = p.d;
+  int last_active = -1, first_active = -1;
+  for (int n = 0; n < d - 2; ++n)
+    if (g->inner[n].active) {
+      if (first_active < 0) first_active = n;
+      last_active = n;
+    }
+  const bool no_inner = first_active < 0;
+  int64_t dims[8];
+  for (int n = 0; n < d - 2; ++n) dims[n] = g->inner[n].active ? p.r[n] : p.I[n];
+  const uint32_t* cur = nullptr;
+  uint32_t* bufs[2] = {g->X0, g->X1};
+  int which = 0;
+  cudaError_t e = cudaSuccess;
   // ---- Adam on the core; C~ (bf16) feeds the expansion chain, or Y' directly
   {
     const bool direct = no_inner;

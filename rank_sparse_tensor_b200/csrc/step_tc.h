@@ -25,15 +25,26 @@ struct TcPlan {
   void* impl = nullptr;  // owned by step_tc.cu (host-side description)
 };
 
-bool tc_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt);
-bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
-             int wdt, AllocFn alloc, void* ctx);
+// proj_mask: bit n set = mode n is projected (normally ranks[n] < shape[n];
+// a mode-0 shard of a split tensor is projected even when r_0 >= its rows).
+bool tc_supported(int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int gdt, int wdt);
+bool tc_plan(TcPlan& p, int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int64_t k,
+             int gdt, int wdt, AllocFn alloc, void* ctx);
 void tc_release(TcPlan& p);
 cudaError_t tc_rebuild(TcPlan& p, const int64_t* omega, int64_t k, const float* const* U,
                        cudaStream_t s);
 cudaError_t tc_step(TcPlan& p, const void* g, void* w, float* sp_m, float* sp_v, float* core_m,
                     float* core_v, const AdamConst& asp, const AdamConst& acore, float decay,
                     float lr, int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx);
+// The step in two halves: the sparse AdamW and the projection into the core
+// buffer (tc_core, fp32 (re, im) pairs in this path's layout), then the core
+// AdamW, the expansion and the weight update.
+cudaError_t tc_step_project(TcPlan& p, const void* grad, float* sp_m, float* sp_v, const AdamConst& asp,
+                            int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx);
+cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, const AdamConst& acore,
+                           float decay, float lr, int* d_err, cudaStream_t s, TimerHook hook,
+                           void* hook_ctx);
+float* tc_core(TcPlan& p);
 // Core moments are stored in the path's internal layout; these convert
 // to/from the canonical row-major r_1 x ... x r_d layout (host buffers).
 cudaError_t tc_core_to_canonical(const TcPlan& p, const float* dev, int comps, float* host_out);

@@ -372,20 +372,20 @@ cudaError_t launch_mode32(bool cplx, bool wupd, const MG32Args& a, int nnt, cuda
 
 }  // namespace
 
-bool tc32_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt) {
+bool tc32_supported(int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int gdt, int wdt) {
   if (!((gdt == TGD_C64 && wdt == TGD_C64) || (gdt == TGD_R32 && wdt == TGD_R32))) return false;
   bool any = false;
   for (int n = 0; n < nd; ++n) {
-    if (ranks[n] < shape[n]) {
+    if ((proj_mask >> n) & 1u) {
       any = true;
-      if (shape[n] > 256) return false;
+      if (shape[n] > 256 || ranks[n] > 256) return false;
     }
   }
   return any;
 }
 
-bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
-               AllocFn alloc, void* ctx) {
+bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int64_t k,
+               int gdt, AllocFn alloc, void* ctx) {
   Tc32Impl* g = new Tc32Impl;
   p.impl = g;
   g->d = nd;
@@ -409,7 +409,7 @@ bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, 
   int64_t maxe = 1, cur = g->N;
   int first = -1;
   for (int n = nd - 1; n >= 0; --n) {
-    if (ranks[n] == shape[n]) continue;
+    if (!((proj_mask >> n) & 1u)) continue;
     if (first < 0) first = n;
     cur = cur / shape[n] * ranks[n];
     maxe = std::max(maxe, cur);
@@ -420,7 +420,7 @@ bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, 
     m.n = n;
     m.I = shape[n];
     m.r = ranks[n];
-    m.active = ranks[n] < shape[n];
+    m.active = ((proj_mask >> n) & 1u) != 0;
     if (m.active) {
       mode_geom(m.I, m.r, g->cplx, m.NTp, m.nntp, m.nkcp);
       mode_geom(m.r, m.I, g->cplx, m.NTe, m.nnte, m.nkce);

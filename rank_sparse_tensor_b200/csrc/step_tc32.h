@@ -16,9 +16,10 @@ struct Tc32Plan {
 
 // fp32 gradients and weights of one kind (both real or both complex), at least
 // one projected mode, projected modes of at most 256 entries.
-bool tc32_supported(int nd, const int64_t* shape, const int64_t* ranks, int gdt, int wdt);
-bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, int64_t k, int gdt,
-               AllocFn alloc, void* ctx);
+// proj_mask: bit n set = mode n is projected (see tc_supported).
+bool tc32_supported(int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int gdt, int wdt);
+bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, uint32_t proj_mask, int64_t k,
+               int gdt, AllocFn alloc, void* ctx);
 void tc32_release(Tc32Plan& p);
 // Omega's per-word ranks and the factor images (after every refresh).
 cudaError_t tc32_rebuild(Tc32Plan& p, const int64_t* omega, int64_t k, const float* const* U,

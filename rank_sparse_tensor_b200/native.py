@@ -35,7 +35,7 @@ class Options(C.Structure):
                 ("complex_adam", C.c_int), ("moments_on_refresh", C.c_int),
                 ("auto_refresh", C.c_int), ("path", C.c_int), ("sm_budget", C.c_int),
                 ("order", C.c_int), ("basis", C.c_int), ("wait_limit_ms", C.c_int),
-                ("test_stall", C.c_int)]
+                ("test_stall", C.c_int), ("sparse_k", C.c_int64), ("mode0_total", C.c_int64)]
 
 
 class Info(C.Structure):
@@ -78,6 +78,9 @@ SIGNATURES = {
     "tgd_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "tgd_refresh": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "tgd_step_host": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "tgd_step_begin": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "tgd_core_buffer": (C.c_int, [C.c_void_p, C.POINTER(C.c_void_p), C.POINTER(C.c_int64)]),
+    "tgd_step_end": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "tgd_sync": (C.c_int, [C.c_void_p, C.c_void_p]),
     "tgd_destroy": (C.c_int, [C.c_void_p]),
     "tgd_query": (C.c_int, [C.c_void_p, C.POINTER(Info)]),
