@@ -11,6 +11,11 @@ already resident in HBM. The default workload is the large complex fp16
 spectral tensor (256, 256, 128, 65) with ranks (64, 64, 32, 16), 5% top-k
 sparse, factors and index set fixed after one untimed refresh.
 
+The default run also records the other workloads at their full step counts
+under "workloads" (the 4-tensor mixed-precision set, the complex64 FNO
+tensor, the 5-way refresh tensor and the small real tensor), each with its
+time per step, roofline fraction, kernel times and clocks.
+
 Multi-GPU (torchrun, one rank per GPU): every rank steps its own tensor
 (independent problems, no data-path collective), value = elements of all
 ranks / the slowest rank's time (weak scaling).
@@ -89,6 +94,8 @@ def kernel_algorithmic_bytes(name: str, wl) -> float:
         "proj_stream": a["grad"] + 8 * wl.k,
         "sparse_adam": moments,
         "recon_stream": a["weight"],
+        # fp32 tensor-core path: the last expansion updates W in place
+        "expand_update32": a["weight"],
         # CUDA-core path
         "weight_update": a["weight"],
         "mode_product": a["grad"],
@@ -288,6 +295,178 @@ def job_throughput(world: int, elems_per_rank: int, steps: int, max_ms: float) -
     return world * elems_per_rank * steps / (max_ms / 1e3)
 
 
+def step_roofline(wl, n_tensors, step_ms, hbm_gbs):
+    """Algorithmic bytes of one step over every tensor, and the fraction of
+    the HBM roofline the step time reaches."""
+    ab = algorithmic_bytes(wl)["total"] * n_tensors
+    gbs = ab / (step_ms / 1e3) / 1e9
+    return {"step_algorithmic_bytes": ab, "step_achieved_gbs": gbs, "step_frac": gbs / hbm_gbs}
+
+
+class Bench:
+    """One rank's tensors of one workload, resident in HBM, and their timing."""
+
+    def __init__(self, wl, args, dev, rank, concurrent_default=True):
+        import torch
+        import rank_sparse_tensor_b200 as rst
+        from rank_sparse_tensor_b200.synth import GradientStream, weights
+        self.wl, self.args, self.dev = wl, args, dev
+        nt = wl.n_tensors
+        self.concurrent = nt > 1 and not args.sequential and concurrent_default
+        n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sm_budget = max(1, n_sms // nt) if self.concurrent else 0
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(nt)] if self.concurrent else None
+        self.tensors = []
+        for gseed, wseed in tensor_seeds(rank, nt):
+            gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=gseed,
+                                outlier_frac=wl.outlier_frac, outlier_scale=wl.outlier_scale,
+                                noise=wl.noise, drift=0.0, device=str(dev))
+            grads = [gs.next() for _ in range(2)]
+            w = weights(wl.shape, wl.weight_dtype, seed=wseed, device=str(dev))
+            opt = rst.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, wl.T, wl.lr, wl.betas, wl.eps,
+                                 wl.wd, wl.dtype, wl.weight_dtype, path=args.path, sm_budget=sm_budget)
+            if wl.T == 0:
+                opt.refresh(grads[0])
+            self.tensors.append((opt, grads, w))
+        torch.cuda.synchronize()
+        in_bytes = sum(g[0].numel() * g[0].element_size() + w.numel() * w.element_size()
+                       for _, g, w in self.tensors)
+        self.flush = in_bytes < 2 * L2_BYTES
+        self.scratch = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if self.flush else None
+
+    def one_step(self, i):
+        import torch
+        if self.streams is None:
+            for opt, grads, w in self.tensors:
+                opt.step(grads[i % 2], w)
+            return
+        # each tensor on its own stream, forked from and joined back into the
+        # timed stream
+        main = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        for (opt, grads, w), st in zip(self.tensors, self.streams):
+            st.wait_event(fork)
+            with torch.cuda.stream(st):
+                opt.step(grads[i % 2], w)
+        for st in self.streams:
+            join = torch.cuda.Event()
+            join.record(st)
+            main.wait_event(join)
+
+    def timed_steps(self, steps, profile, barrier):
+        """`steps` steps between barriers, each bracketed by CUDA events on
+        the launching stream (L2 flushed between steps when inputs fit in
+        it). Returns (total ms, {kernel: [launches, ms]})."""
+        import torch
+        stream = torch.cuda.current_stream()
+        for opt, _, _ in self.tensors:
+            opt.profile(profile)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            evs[i][0].record(stream)
+            self.one_step(i)
+            evs[i][1].record(stream)
+            if self.flush:
+                self.scratch.add_(1.0)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        prof = {}
+        for opt, _, _ in self.tensors:
+            opt.profile(False)
+            if profile:
+                for kname, (n, ms) in opt.profile_read().items():
+                    a = prof.setdefault(kname, [0, 0.0])
+                    a[0] += n
+                    a[1] += ms
+        return sum(a.elapsed_time(b) for a, b in evs), prof
+
+    def close(self):
+        for opt, _, _ in self.tensors:
+            opt.close()
+        self.tensors = []
+
+
+def measure(wl, args, dev, world, rank, local, barrier, steps, warmup):
+    """Warm-up, K timed steps with the clock sampler running, K more with
+    per-kernel events; the per-rank numbers of one workload."""
+    import torch
+    b = Bench(wl, args, dev, rank)
+    for i in range(warmup):
+        b.one_step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local, args.out_dir)
+    time.sleep(1.0)  # the polling process is up before the timed region
+    sampler.mark(True)
+    total_ms, _ = b.timed_steps(steps, False, barrier)
+    sampler.mark(False)
+    clocks = sampler.stop()
+    _, prof = b.timed_steps(steps, True, barrier)
+    max_ms = max_over_ranks(total_ms, world, dev)
+    return b, {"total_ms": total_ms, "max_ms": max_ms, "prof": prof, "clocks": clocks}
+
+
+def kernel_roofline(wl, prof, hbm_gbs):
+    """The slowest per-step kernel's algorithmic bytes per launch over its
+    average launch time (a refresh kernel in the profiled pass is reported
+    in "kernels" but is not a step kernel)."""
+    refresh_kernels = {"select", "mode_gram", "eigh", "dct_select", "rebuild"}
+    step_prof = {k: v for k, v in prof.items() if k not in refresh_kernels}
+    dom = max(step_prof.items(), key=lambda kv: kv[1][1]) if step_prof else ("none", [1, 1.0])
+    dom_name, (dom_n, dom_ms) = dom[0], dom[1]
+    per_launch_ms = dom_ms / max(dom_n, 1)
+    kbytes = kernel_algorithmic_bytes(dom_name, wl)
+    achieved = kbytes / (per_launch_ms / 1e3) / 1e9 if kbytes else None
+    return dom_name, achieved
+
+
+def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs):
+    """A compact record of one more workload at its full step count: time
+    per step, throughput, the step's roofline fraction, kernel times and
+    clocks (refreshes, where the workload's period T calls for them, run
+    inside the timed steps)."""
+    import torch
+    from rank_sparse_tensor_b200.synth import WORKLOADS
+    wl = WORKLOADS[name]
+    steps = wl.steps
+    b, m = measure(wl, args, dev, world, rank, local, barrier, steps, 3)
+    step_ms = m["max_ms"] / steps
+    n_elems = wl.N * len(b.tensors)
+    rec = {"steps": steps, "warmup": 3, "ms_per_step": step_ms,
+           "value": job_throughput(world, n_elems, steps, m["max_ms"]), "unit": UNIT,
+           "shape": list(wl.shape), "ranks": list(wl.ranks), "tensors_per_gpu": len(b.tensors),
+           "T": wl.T, "grad_dtype": wl.dtype, "kernel_path": b.tensors[0][0].info["path"],
+           "l2": "flushed between steps" if b.flush else "inputs larger than L2",
+           "tensor_streams": ("one stream per tensor, 1/%d of the SMs each" % wl.n_tensors)
+           if b.concurrent else "one stream",
+           "roofline": dict(step_roofline(wl, len(b.tensors), step_ms, hbm_gbs), peak=hbm_gbs,
+                            unit="GB/s", bound="hbm"),
+           "kernels": {k: {"launches": v[0], "ms_total": round(v[1], 4)} for k, v in m["prof"].items()},
+           "clocks": m["clocks"]}
+    b.close()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def cpu_single_core(wl_name, target_s):
+    """The oracle's throughput on one host thread, in a fresh process (the
+    oracle fixes its thread count when it starts)."""
+    env = dict(os.environ, TGD_ORACLE_THREADS="1")
+    r = subprocess.run([sys.executable, os.path.abspath(__file__), "--cpu-baseline-only",
+                        "--workload", wl_name, "--cpu-seconds", str(target_s)],
+                       env=env, capture_output=True, text=True, timeout=600)
+    for line in r.stdout.splitlines()[::-1]:
+        if line.startswith("{"):
+            return json.loads(line)
+    return {"error": (r.stderr or r.stdout)[-300:]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -306,12 +485,19 @@ def main():
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the leading mode (and its rank) by this factor: small "
                          "cases of the same kernels, for profiler captures only")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the records of the other workloads in the default run")
+    ap.add_argument("--cpu-baseline-only", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help=argparse.SUPPRESS)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     import dataclasses
     from rank_sparse_tensor_b200.synth import WORKLOADS
     wl = WORKLOADS[args.workload]
+    if args.cpu_baseline_only:
+        print(json.dumps(cpu_baseline(wl, args.cpu_seconds)), flush=True)
+        return 0
     if args.shrink > 1:
         sh, rk, gr = list(wl.shape), list(wl.ranks), list(wl.gen_ranks)
         sh[0] //= args.shrink
@@ -322,11 +508,8 @@ def main():
     if args.impl == "reference":
         return run_reference(args, wl)
 
-    import numpy as np
     import torch
     import torch.distributed as dist
-    import rank_sparse_tensor_b200 as rst
-    from rank_sparse_tensor_b200.synth import GradientStream, weights
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
@@ -340,96 +523,10 @@ def main():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # Inputs resident in HBM before the timed region.
-    nt = wl.n_tensors if args.workload != DEFAULT_WORKLOAD else 1
-    concurrent = nt > 1 and not args.sequential
-    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    sm_budget = max(1, n_sms // nt) if concurrent else 0
-    streams = [torch.cuda.Stream(device=dev) for _ in range(nt)] if concurrent else None
-    tensors = []
-    for gseed, wseed in tensor_seeds(rank, nt):
-        gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=gseed,
-                            outlier_frac=wl.outlier_frac, outlier_scale=wl.outlier_scale,
-                            noise=wl.noise, drift=0.0, device=str(dev))
-        grads = [gs.next() for _ in range(2)]
-        w = weights(wl.shape, wl.weight_dtype, seed=wseed, device=str(dev))
-        T = wl.T
-        opt = rst.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, T, wl.lr, wl.betas, wl.eps, wl.wd,
-                             wl.dtype, wl.weight_dtype, path=args.path, sm_budget=sm_budget)
-        if T == 0:
-            opt.refresh(grads[0])
-        tensors.append((opt, grads, w))
-    torch.cuda.synchronize()
-    in_bytes = sum(g[0].numel() * g[0].element_size() + w.numel() * w.element_size()
-                   for _, g, w in tensors)
-    flush = in_bytes < 2 * L2_BYTES
-    scratch = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if flush else None
-
-    def one_step(i):
-        if streams is None:
-            for opt, grads, w in tensors:
-                opt.step(grads[i % 2], w)
-            return
-        # each tensor on its own stream, forked from and joined back into the
-        # timed stream
-        main = torch.cuda.current_stream()
-        fork = torch.cuda.Event()
-        fork.record(main)
-        for (opt, grads, w), st in zip(tensors, streams):
-            st.wait_event(fork)
-            with torch.cuda.stream(st):
-                opt.step(grads[i % 2], w)
-        for st in streams:
-            join = torch.cuda.Event()
-            join.record(st)
-            main.wait_event(join)
-
-    for i in range(args.warmup):
-        one_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-
-    def timed_steps(profile: bool):
-        """K steps between barriers, each bracketed by CUDA events on the
-        launching stream (L2 flushed between steps when inputs fit in it)."""
-        for opt, _, _ in tensors:
-            opt.profile(profile)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(args.steps):
-            evs[i][0].record(stream)
-            one_step(i)
-            evs[i][1].record(stream)
-            if flush:
-                scratch.add_(1.0)
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        prof = {}
-        for opt, _, _ in tensors:
-            opt.profile(False)
-            if profile:
-                for kname, (n, ms) in opt.profile_read().items():
-                    a = prof.setdefault(kname, [0, 0.0])
-                    a[0] += n
-                    a[1] += ms
-        return sum(a.elapsed_time(b) for a, b in evs), prof
-
-    # the metric: K steps without per-kernel events; then K more with them,
-    # for the per-kernel launch times of the roofline
-    sampler = ClockSampler(local, args.out_dir)
-    time.sleep(1.0)  # the polling process is up before the timed region
-    sampler.mark(True)
-    total_ms, _ = timed_steps(False)
-    sampler.mark(False)
-    clocks = sampler.stop()
-    _, prof = timed_steps(True)
-    max_ms = max_over_ranks(total_ms, world, dev)
+    if args.workload == DEFAULT_WORKLOAD:
+        wl = dataclasses.replace(wl, n_tensors=1)
+    b, m = measure(wl, args, dev, world, rank, local, barrier, args.steps, args.warmup)
+    tensors, prof, clocks, max_ms = b.tensors, m["prof"], m["clocks"], m["max_ms"]
     n_elems = wl.N * len(tensors)
     value = job_throughput(world, n_elems, args.steps, max_ms)
 
@@ -452,18 +549,10 @@ def main():
         e2e = {"value": job_throughput(world, wl.N, args.e2e_steps, 1e3 * el), "unit": UNIT,
                "h2d_bytes_per_step": gh.numel() * gh.element_size() + wh.numel() * wh.element_size(),
                "d2h_bytes_per_step": wh.numel() * wh.element_size()}
+        del gh, wh
 
     hbm_gbs, bf16_tf, peak_src = load_peaks()
-    # the roofline's kernel: the slowest per-step kernel (a refresh that falls
-    # in the profiled pass is reported in "kernels" but is not a step kernel)
-    refresh_kernels = {"select", "mode_gram", "eigh", "rebuild"}
-    step_prof = {k: v for k, v in prof.items() if k not in refresh_kernels}
-    dom = max(step_prof.items(), key=lambda kv: kv[1][1]) if step_prof else ("none", [1, 1.0])
-    dom_name, (dom_n, dom_ms) = dom[0], dom[1]
-    per_launch_ms = dom_ms / max(dom_n, 1)
-    kbytes = kernel_algorithmic_bytes(dom_name, wl)
-    achieved = kbytes / (per_launch_ms / 1e3) / 1e9 if kbytes else None
-    ab = algorithmic_bytes(wl)
+    dom_name, achieved = kernel_roofline(wl, prof, hbm_gbs)
     step_ms = max_ms / args.steps
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
@@ -480,17 +569,14 @@ def main():
                    "sparse_ratio": wl.sparse_ratio, "k": wl.k, "T": wl.T, "tensors_per_gpu": len(tensors),
                    "grad_dtype": wl.dtype, "weight_dtype": wl.weight_dtype,
                    "kernel_path": tensors[0][0].info["path"],
-                   "l2": "flushed between steps" if flush else "inputs larger than L2",
+                   "l2": "flushed between steps" if b.flush else "inputs larger than L2",
                    "parallelism": f"independent tensors per rank x{world}",
-                   "tensor_streams": "one stream per tensor, 1/%d of the SMs each" % nt if concurrent
-                   else "one stream"},
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
-                     "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,
-                     "traffic": traffic, "peak_source": peak_src,
-                     # a step covers every tensor of this rank
-                     "step_algorithmic_bytes": ab["total"] * len(tensors),
-                     "step_achieved_gbs": ab["total"] * len(tensors) / (step_ms / 1e3) / 1e9,
-                     "step_frac": ab["total"] * len(tensors) / (step_ms / 1e3) / 1e9 / hbm_gbs},
+                   "tensor_streams": "one stream per tensor, 1/%d of the SMs each" % wl.n_tensors
+                   if b.concurrent else "one stream"},
+        "roofline": dict({"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
+                          "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,
+                          "traffic": traffic, "peak_source": peak_src},
+                         **step_roofline(wl, len(tensors), step_ms, hbm_gbs)),
         "kernels": {k: {"launches": v[0], "ms_total": round(v[1], 4)} for k, v in prof.items()},
         "gpu_launches": int(sum(v[0] for v in prof.values())),  # per K steps (profiled pass)
         "clocks": clocks,
@@ -498,12 +584,22 @@ def main():
         "optimizer_state": optimizer_state(wl, len(tensors),
                                            sum(t[0].info["device_bytes"] for t in tensors)),
     }
+    b.close()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    # the other workloads, each at its full step count (default run only)
+    if args.workload == DEFAULT_WORKLOAD and not args.no_other_workloads and args.shrink == 1:
+        line["workloads"] = {}
+        for name in ("fno4_c32h_128x128x64x33", "fno_c64_64x64x32x17", "refresh_c64_64x64x32x32x17",
+                     "tiny_r32_16x16x8x8"):
+            line["workloads"][name] = other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+        cb = cpu_baseline(wl)
+        one = cpu_single_core(wl.name, 10.0)
+        cb["single_core"] = {k: one.get(k) for k in ("value", "unit", "cores", "sample")} if "value" in one else one
+        line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for opt, _, _ in tensors:
-        opt.close()
     if world > 1:
         dist.destroy_process_group()
     return 0
