@@ -34,17 +34,6 @@ def orc():
     return oracle
 
 
-def block_rows(I0, nblocks):
-    """Contiguous, balanced blocks of mode 0's rows: [(begin, end), ...]."""
-    base, extra = divmod(I0, nblocks)
-    out, b = [], 0
-    for i in range(nblocks):
-        e = b + base + (1 if i < extra else 0)
-        out.append((b, e))
-        b = e
-    return out
-
-
 # name: (shape, ranks, dtype, blocks, path)
 CASES = {
     "c32h_tensor_core_2": ((8, 8, 64, 33), (4, 4, 16, 8), "c32h", 2, "tcgen05"),
@@ -76,23 +65,18 @@ def test_split_step_equals_whole_step(lib, orc, name):
     w_ref = w0.copy()
     assert o.step(g1, w_ref) == 0
 
-    S = int(np.prod(shape[1:]))  # elements per mode-0 row
-    mc = 2 if cplx else 1
-    vc = 1
+    from rank_sparse_tensor_b200 import split
+    state = dict(mom, omega=omega, U=U, t=2, refreshes=1, has_subspace=True)
     handles, grads, ws = [], [], []
-    for b0, b1 in block_rows(shape[0], nb):
-        # the block's entries of Omega (ascending): a contiguous range
-        e0, e1 = (int(x) for x in np.searchsorted(omega, [b0 * S, b1 * S]))
+    for blk in range(nb):
+        b0, b1 = split.block_rows(shape[0], nb, blk)
+        mine = split.block_state(state, shape, b0, b1, cplx)
         bshape = (b1 - b0,) + tuple(shape[1:])
         h = lib.TensorGRaD(bshape, ranks, rho, 0, lr=1e-3, wd=0.01, grad_dtype=dtype, auto_refresh=0,
-                           path=path, sparse_k=e1 - e0, mode0_total=shape[0])
+                           path=path, sparse_k=mine["k"], mode0_total=shape[0])
         assert h.info["path"] == path
-        assert h.info["k"] == e1 - e0
-        h.set_state({"omega": omega[e0:e1] - b0 * S, "U": [U[0][b0:b1]] + U[1:],
-                     "core_m": mom["core_m"], "core_v": mom["core_v"],
-                     "sparse_m": mom["sparse_m"][e0 * mc:e1 * mc],
-                     "sparse_v": mom["sparse_v"][e0 * vc:e1 * vc],
-                     "t": 2, "refreshes": 1, "has_subspace": True})
+        assert h.info["k"] == mine["k"]
+        h.set_state({key: v for key, v in mine.items() if key != "k"})
         handles.append(h)
         grads.append(torch.from_numpy(np.ascontiguousarray(g1[b0:b1])).cuda())
         ws.append(torch.from_numpy(np.ascontiguousarray(w0[b0:b1])).cuda())

@@ -89,3 +89,86 @@ def test_reference_arm_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _split_worker(rank, world, port, out_dir):
+    """A block of mode-0 rows per rank: the rank's share of the state, its
+    partial core (a numpy projection of the block standing in for the
+    library's, which needs a GPU) and the all-reduce that sums the blocks."""
+    import datetime
+
+    import numpy as np
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from rank_sparse_tensor_b200 import split
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        shape, ranks = (7, 5, 6), (3, 2, 4)
+        rng = np.random.default_rng(0)          # the same whole tensor on every rank
+        G = rng.standard_normal(shape) + 1j * rng.standard_normal(shape)
+        U = [np.linalg.qr(rng.standard_normal((I, r)) + 1j * rng.standard_normal((I, r)))[0]
+             for I, r in zip(shape, ranks)]
+        N = G.size
+        omega = np.sort(rng.choice(N, size=N // 10, replace=False))
+        k = omega.size
+        state = {"omega": omega, "U": U, "t": 3, "refreshes": 1, "has_subspace": 1,
+                 "core_m": np.arange(2 * np.prod(ranks), dtype=np.float32),
+                 "core_v": np.ones(np.prod(ranks), np.float32),
+                 "sparse_m": np.arange(2 * k, dtype=np.float32),
+                 "sparse_v": np.arange(k, dtype=np.float32)}
+
+        def project(X, Us):
+            for n, Un in enumerate(Us):
+                X = np.moveaxis(np.tensordot(Un.conj().T, np.moveaxis(X, n, 0), axes=1), 0, n)
+            return X
+
+        b0, b1 = split.block_rows(shape[0], world, rank)
+        mine = split.block_state(state, shape, b0, b1, cplx=True)
+        R = G.reshape(-1).copy()
+        R[omega] = 0                           # the residual of the whole tensor
+        Rb = R.reshape(shape)[b0:b1]           # this rank's rows
+        part = project(Rb, mine["U"])
+        core = torch.from_numpy(np.stack([part.real, part.imag], -1).reshape(-1).copy())
+        split.allreduce_core(core)
+        whole = project(R.reshape(shape), U)
+        ref = np.stack([whole.real, whole.imag], -1).reshape(-1)
+        with open(os.path.join(out_dir, f"split{rank}.json"), "w") as f:
+            json.dump({"rows": [b0, b1], "k": int(mine["k"]),
+                       "omega": (mine["omega"] + b0 * 30).tolist(),
+                       "sparse_m": mine["sparse_m"].tolist(),
+                       "err": float(np.abs(core.numpy() - ref).max() / np.abs(ref).max()),
+                       "k_total": int(k), "omega_total": omega.tolist()}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_blocks_and_core_allreduce_two_gloo_ranks(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_split_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    res = [json.load(open(tmp_path / f"split{r}.json")) for r in range(2)]
+    # the blocks tile mode 0 (7 rows: 4 + 3)
+    assert res[0]["rows"] == [0, 4] and res[1]["rows"] == [4, 7]
+    # every Omega entry lands in exactly one block, in order, with its moments
+    assert res[0]["omega"] + res[1]["omega"] == res[0]["omega_total"]
+    assert res[0]["k"] + res[1]["k"] == res[0]["k_total"]
+    assert res[0]["sparse_m"] + res[1]["sparse_m"] == list(map(float, range(2 * res[0]["k_total"])))
+    # the summed partial cores are the whole tensor's core on every rank
+    assert res[0]["err"] < 1e-12 and res[1]["err"] < 1e-12
+
+
+def test_block_rows_cover_mode0():
+    sys.path.insert(0, ROOT)
+    from rank_sparse_tensor_b200 import split
+    for I0 in (1, 7, 256):
+        for nb in range(1, min(I0, 9) + 1):
+            blocks = [split.block_rows(I0, nb, b) for b in range(nb)]
+            assert blocks[0][0] == 0 and blocks[-1][1] == I0
+            assert all(blocks[i][1] == blocks[i + 1][0] for i in range(nb - 1))
+            sizes = [e - b for b, e in blocks]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        split.block_rows(4, 5, 0)
