@@ -21,10 +21,11 @@
 // the tensor X[a][k][b]: A = the rows' K values gathered by the threads
 // (coalesced across threads when b varies fastest), B = the factor's
 // embedding (complex products as real 2 x 2 blocks, as in step_tc.cu),
-// accumulators in TMEM. fp32 operands are split into two bf16 parts, x = h +
-// l with h = bf16(x) and l = bf16(x - h), and three products h.h + l.h + h.l
-// are accumulated in fp32: the dropped l.l term and the rounding of l leave a
-// relative error near 2^-16 per product, against 2^-9 for one bf16 operand.
+// accumulators in TMEM. fp32 operands are split into three bf16 parts, x =
+// h + m + l with h = bf16(x), m = bf16(x - h), l = bf16(x - h - m), and the
+// six products hh, hm, mh, hl, lh, mm are accumulated in fp32; the dropped
+// products (ml, lm, ll) and the rounding of l are below 2^-24 of |x||u|, the
+// accuracy of an fp32 FMA, against 2^-9 for one bf16 operand.
 // Every wait is bounded and reports TGD_ERR_TIMEOUT.
 
 #include <algorithm>
@@ -54,12 +55,15 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-// x = h + l (+ a remainder below 2^-16 |x|): the two bf16 parts, packed with
-// the neighbouring K value (lo half = even K)
-__device__ __forceinline__ void split2(float x, float y, uint32_t& h, uint32_t& l) {
+// x = h + m + l (+ a remainder below 2^-24 |x|): the three bf16 parts of two
+// neighbouring K values, packed in pairs (lo half = even K)
+__device__ __forceinline__ void split3(float x, float y, uint32_t& h, uint32_t& m, uint32_t& l) {
   const uint16_t hx = bf16_bits(x), hy = bf16_bits(y);
-  const uint16_t lx = bf16_bits(x - bf16_val(hx)), ly = bf16_bits(y - bf16_val(hy));
+  const float rx = x - bf16_val(hx), ry = y - bf16_val(hy);
+  const uint16_t mx = bf16_bits(rx), my = bf16_bits(ry);
+  const uint16_t lx = bf16_bits(rx - bf16_val(mx)), ly = bf16_bits(ry - bf16_val(my));
   h = (uint32_t)hx | ((uint32_t)hy << 16);
+  m = (uint32_t)mx | ((uint32_t)my << 16);
   l = (uint32_t)lx | ((uint32_t)ly << 16);
 }
 
@@ -69,8 +73,8 @@ struct MG32Args {
   int64_t rows, K, B;     // rows = A * B unfolding rows; K entries along the mode
   float* Y;               // [a][j][b] output (unused when the epilogue updates W)
   int64_t J;
-  const uint8_t* img;     // B operand blocks [n block][k chunk][hi, lo], NT x 64 bf16 each
-  int NT, nkc;
+  const uint8_t* img;     // B operand blocks [n block][k chunk][h, m, l], NT x 64 bf16 each
+  int NT, nkc, nstage;
   uint32_t tmem_cols;
   // epilogue of the last expansion: the weight update
   float* W;               // the weights, the full tensor (Y's layout)
@@ -83,19 +87,22 @@ struct MG32Args {
 
 // Y[a][j][b] = sum_k X[a][k][b] M[k][j] over one 128-row block of the
 // unfolding and one NT-wide block of (j, re/im) columns. K advances in chunks
-// of 32 complex (64 real) values, two stages: the chunk's operand image
-// arrives by bulk copy while the threads split and store their rows' values,
-// and the next chunk's values are loaded while its MMAs run.
+// of 32 complex (64 real) values, in two stages when there are several
+// chunks: the chunk's operand image arrives by bulk copy while the threads
+// split and store their rows' values, and the next chunk's values are loaded
+// while its MMAs run.
 // WUPD: instead of storing Y, W[o] <- W[o] decay - lr (Y[o] + S~[o in Omega]).
 template <bool CPLX, bool WUPD>
 __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t b_bytes = (uint32_t)p.NT * 64 * 2;
-  // stage s: A hi, A lo, B hi, B lo
-  auto Ah = [&](int s) { return smem + (uint32_t)s * 2 * G32_ATILE; };
-  auto Al = [&](int s) { return smem + (uint32_t)s * 2 * G32_ATILE + G32_ATILE; };
-  auto Bh = [&](int s) { return smem + 4 * G32_ATILE + (uint32_t)s * 2 * b_bytes; };
-  uint64_t* bars = (uint64_t*)(smem + 4 * G32_ATILE + 4 * b_bytes);  // [0,1] MMAs done, [2,3] B landed
+  const uint32_t stage_bytes = 3 * G32_ATILE + 3 * b_bytes;
+  // stage s: A parts h, m, l, then B parts h, m, l
+  auto Apart = [&](int s, int part) { return smem + (uint32_t)s * stage_bytes + (uint32_t)part * G32_ATILE; };
+  auto Bpart = [&](int s, int part) {
+    return smem + (uint32_t)s * stage_bytes + 3 * G32_ATILE + (uint32_t)part * b_bytes;
+  };
+  uint64_t* bars = (uint64_t*)(smem + (uint32_t)p.nstage * stage_bytes);  // [0,1] MMAs done, [2,3] B landed
   uint32_t* tslot = (uint32_t*)(bars + 4);
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -117,7 +124,7 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   const uint32_t dt = *tslot;
   const uint32_t lbo_b = (uint32_t)(p.NT / 8) * 128;
   const uint32_t idesc = idesc_f16(1, 128, p.NT);
-  const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * 2 * b_bytes;
+  const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * 3 * b_bytes;
   uint32_t issued[2] = {0, 0}, waited[2] = {0, 0}, bloaded[2] = {0, 0};
   constexpr int KE = CPLX ? 32 : 64;  // entries per chunk
   constexpr int NV = 64;              // fp32 values per chunk and row
@@ -153,27 +160,29 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
     }
   };
   load_x(0);
+  const int ns = p.nstage;
   for (int kc = 0; kc < p.nkc; ++kc) {
-    const int s = kc & 1;
-    if (kc >= 2) {
+    const int s = kc % ns;
+    if (kc >= ns) {
       const bool ok = wait_all(&bars[s], waited[s] & 1u);
       waited[s]++;
       if (!ok) break;
       tc_fence_after();
     }
     if (tid == 0) {
-      mbar_expect_tx(&bars[2 + s], 2 * b_bytes);
-      bulk_g2s(Bh(s), img + (int64_t)kc * 2 * b_bytes, 2 * b_bytes, &bars[2 + s]);
+      mbar_expect_tx(&bars[2 + s], 3 * b_bytes);
+      bulk_g2s(Bpart(s, 0), img + (int64_t)kc * 3 * b_bytes, 3 * b_bytes, &bars[2 + s]);
       bloaded[s]++;
     }
-    // this row's 64 K values -> the hi and lo A tiles (8 core matrices each)
+    // this row's 64 K values -> the h, m and l A tiles (8 core matrices each)
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      uint32_t h[4], l[4];
+      uint32_t h[4], m[4], l[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) split2(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], h[u], l[u]);
-      *(uint4*)(Ah(s) + q * G32_LBO + tid * 16) = make_uint4(h[0], h[1], h[2], h[3]);
-      *(uint4*)(Al(s) + q * G32_LBO + tid * 16) = make_uint4(l[0], l[1], l[2], l[3]);
+      for (int u = 0; u < 4; ++u) split3(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], h[u], m[u], l[u]);
+      *(uint4*)(Apart(s, 0) + q * G32_LBO + tid * 16) = make_uint4(h[0], h[1], h[2], h[3]);
+      *(uint4*)(Apart(s, 1) + q * G32_LBO + tid * 16) = make_uint4(m[0], m[1], m[2], m[3]);
+      *(uint4*)(Apart(s, 2) + q * G32_LBO + tid * 16) = make_uint4(l[0], l[1], l[2], l[3]);
     }
     if (kc + 1 < p.nkc) load_x(kc + 1);
     fence_async_smem();
@@ -186,16 +195,16 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
         atomicOr(p.err, DEV_ERR_TIMEOUT);
         s_abort = 1;
       } else {
-        const uint32_t ah = smem_u32(Ah(s)), al = smem_u32(Al(s));
-        const uint32_t bh = smem_u32(Bh(s)), bl = bh + b_bytes;
+        const uint32_t a0 = smem_u32(Apart(s, 0)), b0 = smem_u32(Bpart(s, 0));
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t dah = sdesc(ah + kk * 2 * G32_LBO, G32_LBO, 128);
-          const uint64_t dal = sdesc(al + kk * 2 * G32_LBO, G32_LBO, 128);
-          const uint64_t dbh = sdesc(bh + kk * 2 * lbo_b, lbo_b, 128);
-          const uint64_t dbl = sdesc(bl + kk * 2 * lbo_b, lbo_b, 128);
-          mma_f16(dt, dah, dbh, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-          mma_f16(dt, dal, dbh, idesc, 1u);
-          mma_f16(dt, dah, dbl, idesc, 1u);
+          // (A part, B part): hh, hm, mh, hl, lh, mm
+#pragma unroll
+          for (int pr = 0; pr < 6; ++pr) {
+            const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
+            const uint64_t da = sdesc(a0 + pa * G32_ATILE + kk * 2 * G32_LBO, G32_LBO, 128);
+            const uint64_t db = sdesc(b0 + pb * b_bytes + kk * 2 * lbo_b, lbo_b, 128);
+            mma_f16(dt, da, db, idesc, (kc > 0 || kk > 0 || pr > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&bars[s]);
         issued[s]++;
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   }
   __syncthreads();
   if (!s_abort) {
-    const int s = (p.nkc - 1) & 1;
+    const int s = (p.nkc - 1) % ns;
     wait_all(&bars[s], waited[s] & 1u);
     waited[s]++;
     tc_fence_after();
@@ -267,8 +276,9 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
 // Jc = r), kind 1 expansion M = U^T (Kc = r, Jc = I). Complex M as the real
 // embedding E[(kk,0)][(j,0)] = Mr, E[(kk,1)][(j,0)] = -Mi, E[(kk,0)][(j,1)] =
 // Mi, E[(kk,1)][(j,1)] = Mr; real M as itself. Zero padded to Np x Kp, stored
-// as [n block][k chunk][hi, lo] blocks of NT x 64, each K-major no-swizzle
-// with 8-row groups 128 B apart and K core matrices NT / 8 * 128 B apart.
+// as [n block][k chunk][h, m, l] blocks of NT x 64 (the three bf16 parts of
+// each fp32 entry), each K-major no-swizzle with 8-row groups 128 B apart and
+// K core matrices NT / 8 * 128 B apart.
 __global__ void embed32_kernel(const float2* U, int I, int r, int kind, int cplx, int Np, int Kp, int NT,
                                uint16_t* img) {
   const int nkb = Kp / 64;
@@ -287,12 +297,15 @@ __global__ void embed32_kernel(const float2* U, int I, int r, int kind, int cplx
     } else if (n < Jc && k < Kc) {
       val = kind == 0 ? U[(int64_t)k * r + n].x : U[(int64_t)n * r + k].x;
     }
-    const uint16_t h = bf16_bits(val), l = bf16_bits(val - bf16_val(h));
+    const uint16_t h = bf16_bits(val);
+    const float r = val - bf16_val(h);
+    const uint16_t m = bf16_bits(r), l = bf16_bits(r - bf16_val(m));
     const int nb = n / NT, nl = n - nb * NT, kb = k / 64, kl = k - kb * 64;
-    const int64_t base = ((int64_t)nb * nkb + kb) * 2 * NT * 64;
+    const int64_t base = ((int64_t)nb * nkb + kb) * 3 * NT * 64;
     const uint32_t off = kmaj((uint32_t)nl, (uint32_t)kl, (uint32_t)(NT / 8) * 128u) / 2;
     img[base + off] = h;
-    img[base + (int64_t)NT * 64 + off] = l;
+    img[base + (int64_t)NT * 64 + off] = m;
+    img[base + 2 * (int64_t)NT * 64 + off] = l;
   }
 }
 
@@ -341,22 +354,26 @@ int pow2_cols32(int n) {
   while (c < n) c <<= 1;
   return c;
 }
-size_t g32_smem(int NT) { return 4 * (size_t)G32_ATILE + 4 * (size_t)NT * 64 * 2 + 64; }
+// stages x (three A tiles + three B blocks) + barriers
+size_t g32_smem(int NT, int nstage) {
+  return (size_t)nstage * (3 * (size_t)G32_ATILE + 3 * (size_t)NT * 64 * 2) + 64;
+}
 
 Tc32Impl* impl32(Tc32Plan& p) { return (Tc32Impl*)p.impl; }
 
 // Geometry of one mode's GEMM: N = 2 Jc (complex) or Jc columns in blocks of
-// at most 256; K chunks of 64 real values (32 complex).
+// at most 128 (two stages of three A tiles and three B blocks fit shared
+// memory); K chunks of 64 real values (32 complex).
 void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc) {
   const int Np = r16i((int)(cplx ? 2 * Jc : Jc));
-  NT = Np <= 256 ? Np : 256;
+  NT = Np <= 128 ? Np : 128;
   nnt = (int)ceil_div(Np, NT);
   nkc = (int)ceil_div(cplx ? 2 * Kc : Kc, 64);
 }
 
 template <bool CPLX, bool WUPD>
 cudaError_t launch32(const MG32Args& a, int nnt, cudaStream_t s) {
-  const size_t sm = g32_smem(a.NT);
+  const size_t sm = g32_smem(a.NT, a.nstage);
   cudaError_t e = cudaFuncSetAttribute(mode_gemm32_kernel<CPLX, WUPD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
@@ -424,8 +441,8 @@ bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, 
     if (m.active) {
       mode_geom(m.I, m.r, g->cplx, m.NTp, m.nntp, m.nkcp);
       mode_geom(m.r, m.I, g->cplx, m.NTe, m.nnte, m.nkce);
-      ok &= A((void**)&m.img_p, (size_t)m.nntp * m.nkcp * 2 * m.NTp * 64 * 2);
-      ok &= A((void**)&m.img_e, (size_t)m.nnte * m.nkce * 2 * m.NTe * 64 * 2);
+      ok &= A((void**)&m.img_p, (size_t)m.nntp * m.nkcp * 3 * m.NTp * 64 * 2);
+      ok &= A((void**)&m.img_e, (size_t)m.nnte * m.nkce * 3 * m.NTe * 64 * 2);
     }
     g->modes.push_back(m);
   }
@@ -502,6 +519,7 @@ cudaError_t tc32_project(Tc32Plan& p, const void* grad, const uint32_t* bits, in
     a.img = (const uint8_t*)m.img_p;
     a.NT = m.NTp;
     a.nkc = m.nkcp;
+    a.nstage = m.nkcp > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTp);
     a.err = d_err;
     if (hook) hook(hook_ctx, 0, "mode_gemm32", s);
@@ -547,6 +565,7 @@ cudaError_t tc32_expand_update(Tc32Plan& p, void* w, const uint32_t* bits, float
     a.img = (const uint8_t*)m.img_e;
     a.NT = m.NTe;
     a.nkc = m.nkce;
+    a.nstage = m.nkce > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTe);
     a.W = (float*)w;
     a.S = g->S;

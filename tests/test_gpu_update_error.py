@@ -24,18 +24,19 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 # Bound on max |dW_gpu - dW_ref| / max |dW_ref| for one step:
-# - generic path: fp32 FFMA chains, a few hundred terms per sum: ~1e-6, bound 1e-4;
-# - tensor-core path, fp16 gradients: the gradient and U_b are exact or
-#   rounded once to fp16 (2^-11); the intermediates between the GEMMs are
-#   16-bit (Y, Y', C~ and P': four roundings of 2^-9 each for bf16) and the
-#   factor images U_a, U_n are 16-bit too. Four to six roundings of 2^-9 add
-#   to about 1e-2 in the worst case; the bound keeps a factor 2 for the
-#   element where the max is taken.
-# - tensor-core path, fp32 gradients: every operand is split into two bf16
-#   parts and three products are kept (relative error near 2^-16 per
-#   product); about eight GEMMs in the chain: ~1e-4 worst case, bound 1e-4.
+# - generic path: fp32 FFMA chains, a few hundred terms per sum: ~1e-6
+#   measured, bound 1e-4;
+# - tensor-core path, fp16 gradients: the gradient and U_b enter exactly or
+#   rounded once to fp16 (2^-11); the intermediates between the GEMMs (Y, Y',
+#   C~, P') and the other factor images are bf16, each rounding within 2^-9
+#   (2.0e-3) of its value. The roundings of one chain are independent and
+#   largely cancel in the sums that follow: measured 2e-4 to 4.3e-4 on the
+#   cases below, so the bound is one bf16 rounding, 2e-3;
+# - tensor-core path, fp32 gradients: every operand split into three bf16
+#   parts, six products kept (the accuracy of an fp32 FMA): bound 1e-4, as
+#   the generic path.
 UPDATE_TOL = {("generic", "c32h"): 1e-4, ("generic", "c64"): 1e-4, ("generic", "r32"): 1e-4,
-              ("tcgen05", "c32h"): 2e-2, ("tcgen05", "c64"): 1e-4, ("tcgen05", "r32"): 1e-4}
+              ("tcgen05", "c32h"): 2e-3, ("tcgen05", "c64"): 1e-4, ("tcgen05", "r32"): 1e-4}
 
 
 @pytest.fixture(scope="module")
@@ -140,17 +141,29 @@ def test_full_size_factor_parity(lib, orc, wl_name, omega_mode):
     st = gpu.get_state()
     o = orc.Oracle(wl.shape, wl.ranks, wl.sparse_ratio, 0, grad_dtype=wl.dtype,
                    weight_dtype=wl.weight_dtype, omega_mode=omega_mode, seed=9, auto_refresh=0)
-    o.refresh(to_np(g_dev))
+    g = to_np(g_dev)
+    o.refresh(g)
     assert np.array_equal(st["omega"], o.omega)
-    checked = 0
+    # the residual R = G with Omega zeroed, for the captured energy below
+    if wl.dtype == "c32h":
+        R = g[..., 0].astype(np.float64) + 1j * g[..., 1].astype(np.float64)
+    else:
+        R = g.astype(np.complex128)
+    R.reshape(-1)[o.omega] = 0
     for n, (I, r) in enumerate(zip(wl.shape, wl.ranks)):
         if r == I:
             continue
-        Uo = o.get_U(n)
-        gap = eigengap(o.eigvals(n), r)
-        d = projector_distance(st["U"][n], Uo)
-        assert np.allclose(st["U"][n].conj().T @ st["U"][n], np.eye(r), atol=1e-5)
+        Ug = st["U"][n].astype(np.complex128)
+        assert np.allclose(Ug.conj().T @ Ug, np.eye(r), atol=1e-5)
+        ev = o.eigvals(n)
+        gap = eigengap(ev, r)
         if gap > 1e-3:
+            # an open gap: the subspace is unique
+            d = projector_distance(Ug, o.get_U(n))
             assert d <= 1e-3, (n, d, gap)
-            checked += 1
-    assert checked >= 1
+        # any gap: the device factor captures the optimal energy of the mode-n
+        # Gram, ||U^H R_(n)||_F^2 = sum of its r largest eigenvalues (Ky Fan)
+        captured = float(np.sum(np.abs(np.tensordot(Ug.conj().T, R, axes=([1], [n]))) ** 2))
+        best = float(np.sum(ev[:r]))
+        assert captured <= best * (1 + 1e-6), (n, captured, best)
+        assert captured >= best * (1 - 1e-5), (n, captured, best)
