@@ -654,16 +654,19 @@ __global__ void __launch_bounds__(MGT) mode_gemm_kernel(const MGArgs p) {
     for (int q = 0; q < 8; ++q)
       *(uint4*)(As[s] + q * LBO_M128 + tid * 16) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     if (kc + 2 < p.nkc) load_x(v, kc + 2);
+    // the operand image has landed (checked before the barrier, so that
+    // every thread reads the same abort flag after it)
+    if (tid == 0 && !mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (s_abort) return false;
     if (tid == 0) {
-      if (!mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, WAIT_NS)) {
-        atomicOr(p.err, DEV_ERR_TIMEOUT);
-        s_abort = 1;
-      } else {
+      {
         const uint32_t sa = smem_u32(As[s]), sb = smem_u32(Bs[s]);
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(dt, sdesc(sa + kk * 2 * LBO_M128, LBO_M128, 128), sdesc(sb + kk * 2 * lbo_b, lbo_b, 128),

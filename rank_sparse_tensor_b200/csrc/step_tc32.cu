@@ -82,6 +82,10 @@ struct MG32Args {
   const int64_t* wrank;   // Omega entries before each 32-element word of the mask
   const uint32_t* wbits;  // Omega's bit mask for the update
   float decay, lr;
+  // B == 1 (the innermost mode): a CTA's rows of X, and of Y or W, are one
+  // contiguous range each; they then move by bulk copy through shared memory
+  // at these offsets (0: not staged)
+  uint32_t xs_off, os_off;
   int* err;
 };
 
@@ -102,8 +106,9 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   auto Bpart = [&](int s, int part) {
     return smem + (uint32_t)s * stage_bytes + 3 * G32_ATILE + (uint32_t)part * b_bytes;
   };
-  uint64_t* bars = (uint64_t*)(smem + (uint32_t)p.nstage * stage_bytes);  // [0,1] MMAs done, [2,3] B landed
-  uint32_t* tslot = (uint32_t*)(bars + 4);
+  // [0,1] MMAs done, [2,3] B landed, [4] staged rows landed
+  uint64_t* bars = (uint64_t*)(smem + (uint32_t)p.nstage * stage_bytes);
+  uint32_t* tslot = (uint32_t*)(bars + 5);
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -111,10 +116,26 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   const bool valid = rho < p.rows;
   const int64_t a = valid ? rho / p.B : 0, b = valid ? rho - a * p.B : 0;
   const int64_t xbase = a * p.K * p.B + b;  // element index of (a, k = 0, b)
+  // staging applies to CTAs whose 128 rows all exist
+  const bool full_cta = ((int64_t)blockIdx.x + 1) * G32T <= p.rows;
+  const bool st_in = p.xs_off != 0 && full_cta;
+  const bool st_out = p.os_off != 0 && full_cta;
+  constexpr int ESZ = CPLX ? 8 : 4;
+  float* xs = (float*)(smem + p.xs_off);
+  float* os = (float*)(smem + p.os_off);
+  const int64_t a0 = (int64_t)blockIdx.x * G32T;  // first row (B == 1 when staged)
   if (tid == 0) {
     s_abort = 0;
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
+    // the staged rows: X (and W, whose update happens in shared memory)
+    const uint32_t xb = st_in ? (uint32_t)(G32T * p.K * ESZ) : 0u;
+    const uint32_t wb = (st_out && WUPD) ? (uint32_t)(G32T * p.J * ESZ) : 0u;
+    if (xb + wb) {
+      mbar_expect_tx(&bars[4], xb + wb);
+      if (xb) bulk_g2s(xs, (const uint8_t*)p.X + a0 * p.K * ESZ, xb, &bars[4]);
+      if (wb) bulk_g2s(os, (const uint8_t*)p.W + a0 * p.J * ESZ, wb, &bars[4]);
+    }
   }
   __syncthreads();
   if (warp == 0) tmem_alloc(tslot, p.tmem_cols);
@@ -136,7 +157,39 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
     __syncthreads();
     return s_abort == 0;
   };
+  // every thread waits (bounded) for the staged rows: the data of a bulk copy
+  // is visible to the threads that observe its barrier phase complete
+  auto wait_staged = [&]() -> bool {
+    if (!mbar_wait(&bars[4], 0, G32_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    return s_abort == 0;
+  };
   float v[NV];
+  // this row's values from the staged rows (one chunk: K <= 32 complex / 64 real)
+  auto load_x_staged = [&]() {
+#pragma unroll
+    for (int i = 0; i < KE; ++i) {
+      float2 x = make_float2(0.f, 0.f);
+      if (i < p.K) {
+        const int64_t idx = xbase + i;
+        if (!(p.bits && ((__ldg(p.bits + (idx >> 5)) >> (idx & 31)) & 1u))) {
+          if (CPLX)
+            x = ((const float2*)xs)[tid * p.K + i];
+          else
+            x.x = xs[tid * p.K + i];
+        }
+      }
+      if (CPLX) {
+        v[2 * i] = x.x;
+        v[2 * i + 1] = x.y;
+      } else {
+        v[i] = x.x;
+      }
+    }
+  };
   auto load_x = [&](int kc) {
 #pragma unroll
     for (int i = 0; i < KE; ++i) {
@@ -159,9 +212,17 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       }
     }
   };
-  load_x(0);
+  bool staged_waited = false;
+  if (st_in) {
+    staged_waited = true;
+    if (wait_staged()) load_x_staged();
+  } else {
+    load_x(0);
+  }
   const int ns = p.nstage;
-  for (int kc = 0; kc < p.nkc; ++kc) {
+  // (s_abort is read right after barriers only, where every thread sees the
+  // same value)
+  for (int kc = 0; kc < p.nkc && !s_abort; ++kc) {
     const int s = kc % ns;
     if (kc >= ns) {
       const bool ok = wait_all(&bars[s], waited[s] & 1u);
@@ -185,16 +246,19 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       *(uint4*)(Apart(s, 2) + q * G32_LBO + tid * 16) = make_uint4(l[0], l[1], l[2], l[3]);
     }
     if (kc + 1 < p.nkc) load_x(kc + 1);
+    // the chunk's operand image has landed (checked before the barrier, so
+    // that every thread reads the same abort flag after it)
+    if (tid == 0 && !mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, G32_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (s_abort) break;
     if (tid == 0) {
-      if (!mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, G32_WAIT_NS)) {
-        atomicOr(p.err, DEV_ERR_TIMEOUT);
-        s_abort = 1;
-      } else {
+      {
         const uint32_t a0 = smem_u32(Apart(s, 0)), b0 = smem_u32(Bpart(s, 0));
         for (int kk = 0; kk < 4; ++kk) {
           // (A part, B part): hh, hm, mh, hl, lh, mm
@@ -218,7 +282,61 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
     waited[s]++;
     tc_fence_after();
   }
-  if (!s_abort) {
+  if (!s_abort && st_out && WUPD && !staged_waited) {
+    staged_waited = true;
+    wait_staged();
+  }
+  if (!s_abort && st_out) {
+    // rows staged in shared memory: Y written there, or W updated in place
+    // (row-major [row][j], the layout of the contiguous range), then one bulk
+    // store of the range
+    for (int c0 = 0; c0 < p.NT; c0 += 16) {
+      float y[16];
+      tmem_ld16(dt + lane_base + c0, y);
+      constexpr int PER = CPLX ? 8 : 16;
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int64_t j = (CPLX ? c0 / 2 : c0) + u;
+        if (j >= p.J) continue;
+        const int64_t so = (int64_t)tid * p.J + j;
+        float dr = CPLX ? y[2 * u] : y[u], di = CPLX ? y[2 * u + 1] : 0.f;
+        if (!WUPD) {
+          if (CPLX)
+            ((float2*)os)[so] = make_float2(dr, di);
+          else
+            os[so] = dr;
+        } else {
+          const int64_t o = (a0 + tid) * p.J + j;
+          const uint32_t word = __ldg(p.wbits + (o >> 5));
+          const uint32_t bit = (uint32_t)(o & 31);
+          if ((word >> bit) & 1u) {
+            const int64_t e = __ldg(p.wrank + (o >> 5)) + __popc(word & ((1u << bit) - 1u));
+            if (CPLX) {
+              const float2 sv = __ldg((const float2*)p.S + e);
+              dr += sv.x;
+              di += sv.y;
+            } else {
+              dr += __ldg(p.S + e);
+            }
+          }
+          if (CPLX) {
+            const float2 w = ((float2*)os)[so];
+            ((float2*)os)[so] = make_float2(__fmaf_rn(-p.lr, dr, w.x * p.decay), __fmaf_rn(-p.lr, di, w.y * p.decay));
+          } else {
+            os[so] = __fmaf_rn(-p.lr, dr, os[so] * p.decay);
+          }
+        }
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      uint8_t* dst = WUPD ? (uint8_t*)p.W : (uint8_t*)p.Y;
+      bulk_s2g(dst + a0 * p.J * ESZ, os, (uint32_t)(G32T * p.J * ESZ));
+      bulk_commit();
+      bulk_wait_all0();
+    }
+  } else if (!s_abort) {
     const int64_t j0 = (int64_t)blockIdx.y * (CPLX ? p.NT / 2 : p.NT);
     for (int c0 = 0; c0 < p.NT; c0 += 16) {
       float y[16];
@@ -265,6 +383,7 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       if (issued[s] > waited[s]) mbar_wait(&bars[s], (issued[s] - 1) & 1u, G32_WAIT_NS / 4);
       if (bloaded[s] > 0) mbar_wait(&bars[2 + s], (bloaded[s] - 1) & 1u, G32_WAIT_NS / 4);
     }
+    if (st_in || (st_out && WUPD)) mbar_wait(&bars[4], 0, G32_WAIT_NS / 4);
   }
   tc_fence_before();
   __syncthreads();
@@ -358,6 +477,8 @@ int pow2_cols32(int n) {
 size_t g32_smem(int NT, int nstage) {
   return (size_t)nstage * (3 * (size_t)G32_ATILE + 3 * (size_t)NT * 64 * 2) + 64;
 }
+constexpr size_t G32_SMEM_LIMIT = 227 * 1024 - 1024;
+size_t al128(size_t x) { return (x + 127) / 128 * 128; }
 
 Tc32Impl* impl32(Tc32Plan& p) { return (Tc32Impl*)p.impl; }
 
@@ -371,9 +492,34 @@ void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc) {
   nkc = (int)ceil_div(cplx ? 2 * Kc : Kc, 64);
 }
 
+// Staging of the contiguous row ranges of an innermost-mode product (B == 1):
+// the input when its K fits one chunk, the output when it is one N block;
+// both only where the addresses allow bulk copies and shared memory suffices.
 template <bool CPLX, bool WUPD>
-cudaError_t launch32(const MG32Args& a, int nnt, cudaStream_t s) {
-  const size_t sm = g32_smem(a.NT, a.nstage);
+cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
+  const size_t esz = CPLX ? 8 : 4;
+  size_t sm = g32_smem(a.NT, a.nstage);
+  a.xs_off = 0;
+  a.os_off = 0;
+  if (a.B == 1) {
+    size_t off = al128(sm);
+    if (a.nkc == 1 && ((uintptr_t)a.X % 16) == 0) {
+      const size_t need = off + al128((size_t)G32T * a.K * esz);
+      if (need <= G32_SMEM_LIMIT) {
+        a.xs_off = (uint32_t)off;
+        off = need;
+      }
+    }
+    const void* out = WUPD ? (const void*)a.W : (const void*)a.Y;
+    if (nnt == 1 && ((uintptr_t)out % 16) == 0) {
+      const size_t need = off + al128((size_t)G32T * a.J * esz);
+      if (need <= G32_SMEM_LIMIT) {
+        a.os_off = (uint32_t)off;
+        off = need;
+      }
+    }
+    sm = off;
+  }
   cudaError_t e = cudaFuncSetAttribute(mode_gemm32_kernel<CPLX, WUPD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
@@ -383,6 +529,7 @@ cudaError_t launch32(const MG32Args& a, int nnt, cudaStream_t s) {
 }
 
 cudaError_t launch_mode32(bool cplx, bool wupd, const MG32Args& a, int nnt, cudaStream_t s) {
+  // (a is copied: the launcher fills in the staging offsets)
   if (cplx) return wupd ? launch32<true, true>(a, nnt, s) : launch32<true, false>(a, nnt, s);
   return wupd ? launch32<false, true>(a, nnt, s) : launch32<false, false>(a, nnt, s);
 }
