@@ -306,7 +306,7 @@ def step_roofline(wl, n_tensors, step_ms, hbm_gbs):
 class Bench:
     """One rank's tensors of one workload, resident in HBM, and their timing."""
 
-    def __init__(self, wl, args, dev, rank, concurrent_default=True):
+    def __init__(self, wl, args, dev, rank, concurrent_default=True, opts=None):
         import torch
         import rank_sparse_tensor_b200 as rst
         from rank_sparse_tensor_b200.synth import GradientStream, weights
@@ -324,7 +324,8 @@ class Bench:
             grads = [gs.next() for _ in range(2)]
             w = weights(wl.shape, wl.weight_dtype, seed=wseed, device=str(dev))
             opt = rst.TensorGRaD(wl.shape, wl.ranks, wl.sparse_ratio, wl.T, wl.lr, wl.betas, wl.eps,
-                                 wl.wd, wl.dtype, wl.weight_dtype, path=args.path, sm_budget=sm_budget)
+                                 wl.wd, wl.dtype, wl.weight_dtype, path=args.path, sm_budget=sm_budget,
+                                 **(opts or {}))
             if wl.T == 0:
                 opt.refresh(grads[0])
             self.tensors.append((opt, grads, w))
@@ -392,11 +393,11 @@ class Bench:
         self.tensors = []
 
 
-def measure(wl, args, dev, world, rank, local, barrier, steps, warmup):
+def measure(wl, args, dev, world, rank, local, barrier, steps, warmup, opts=None):
     """Warm-up, K timed steps with the clock sampler running, K more with
     per-kernel events; the per-rank numbers of one workload."""
     import torch
-    b = Bench(wl, args, dev, rank)
+    b = Bench(wl, args, dev, rank, opts=opts)
     for i in range(warmup):
         b.one_step(i)
     torch.cuda.synchronize()
@@ -425,16 +426,18 @@ def kernel_roofline(wl, prof, hbm_gbs):
     return dom_name, achieved
 
 
-def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs):
+def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs, opts=None, oracle_steps=0):
     """A compact record of one more workload at its full step count: time
     per step, throughput, the step's roofline fraction, kernel times and
     clocks (refreshes, where the workload's period T calls for them, run
-    inside the timed steps)."""
+    inside the timed steps). opts: options of the method's variants (the
+    decomposition order, the factor basis). oracle_steps > 0: the oracle's
+    throughput on the same workload (rank 0, after the GPU timing)."""
     import torch
     from rank_sparse_tensor_b200.synth import WORKLOADS
     wl = WORKLOADS[name]
     steps = wl.steps
-    b, m = measure(wl, args, dev, world, rank, local, barrier, steps, 3)
+    b, m = measure(wl, args, dev, world, rank, local, barrier, steps, 3, opts=opts)
     step_ms = m["max_ms"] / steps
     n_elems = wl.N * len(b.tensors)
     rec = {"steps": steps, "warmup": 3, "ms_per_step": step_ms,
@@ -448,10 +451,34 @@ def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs):
                             unit="GB/s", bound="hbm"),
            "kernels": {k: {"launches": v[0], "ms_total": round(v[1], 4)} for k, v in m["prof"].items()},
            "clocks": m["clocks"]}
+    if opts:
+        rec["options"] = dict(opts)
     b.close()
+    if oracle_steps and rank == 0:
+        rec["cpu_baseline"] = oracle_full(wl, oracle_steps, opts)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return rec
+
+
+def oracle_full(wl, steps, opts=None):
+    """The oracle on the whole workload (not a sample) for `steps` steps
+    from create, its refreshes at the workload's period included."""
+    import oracle
+    from rank_sparse_tensor_b200.synth import GradientStream, weights
+    gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, 1, outlier_frac=wl.outlier_frac,
+                        outlier_scale=wl.outlier_scale)
+    g = [gs.next().numpy() for _ in range(2)]
+    w = weights(wl.shape, wl.weight_dtype, 1).numpy()
+    o = oracle.Oracle(wl.shape, wl.ranks, wl.sparse_ratio, wl.T, wl.lr, wl.betas, wl.eps, wl.wd,
+                      wl.dtype, wl.weight_dtype, **(opts or {}))
+    t0 = time.perf_counter()
+    for i in range(steps):
+        o.step(g[i % 2], w)
+    el = time.perf_counter() - t0
+    return {"value": wl.N * steps / el, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{steps} oracle steps of the whole workload from create (refreshes every "
+                      f"{wl.T} steps included): {el:.1f} s"}
 
 
 def cpu_single_core(wl_name, target_s):
@@ -590,9 +617,22 @@ def main():
     # the other workloads, each at its full step count (default run only)
     if args.workload == DEFAULT_WORKLOAD and not args.no_other_workloads and args.shrink == 1:
         line["workloads"] = {}
-        for name in ("fno4_c32h_128x128x64x33", "fno_c64_64x64x32x17", "refresh_c64_64x64x32x32x17",
-                     "tiny_r32_16x16x8x8"):
-            line["workloads"][name] = other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs)
+        ow = line["workloads"]
+        cpu = world == 1 and not args.no_cpu_baseline
+        ow["fno4_c32h_128x128x64x33"] = other_workload("fno4_c32h_128x128x64x33", args, dev, world, rank,
+                                                       local, barrier, hbm_gbs)
+        ow["fno_c64_64x64x32x17"] = other_workload("fno_c64_64x64x32x17", args, dev, world, rank, local,
+                                                   barrier, hbm_gbs, oracle_steps=200 if cpu else 0)
+        # the method's ablated variants on the same tensor: the low-rank part
+        # first, and the DCT column-selection basis instead of HOSVD factors
+        ow["fno_c64_64x64x32x17/lowrank_first"] = other_workload(
+            "fno_c64_64x64x32x17", args, dev, world, rank, local, barrier, hbm_gbs, opts={"order": 1})
+        ow["fno_c64_64x64x32x17/dct_basis"] = other_workload(
+            "fno_c64_64x64x32x17", args, dev, world, rank, local, barrier, hbm_gbs, opts={"basis": 1})
+        ow["refresh_c64_64x64x32x32x17"] = other_workload("refresh_c64_64x64x32x32x17", args, dev, world,
+                                                          rank, local, barrier, hbm_gbs)
+        ow["tiny_r32_16x16x8x8"] = other_workload("tiny_r32_16x16x8x8", args, dev, world, rank, local,
+                                                  barrier, hbm_gbs, oracle_steps=10 if cpu else 0)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl)
         one = cpu_single_core(wl.name, 10.0)
