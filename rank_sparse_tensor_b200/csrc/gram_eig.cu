@@ -329,8 +329,8 @@ template <int DT>
 __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* tiles = smem;                                      // [stage][part] tiles
-  int64_t* colbase = (int64_t*)(smem + 6 * TG_TILE);          // [2][TG_COLS]
-  uint64_t* done = (uint64_t*)(colbase + 2 * TG_COLS);        // [2] MMAs of a stage done
+  int64_t* colbase = (int64_t*)(smem + 6 * TG_TILE);          // [3][TG_COLS]
+  uint64_t* done = (uint64_t*)(colbase + 3 * TG_COLS);        // [2] MMAs of a stage done
   uint32_t* tslot = (uint32_t*)(done + 2);
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -362,6 +362,7 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
     }
   };
   set_colbase(0, c_begin);
+  set_colbase(1, c_begin + TG_COLS);
   __syncthreads();
   if (warp == 0) ptx::tmem_alloc(tslot, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
   ptx::tc_fence_before();
@@ -369,8 +370,10 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
   ptx::tc_fence_after();
   const uint32_t dt_base = *tslot;
   const uint32_t idesc = ptx::idesc_f16(1, 128, p.N);
-  float2 v[16];
-  auto load = [&](int slot) {
+  // two register sets: chunk kc + 2 is loaded while chunk kc is converted and
+  // its MMAs run (column offsets in a ring of three slots)
+  float2 va[16], vb[16];
+  auto load = [&](float2 (&v)[16], int slot) {
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
       float2 x = make_float2(0.f, 0.f);
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
     }
   };
   // this thread's columns of the chunk -> rows i and I + i of the three tiles of stage s
-  auto store = [&](int s) {
+  auto store = [&](const float2 (&v)[16], int s) {
     if (!row_ok) return;
 #pragma unroll
     for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
@@ -415,8 +418,12 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
     }
   };
   uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
-  load(0);
-  for (int kc = 0; kc < nch; ++kc) {
+  if (nch > 0) load(va, 0);
+  if (nch > 1) load(vb, 1);
+  // one chunk: wait for its stage, convert and store the registers, publish
+  // the next-but-one chunk's column offsets, barrier, refill the registers
+  // with chunk kc + 2, issue the MMAs
+  auto chunk = [&](float2 (&v)[16], int kc) -> bool {
     const int s = kc & 1;
     if (kc >= 2) {
       if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
@@ -424,17 +431,17 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
         s_abort = 1;
       }
       __syncthreads();
-      if (s_abort) break;
+      if (s_abort) return false;
       waited[s]++;
       ptx::tc_fence_after();
     }
-    store(s);
-    set_colbase((kc + 1) & 1, c_begin + (int64_t)(kc + 1) * TG_COLS);
+    store(v, s);
+    set_colbase((kc + 2) % 3, c_begin + (int64_t)(kc + 2) * TG_COLS);
     ptx::fence_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (kc + 1 < nch) load((kc + 1) & 1);
+    if (kc + 2 < nch) load(v, (kc + 2) % 3);
     if (tid == 0) {
       const uint32_t base = ptx::smem_u32(tiles + (size_t)s * 3 * TG_TILE);
       // (A part, B part): hh, hm, mh, hl, lh, mm
@@ -451,6 +458,11 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
       ptx::mma_commit(&done[s]);
       issued[s]++;
     }
+    return true;
+  };
+  for (int kc = 0; kc < nch; kc += 2) {
+    if (!chunk(va, kc)) break;
+    if (kc + 1 < nch && !chunk(vb, kc + 1)) break;
   }
   __syncthreads();
   bool ok = !s_abort;
@@ -493,7 +505,7 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
   if (warp == 0) ptx::tmem_dealloc(dt_base, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
 }
 
-size_t tg_smem_bytes() { return 6 * (size_t)TG_TILE + 2 * TG_COLS * 8 + 2 * 8 + 16; }
+size_t tg_smem_bytes() { return 6 * (size_t)TG_TILE + 3 * TG_COLS * 8 + 2 * 8 + 16; }
 
 struct TcGramGeom {
   int64_t I, B, ncol, cols_per_split;
@@ -510,8 +522,8 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
   g.ncol = A * g.B;
   g.N = (int)((2 * g.I + 15) / 16 * 16);
   g.R = g.I <= 32 ? 32 : 64;
-  // two CTAs per SM, a few waves; at least four chunks per split; partials under 32 MB
-  int64_t ns = std::min<int64_t>(148 * 2 * 3, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
+  // one wave of two CTAs per SM; at least four chunks per split; partials under 32 MB
+  int64_t ns = std::min<int64_t>(148 * 2, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
   ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
   g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), TG_COLS) * TG_COLS;
   g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
