@@ -55,6 +55,8 @@ struct tgd_ctx {
   double* gram[TGD_MAX_NDIM] = {};
   double* evals[TGD_MAX_NDIM] = {};
   double* eig_work[TGD_MAX_NDIM] = {};
+  double* eig_v[TGD_MAX_NDIM] = {};  // each mode's eigenvectors of the last refresh
+  bool eig_warm = false;             // eig_v holds them (every projected mode <= 128)
   EigJob* jobs_dev = nullptr;
   std::vector<EigJob> jobs;
   // generic step scratch
@@ -212,6 +214,14 @@ AdamConst adam_const(const tgd_ctx* h, double scale) {
 
 bool mode_active(const tgd_ctx* h, int n) { return ((h->proj >> n) & 1u) != 0; }
 
+// The block eigensolver (every projected mode of at most 128 entries) keeps
+// each mode's eigenvectors, and the next refresh starts from them.
+bool eig_keeps_vectors(const tgd_ctx* h) {
+  for (int n = 0; n < h->d; ++n)
+    if (mode_active(h, n) && h->I[n] > 128) return false;
+  return true;
+}
+
 // Derived device data that depends on Omega and U: the Omega bitmask, the
 // coefficient matrices of the generic path and the tensor-core operands.
 tgd_status rebuild_derived(tgd_ctx* h, cudaStream_t s) {
@@ -319,6 +329,8 @@ tgd_status do_refresh_lowrank_first(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.work = h->eig_work[n];
     j.U = h->U[n];
     j.evals = h->evals[n];
+    j.vprev = h->eig_v[n];
+    j.warm = h->eig_warm ? 1 : 0;
     j.n = (int)h->I[n];
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
@@ -326,6 +338,7 @@ tgd_status do_refresh_lowrank_first(tgd_ctx* h, const void* g, cudaStream_t s) {
   {
     TIMED(h, s, "eigh");
     TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+    h->eig_warm = eig_keeps_vectors(h);
   }
   for (int n = 0; n < h->d; ++n)
     if (mode_active(h, n)) TGD_CUDA(h, coef_matrices(h->U[n], h->I[n], h->r[n], h->cplx, h->P[n], h->E[n], s));
@@ -416,6 +429,8 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.work = h->eig_work[n];
     j.U = h->U[n];
     j.evals = h->evals[n];
+    j.vprev = h->eig_v[n];
+    j.warm = h->eig_warm ? 1 : 0;
     j.n = (int)h->I[n];
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
@@ -426,6 +441,7 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
   } else {
     TIMED(h, s, "eigh");
     TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+    h->eig_warm = eig_keeps_vectors(h);
   }
   tgd_status st = rebuild_derived(h, s);
   if (st != TGD_OK) return st;
@@ -703,6 +719,7 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
       ok &= dalloc_t(h, &h->gram[n], (size_t)shape[n] * shape[n] * 2);
       ok &= dalloc_t(h, &h->evals[n], (size_t)shape[n]);
       ok &= dalloc_t(h, &h->eig_work[n], eig_work_doubles((int)shape[n]));
+      ok &= dalloc_t(h, &h->eig_v[n], (size_t)2 * shape[n] * shape[n]);
     }
   ok &= dalloc(h, (void**)&h->gram_part, gp);
   ok &= dalloc_t(h, &h->jobs_dev, TGD_MAX_NDIM);

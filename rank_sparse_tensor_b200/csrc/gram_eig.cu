@@ -731,10 +731,49 @@ __global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
   double2* T = dyn;  // packed upper triangle of A
   double2* Vt = n <= 64 ? dyn + ntri : (double2*)J.work;
   const double2* G = (const double2*)J.gram;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int i = e / n, j = e - i * n;
-    if (i <= j) T[tri_idx(i, j, n)] = G[e];
-    Vt[e] = make_double2(i == j ? 1.0 : 0.0, 0.0);
+  if (J.warm) {
+    // Start from the previous refresh's eigenvectors V (rows of Vt): the
+    // rotated matrix V^H A V is nearly diagonal when the subspaces move
+    // little between refreshes, so the sweeps below end after one or two.
+    // Jacobi converges from any unitary start; the results are the
+    // eigenpairs of A either way.
+    const double2* Vp = (const double2*)J.vprev;
+    double2* W = (double2*)J.work + (size_t)n * n;  // W = A V (n x n)
+    for (int e = threadIdx.x; e < n * n; e += blockDim.x) Vt[e] = Vp[e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+      const int i = e / n, l = e - i * n;
+      double2 acc = make_double2(0.0, 0.0);
+      for (int j = 0; j < n; ++j) {
+        const double2 g = G[i * n + j], v = Vt[l * n + j];
+        acc.x += g.x * v.x - g.y * v.y;
+        acc.y += g.x * v.y + g.y * v.x;
+      }
+      W[e] = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
+      int k = 0, r = e;
+      while (r >= n - k) {
+        r -= n - k;
+        ++k;
+      }
+      const int l = k + r;
+      double2 acc = make_double2(0.0, 0.0);  // sum_i conj(V[i][k]) W[i][l]
+      for (int i = 0; i < n; ++i) {
+        const double2 v = Vt[k * n + i], w = W[i * n + l];
+        acc.x += v.x * w.x + v.y * w.y;
+        acc.y += v.x * w.y - v.y * w.x;
+      }
+      if (l == k) acc.y = 0.0;  // Hermitian: a real diagonal
+      T[e] = acc;
+    }
+  } else {
+    for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+      const int i = e / n, j = e - i * n;
+      if (i <= j) T[tri_idx(i, j, n)] = G[e];
+      Vt[e] = make_double2(i == j ? 1.0 : 0.0, 0.0);
+    }
   }
   const int m = n + (n & 1);
   const int npairs = m / 2;
@@ -913,6 +952,9 @@ __global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
       ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
     }
   }
+  // the eigenvectors, the start of the next refresh
+  if (J.vprev)
+    for (int e = threadIdx.x; e < n * n; e += blockDim.x) ((double2*)J.vprev)[e] = Vt[e];
 }
 
 // ------------------------------------------------------- DCT column selection
@@ -1059,7 +1101,7 @@ cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const
   return cudaGetLastError();
 }
 
-size_t eig_work_doubles(int n) { return n > 64 ? (size_t)4 * n * n : 0; }
+size_t eig_work_doubles(int n) { return (size_t)4 * n * n; }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;

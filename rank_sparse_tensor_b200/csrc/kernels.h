@@ -37,10 +37,13 @@ cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const
 
 struct EigJob {
   const double* gram;  // n x n complex (interleaved doubles)
-  double* work;        // 2 * n * n complex doubles of global scratch (used when n > 64)
+  double* work;        // 2 * n * n complex doubles of global scratch
   float* U;            // out: n x r complex fp32, row-major
   double* evals;       // out: n eigenvalues, descending
+  double* vprev;       // n x n complex: a unitary basis to start from (rows = vectors), and
+                       // out: the eigenvectors found (n <= 128; any order)
   int n, r;
+  int warm;            // 1: start from vprev, 0: from the identity
 };
 size_t eig_work_doubles(int n);
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);

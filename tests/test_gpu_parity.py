@@ -232,3 +232,27 @@ def test_step_host_equals_device_step(lib, dtype, shape, ranks, path):
     assert np.array_equal(to_np(w_dev).view(np.uint8), w_host.view(np.uint8))
     assert not np.array_equal(w_host, to_np(w))
     assert a.get_state()["t"] == b.get_state()["t"] == 1
+
+
+@pytest.mark.parametrize("name", ["c64_64x64x32x17", "c32h_24x16x64x33", "c64_gram_pairs_130x20x9"])
+def test_second_refresh_starts_from_the_first(lib, orc, name):
+    """A refresh after the first starts the eigensolver from the previous
+    eigenvectors; its factors must still be those of the new gradient's
+    Grams (projector distance to the oracle's cold solve where the gap is
+    open), and orthonormal."""
+    shape, ranks, gen_ranks, dtype, rho = CASES[name]
+    grads, _ = _inputs(shape, gen_ranks, dtype, seed=21, steps=3)
+    g = _gpu(lib, shape, ranks, rho, dtype)
+    for gr in grads:
+        g.refresh(torch.from_numpy(gr).cuda())
+    st = g.get_state()
+    o = orc.Oracle(shape, ranks, rho, 0, grad_dtype=dtype, auto_refresh=0)
+    o.refresh(grads[-1])
+    assert np.array_equal(st["omega"], o.omega)
+    for n in range(len(shape)):
+        if ranks[n] == shape[n]:
+            continue
+        U = st["U"][n].astype(np.complex128)
+        assert np.allclose(U.conj().T @ U, np.eye(ranks[n]), atol=1e-5)
+        if eigengap(o.eigvals(n), ranks[n]) > 1e-3:
+            assert projector_distance(U, o.get_U(n)) <= 1e-3
