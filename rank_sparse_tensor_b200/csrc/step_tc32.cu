@@ -43,7 +43,7 @@ using namespace ptx;
 
 constexpr int G32T = 128;                    // threads = GEMM rows per CTA
 constexpr uint32_t G32_LBO = 2048;           // A tile: 128 rows x 16 B between K core matrices
-constexpr uint32_t G32_ATILE = 8 * G32_LBO;  // 128 rows x 64 bf16
+constexpr int G32_KMAX = 64;                 // bf16 K values per chunk at most
 constexpr uint64_t G32_WAIT_NS = 2000000000ull;
 
 __host__ __device__ __forceinline__ uint32_t kmaj(uint32_t row, uint32_t k, uint32_t lbo) {
@@ -73,8 +73,9 @@ struct MG32Args {
   int64_t rows, K, B;     // rows = A * B unfolding rows; K entries along the mode
   float* Y;               // [a][j][b] output (unused when the epilogue updates W)
   int64_t J;
-  const uint8_t* img;     // B operand blocks [n block][k chunk][h, m, l], NT x 64 bf16 each
+  const uint8_t* img;     // B operand blocks [n block][k chunk][h, m, l], NT x kp bf16 each
   int NT, nkc, nstage;
+  int kp;                 // bf16 K values per chunk: a multiple of 16, at most 64
   uint32_t tmem_cols;
   // epilogue of the last expansion: the weight update
   float* W;               // the weights, the full tensor (Y's layout)
@@ -91,7 +92,8 @@ struct MG32Args {
 
 // Y[a][j][b] = sum_k X[a][k][b] M[k][j] over one 128-row block of the
 // unfolding and one NT-wide block of (j, re/im) columns. K advances in chunks
-// of 32 complex (64 real) values, in two stages when there are several
+// of kp real values (kp / 2 complex; kp = 64, or the whole K rounded up to 16
+// when it fits one chunk), in two stages when there are several
 // chunks: the chunk's operand image arrives by bulk copy while the threads
 // split and store their rows' values, and the next chunk's values are loaded
 // while its MMAs run.
@@ -99,12 +101,14 @@ struct MG32Args {
 template <bool CPLX, bool WUPD>
 __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t b_bytes = (uint32_t)p.NT * 64 * 2;
-  const uint32_t stage_bytes = 3 * G32_ATILE + 3 * b_bytes;
+  const int kq = p.kp / 8;                       // K core matrices per chunk
+  const uint32_t atile = (uint32_t)kq * G32_LBO;  // one part of A: 128 rows x kp bf16
+  const uint32_t b_bytes = (uint32_t)p.NT * p.kp * 2;
+  const uint32_t stage_bytes = 3 * atile + 3 * b_bytes;
   // stage s: A parts h, m, l, then B parts h, m, l
-  auto Apart = [&](int s, int part) { return smem + (uint32_t)s * stage_bytes + (uint32_t)part * G32_ATILE; };
+  auto Apart = [&](int s, int part) { return smem + (uint32_t)s * stage_bytes + (uint32_t)part * atile; };
   auto Bpart = [&](int s, int part) {
-    return smem + (uint32_t)s * stage_bytes + 3 * G32_ATILE + (uint32_t)part * b_bytes;
+    return smem + (uint32_t)s * stage_bytes + 3 * atile + (uint32_t)part * b_bytes;
   };
   // [0,1] MMAs done, [2,3] B landed, [4] staged rows landed
   uint64_t* bars = (uint64_t*)(smem + (uint32_t)p.nstage * stage_bytes);
@@ -147,8 +151,9 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   const uint32_t idesc = idesc_f16(1, 128, p.NT);
   const uint8_t* img = p.img + (int64_t)blockIdx.y * p.nkc * 3 * b_bytes;
   uint32_t issued[2] = {0, 0}, waited[2] = {0, 0}, bloaded[2] = {0, 0};
-  constexpr int KE = CPLX ? 32 : 64;  // entries per chunk
-  constexpr int NV = 64;              // fp32 values per chunk and row
+  constexpr int KE = CPLX ? G32_KMAX / 2 : G32_KMAX;  // entries per chunk at most
+  constexpr int NV = G32_KMAX;                        // fp32 values per chunk and row
+  const int ke = CPLX ? p.kp / 2 : p.kp;              // entries per chunk
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (tid == 0 && !mbar_wait(bar, parity, G32_WAIT_NS)) {
       atomicOr(p.err, DEV_ERR_TIMEOUT);
@@ -172,6 +177,7 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   auto load_x_staged = [&]() {
 #pragma unroll
     for (int i = 0; i < KE; ++i) {
+      if (i >= ke) break;
       float2 x = make_float2(0.f, 0.f);
       if (i < p.K) {
         const int64_t idx = xbase + i;
@@ -193,7 +199,8 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   auto load_x = [&](int kc) {
 #pragma unroll
     for (int i = 0; i < KE; ++i) {
-      const int64_t k = (int64_t)kc * KE + i;
+      if (i >= ke) break;
+      const int64_t k = (int64_t)kc * ke + i;
       float2 x = make_float2(0.f, 0.f);
       if (valid && k < p.K) {
         const int64_t idx = xbase + k * p.B;
@@ -237,7 +244,8 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
     }
     // this row's 64 K values -> the h, m and l A tiles (8 core matrices each)
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < G32_KMAX / 8; ++q) {
+      if (q >= kq) break;
       uint32_t h[4], m[4], l[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) split3(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], h[u], m[u], l[u]);
@@ -260,12 +268,12 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
     if (tid == 0) {
       {
         const uint32_t a0 = smem_u32(Apart(s, 0)), b0 = smem_u32(Bpart(s, 0));
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < kq / 2; ++kk) {
           // (A part, B part): hh, hm, mh, hl, lh, mm
 #pragma unroll
           for (int pr = 0; pr < 6; ++pr) {
             const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
-            const uint64_t da = sdesc(a0 + pa * G32_ATILE + kk * 2 * G32_LBO, G32_LBO, 128);
+            const uint64_t da = sdesc(a0 + pa * atile + kk * 2 * G32_LBO, G32_LBO, 128);
             const uint64_t db = sdesc(b0 + pb * b_bytes + kk * 2 * lbo_b, lbo_b, 128);
             mma_f16(dt, da, db, idesc, (kc > 0 || kk > 0 || pr > 0) ? 1u : 0u);
           }
@@ -399,8 +407,8 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
 // each fp32 entry), each K-major no-swizzle with 8-row groups 128 B apart and
 // K core matrices NT / 8 * 128 B apart.
 __global__ void embed32_kernel(const float2* U, int I, int r, int kind, int cplx, int Np, int Kp, int NT,
-                               uint16_t* img) {
-  const int nkb = Kp / 64;
+                               int kp, uint16_t* img) {
+  const int nkb = Kp / kp;
   const int Kc = kind == 0 ? I : r, Jc = kind == 0 ? r : I;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)Np * Kp;
        e += (int64_t)gridDim.x * blockDim.x) {
@@ -419,12 +427,12 @@ __global__ void embed32_kernel(const float2* U, int I, int r, int kind, int cplx
     const uint16_t h = bf16_bits(val);
     const float r = val - bf16_val(h);
     const uint16_t m = bf16_bits(r), l = bf16_bits(r - bf16_val(m));
-    const int nb = n / NT, nl = n - nb * NT, kb = k / 64, kl = k - kb * 64;
-    const int64_t base = ((int64_t)nb * nkb + kb) * 3 * NT * 64;
+    const int nb = n / NT, nl = n - nb * NT, kb = k / kp, kl = k - kb * kp;
+    const int64_t base = ((int64_t)nb * nkb + kb) * 3 * NT * kp;
     const uint32_t off = kmaj((uint32_t)nl, (uint32_t)kl, (uint32_t)(NT / 8) * 128u) / 2;
     img[base + off] = h;
-    img[base + (int64_t)NT * 64 + off] = m;
-    img[base + 2 * (int64_t)NT * 64 + off] = l;
+    img[base + (int64_t)NT * kp + off] = m;
+    img[base + 2 * (int64_t)NT * kp + off] = l;
   }
 }
 
@@ -452,6 +460,7 @@ struct Mode32 {
   uint16_t* img_p = nullptr;  // projection image
   uint16_t* img_e = nullptr;  // expansion image
   int NTp = 0, nntp = 0, nkcp = 0, NTe = 0, nnte = 0, nkce = 0;
+  int kpp = 64, kpe = 64;     // bf16 K values per chunk
 };
 
 struct Tc32Impl {
@@ -474,8 +483,8 @@ int pow2_cols32(int n) {
   return c;
 }
 // stages x (three A tiles + three B blocks) + barriers
-size_t g32_smem(int NT, int nstage) {
-  return (size_t)nstage * (3 * (size_t)G32_ATILE + 3 * (size_t)NT * 64 * 2) + 64;
+size_t g32_smem(int NT, int nstage, int kp) {
+  return (size_t)nstage * (3 * (size_t)(kp / 8) * G32_LBO + 3 * (size_t)NT * kp * 2) + 64;
 }
 constexpr size_t G32_SMEM_LIMIT = 227 * 1024 - 1024;
 size_t al128(size_t x) { return (x + 127) / 128 * 128; }
@@ -484,12 +493,15 @@ Tc32Impl* impl32(Tc32Plan& p) { return (Tc32Impl*)p.impl; }
 
 // Geometry of one mode's GEMM: N = 2 Jc (complex) or Jc columns in blocks of
 // at most 128 (two stages of three A tiles and three B blocks fit shared
-// memory); K chunks of 64 real values (32 complex).
-void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc) {
+// memory); K in chunks of 64 real values (32 complex), or one chunk of K
+// rounded up to 16 when it fits.
+void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc, int& kp) {
   const int Np = r16i((int)(cplx ? 2 * Jc : Jc));
   NT = Np <= 128 ? Np : 128;
   nnt = (int)ceil_div(Np, NT);
-  nkc = (int)ceil_div(cplx ? 2 * Kc : Kc, 64);
+  const int64_t kreal = cplx ? 2 * Kc : Kc;
+  nkc = (int)ceil_div(kreal, G32_KMAX);
+  kp = nkc == 1 ? r16i((int)kreal) : G32_KMAX;
 }
 
 // Staging of the contiguous row ranges of an innermost-mode product (B == 1):
@@ -498,7 +510,7 @@ void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc) {
 template <bool CPLX, bool WUPD>
 cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
   const size_t esz = CPLX ? 8 : 4;
-  size_t sm = g32_smem(a.NT, a.nstage);
+  size_t sm = g32_smem(a.NT, a.nstage, a.kp);
   a.xs_off = 0;
   a.os_off = 0;
   if (a.B == 1) {
@@ -586,10 +598,10 @@ bool tc32_plan(Tc32Plan& p, int nd, const int64_t* shape, const int64_t* ranks, 
     m.r = ranks[n];
     m.active = ((proj_mask >> n) & 1u) != 0;
     if (m.active) {
-      mode_geom(m.I, m.r, g->cplx, m.NTp, m.nntp, m.nkcp);
-      mode_geom(m.r, m.I, g->cplx, m.NTe, m.nnte, m.nkce);
-      ok &= A((void**)&m.img_p, (size_t)m.nntp * m.nkcp * 3 * m.NTp * 64 * 2);
-      ok &= A((void**)&m.img_e, (size_t)m.nnte * m.nkce * 3 * m.NTe * 64 * 2);
+      mode_geom(m.I, m.r, g->cplx, m.NTp, m.nntp, m.nkcp, m.kpp);
+      mode_geom(m.r, m.I, g->cplx, m.NTe, m.nnte, m.nkce, m.kpe);
+      ok &= A((void**)&m.img_p, (size_t)m.nntp * m.nkcp * 3 * m.NTp * m.kpp * 2);
+      ok &= A((void**)&m.img_e, (size_t)m.nnte * m.nkce * 3 * m.NTe * m.kpe * 2);
     }
     g->modes.push_back(m);
   }
@@ -620,13 +632,13 @@ cudaError_t tc32_rebuild(Tc32Plan& p, const int64_t* omega, int64_t k, const flo
   for (auto& m : g->modes) {
     if (!m.active) continue;
     const float2* Un = (const float2*)U[m.n];
-    int Np = m.nntp * m.NTp, Kp = m.nkcp * 64;
+    int Np = m.nntp * m.NTp, Kp = m.nkcp * m.kpp;
     embed32_kernel<<<blocks((int64_t)Np * Kp), 256, 0, s>>>(Un, (int)m.I, (int)m.r, 0, g->cplx ? 1 : 0, Np, Kp,
-                                                            m.NTp, m.img_p);
+                                                            m.NTp, m.kpp, m.img_p);
     Np = m.nnte * m.NTe;
-    Kp = m.nkce * 64;
+    Kp = m.nkce * m.kpe;
     embed32_kernel<<<blocks((int64_t)Np * Kp), 256, 0, s>>>(Un, (int)m.I, (int)m.r, 1, g->cplx ? 1 : 0, Np, Kp,
-                                                            m.NTe, m.img_e);
+                                                            m.NTe, m.kpe, m.img_e);
   }
   return cudaGetLastError();
 }
@@ -666,6 +678,7 @@ cudaError_t tc32_project(Tc32Plan& p, const void* grad, const uint32_t* bits, in
     a.img = (const uint8_t*)m.img_p;
     a.NT = m.NTp;
     a.nkc = m.nkcp;
+    a.kp = m.kpp;
     a.nstage = m.nkcp > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTp);
     a.err = d_err;
@@ -712,6 +725,7 @@ cudaError_t tc32_expand_update(Tc32Plan& p, void* w, const uint32_t* bits, float
     a.img = (const uint8_t*)m.img_e;
     a.NT = m.NTe;
     a.nkc = m.nkce;
+    a.kp = m.kpe;
     a.nstage = m.nkce > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTe);
     a.W = (float*)w;
