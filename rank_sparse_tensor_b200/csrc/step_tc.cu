@@ -765,6 +765,7 @@ __device__ __forceinline__ float2 wload(const float2* p) { return *p; }
 __device__ __forceinline__ void wstore(float2* p, float x, float y) { *p = make_float2(x, y); }
 
 constexpr int R3T = 512;
+constexpr int PREP_ITEMS = 2;  // B1 items per prep thread whose addressing is precomputed
 constexpr int R3_NS_MAX = 6;  // W stages
 constexpr int EPF = 4;  // Omega entries per epilogue thread prefetched for the next tile
 
@@ -980,6 +981,25 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     const int nkc = p.K1 / 8;  // 16-byte K chunks of a B1 row (4 complex j_a each)
     const bool vec = (p.ra & 3) == 0;  // a chunk's 4 j_a lie in one slab, 16-byte aligned
     bool ok = true;
+    // Where each B1 item of this thread reads Y' in a stage and writes B1: the
+    // same for every tile, so the divisions are done once (for the first
+    // PREP_ITEMS items of the thread; further items, on large ranks, per tile).
+    const int n_items = p.rb * nkc;
+    auto item_addr = [&](int e, int (&src)[4], int (&sl)[4], uint32_t& dst) {
+      const int kc = e % nkc, jb = e / nkc;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kp = 4 * kc + u;
+        sl[u] = kp / p.ra;
+        src[u] = sl[u] * (int)p.yp_bs + jb * p.ra + (kp - sl[u] * p.ra);
+      }
+      dst = kmaj_off((uint32_t)(2 * jb), (uint32_t)(8 * kc), p.lbo_b1);
+    };
+    int it_src[PREP_ITEMS][4], it_sl[PREP_ITEMS][4];
+    uint32_t it_dst[PREP_ITEMS];
+#pragma unroll
+    for (int q = 0; q < PREP_ITEMS; ++q)
+      if (row + 128 * q < n_items) item_addr(row + 128 * q, it_src[q], it_sl[q], it_dst[q]);
     auto build = [&](int64_t it) -> bool {
       const int b = (int)(it & 1), s = (int)(it % ns);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
@@ -992,23 +1012,18 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       const uint32_t* ys = (const uint32_t*)yst(s);
       const int64_t vs = p.n_slabs - t * p.spb;
       const int vslabs = vs < p.spb ? (int)vs : p.spb;
-      for (int e = row; e < p.rb * nkc; e += 128) {
-        const int kc = e % nkc, jb = e / nkc;
+      auto item = [&](const int (&src)[4], const int (&sl)[4], uint32_t dst) {
         uint32_t yv[4];
         if (vec) {
-          const int sl = 4 * kc / p.ra, ja0 = 4 * kc - sl * p.ra;
           uint4 y4 = make_uint4(0, 0, 0, 0);
-          if (sl < vslabs) y4 = *(const uint4*)(ys + sl * p.yp_bs + jb * p.ra + ja0);
+          if (sl[0] < vslabs) y4 = *(const uint4*)(ys + src[0]);
           yv[0] = y4.x;
           yv[1] = y4.y;
           yv[2] = y4.z;
           yv[3] = y4.w;
         } else {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int kp = 4 * kc + u, sl = kp / p.ra, ja = kp - sl * p.ra;
-            yv[u] = sl < vslabs ? ys[sl * p.yp_bs + jb * p.ra + ja] : 0u;
-          }
+          for (int u = 0; u < 4; ++u) yv[u] = sl[u] < vslabs ? ys[src[u]] : 0u;
         }
         uint32_t lo[4], hi[4];
 #pragma unroll
@@ -1017,10 +1032,18 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
           lo[u] = f2_to_bf2(y.x, -y.y);
           hi[u] = f2_to_bf2(y.y, y.x);
         }
-        *(uint4*)(B1 + kmaj_off((uint32_t)(2 * jb), (uint32_t)(8 * kc), p.lbo_b1)) =
-            make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *(uint4*)(B1 + kmaj_off((uint32_t)(2 * jb + 1), (uint32_t)(8 * kc), p.lbo_b1)) =
-            make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        // rows 2 j_b and 2 j_b + 1 sit in one 8-row group, 16 bytes apart
+        *(uint4*)(B1 + dst) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *(uint4*)(B1 + dst + 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      };
+#pragma unroll
+      for (int q = 0; q < PREP_ITEMS; ++q)
+        if (row + 128 * q < n_items) item(it_src[q], it_sl[q], it_dst[q]);
+      for (int e = row + 128 * PREP_ITEMS; e < n_items; e += 128) {
+        int src[4], sl[4];
+        uint32_t dst;
+        item_addr(e, src, sl, dst);
+        item(src, sl, dst);
       }
       fence_async_smem();
       mbar_arrive(&b1full[b]);
