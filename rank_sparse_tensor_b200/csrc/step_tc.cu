@@ -331,10 +331,8 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int Ib = p.Ib;
     // GEMM1's A row in TMEM: K1 / 2 columns (one complex fp16 pair each) in
-    // chunks of 8; the two halves of the converters take a range each, split
-    // so that both hold about half of the row's I_b valid pairs (the
-    // padding chunk costs no loads)
-    const int nch = p.K1 / 16, nch0 = min(nch, max(1, (Ib + 8) / 16));
+    // chunks of 8; the two halves of the converters take alternate ranges
+    const int nch = p.K1 / 16, nch0 = (nch + 1) / 2;
     const int ch_lo = half ? nch0 : 0, ch_hi = half ? nch : nch0;
     int64_t cur_e0 = 0, cur_e1 = 0, nx_e0 = 0, nx_e1 = 0, nn_e0 = 0, nn_e1 = 0;
     uint32_t pf_loc[PF];
@@ -1080,9 +1078,10 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     const int et = tid - 256;  // 0..255
     const int row = et & 127, half = et >> 7;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    // column halves of Delta in chunks of 8 complex values, split so that
-    // both halves update about half of the row's I_b weights
-    const int nch = p.N2 / 16, nch0 = min(nch, max(1, (p.Ib + 8) / 16));
+    // column halves of Delta in chunks of 8 complex values (the first half
+    // takes the larger share of whole chunks; the partial last chunk, with
+    // its per-element bounds, falls to the second)
+    const int nch = p.N2 / 16, nch0 = (nch + 1) / 2;
     const int c_lo = half ? nch0 : 0, c_hi = half ? nch : nch0;
     const int sl_row = row >> p.log2Ia;
     const uint32_t erow = (uint32_t)row * p.Ib;
