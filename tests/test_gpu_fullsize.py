@@ -143,3 +143,55 @@ def test_full_size_omega_bit_exact(lib, orc, wl_name, omega_mode):
     om = gpu.get_state()["omega"]
     ref = orc.topk(to_np(g_dev), wl.dtype, k) if omega_mode == 0 else orc.random_omega(9, 0, N, k)
     assert np.array_equal(om, ref)
+
+
+def test_fno4_four_tensors_side_by_side(lib, orc):
+    """The 4-tensor workload as the benchmark runs it: four (128,128,64,33)
+    complex fp16 tensors stepped at once, each on its own stream with a
+    quarter of the SMs (sm_budget), every tensor's weights compared with the
+    oracle's teacher-forced step element by element."""
+    import math
+    from rank_sparse_tensor_b200.synth import WORKLOADS, GradientStream, weights
+    wl = WORKLOADS["fno4_c32h_128x128x64x33"]
+    shape, ranks = wl.shape, wl.ranks
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    budget = max(1, n_sms // 4)
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    runs = []
+    for j in range(4):
+        gs = GradientStream(shape, wl.gen_ranks, wl.dtype, 40 + j, outlier_frac=wl.outlier_frac,
+                            outlier_scale=wl.outlier_scale, device="cuda")
+        g_dev = gs.next()
+        w_dev = weights(shape, wl.weight_dtype, 40 + j, device="cuda")
+        g, w0 = to_np(g_dev), to_np(w_dev)
+        k = math.floor(wl.sparse_ratio * math.prod(shape))
+        omega = orc.topk(g, wl.dtype, k)
+        U = _factors(shape, ranks, True, 50 + j)
+        gpu = lib.TensorGRaD(shape, ranks, wl.sparse_ratio, 0, wl.lr, wl.betas, wl.eps, wl.wd,
+                             wl.dtype, wl.weight_dtype, auto_refresh=0, sm_budget=budget)
+        assert gpu.info["path"] == "tcgen05"
+        mom = random_moments(np.random.default_rng(60 + j), gpu.info, True)
+        gpu.set_state(dict(mom, omega=omega, U=U, t=4, refreshes=1, has_subspace=True))
+        runs.append((gpu, g_dev, w_dev, g, w0, omega, U, mom))
+    torch.cuda.synchronize()
+    main = torch.cuda.current_stream()
+    fork = torch.cuda.Event()
+    fork.record(main)
+    for (gpu, g_dev, w_dev, *_), st in zip(runs, streams):
+        st.wait_event(fork)
+        with torch.cuda.stream(st):
+            gpu.step(g_dev, w_dev)
+    torch.cuda.synchronize()
+    for gpu, g_dev, w_dev, g, w0, omega, U, mom in runs:
+        gpu.sync()
+        o = orc.Oracle(shape, ranks, wl.sparse_ratio, 0, wl.lr, wl.betas, wl.eps, wl.wd, wl.dtype,
+                       wl.weight_dtype, auto_refresh=0)
+        o.omega = omega
+        for n in range(len(shape)):
+            o.set_U(n, U[n])
+        for key, v in mom.items():
+            o.set_moment(key, v)
+        o.set_counters(4, 1, True)
+        w_ref = w0.copy()
+        assert o.step(g, w_ref) == 0
+        assert rel_err(to_np(w_dev), w_ref, wl.dtype) <= TOL[wl.dtype]
