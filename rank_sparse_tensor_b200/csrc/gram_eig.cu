@@ -310,19 +310,18 @@ struct TcGramArgs {
   int* err;
 };
 
-__device__ __forceinline__ uint16_t bf16_bits(float x) {
-  __nv_bfloat16 h = __float2bfloat16_rn(x);
-  return *reinterpret_cast<uint16_t*>(&h);
+// x = h + m + l (bf16 parts, each the rounding of what the earlier leave).
+// The three parts of x and y at once, packed as bf16 pairs (x in the low
+// half); each part the rounding to nearest of what the earlier parts leave.
+__device__ __forceinline__ uint32_t bf2_bits(float x, float y) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ float bf16_val(uint16_t b) {
-  return __uint_as_float((uint32_t)b << 16);
-}
-// x = h + m + l (bf16 parts, each the rounding of what the earlier leave)
-__device__ __forceinline__ void split3(float x, uint16_t& h, uint16_t& m, uint16_t& l) {
-  h = bf16_bits(x);
-  const float r1 = x - bf16_val(h);
-  m = bf16_bits(r1);
-  l = bf16_bits(r1 - bf16_val(m));
+__device__ __forceinline__ void split3_pair(float x, float y, uint32_t& h, uint32_t& m, uint32_t& l) {
+  h = bf2_bits(x, y);
+  const float rx = x - __uint_as_float(h << 16), ry = y - __uint_as_float(h & 0xffff0000u);
+  m = bf2_bits(rx, ry);
+  l = bf2_bits(rx - __uint_as_float(m << 16), ry - __uint_as_float(m & 0xffff0000u));
 }
 
 template <int DT>
@@ -397,16 +396,12 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float2 x = v[gq * 4 + u];
-        uint16_t rh, rm, rl, ih, im, il;
-        split3(x.x, rh, rm, rl);
-        split3(x.y, ih, im, il);
-        // x row: (re, im); J x row: (-im, re); the low half holds the even K
-        xr[0][u] = (uint32_t)rh | ((uint32_t)ih << 16);
-        xr[1][u] = (uint32_t)rm | ((uint32_t)im << 16);
-        xr[2][u] = (uint32_t)rl | ((uint32_t)il << 16);
-        jr[0][u] = (uint32_t)(ih ^ 0x8000u) | ((uint32_t)rh << 16);
-        jr[1][u] = (uint32_t)(im ^ 0x8000u) | ((uint32_t)rm << 16);
-        jr[2][u] = (uint32_t)(il ^ 0x8000u) | ((uint32_t)rl << 16);
+        // x row: (re, im), the three parts of both in packed pairs (the low
+        // half holds the even K); J x row: (-im, re), the halves swapped and
+        // the new low half negated
+        split3_pair(x.x, x.y, xr[0][u], xr[1][u], xr[2][u]);
+#pragma unroll
+        for (int part = 0; part < 3; ++part) jr[part][u] = __byte_perm(xr[part][u], 0u, 0x1032) ^ 0x8000u;
       }
       const uint32_t kg = (uint32_t)(q * cpt / 4 + gq);
 #pragma unroll

@@ -57,14 +57,15 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 // x = h + m + l (+ a remainder below 2^-24 |x|): the three bf16 parts of two
 // neighbouring K values, packed in pairs (lo half = even K)
+__device__ __forceinline__ uint32_t bf2_bits(float x, float y) {  // (x lo, y hi), each rounded to nearest
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 __device__ __forceinline__ void split3(float x, float y, uint32_t& h, uint32_t& m, uint32_t& l) {
-  const uint16_t hx = bf16_bits(x), hy = bf16_bits(y);
-  const float rx = x - bf16_val(hx), ry = y - bf16_val(hy);
-  const uint16_t mx = bf16_bits(rx), my = bf16_bits(ry);
-  const uint16_t lx = bf16_bits(rx - bf16_val(mx)), ly = bf16_bits(ry - bf16_val(my));
-  h = (uint32_t)hx | ((uint32_t)hy << 16);
-  m = (uint32_t)mx | ((uint32_t)my << 16);
-  l = (uint32_t)lx | ((uint32_t)ly << 16);
+  h = bf2_bits(x, y);
+  const float rx = x - __uint_as_float(h << 16), ry = y - __uint_as_float(h & 0xffff0000u);
+  m = bf2_bits(rx, ry);
+  l = bf2_bits(rx - __uint_as_float(m << 16), ry - __uint_as_float(m & 0xffff0000u));
 }
 
 struct MG32Args {
