@@ -294,8 +294,16 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
 // leave), and the six products hh, hm, mh, hl, lh, mm are accumulated in
 // fp32 in TMEM, which keeps about fp32 accuracy; the products of the two
 // smallest parts (ml, lm, ll, below 2^-24 of the result) are dropped.
-constexpr int TG_THREADS = 128;
+//
+// The chunks' raw elements reach shared memory by asynchronous copies
+// (cp.async, one element each, consecutive threads on consecutive memory)
+// into a ring of TG_NS stages, issued TG_NS - 1 chunks ahead, so each CTA
+// keeps three chunks of loads in flight while it converts one chunk into the
+// bf16 tiles and its MMAs run.
+constexpr int TG_THREADS = 256;
 constexpr int TG_COLS = 32;                 // complex columns per chunk: K = 64 bf16 values
+constexpr int TG_NS = 4;                    // staging stages
+constexpr int TG_SROW = TG_COLS + 1;        // staged row stride (elements), general layout
 constexpr uint32_t TG_LBO = 2048;           // 128 rows x 16 B between K core matrices
 constexpr uint32_t TG_TILE = 8 * TG_LBO;    // 128 rows x 64 K values of bf16
 constexpr uint64_t TG_WAIT_NS = 2000000000ull;
@@ -305,7 +313,7 @@ struct TcGramArgs {
   const uint32_t* bits;
   int64_t I, B, ncol, cols_per_split;
   int N;     // MMA N: 2I rounded up to 16
-  int R;     // rows per thread pass: 32 (I <= 32) or 64
+  int R;     // rows of a conversion pass: 32 (I <= 32) or 64
   float* partial;  // [split][I][I] complex, interleaved
   int* err;
 };
@@ -324,18 +332,55 @@ __device__ __forceinline__ void split3_pair(float x, float y, uint32_t& h, uint3
   l = bf2_bits(rx - __uint_as_float(m << 16), ry - __uint_as_float(m & 0xffff0000u));
 }
 
+// One element of ES bytes global -> shared: asynchronous for 4 and 8 bytes
+// (cp.async), a plain copy for 2-byte elements (below cp.async's minimum).
+template <int ES>
+__device__ __forceinline__ void cp_async_elem(void* dst, const void* src) {
+  if constexpr (ES == 8)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
+  else if constexpr (ES == 4)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
+  else
+    *(uint16_t*)dst = __ldg((const unsigned short*)src);
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Element (re, im) of storage type DT from raw staged bytes.
 template <int DT>
-__global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p) {
+__device__ __forceinline__ float2 staged_elem(const uint8_t* p) {
+  if constexpr (DT == TGD_R32) {
+    return make_float2(*(const float*)p, 0.f);
+  } else if constexpr (DT == TGD_C64) {
+    return *(const float2*)p;
+  } else if constexpr (DT == TGD_C32H) {
+    return __half22float2(*(const __half2*)p);
+  } else {
+    return make_float2(__half2float(*(const __half*)p), 0.f);
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs p) {
+  constexpr int ES = Dt<DT>::bytes;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* tiles = smem;                                      // [stage][part] tiles
-  int64_t* colbase = (int64_t*)(smem + 6 * TG_TILE);          // [3][TG_COLS]
-  uint64_t* done = (uint64_t*)(colbase + 3 * TG_COLS);        // [2] MMAs of a stage done
+  uint8_t* tiles = smem;                                           // [stage][part] tiles
+  uint8_t* stage = smem + 6 * TG_TILE;                             // [TG_NS] raw chunks
+  const uint32_t stage_bytes = (uint32_t)(64 * TG_SROW * ES + 15) / 16 * 16;
+  int64_t* colbase = (int64_t*)(stage + TG_NS * stage_bytes);      // [TG_NS][TG_COLS]
+  uint64_t* done = (uint64_t*)(colbase + TG_NS * TG_COLS);         // [2] MMAs of a stage done
   uint32_t* tslot = (uint32_t*)(done + 2);
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int Q = TG_THREADS / p.R, cpt = TG_COLS / Q;          // column blocks, columns per thread
+  const int I = (int)p.I;
+  const bool contig = p.B == 1;  // the innermost mode: a chunk's columns are one block
+  // staged element (i, c) at i * rs + c * cs
+  const int rs = contig ? 1 : TG_SROW, cs = contig ? I : 1;
+  // conversion: row i of the pass, column block q, cpt columns per thread
+  const int Q = TG_THREADS / p.R, cpt = TG_COLS / Q;
   const int i = tid % p.R, q = tid / p.R;
-  const bool row_ok = i < p.I;
+  const bool conv = i < I;
   const int64_t c_begin = (int64_t)blockIdx.y * p.cols_per_split;
   const int64_t c_end = c_begin + p.cols_per_split < p.ncol ? c_begin + p.cols_per_split : p.ncol;
   const int nch = (int)((c_end - c_begin + TG_COLS - 1) / TG_COLS);
@@ -349,7 +394,16 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
     ptx::mbar_init(&done[1], 1);
     ptx::fence_mbar_init();
   }
-  auto set_colbase = [&](int slot, int64_t c0) {
+  // Copies of chunk kc into its stage, and the element offsets of its
+  // columns (for the residual's mask). General layout: thread t copies
+  // column t % 32 of rows t / 32, + 8, ... (consecutive threads read
+  // consecutive columns); the innermost mode: the chunk's contiguous block,
+  // consecutive threads on consecutive elements.
+  const uint8_t* gb = (const uint8_t*)p.g;
+  auto issue = [&](int kc) {
+    const int slot = kc % TG_NS;
+    uint8_t* st = stage + slot * stage_bytes;
+    const int64_t c0 = c_begin + (int64_t)kc * TG_COLS;
     if (tid < TG_COLS) {
       const int64_t c = c0 + tid;
       int64_t off = -1;
@@ -359,9 +413,25 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
       }
       colbase[slot * TG_COLS + tid] = off;
     }
+    if (c0 >= c_end) return;
+    if (contig) {
+      const int ncols = (int)(c_end - c0 < TG_COLS ? c_end - c0 : TG_COLS);
+      const int64_t e0 = c0 * p.I;
+      for (int e = tid; e < ncols * I; e += TG_THREADS) cp_async_elem<ES>(st + e * ES, gb + (e0 + e) * ES);
+    } else {
+      const int col = tid & (TG_COLS - 1);
+      const int64_t c = c0 + col;
+      if (c < c_end) {
+        const int64_t a = c / p.B, base = a * IB + (c - a * p.B);
+        for (int r = tid >> 5; r < I; r += TG_THREADS / TG_COLS)
+          cp_async_elem<ES>(st + (r * TG_SROW + col) * ES, gb + (base + (int64_t)r * p.B) * ES);
+      }
+    }
   };
-  set_colbase(0, c_begin);
-  set_colbase(1, c_begin + TG_COLS);
+  for (int kc = 0; kc < TG_NS - 1; ++kc) {
+    if (kc < nch) issue(kc);
+    cp_async_commit();
+  }
   __syncthreads();
   if (warp == 0) ptx::tmem_alloc(tslot, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
   ptx::tc_fence_before();
@@ -369,33 +439,26 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
   ptx::tc_fence_after();
   const uint32_t dt_base = *tslot;
   const uint32_t idesc = ptx::idesc_f16(1, 128, p.N);
-  // two register sets: chunk kc + 2 is loaded while chunk kc is converted and
-  // its MMAs run (column offsets in a ring of three slots)
-  float2 va[16], vb[16];
-  auto load = [&](float2 (&v)[16], int slot) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      float2 x = make_float2(0.f, 0.f);
-      if (u < cpt && row_ok) {
-        const int64_t cb = colbase[slot * TG_COLS + q * cpt + u];
-        if (cb >= 0) {
-          const int64_t idx = cb + (int64_t)i * p.B;
-          if (!(p.bits && mask_bit(p.bits, idx))) x = load_elem<DT>(p.g, idx);
-        }
-      }
-      v[u] = x;
-    }
-  };
-  // this thread's columns of the chunk -> rows i and I + i of the three tiles of stage s
-  auto store = [&](const float2 (&v)[16], int s) {
-    if (!row_ok) return;
+  // this thread's columns of a staged chunk -> rows i and I + i of the three
+  // tiles of stage s (Omega's entries zeroed: the residual)
+  auto convert = [&](int kc, int s) {
+    if (!conv) return;
+    const int slot = kc % TG_NS;
+    const uint8_t* st = stage + slot * stage_bytes;
+    const int64_t* cb = colbase + slot * TG_COLS;
 #pragma unroll
     for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
       if (gq * 4 >= cpt) break;
       uint32_t xr[3][4], jr[3][4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float2 x = v[gq * 4 + u];
+        const int col = q * cpt + gq * 4 + u;
+        float2 x = make_float2(0.f, 0.f);
+        const int64_t base = cb[col];
+        if (base >= 0) {
+          const int64_t idx = base + (int64_t)i * p.B;
+          if (!(p.bits && mask_bit(p.bits, idx))) x = staged_elem<DT>(st + (i * rs + col * cs) * ES);
+        }
         // x row: (re, im), the three parts of both in packed pairs (the low
         // half holds the even K); J x row: (-im, re), the halves swapped and
         // the new low half negated
@@ -408,35 +471,33 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
       for (int part = 0; part < 3; ++part) {
         uint8_t* t = tiles + (size_t)(s * 3 + part) * TG_TILE + kg * TG_LBO;
         *(uint4*)(t + (uint32_t)i * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
-        *(uint4*)(t + (uint32_t)(p.I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
+        *(uint4*)(t + (uint32_t)(I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
       }
     }
   };
   uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
-  if (nch > 0) load(va, 0);
-  if (nch > 1) load(vb, 1);
-  // one chunk: wait for its stage, convert and store the registers, publish
-  // the next-but-one chunk's column offsets, barrier, refill the registers
-  // with chunk kc + 2, issue the MMAs
-  auto chunk = [&](float2 (&v)[16], int kc) -> bool {
+  for (int kc = 0; kc < nch; ++kc) {
     const int s = kc & 1;
+    // the copies TG_NS - 1 chunks ahead (into the stage chunk kc - 1 used)
+    if (kc + TG_NS - 1 < nch) issue(kc + TG_NS - 1);
+    cp_async_commit();
+    cp_async_wait<TG_NS - 1>();  // this thread's copies of chunk kc have landed
+    // the tiles of stage s are free once chunk kc - 2's MMAs are done
+    if (kc >= 2 && tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    if (s_abort) break;
     if (kc >= 2) {
-      if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
-        atomicOr(p.err, DEV_ERR_TIMEOUT);
-        s_abort = 1;
-      }
-      __syncthreads();
-      if (s_abort) return false;
       waited[s]++;
       ptx::tc_fence_after();
     }
-    store(v, s);
-    set_colbase((kc + 2) % 3, c_begin + (int64_t)(kc + 2) * TG_COLS);
+    convert(kc, s);
     ptx::fence_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (kc + 2 < nch) load(v, (kc + 2) % 3);
     if (tid == 0) {
       const uint32_t base = ptx::smem_u32(tiles + (size_t)s * 3 * TG_TILE);
       // (A part, B part): hh, hm, mh, hl, lh, mm
@@ -453,12 +514,8 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
       ptx::mma_commit(&done[s]);
       issued[s]++;
     }
-    return true;
-  };
-  for (int kc = 0; kc < nch; kc += 2) {
-    if (!chunk(va, kc)) break;
-    if (kc + 1 < nch && !chunk(vb, kc + 1)) break;
   }
+  cp_async_wait<0>();  // no copy may still target this CTA's shared memory
   __syncthreads();
   bool ok = !s_abort;
   if (ok && nch > 0) {
@@ -471,7 +528,7 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
     ok = !s_abort;
     ptx::tc_fence_after();
   }
-  if (ok) {
+  if (ok && warp < 4) {
     // lane = row of D; columns j < I the real part, I <= j < 2I the imaginary part
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int row = tid;
@@ -490,7 +547,7 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
         }
       }
     }
-  } else if (tid == 0) {
+  } else if (!ok && tid == 0) {
     // bounded waits for MMAs still in flight
     for (int st = 0; st < 2; ++st)
       if (issued[st] > waited[st]) ptx::mbar_wait(&done[st], (issued[st] - 1) & 1u, TG_WAIT_NS / 4);
@@ -500,7 +557,10 @@ __global__ void __launch_bounds__(TG_THREADS) gram_tc_kernel(const TcGramArgs p)
   if (warp == 0) ptx::tmem_dealloc(dt_base, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
 }
 
-size_t tg_smem_bytes() { return 6 * (size_t)TG_TILE + 3 * TG_COLS * 8 + 2 * 8 + 16; }
+size_t tg_smem_bytes(int es) {
+  const size_t stage_bytes = ((size_t)64 * TG_SROW * es + 15) / 16 * 16;
+  return 6 * (size_t)TG_TILE + TG_NS * stage_bytes + TG_NS * TG_COLS * 8 + 2 * 8 + 16;
+}
 
 struct TcGramGeom {
   int64_t I, B, ncol, cols_per_split;
@@ -517,8 +577,9 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
   g.ncol = A * g.B;
   g.N = (int)((2 * g.I + 15) / 16 * 16);
   g.R = g.I <= 32 ? 32 : 64;
-  // one wave of two CTAs per SM; at least four chunks per split; partials under 32 MB
-  int64_t ns = std::min<int64_t>(148 * 2, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
+  // one CTA per SM (a persistent split each); at least four chunks per split;
+  // partials under 32 MB
+  int64_t ns = std::min<int64_t>(148, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
   ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
   g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), TG_COLS) * TG_COLS;
   g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
@@ -1034,7 +1095,7 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
   a.R = t.R;
   a.partial = partial;
   a.err = err;
-  const size_t smem = tg_smem_bytes();
+  const size_t smem = tg_smem_bytes(dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4));
   const dim3 grid(1, t.nsplit);
   cudaError_t e = cudaSuccess;
   switch (dt) {
