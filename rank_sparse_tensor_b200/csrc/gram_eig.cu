@@ -288,8 +288,9 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
 // K-major tile holds, for each split part, the rows x_i (rows 0..I-1) and
 // J x_i (rows I..2I-1), where J maps each (re, im) pair of a column to
 // (-im, re); the rest are zero. With K = (column, re/im), the product of the
-// tile with its first N = 2I rows gives D[i][j] = Re sum_c x_ic conj(x_jc) and
-// D[i][I + j] = Im sum_c x_ic conj(x_jc). Each fp32 value is split into three
+// whole tile (M = 128) with its first I rows (N = I rounded up to 16) gives
+// D[i][j] = Re sum_c x_ic conj(x_jc) and D[I + i][j] = -Im sum_c x_ic
+// conj(x_jc) (columns j >= I of D are not read). Each fp32 value is split into three
 // bf16 parts h + m + l (each the bf16 rounding of what the earlier parts
 // leave), and the six products hh, hm, mh, hl, lh, mm are accumulated in
 // fp32 in TMEM, which keeps about fp32 accuracy; the products of the two
@@ -299,7 +300,9 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
 // (cp.async, one element each, consecutive threads on consecutive memory)
 // into a ring of TG_NS stages, issued TG_NS - 1 chunks ahead, so each CTA
 // keeps three chunks of loads in flight while it converts one chunk into the
-// bf16 tiles and its MMAs run.
+// bf16 tiles and its MMAs run. The word of Omega's bitmask that holds each
+// element's bit travels the same way, beside the element, so no conversion
+// waits on a global load.
 constexpr int TG_THREADS = 256;
 constexpr int TG_COLS = 32;                 // complex columns per chunk: K = 64 bf16 values
 constexpr int TG_NS = 4;                    // staging stages
@@ -312,7 +315,7 @@ struct TcGramArgs {
   const void* g;
   const uint32_t* bits;
   int64_t I, B, ncol, cols_per_split;
-  int N;     // MMA N: 2I rounded up to 16
+  int N;     // MMA N: I rounded up to 16
   int R;     // rows of a conversion pass: 32 (I <= 32) or 64
   float* partial;  // [split][I][I] complex, interleaved
   int* err;
@@ -368,7 +371,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
   uint8_t* tiles = smem;                                           // [stage][part] tiles
   uint8_t* stage = smem + 6 * TG_TILE;                             // [TG_NS] raw chunks
   const uint32_t stage_bytes = (uint32_t)(64 * TG_SROW * ES + 15) / 16 * 16;
-  int64_t* colbase = (int64_t*)(stage + TG_NS * stage_bytes);      // [TG_NS][TG_COLS]
+  uint8_t* mstage = stage + TG_NS * stage_bytes;                    // [TG_NS] mask words
+  const uint32_t mstage_bytes = 64 * TG_SROW * 4;
+  int64_t* colbase = (int64_t*)(mstage + TG_NS * mstage_bytes);    // [TG_NS][TG_COLS]
   uint64_t* done = (uint64_t*)(colbase + TG_NS * TG_COLS);         // [2] MMAs of a stage done
   uint32_t* tslot = (uint32_t*)(done + 2);
   __shared__ int s_abort;
@@ -400,9 +405,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
   // consecutive columns); the innermost mode: the chunk's contiguous block,
   // consecutive threads on consecutive elements.
   const uint8_t* gb = (const uint8_t*)p.g;
+  const bool masked = p.bits != nullptr;
   auto issue = [&](int kc) {
     const int slot = kc % TG_NS;
     uint8_t* st = stage + slot * stage_bytes;
+    uint8_t* mw = mstage + slot * mstage_bytes;
     const int64_t c0 = c_begin + (int64_t)kc * TG_COLS;
     if (tid < TG_COLS) {
       const int64_t c = c0 + tid;
@@ -417,14 +424,20 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
     if (contig) {
       const int ncols = (int)(c_end - c0 < TG_COLS ? c_end - c0 : TG_COLS);
       const int64_t e0 = c0 * p.I;
-      for (int e = tid; e < ncols * I; e += TG_THREADS) cp_async_elem<ES>(st + e * ES, gb + (e0 + e) * ES);
+      for (int e = tid; e < ncols * I; e += TG_THREADS) {
+        cp_async_elem<ES>(st + e * ES, gb + (e0 + e) * ES);
+        if (masked) cp_async_elem<4>(mw + e * 4, p.bits + ((e0 + e) >> 5));
+      }
     } else {
       const int col = tid & (TG_COLS - 1);
       const int64_t c = c0 + col;
       if (c < c_end) {
         const int64_t a = c / p.B, base = a * IB + (c - a * p.B);
-        for (int r = tid >> 5; r < I; r += TG_THREADS / TG_COLS)
-          cp_async_elem<ES>(st + (r * TG_SROW + col) * ES, gb + (base + (int64_t)r * p.B) * ES);
+        for (int r = tid >> 5; r < I; r += TG_THREADS / TG_COLS) {
+          const int64_t idx = base + (int64_t)r * p.B;
+          cp_async_elem<ES>(st + (r * TG_SROW + col) * ES, gb + idx * ES);
+          if (masked) cp_async_elem<4>(mw + (r * TG_SROW + col) * 4, p.bits + (idx >> 5));
+        }
       }
     }
   };
@@ -445,6 +458,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
     if (!conv) return;
     const int slot = kc % TG_NS;
     const uint8_t* st = stage + slot * stage_bytes;
+    const uint32_t* mw = (const uint32_t*)(mstage + slot * mstage_bytes);
     const int64_t* cb = colbase + slot * TG_COLS;
 #pragma unroll
     for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
@@ -456,8 +470,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
         float2 x = make_float2(0.f, 0.f);
         const int64_t base = cb[col];
         if (base >= 0) {
-          const int64_t idx = base + (int64_t)i * p.B;
-          if (!(p.bits && mask_bit(p.bits, idx))) x = staged_elem<DT>(st + (i * rs + col * cs) * ES);
+          const int e = i * rs + col * cs;
+          const uint32_t bit = (uint32_t)(base + (int64_t)i * p.B) & 31u;
+          if (!(masked && ((mw[e] >> bit) & 1u))) x = staged_elem<DT>(st + e * ES);
         }
         // x row: (re, im), the three parts of both in packed pairs (the low
         // half holds the even K); J x row: (-im, re), the halves swapped and
@@ -529,21 +544,21 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
     ptx::tc_fence_after();
   }
   if (ok && warp < 4) {
-    // lane = row of D; columns j < I the real part, I <= j < 2I the imaginary part
+    // lane = row of D: rows r < I the real parts of row r, rows I <= r < 2I
+    // the negated imaginary parts of row r - I; columns j < I
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int row = tid;
+    const bool re = row < I;
+    const int64_t orow = re ? row : row - I;
     float* out = p.partial + (size_t)blockIdx.y * p.I * p.I * 2;
     for (int c0 = 0; c0 < p.N; c0 += 16) {
       float y[16];
       ptx::tmem_ld16(dt_base + lane_base + c0, y);
-      if (row < p.I) {
+      if (row < 2 * I) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int j = c0 + u;
-          if (j < p.I)
-            out[((int64_t)row * p.I + j) * 2] = nch > 0 ? y[u] : 0.f;
-          else if (j < 2 * p.I)
-            out[((int64_t)row * p.I + (j - p.I)) * 2 + 1] = nch > 0 ? y[u] : 0.f;
+          if (j < I) out[(orow * p.I + j) * 2 + (re ? 0 : 1)] = nch > 0 ? (re ? y[u] : -y[u]) : 0.f;
         }
       }
     }
@@ -559,7 +574,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs
 
 size_t tg_smem_bytes(int es) {
   const size_t stage_bytes = ((size_t)64 * TG_SROW * es + 15) / 16 * 16;
-  return 6 * (size_t)TG_TILE + TG_NS * stage_bytes + TG_NS * TG_COLS * 8 + 2 * 8 + 16;
+  return 6 * (size_t)TG_TILE + TG_NS * (stage_bytes + 64 * TG_SROW * 4) + TG_NS * TG_COLS * 8 + 2 * 8 + 16;
 }
 
 struct TcGramGeom {
@@ -575,7 +590,7 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
   for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
   g.I = dims[n];
   g.ncol = A * g.B;
-  g.N = (int)((2 * g.I + 15) / 16 * 16);
+  g.N = (int)((g.I + 15) / 16 * 16);
   g.R = g.I <= 32 ? 32 : 64;
   // one CTA per SM (a persistent split each); at least four chunks per split;
   // partials under 32 MB
