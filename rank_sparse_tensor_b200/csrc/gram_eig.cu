@@ -24,7 +24,10 @@
 // r_n eigenvectors, each scaled by a unit phase that makes its largest-
 // magnitude entry (ties to the lowest row) real and positive.
 
+#include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -284,42 +287,109 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
 }
 
 // ------------------------------------------------ tensor-core Gram (I_n <= 64)
-// The Gram as one tcgen05 GEMM per chunk of 32 unfolding columns. A 128-row
-// K-major tile holds, for each split part, the rows x_i (rows 0..I-1) and
-// J x_i (rows I..2I-1), where J maps each (re, im) pair of a column to
-// (-im, re); the rest are zero. With K = (column, re/im), the product of the
-// whole tile (M = 128) with its first I rows (N = I rounded up to 16) gives
-// D[i][j] = Re sum_c x_ic conj(x_jc) and D[I + i][j] = -Im sum_c x_ic
-// conj(x_jc) (columns j >= I of D are not read). Each fp32 value is split into three
-// bf16 parts h + m + l (each the bf16 rounding of what the earlier parts
-// leave), and the six products hh, hm, mh, hl, lh, mm are accumulated in
-// fp32 in TMEM, which keeps about fp32 accuracy; the products of the two
-// smallest parts (ml, lm, ll, below 2^-24 of the result) are dropped.
+// The Gram as tcgen05 GEMMs over chunks of at most 32 unfolding columns
+// (K = (column, re/im) pairs: 64 bf16 values). Each fp32 value is split into
+// three bf16 parts h + m + l (each the bf16 rounding of what the earlier
+// parts leave); the Gram is the sum of the part products, of which hh, hm,
+// mh, hl, lh and mm (and, where they come free, ml, lm, ll) are formed,
+// which keeps about fp32 accuracy.
 //
-// The chunks' raw elements reach shared memory by asynchronous copies
-// (cp.async, one element each, consecutive threads on consecutive memory)
-// into a ring of TG_NS stages, issued TG_NS - 1 chunks ahead, so each CTA
-// keeps three chunks of loads in flight while it converts one chunk into the
-// bf16 tiles and its MMAs run. The word of Omega's bitmask that holds each
-// element's bit travels the same way, beside the element, so no conversion
-// waits on a global load.
-constexpr int TG_THREADS = 256;
-constexpr int TG_COLS = 32;                 // complex columns per chunk: K = 64 bf16 values
+// For part p a K-major tile holds the rows x_i and J x_i, where J maps each
+// (re, im) pair of a column to (-im, re). With Y = [x_h; x_m; x_l] (3I rows,
+// the B operand), the product of [x_p; J x_p] with Y gives, in column block
+// q of D, Re sum_c x_ic conj(y_jc) in the x rows and -Im sum_c x_ic conj(y_jc)
+// in the J x rows. An MMA costs about the same below N = 128 whatever its
+// N, so the parts are packed as densely as the 128 rows of an A tile allow:
+// P_A = min(3, 64 / I) parts per A tile (one MMA per K step for I <= 21,
+// two for I <= 32, three for I <= 64), each A tile multiplied with the part
+// blocks of Y it needs. Every product lands in D at the row of its A part
+// and the column block of its B part; the epilogue adds the column blocks
+// and the stacked part rows in a fixed order.
+//
+// The unfolding is viewed as [A][I][B] (A, B the products of the dimensions
+// before and after mode n), column c = a B + b. One CTA per SM owns a range
+// of chunks and runs a pipeline whose roles hand stages over through
+// mbarriers:
+// - a producer warp brings each chunk into a ring of TG_NS shared-memory
+//   stages: when B is a multiple of 32, a chunk is 32 columns of one slab a,
+//   fetched by one TMA tensor copy of its I x 32 box (TG_ROWS); when B < 32,
+//   a chunk is floor(32 / B) whole slabs, one contiguous bulk copy
+//   (TG_SLABS); any other layout goes element by element (TG_ELEMS). The
+//   words of Omega's bitmask the chunk needs (two per row, or the block's)
+//   come by asynchronous copies beside it (TG_ELEMS, the fallback, reads the
+//   bits where it converts);
+// - two groups of four converter warps take alternate chunks, each group
+//   turning its chunk into the bf16 tiles of its own tile set (one thread:
+//   one row, four columns), the entries of Omega read as zero (the
+//   residual);
+// - one thread issues the chunk's MMAs and commits them to the tile set's
+//   free barrier.
+constexpr int TG_CONV_WARPS = 8;
+constexpr int TG_GROUP_WARPS = 4;           // converter warps per tile set
+constexpr int TG_PROD_WARP = TG_CONV_WARPS;
+constexpr int TG_MMA_WARP = TG_CONV_WARPS + 1;
+constexpr int TG_THREADS = 32 * (TG_CONV_WARPS + 2);
+constexpr int TG_COLS = 32;                 // column capacity of a chunk
 constexpr int TG_NS = 4;                    // staging stages
-constexpr int TG_SROW = TG_COLS + 1;        // staged row stride (elements), general layout
-constexpr uint32_t TG_LBO = 2048;           // 128 rows x 16 B between K core matrices
-constexpr uint32_t TG_TILE = 8 * TG_LBO;    // 128 rows x 64 K values of bf16
+constexpr uint32_t TG_LBO_A = 2048;         // A tile: 128 rows x 16 B between K core matrices
+constexpr uint32_t TG_TILE_A = 8 * TG_LBO_A;
+constexpr uint32_t TG_LBO_B = 3072;         // Y tile: 192 rows x 16 B
+constexpr uint32_t TG_TILE_B = 8 * TG_LBO_B;
+constexpr uint32_t TG_SET = 3 * TG_TILE_A + TG_TILE_B;   // one tile set: up to three A tiles and Y
+constexpr int TG_MASK_WORDS = 128;          // two per row, or a block of <= 2048 bits + 1
 constexpr uint64_t TG_WAIT_NS = 2000000000ull;
+
+enum TgMode { TG_ROWS = 0, TG_SLABS = 1, TG_ELEMS = 2 };
 
 struct TcGramArgs {
   const void* g;
   const uint32_t* bits;
-  int64_t I, B, ncol, cols_per_split;
-  int N;     // MMA N: I rounded up to 16
-  int R;     // rows of a conversion pass: 32 (I <= 32) or 64
-  float* partial;  // [split][I][I] complex, interleaved
+  int64_t A, I, B;            // the unfolding as [A][I][B]
+  int64_t nchunk;             // chunks of the whole unfolding
+  int64_t chunks_per_split;
+  int mode;                   // TgMode
+  int slabs;                  // slabs per chunk (TG_SLABS)
+  float* partial;             // [split][I][I] complex, interleaved
   int* err;
 };
+
+// What the converters need of a staged chunk besides its elements.
+struct TgMeta {
+  int ncols;                  // valid columns
+  int rs;                     // staged stride between rows (elements)
+  int sh;                     // bit offset in its first word: of the block (TG_SLABS), of row 0 (TG_ROWS)
+  int bsh;                    // TG_ROWS: B mod 32 (row i's offset is sh + i bsh, mod 32)
+  int colofs[TG_COLS];        // staged offset of each column's row 0 (elements)
+  int64_t gcol[TG_COLS];      // TG_ELEMS: element index of each column's row 0
+  uint32_t wm[TG_MASK_WORDS]; // Omega's words: two per row (TG_ROWS), the block's (TG_SLABS)
+};
+
+// Parts per A tile for mode size I, and the number of A tiles.
+// Byte offset of element (i, col) in a TG_ROWS / TG_ELEMS stage. 8- and
+// 4-byte elements: rows of 128 bytes (a box of 16, or of 32, columns; 8-byte
+// elements fill two boxes, each starting on a 1024-byte boundary), the
+// 16-byte units of row i permuted by XOR with i mod 8 (the TMA 128-byte
+// swizzle), so that eight consecutive rows read or written at one column
+// fall in different banks; 2-byte elements: plain 64-byte rows.
+template <int ES>
+__host__ __device__ __forceinline__ uint32_t tg_soff(int i, int col, uint32_t boxb) {
+  if constexpr (ES == 8) {
+    const uint32_t byte = (uint32_t)(col & 15) * 8;
+    return (uint32_t)(col >> 4) * boxb + (uint32_t)i * 128 + ((((byte >> 4) ^ (uint32_t)(i & 7)) << 4) | (byte & 15));
+  } else if constexpr (ES == 4) {
+    const uint32_t byte = (uint32_t)col * 4;
+    return (uint32_t)i * 128 + ((((byte >> 4) ^ (uint32_t)(i & 7)) << 4) | (byte & 15));
+  } else {
+    return (uint32_t)i * 64 + (uint32_t)col * 2;
+  }
+}
+__host__ __device__ constexpr uint32_t tg_boxb(int I) { return ((uint32_t)I * 128 + 1023) / 1024 * 1024; }
+
+__host__ __device__ constexpr int tg_parts_per_a(int I) { return I <= 21 ? 3 : (I <= 32 ? 2 : 1); }
+__host__ __device__ constexpr int tg_a_tiles(int I) { return (3 + tg_parts_per_a(I) - 1) / tg_parts_per_a(I); }
+// MMA N of A tile a: the Y part blocks its parts need (p + q <= 2 for the
+// tile's first part p), rounded up to 16.
+__host__ __device__ constexpr int tg_n_of(int I, int a) { return ((3 - a * tg_parts_per_a(I)) * I + 15) / 16 * 16; }
 
 // x = h + m + l (bf16 parts, each the rounding of what the earlier leave).
 // The three parts of x and y at once, packed as bf16 pairs (x in the low
@@ -346,9 +416,40 @@ __device__ __forceinline__ void cp_async_elem(void* dst, const void* src) {
   else
     *(uint16_t*)dst = __ldg((const unsigned short*)src);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// The mbarrier gets one more pending arrival, made when this thread's
+// earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(ptx::smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tg_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_u32(bar)) : "memory");
+}
+// TMA copy of the box at (x, y, z) of a 3-D tensor map into shared memory,
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          ptx::smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(ptx::smem_u32(bar))
+      : "memory");
+}
+// Lane 0 waits (bounded) for the phase, the warp learns the outcome; on
+// expiry the error is recorded and the abort flag raised.
+__device__ __forceinline__ bool tg_waitw(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    if (*abort) {
+      ok = 0;
+    } else if (!ptx::mbar_wait(bar, parity, TG_WAIT_NS)) {
+      atomicOr(err, DEV_ERR_TIMEOUT);
+      *abort = 1;
+      ok = 0;
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
 
 // Element (re, im) of storage type DT from raw staged bytes.
 template <int DT>
@@ -365,239 +466,363 @@ __device__ __forceinline__ float2 staged_elem(const uint8_t* p) {
 }
 
 template <int DT>
-__global__ void __launch_bounds__(TG_THREADS, 1) gram_tc_kernel(const TcGramArgs p) {
+__global__ void __launch_bounds__(TG_THREADS, 1)
+    gram_tc_kernel(const TcGramArgs p, const __grid_constant__ CUtensorMap rows_map) {
   constexpr int ES = Dt<DT>::bytes;
+  constexpr uint32_t STAGE = 64 * TG_COLS * ES;                // a dense 64 x 32 box, or a block of <= 2048 elements
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* tiles = smem;                                           // [stage][part] tiles
-  uint8_t* stage = smem + 6 * TG_TILE;                             // [TG_NS] raw chunks
-  const uint32_t stage_bytes = (uint32_t)(64 * TG_SROW * ES + 15) / 16 * 16;
-  uint8_t* mstage = stage + TG_NS * stage_bytes;                    // [TG_NS] mask words
-  const uint32_t mstage_bytes = 64 * TG_SROW * 4;
-  int64_t* colbase = (int64_t*)(mstage + TG_NS * mstage_bytes);    // [TG_NS][TG_COLS]
-  uint64_t* done = (uint64_t*)(colbase + TG_NS * TG_COLS);         // [2] MMAs of a stage done
-  uint32_t* tslot = (uint32_t*)(done + 2);
+  uint8_t* tiles = smem;                                        // [2] tile sets
+  uint8_t* stage = smem + 2 * TG_SET;                           // [TG_NS] staged chunks
+  TgMeta* meta = (TgMeta*)(stage + TG_NS * STAGE);              // [TG_NS]
+  uint64_t* full = (uint64_t*)(meta + TG_NS);                   // [TG_NS] chunk staged
+  uint64_t* sfree = full + TG_NS;                               // [TG_NS] stage read
+  uint64_t* tfull = sfree + TG_NS;                              // [2] tile set written
+  uint64_t* tfree = tfull + 2;                                  // [2] tile set's MMAs done
+  int* tks = (int*)(tfree + 2);                                 // [2] K steps of the set's chunk
+  uint32_t* tslot = (uint32_t*)(tks + 2);
   __shared__ int s_abort;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  volatile int* abort = &s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int I = (int)p.I;
-  const bool contig = p.B == 1;  // the innermost mode: a chunk's columns are one block
-  // staged element (i, c) at i * rs + c * cs
-  const int rs = contig ? 1 : TG_SROW, cs = contig ? I : 1;
-  // conversion: row i of the pass, column block q, cpt columns per thread
-  const int Q = TG_THREADS / p.R, cpt = TG_COLS / Q;
-  const int i = tid % p.R, q = tid / p.R;
-  const bool conv = i < I;
-  const int64_t c_begin = (int64_t)blockIdx.y * p.cols_per_split;
-  const int64_t c_end = c_begin + p.cols_per_split < p.ncol ? c_begin + p.cols_per_split : p.ncol;
-  const int nch = (int)((c_end - c_begin + TG_COLS - 1) / TG_COLS);
+  const int PA = tg_parts_per_a(I), NA = tg_a_tiles(I);
+  const int N0 = tg_n_of(I, 0);
+  const uint32_t tmem_cols = N0 <= 32 ? 32u : (N0 <= 64 ? 64u : (N0 <= 128 ? 128u : 256u));
   const int64_t IB = p.I * p.B;
-  // zero every tile once: rows 2I..127 stay zero, rows 0..2I-1 are rewritten per chunk
-  for (uint32_t o = tid * 16; o < 6 * TG_TILE; o += TG_THREADS * 16)
-    *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
+  const int64_t q_begin = (int64_t)blockIdx.x * p.chunks_per_split;
+  const int64_t q_end = q_begin + p.chunks_per_split < p.nchunk ? q_begin + p.chunks_per_split : p.nchunk;
+  const int nch = q_end > q_begin ? (int)(q_end - q_begin) : 0;
+  const bool masked = p.bits != nullptr;
+  // rows no part uses stay zero in every tile
+  for (uint32_t o = tid * 16; o < 2 * TG_SET; o += TG_THREADS * 16) *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
     s_abort = 0;
-    ptx::mbar_init(&done[0], 1);
-    ptx::mbar_init(&done[1], 1);
+    for (int s = 0; s < TG_NS; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&sfree[s], TG_GROUP_WARPS);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(&tfull[t], TG_GROUP_WARPS);
+      ptx::mbar_init(&tfree[t], 1);
+    }
     ptx::fence_mbar_init();
   }
-  // Copies of chunk kc into its stage, and the element offsets of its
-  // columns (for the residual's mask). General layout: thread t copies
-  // column t % 32 of rows t / 32, + 8, ... (consecutive threads read
-  // consecutive columns); the innermost mode: the chunk's contiguous block,
-  // consecutive threads on consecutive elements.
-  const uint8_t* gb = (const uint8_t*)p.g;
-  const bool masked = p.bits != nullptr;
-  auto issue = [&](int kc) {
-    const int slot = kc % TG_NS;
-    uint8_t* st = stage + slot * stage_bytes;
-    uint8_t* mw = mstage + slot * mstage_bytes;
-    const int64_t c0 = c_begin + (int64_t)kc * TG_COLS;
-    if (tid < TG_COLS) {
-      const int64_t c = c0 + tid;
-      int64_t off = -1;
-      if (c < c_end) {
-        const int64_t a = c / p.B;
-        off = a * IB + (c - a * p.B);
-      }
-      colbase[slot * TG_COLS + tid] = off;
-    }
-    if (c0 >= c_end) return;
-    if (contig) {
-      const int ncols = (int)(c_end - c0 < TG_COLS ? c_end - c0 : TG_COLS);
-      const int64_t e0 = c0 * p.I;
-      for (int e = tid; e < ncols * I; e += TG_THREADS) {
-        cp_async_elem<ES>(st + e * ES, gb + (e0 + e) * ES);
-        if (masked) cp_async_elem<4>(mw + e * 4, p.bits + ((e0 + e) >> 5));
-      }
-    } else {
-      const int col = tid & (TG_COLS - 1);
-      const int64_t c = c0 + col;
-      if (c < c_end) {
-        const int64_t a = c / p.B, base = a * IB + (c - a * p.B);
-        for (int r = tid >> 5; r < I; r += TG_THREADS / TG_COLS) {
-          const int64_t idx = base + (int64_t)r * p.B;
-          cp_async_elem<ES>(st + (r * TG_SROW + col) * ES, gb + idx * ES);
-          if (masked) cp_async_elem<4>(mw + (r * TG_SROW + col) * 4, p.bits + (idx >> 5));
-        }
-      }
-    }
-  };
-  for (int kc = 0; kc < TG_NS - 1; ++kc) {
-    if (kc < nch) issue(kc);
-    cp_async_commit();
-  }
-  __syncthreads();
-  if (warp == 0) ptx::tmem_alloc(tslot, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+  if (warp == 0) ptx::tmem_alloc(tslot, tmem_cols);
+  ptx::fence_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t dt_base = *tslot;
-  const uint32_t idesc = ptx::idesc_f16(1, 128, p.N);
-  // this thread's columns of a staged chunk -> rows i and I + i of the three
-  // tiles of stage s (Omega's entries zeroed: the residual)
-  auto convert = [&](int kc, int s) {
-    if (!conv) return;
-    const int slot = kc % TG_NS;
-    const uint8_t* st = stage + slot * stage_bytes;
-    const uint32_t* mw = (const uint32_t*)(mstage + slot * mstage_bytes);
-    const int64_t* cb = colbase + slot * TG_COLS;
-#pragma unroll
-    for (int gq = 0; gq < 4; ++gq) {         // K core matrices: 4 complex columns each
-      if (gq * 4 >= cpt) break;
-      uint32_t xr[3][4], jr[3][4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int col = q * cpt + gq * 4 + u;
-        float2 x = make_float2(0.f, 0.f);
-        const int64_t base = cb[col];
-        if (base >= 0) {
-          const int e = i * rs + col * cs;
-          const uint32_t bit = (uint32_t)(base + (int64_t)i * p.B) & 31u;
-          if (!(masked && ((mw[e] >> bit) & 1u))) x = staged_elem<DT>(st + e * ES);
+  const uint8_t* gb = (const uint8_t*)p.g;
+
+  if (warp == TG_PROD_WARP) {
+    // ------------------------------------------------------------ producer
+    int issued = 0;
+    for (int kc = 0; kc < nch; ++kc) {
+      const int slot = kc % TG_NS;
+      if (kc >= TG_NS && !tg_waitw(&sfree[slot], (uint32_t)((kc / TG_NS - 1) & 1), abort, p.err)) break;
+      TgMeta* m = &meta[slot];
+      uint8_t* st = stage + slot * STAGE;
+      const int64_t q = q_begin + kc;
+      if (p.mode == TG_SLABS) {
+        const int64_t a0 = q * p.slabs;
+        const int64_t a1 = a0 + p.slabs < p.A ? a0 + p.slabs : p.A;
+        const int ncols = (int)((a1 - a0) * p.B);
+        const int64_t blk = a0 * IB, nel = (a1 - a0) * IB;
+        if (masked) {
+          const int64_t w0 = blk >> 5, nw = ((blk + nel - 1) >> 5) - w0 + 1;
+          for (int w = lane; w < nw; w += 32) cp_async_elem<4>(&m->wm[w], p.bits + w0 + w);
         }
-        // x row: (re, im), the three parts of both in packed pairs (the low
-        // half holds the even K); J x row: (-im, re), the halves swapped and
-        // the new low half negated
-        split3_pair(x.x, x.y, xr[0][u], xr[1][u], xr[2][u]);
-#pragma unroll
-        for (int part = 0; part < 3; ++part) jr[part][u] = __byte_perm(xr[part][u], 0u, 0x1032) ^ 0x8000u;
+        m->colofs[lane] = lane < ncols ? (int)((lane / p.B) * IB + lane % p.B) : 0;
+        if (lane == 0) {
+          m->ncols = ncols;
+          m->rs = (int)p.B;
+          m->sh = (int)(blk & 31);
+        }
+        cp_async_arrive(&full[slot]);
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bytes = (uint32_t)((nel * ES + 15) / 16 * 16);
+          ptx::mbar_expect_tx(&full[slot], bytes);
+          ptx::bulk_g2s(st, gb + blk * ES, bytes, &full[slot]);
+        }
+      } else if (p.mode == TG_ROWS) {
+        const int64_t c0 = q * TG_COLS;
+        const int64_t a = c0 / p.B;
+        const int64_t b0 = c0 - a * p.B;
+        const int64_t base0 = a * IB + b0;
+        if (masked)
+          for (int i = lane; i < I; i += 32) {
+            // row i's 32 bits start at bit rb: its word and, unless rb is a
+            // word boundary, the next
+            const int64_t rb = base0 + (int64_t)i * p.B;
+            cp_async_elem<4>(&m->wm[2 * i], p.bits + (rb >> 5));
+            if (rb & 31) cp_async_elem<4>(&m->wm[2 * i + 1], p.bits + (rb >> 5) + 1);
+          }
+        m->colofs[lane] = lane;
+        if (lane == 0) {
+          m->ncols = TG_COLS;
+          m->rs = TG_COLS;
+          m->sh = (int)(base0 & 31);
+          m->bsh = (int)(p.B & 31);
+        }
+        cp_async_arrive(&full[slot]);
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_expect_tx(&full[slot], (uint32_t)(I * TG_COLS * ES));
+          // the I rows x 32 columns at column b0 of slab a; 8-byte elements
+          // are addressed as pairs of 4-byte ones, in two boxes of 16 columns
+          if constexpr (ES == 8) {
+            tma_load_3d(st, &rows_map, (int)(2 * b0), 0, (int)a, &full[slot]);
+            tma_load_3d(st + tg_boxb(I), &rows_map, (int)(2 * b0 + 32), 0, (int)a, &full[slot]);
+          } else {
+            tma_load_3d(st, &rows_map, (int)b0, 0, (int)a, &full[slot]);
+          }
+        }
+      } else {
+        const int64_t c0 = q * TG_COLS;
+        const int64_t ncol = p.A * p.B;
+        const int ncols = (int)(ncol - c0 < TG_COLS ? ncol - c0 : TG_COLS);
+        const bool valid = lane < ncols;
+        int64_t cb = 0;
+        if (valid) {
+          const int64_t c = c0 + lane, a = c / p.B;
+          cb = a * IB + (c - a * p.B);
+        }
+        if (valid)
+          for (int i = 0; i < I; ++i)
+            cp_async_elem<ES>(st + tg_soff<ES>(i, lane, tg_boxb(I)), gb + (cb + (int64_t)i * p.B) * ES);
+        m->colofs[lane] = lane;
+        m->gcol[lane] = cb;
+        if (lane == 0) {
+          m->ncols = ncols;
+          m->rs = TG_COLS;
+          m->sh = 0;
+        }
+        cp_async_arrive(&full[slot]);
+        __syncwarp();
+        if (lane == 0) tg_arrive(&full[slot]);
       }
-      const uint32_t kg = (uint32_t)(q * cpt / 4 + gq);
+      issued = kc + 1;
+    }
+    // no copy may still target this CTA's shared memory at exit
+    if (lane == 0)
+      for (int kc = issued > TG_NS ? issued - TG_NS : 0; kc < issued; ++kc)
+        ptx::mbar_wait(&full[kc % TG_NS], (uint32_t)((kc / TG_NS) & 1), TG_WAIT_NS / 4);
+    __syncwarp();
+  } else if (warp == TG_MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t idesc[3];
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        uint8_t* t = tiles + (size_t)(s * 3 + part) * TG_TILE + kg * TG_LBO;
-        *(uint4*)(t + (uint32_t)i * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
-        *(uint4*)(t + (uint32_t)(I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
-      }
-    }
-  };
-  uint32_t issued[2] = {0, 0}, waited[2] = {0, 0};
-  for (int kc = 0; kc < nch; ++kc) {
-    const int s = kc & 1;
-    // the copies TG_NS - 1 chunks ahead (into the stage chunk kc - 1 used)
-    if (kc + TG_NS - 1 < nch) issue(kc + TG_NS - 1);
-    cp_async_commit();
-    cp_async_wait<TG_NS - 1>();  // this thread's copies of chunk kc have landed
-    // the tiles of stage s are free once chunk kc - 2's MMAs are done
-    if (kc >= 2 && tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
-      atomicOr(p.err, DEV_ERR_TIMEOUT);
-      s_abort = 1;
-    }
-    __syncthreads();
-    if (s_abort) break;
-    if (kc >= 2) {
-      waited[s]++;
+    for (int a = 0; a < 3; ++a) idesc[a] = ptx::idesc_f16(1, 128, a < NA ? tg_n_of(I, a) : 16);
+    // descriptors of set 0's first A tile and of its Y tile; the others by
+    // adding to the start address field, which counts 16-byte units
+    const uint64_t da_base = ptx::sdesc(ptx::smem_u32(tiles), TG_LBO_A, 128);
+    const uint64_t dy_base = ptx::sdesc(ptx::smem_u32(tiles + 3 * TG_TILE_A), TG_LBO_B, 128);
+    int issued[2] = {0, 0};
+    for (int kc = 0; kc < nch; ++kc) {
+      const int t = kc & 1;
+      if (!tg_waitw(&tfull[t], (uint32_t)((kc >> 1) & 1), abort, p.err)) break;
       ptx::tc_fence_after();
-    }
-    convert(kc, s);
-    ptx::fence_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    if (tid == 0) {
-      const uint32_t base = ptx::smem_u32(tiles + (size_t)s * 3 * TG_TILE);
-      // (A part, B part): hh, hm, mh, hl, lh, mm
+      if (lane == 0) {
+        const int nks = tks[t];
+        const uint32_t set = (uint32_t)t * TG_SET;
+        for (int kk = 0; kk < nks; ++kk) {
+          const uint64_t dy = dy_base + ((set + kk * 2 * TG_LBO_B) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int pr = 0; pr < 6; ++pr) {
-          const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
-          const uint32_t ka = base + pa * TG_TILE + kk * 2 * TG_LBO;
-          const uint32_t kb = base + pb * TG_TILE + kk * 2 * TG_LBO;
-          ptx::mma_f16(dt_base, ptx::sdesc(ka, TG_LBO, 128), ptx::sdesc(kb, TG_LBO, 128), idesc,
-                       (kc > 0 || kk > 0 || pr > 0) ? 1u : 0u);
+          for (int a = 0; a < 3; ++a)
+            if (a < NA)
+              ptx::mma_f16(dt_base, da_base + ((set + a * TG_TILE_A + kk * 2 * TG_LBO_A) >> 4), dy, idesc[a],
+                           (kc > 0 || kk > 0 || a > 0) ? 1u : 0u);
         }
-      ptx::mma_commit(&done[s]);
-      issued[s]++;
+        ptx::mma_commit(&tfree[t]);
+      }
+      __syncwarp();
+      issued[t] = (kc >> 1) + 1;
     }
-  }
-  cp_async_wait<0>();  // no copy may still target this CTA's shared memory
-  __syncthreads();
-  bool ok = !s_abort;
-  if (ok && nch > 0) {
-    const int s = (nch - 1) & 1;
-    if (tid == 0 && !ptx::mbar_wait(&done[s], waited[s] & 1u, TG_WAIT_NS)) {
-      atomicOr(p.err, DEV_ERR_TIMEOUT);
-      s_abort = 1;
-    }
-    __syncthreads();
-    ok = !s_abort;
-    ptx::tc_fence_after();
-  }
-  if (ok && warp < 4) {
-    // lane = row of D: rows r < I the real parts of row r, rows I <= r < 2I
-    // the negated imaginary parts of row r - I; columns j < I
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int row = tid;
-    const bool re = row < I;
-    const int64_t orow = re ? row : row - I;
-    float* out = p.partial + (size_t)blockIdx.y * p.I * p.I * 2;
-    for (int c0 = 0; c0 < p.N; c0 += 16) {
-      float y[16];
-      ptx::tmem_ld16(dt_base + lane_base + c0, y);
-      if (row < 2 * I) {
+    // every committed MMA has finished before TMEM is read or freed
+    if (lane == 0)
+      for (int t = 0; t < 2; ++t)
+        if (issued[t] > 0 && !ptx::mbar_wait(&tfree[t], (uint32_t)((issued[t] - 1) & 1), TG_WAIT_NS)) {
+          atomicOr(p.err, DEV_ERR_TIMEOUT);
+          *abort = 1;
+        }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ converters
+    // group g converts the chunks kc = g, g + 2, ... into tile set g; a warp
+    // item is 8 rows x 16 columns, lane = (row, group of four columns), so
+    // that a tile store of the warp covers 8 consecutive rows (128 bytes) of
+    // four K groups
+    const int grp = warp / TG_GROUP_WARPS, gw = warp % TG_GROUP_WARPS;
+    const int rb_n = (I + 7) / 8;
+    const uint32_t boxb = tg_boxb(I);
+    uint8_t* set = tiles + (size_t)grp * TG_SET;
+    for (int kc = grp; kc < nch; kc += 2) {
+      const int slot = kc % TG_NS;
+      if (!tg_waitw(&full[slot], (uint32_t)((kc / TG_NS) & 1), abort, p.err)) break;
+      if (kc >= 2 && !tg_waitw(&tfree[grp], (uint32_t)(((kc >> 1) - 1) & 1), abort, p.err)) break;
+      ptx::tc_fence_after();
+      const TgMeta* m = &meta[slot];
+      const uint8_t* st = stage + slot * STAGE;
+      const int ncols = m->ncols, rs = m->rs, sh = m->sh, bsh = m->bsh;
+      const int nks = (ncols + 7) / 8, ngroups = 2 * nks;
+      const int halves = ngroups > 4 ? 2 : 1;
+      for (int it = gw; it < rb_n * halves; it += TG_GROUP_WARPS) {
+        const int i = (it % rb_n) * 8 + (lane & 7);
+        const int g = (it / rb_n) * 4 + (lane >> 3);
+        if (i >= I || g >= ngroups) continue;
+        const int col0 = 4 * g;
+        // the four elements and their Omega bits, loaded before any use
+        float2 x[4];
+        uint32_t zbits = 0;
+        if (p.mode != TG_SLABS && col0 + 3 < ncols) {
+          if constexpr (ES == 8) {
+            // columns col0..col0+3: two 16-byte units of row i in box g / 4
+            const uint8_t* rowp = st + (uint32_t)(g >> 2) * boxb + (uint32_t)i * 128;
+            const uint32_t c0 = 2u * (uint32_t)(g & 3), sw = (uint32_t)(i & 7);
+            const float4 v0 = *(const float4*)(rowp + ((c0 ^ sw) << 4));
+            const float4 v1 = *(const float4*)(rowp + (((c0 + 1) ^ sw) << 4));
+            x[0] = make_float2(v0.x, v0.y);
+            x[1] = make_float2(v0.z, v0.w);
+            x[2] = make_float2(v1.x, v1.y);
+            x[3] = make_float2(v1.z, v1.w);
+          } else {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = c0 + u;
-          if (j < I) out[(orow * p.I + j) * 2 + (re ? 0 : 1)] = nch > 0 ? (re ? y[u] : -y[u]) : 0.f;
+            for (int u = 0; u < 4; ++u) x[u] = staged_elem<DT>(st + tg_soff<ES>(i, col0 + u, boxb));
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int col = col0 + u;
+            const bool v = col < ncols;
+            if (p.mode == TG_SLABS) {
+              const int off = (v ? m->colofs[col] : 0) + i * rs;
+              x[u] = v ? staged_elem<DT>(st + (size_t)off * ES) : make_float2(0.f, 0.f);
+              if (masked) {
+                const int pos = sh + off;
+                zbits |= ((m->wm[pos >> 5] >> (pos & 31)) & 1u) << u;
+              }
+            } else {
+              x[u] = v ? staged_elem<DT>(st + tg_soff<ES>(i, col, boxb)) : make_float2(0.f, 0.f);
+            }
+          }
+        }
+        if (masked) {
+          if (p.mode == TG_ROWS) {
+            const uint32_t rowbits = __funnelshift_r(m->wm[2 * i], m->wm[2 * i + 1], (uint32_t)(sh + i * bsh) & 31u);
+            zbits = (rowbits >> col0) & 0xFu;
+          } else if (p.mode == TG_ELEMS) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (col0 + u < ncols) zbits |= (uint32_t)mask_bit(p.bits, m->gcol[col0 + u] + (int64_t)i * p.B) << u;
+          }
+        }
+        uint32_t xr[3][4], jr[3][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 v = (zbits >> u) & 1u ? make_float2(0.f, 0.f) : x[u];
+          // x row: (re, im), the three parts of both in packed pairs (the low
+          // half holds the even K); J x row: (-im, re), the halves swapped and
+          // the new low half negated
+          split3_pair(v.x, v.y, xr[0][u], xr[1][u], xr[2][u]);
+#pragma unroll
+          for (int part = 0; part < 3; ++part) jr[part][u] = __byte_perm(xr[part][u], 0u, 0x1032) ^ 0x8000u;
+        }
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          const int at = part / PA, arow = 2 * I * (part % PA);
+          uint8_t* ap = set + (size_t)at * TG_TILE_A + (uint32_t)g * TG_LBO_A;
+          *(uint4*)(ap + (uint32_t)(arow + i) * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
+          *(uint4*)(ap + (uint32_t)(arow + I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
+          uint8_t* yp = set + 3 * TG_TILE_A + (uint32_t)g * TG_LBO_B;
+          *(uint4*)(yp + (uint32_t)(part * I + i) * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
         }
       }
+      ptx::fence_async_smem();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (gw == 0) tks[grp] = nks;
+        tg_arrive(&tfull[grp]);
+        tg_arrive(&sfree[slot]);
+      }
     }
-  } else if (!ok && tid == 0) {
-    // bounded waits for MMAs still in flight
-    for (int st = 0; st < 2; ++st)
-      if (issued[st] > waited[st]) ptx::mbar_wait(&done[st], (issued[st] - 1) & 1u, TG_WAIT_NS / 4);
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(dt_base, p.N <= 32 ? 32 : (p.N <= 64 ? 64 : 128));
+  ptx::tc_fence_after();
+  const bool ok = !*abort;
+  // D (128 lanes x N0 columns) -> shared memory S over the tile sets, which
+  // no MMA reads any more; warp w reads TMEM lanes 32w..32w+31
+  constexpr int SP = 193;  // S row pitch (floats)
+  float* S = (float*)tiles;
+  if (warp < 4) {
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    for (int c0 = 0; c0 < N0; c0 += 16) {
+      float y[16];
+      ptx::tmem_ld16(dt_base + lane_base + c0, y);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) S[tid * SP + c0 + u] = y[u];
+    }
+  }
+  __syncthreads();
+  // stacked row r < 2I (x rows: the real part of row r; J x rows: the
+  // negated imaginary part of row r - I), column j < I: the sum over the A
+  // tile's part slots s and Y's column blocks q, in that order
+  float* out = p.partial + (size_t)blockIdx.x * p.I * p.I * 2;
+  for (int e = tid; e < 2 * I * I; e += TG_THREADS) {
+    const int r = e / I, j = e % I;
+    float v = 0.f;
+    if (ok && nch > 0)
+      for (int s = 0; s < PA; ++s)
+        for (int q = 0; q < 3; ++q) v += S[(2 * I * s + r) * SP + q * I + j];
+    const bool re = r < I;
+    out[((int64_t)(re ? r : r - I) * I + j) * 2 + (re ? 0 : 1)] = re ? v : -v;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(dt_base, tmem_cols);
 }
 
 size_t tg_smem_bytes(int es) {
-  const size_t stage_bytes = ((size_t)64 * TG_SROW * es + 15) / 16 * 16;
-  return 6 * (size_t)TG_TILE + TG_NS * (stage_bytes + 64 * TG_SROW * 4) + TG_NS * TG_COLS * 8 + 2 * 8 + 16;
+  return 2 * (size_t)TG_SET + TG_NS * ((size_t)64 * TG_COLS * es + sizeof(TgMeta)) +
+         (2 * TG_NS + 4) * sizeof(uint64_t) + 2 * sizeof(int) + 16;
 }
 
 struct TcGramGeom {
-  int64_t I, B, ncol, cols_per_split;
-  int nsplit, N, R;
+  int64_t A, I, B, nchunk, chunks_per_split;
+  int nsplit, mode, slabs;
 };
 
-TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n) {
+constexpr int TG_MAX_SPLITS = 148;  // one CTA per SM
+
+// How mode n's unfolding is staged (see gram_tc_kernel) and split over CTAs.
+TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned16) {
   TcGramGeom g;
+  g.A = 1;
   g.B = 1;
-  int64_t A = 1;
-  for (int q = 0; q < n; ++q) A *= dims[q];
+  for (int q = 0; q < n; ++q) g.A *= dims[q];
   for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
   g.I = dims[n];
-  g.ncol = A * g.B;
-  g.N = (int)((g.I + 15) / 16 * 16);
-  g.R = g.I <= 32 ? 32 : 64;
-  // one CTA per SM (a persistent split each); at least four chunks per split;
-  // partials under 32 MB
-  int64_t ns = std::min<int64_t>(148, std::max<int64_t>(1, ceil_div(g.ncol, 4 * TG_COLS)));
-  ns = std::min<int64_t>(ns, std::max<int64_t>(1, (32 << 20) / (8 * g.I * g.I)));
-  g.cols_per_split = ceil_div(ceil_div(g.ncol, ns), TG_COLS) * TG_COLS;
-  g.nsplit = (int)ceil_div(g.ncol, g.cols_per_split);
+  g.slabs = 1;
+  const int64_t total_bytes = g.A * g.I * g.B * es;
+  // TMA coordinates are 32-bit: the column (in 4-byte units for 8-byte
+  // elements) and the slab
+  const bool tma_ok = g.A < (1ll << 31) && 2 * g.B < (1ll << 31);
+  if (aligned16 && g.B < TG_COLS && (TG_COLS / g.B) * g.I * g.B * es % 16 == 0 && total_bytes % 16 == 0) {
+    g.mode = TG_SLABS;
+    g.slabs = (int)(TG_COLS / g.B);
+    g.nchunk = ceil_div(g.A, (int64_t)g.slabs);
+  } else if (aligned16 && tma_ok && g.B % TG_COLS == 0) {
+    g.mode = TG_ROWS;
+    g.nchunk = g.A * g.B / TG_COLS;
+  } else {
+    g.mode = TG_ELEMS;
+    g.nchunk = ceil_div(g.A * g.B, (int64_t)TG_COLS);
+  }
+  const int64_t ns = std::max<int64_t>(1, std::min<int64_t>(TG_MAX_SPLITS, g.nchunk));
+  g.chunks_per_split = ceil_div(g.nchunk, ns);
+  g.nsplit = (int)ceil_div(g.nchunk, g.chunks_per_split);
   return g;
 }
 
@@ -1087,48 +1312,92 @@ cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);
   size_t b = sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
-  if (g.I <= 64) {
-    TcGramGeom t = tc_gram_geom(nd, dims, n);
-    b = std::max(b, sizeof(float2) * (size_t)t.nsplit * t.I * t.I);
-  }
+  if (g.I <= 64) b = std::max(b, sizeof(float2) * (size_t)TG_MAX_SPLITS * g.I * g.I);
   return b;
+}
+
+// The driver's tensor-map encoder, looked up once through the runtime (the
+// library does not link the driver library itself).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+// Tensor map of the unfolding [A][I][B] for TG_ROWS: boxes of 32 columns x
+// I rows of one slab (8-byte elements as pairs of 4-byte ones).
+static cudaError_t rows_tensor_map(CUtensorMap* map, const void* g, int es, const TcGramGeom& t) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return cudaErrorNotSupported;
+  const int ue = es == 8 ? 4 : es;  // unit element bytes
+  const int per = es / ue;
+  const cuuint64_t dim[3] = {(cuuint64_t)(t.B * per), (cuuint64_t)t.I, (cuuint64_t)t.A};
+  const cuuint64_t stride[2] = {(cuuint64_t)(t.B * es), (cuuint64_t)(t.I * t.B * es)};
+  // 128-byte box rows, swizzled (see tg_soff); 2-byte elements: 64-byte rows as they are
+  const cuuint32_t box[3] = {(cuuint32_t)(es == 8 ? 32 : TG_COLS), (cuuint32_t)t.I, 1};
+  const CUtensorMapSwizzle swz = es == 2 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType type = ue == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  const CUresult r = fn(map, type, 3, const_cast<void*>(g), dim, stride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 // Tensor-core Gram for I_n <= 64 (see gram_tc_kernel); the split partials are
 // summed by the same fixed-order fp64 reduction.
 cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
                          int n, float* partial, double* gram, int* err, cudaStream_t s) {
-  const TcGramGeom t = tc_gram_geom(nd, dims, n);
+  const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
+  const TcGramGeom t = tc_gram_geom(nd, dims, n, es, ((uintptr_t)g & 15) == 0);
   TcGramArgs a;
   a.g = g;
   a.bits = bits;
+  a.A = t.A;
   a.I = t.I;
   a.B = t.B;
-  a.ncol = t.ncol;
-  a.cols_per_split = t.cols_per_split;
-  a.N = t.N;
-  a.R = t.R;
+  a.nchunk = t.nchunk;
+  a.chunks_per_split = t.chunks_per_split;
+  a.mode = t.mode;
+  a.slabs = t.slabs;
   a.partial = partial;
   a.err = err;
-  const size_t smem = tg_smem_bytes(dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4));
-  const dim3 grid(1, t.nsplit);
+  CUtensorMap map;
+  memset(&map, 0, sizeof(map));
+  if (t.mode == TG_ROWS) {
+    const cudaError_t e = rows_tensor_map(&map, g, es, t);
+    if (e != cudaSuccess) return e;
+  }
+  const size_t smem = tg_smem_bytes(es);
+  const dim3 grid(t.nsplit);
   cudaError_t e = cudaSuccess;
   switch (dt) {
     case TGD_R32:
       e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) gram_tc_kernel<TGD_R32><<<grid, TG_THREADS, smem, s>>>(a);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R32><<<grid, TG_THREADS, smem, s>>>(a, map);
       break;
     case TGD_C64:
       e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) gram_tc_kernel<TGD_C64><<<grid, TG_THREADS, smem, s>>>(a);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C64><<<grid, TG_THREADS, smem, s>>>(a, map);
       break;
     case TGD_C32H:
       e = cudaFuncSetAttribute(gram_tc_kernel<TGD_C32H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) gram_tc_kernel<TGD_C32H><<<grid, TG_THREADS, smem, s>>>(a);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_C32H><<<grid, TG_THREADS, smem, s>>>(a, map);
       break;
     case TGD_R16:
       e = cudaFuncSetAttribute(gram_tc_kernel<TGD_R16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) gram_tc_kernel<TGD_R16><<<grid, TG_THREADS, smem, s>>>(a);
+      if (e == cudaSuccess) gram_tc_kernel<TGD_R16><<<grid, TG_THREADS, smem, s>>>(a, map);
       break;
     default:
       return cudaErrorInvalidValue;
