@@ -329,13 +329,10 @@ constexpr int TG_GROUP_WARPS = 4;           // converter warps per tile set
 constexpr int TG_PROD_WARP = TG_CONV_WARPS;
 constexpr int TG_MMA_WARP = TG_CONV_WARPS + 1;
 constexpr int TG_THREADS = 32 * (TG_CONV_WARPS + 2);
-constexpr int TG_COLS = 32;                 // column capacity of a chunk
-constexpr int TG_NS = 4;                    // staging stages
+constexpr int TG_COLS = 32;                 // columns of a TG_ROWS / TG_ELEMS chunk
+constexpr int TG_KC_MAX = 64;               // column capacity of a chunk (TG_SLABS may take 64)
+constexpr int TG_NS_MAX = 4;                // staging stages
 constexpr uint32_t TG_LBO_A = 2048;         // A tile: 128 rows x 16 B between K core matrices
-constexpr uint32_t TG_TILE_A = 8 * TG_LBO_A;
-constexpr uint32_t TG_LBO_B = 3072;         // Y tile: 192 rows x 16 B
-constexpr uint32_t TG_TILE_B = 8 * TG_LBO_B;
-constexpr uint32_t TG_SET = 3 * TG_TILE_A + TG_TILE_B;   // one tile set: up to three A tiles and Y
 constexpr int TG_MASK_WORDS = 128;          // two per row, or a block of <= 2048 bits + 1
 constexpr uint64_t TG_WAIT_NS = 2000000000ull;
 
@@ -349,6 +346,8 @@ struct TcGramArgs {
   int64_t chunks_per_split;
   int mode;                   // TgMode
   int slabs;                  // slabs per chunk (TG_SLABS)
+  int kc;                     // column capacity of a chunk: 32, or 64 (TG_SLABS)
+  int ns;                     // staging stages
   float* partial;             // [split][I][I] complex, interleaved
   int* err;
 };
@@ -359,7 +358,7 @@ struct TgMeta {
   int rs;                     // staged stride between rows (elements)
   int sh;                     // bit offset in its first word: of the block (TG_SLABS), of row 0 (TG_ROWS)
   int bsh;                    // TG_ROWS: B mod 32 (row i's offset is sh + i bsh, mod 32)
-  int colofs[TG_COLS];        // staged offset of each column's row 0 (elements)
+  int colofs[TG_KC_MAX];      // staged offset of each column's row 0 (elements)
   int64_t gcol[TG_COLS];      // TG_ELEMS: element index of each column's row 0
   uint32_t wm[TG_MASK_WORDS]; // Omega's words: two per row (TG_ROWS), the block's (TG_SLABS)
 };
@@ -390,6 +389,24 @@ __host__ __device__ constexpr int tg_a_tiles(int I) { return (3 + tg_parts_per_a
 // MMA N of A tile a: the Y part blocks its parts need (p + q <= 2 for the
 // tile's first part p), rounded up to 16.
 __host__ __device__ constexpr int tg_n_of(int I, int a) { return ((3 - a * tg_parts_per_a(I)) * I + 15) / 16 * 16; }
+
+// Shared-memory layout for mode size I, chunk capacity kc and element size
+// es: a tile set holds the A tiles (128 rows x 2 kc bf16 values each) and Y
+// (N0 rows); a stage holds a chunk (the swizzled boxes, or a block).
+struct TgLayout {
+  uint32_t tile_a, lbo_b, set, stage;
+};
+__host__ __device__ inline TgLayout tg_layout(int I, int kc, int es) {
+  TgLayout L;
+  const uint32_t kg = (uint32_t)kc / 4;
+  L.tile_a = kg * TG_LBO_A;
+  L.lbo_b = (uint32_t)tg_n_of(I, 0) * 16;
+  L.set = (uint32_t)tg_a_tiles(I) * L.tile_a + kg * L.lbo_b;
+  uint32_t st = (uint32_t)kc * I * es;
+  if (es == 8 && 2 * tg_boxb(I) > st) st = 2 * tg_boxb(I);
+  L.stage = (st + 1023) / 1024 * 1024;
+  return L;
+}
 
 // x = h + m + l (bf16 parts, each the rounding of what the earlier leave).
 // The three parts of x and y at once, packed as bf16 pairs (x in the low
@@ -469,14 +486,16 @@ template <int DT>
 __global__ void __launch_bounds__(TG_THREADS, 1)
     gram_tc_kernel(const TcGramArgs p, const __grid_constant__ CUtensorMap rows_map) {
   constexpr int ES = Dt<DT>::bytes;
-  constexpr uint32_t STAGE = 64 * TG_COLS * ES;                // a dense 64 x 32 box, or a block of <= 2048 elements
+  const TgLayout L = tg_layout((int)p.I, p.kc, ES);
+  const int NS = p.ns;
+  const uint32_t STAGE = L.stage;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* tiles = smem;                                        // [2] tile sets
-  uint8_t* stage = smem + 2 * TG_SET;                           // [TG_NS] staged chunks
-  TgMeta* meta = (TgMeta*)(stage + TG_NS * STAGE);              // [TG_NS]
-  uint64_t* full = (uint64_t*)(meta + TG_NS);                   // [TG_NS] chunk staged
-  uint64_t* sfree = full + TG_NS;                               // [TG_NS] stage read
-  uint64_t* tfull = sfree + TG_NS;                              // [2] tile set written
+  uint8_t* stage = smem + 2 * L.set;                            // [NS] staged chunks
+  TgMeta* meta = (TgMeta*)(stage + NS * STAGE);                 // [NS]
+  uint64_t* full = (uint64_t*)(meta + NS);                      // [NS] chunk staged
+  uint64_t* sfree = full + TG_NS_MAX;                           // [NS] stage read
+  uint64_t* tfull = sfree + TG_NS_MAX;                              // [2] tile set written
   uint64_t* tfree = tfull + 2;                                  // [2] tile set's MMAs done
   int* tks = (int*)(tfree + 2);                                 // [2] K steps of the set's chunk
   uint32_t* tslot = (uint32_t*)(tks + 2);
@@ -493,10 +512,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   const int nch = q_end > q_begin ? (int)(q_end - q_begin) : 0;
   const bool masked = p.bits != nullptr;
   // rows no part uses stay zero in every tile
-  for (uint32_t o = tid * 16; o < 2 * TG_SET; o += TG_THREADS * 16) *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
+  for (uint32_t o = tid * 16; o < 2 * L.set; o += TG_THREADS * 16) *(uint4*)(tiles + o) = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
     s_abort = 0;
-    for (int s = 0; s < TG_NS; ++s) {
+    for (int s = 0; s < NS; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&sfree[s], TG_GROUP_WARPS);
     }
@@ -517,9 +536,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   if (warp == TG_PROD_WARP) {
     // ------------------------------------------------------------ producer
     int issued = 0;
+    // TG_SLABS: staged offset of column lane (and lane + 32) of a block
+    const int co_lo = (int)((lane / p.B) * IB + lane % p.B);
+    const int co_hi = (int)(((lane + 32) / p.B) * IB + (lane + 32) % p.B);
     for (int kc = 0; kc < nch; ++kc) {
-      const int slot = kc % TG_NS;
-      if (kc >= TG_NS && !tg_waitw(&sfree[slot], (uint32_t)((kc / TG_NS - 1) & 1), abort, p.err)) break;
+      const int slot = kc % NS;
+      if (kc >= NS && !tg_waitw(&sfree[slot], (uint32_t)((kc / NS - 1) & 1), abort, p.err)) break;
       TgMeta* m = &meta[slot];
       uint8_t* st = stage + slot * STAGE;
       const int64_t q = q_begin + kc;
@@ -532,7 +554,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
           const int64_t w0 = blk >> 5, nw = ((blk + nel - 1) >> 5) - w0 + 1;
           for (int w = lane; w < nw; w += 32) cp_async_elem<4>(&m->wm[w], p.bits + w0 + w);
         }
-        m->colofs[lane] = lane < ncols ? (int)((lane / p.B) * IB + lane % p.B) : 0;
+        m->colofs[lane] = co_lo;
+        m->colofs[lane + 32] = co_hi;
         if (lane == 0) {
           m->ncols = ncols;
           m->rs = (int)p.B;
@@ -606,8 +629,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
     }
     // no copy may still target this CTA's shared memory at exit
     if (lane == 0)
-      for (int kc = issued > TG_NS ? issued - TG_NS : 0; kc < issued; ++kc)
-        ptx::mbar_wait(&full[kc % TG_NS], (uint32_t)((kc / TG_NS) & 1), TG_WAIT_NS / 4);
+      for (int kc = issued > NS ? issued - NS : 0; kc < issued; ++kc)
+        ptx::mbar_wait(&full[kc % NS], (uint32_t)((kc / NS) & 1), TG_WAIT_NS / 4);
     __syncwarp();
   } else if (warp == TG_MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -617,7 +640,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
     // descriptors of set 0's first A tile and of its Y tile; the others by
     // adding to the start address field, which counts 16-byte units
     const uint64_t da_base = ptx::sdesc(ptx::smem_u32(tiles), TG_LBO_A, 128);
-    const uint64_t dy_base = ptx::sdesc(ptx::smem_u32(tiles + 3 * TG_TILE_A), TG_LBO_B, 128);
+    const uint64_t dy_base = ptx::sdesc(ptx::smem_u32(tiles + NA * L.tile_a), L.lbo_b, 128);
     int issued[2] = {0, 0};
     for (int kc = 0; kc < nch; ++kc) {
       const int t = kc & 1;
@@ -625,13 +648,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
       ptx::tc_fence_after();
       if (lane == 0) {
         const int nks = tks[t];
-        const uint32_t set = (uint32_t)t * TG_SET;
+        const uint32_t set = (uint32_t)t * L.set;
         for (int kk = 0; kk < nks; ++kk) {
-          const uint64_t dy = dy_base + ((set + kk * 2 * TG_LBO_B) >> 4);
+          const uint64_t dy = dy_base + ((set + kk * 2 * L.lbo_b) >> 4);
 #pragma unroll
           for (int a = 0; a < 3; ++a)
             if (a < NA)
-              ptx::mma_f16(dt_base, da_base + ((set + a * TG_TILE_A + kk * 2 * TG_LBO_A) >> 4), dy, idesc[a],
+              ptx::mma_f16(dt_base, da_base + ((set + a * L.tile_a + kk * 2 * TG_LBO_A) >> 4), dy, idesc[a],
                            (kc > 0 || kk > 0 || a > 0) ? 1u : 0u);
         }
         ptx::mma_commit(&tfree[t]);
@@ -656,17 +679,17 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
     const int grp = warp / TG_GROUP_WARPS, gw = warp % TG_GROUP_WARPS;
     const int rb_n = (I + 7) / 8;
     const uint32_t boxb = tg_boxb(I);
-    uint8_t* set = tiles + (size_t)grp * TG_SET;
+    uint8_t* set = tiles + (size_t)grp * L.set;
     for (int kc = grp; kc < nch; kc += 2) {
-      const int slot = kc % TG_NS;
-      if (!tg_waitw(&full[slot], (uint32_t)((kc / TG_NS) & 1), abort, p.err)) break;
+      const int slot = kc % NS;
+      if (!tg_waitw(&full[slot], (uint32_t)((kc / NS) & 1), abort, p.err)) break;
       if (kc >= 2 && !tg_waitw(&tfree[grp], (uint32_t)(((kc >> 1) - 1) & 1), abort, p.err)) break;
       ptx::tc_fence_after();
       const TgMeta* m = &meta[slot];
       const uint8_t* st = stage + slot * STAGE;
       const int ncols = m->ncols, rs = m->rs, sh = m->sh, bsh = m->bsh;
       const int nks = (ncols + 7) / 8, ngroups = 2 * nks;
-      const int halves = ngroups > 4 ? 2 : 1;
+      const int halves = (ngroups + 3) / 4;
       for (int it = gw; it < rb_n * halves; it += TG_GROUP_WARPS) {
         const int i = (it % rb_n) * 8 + (lane & 7);
         const int g = (it / rb_n) * 4 + (lane >> 3);
@@ -731,10 +754,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
 #pragma unroll
         for (int part = 0; part < 3; ++part) {
           const int at = part / PA, arow = 2 * I * (part % PA);
-          uint8_t* ap = set + (size_t)at * TG_TILE_A + (uint32_t)g * TG_LBO_A;
+          uint8_t* ap = set + (size_t)at * L.tile_a + (uint32_t)g * TG_LBO_A;
           *(uint4*)(ap + (uint32_t)(arow + i) * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
           *(uint4*)(ap + (uint32_t)(arow + I + i) * 16) = make_uint4(jr[part][0], jr[part][1], jr[part][2], jr[part][3]);
-          uint8_t* yp = set + 3 * TG_TILE_A + (uint32_t)g * TG_LBO_B;
+          uint8_t* yp = set + NA * L.tile_a + (uint32_t)g * L.lbo_b;
           *(uint4*)(yp + (uint32_t)(part * I + i) * 16) = make_uint4(xr[part][0], xr[part][1], xr[part][2], xr[part][3]);
         }
       }
@@ -754,7 +777,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   const bool ok = !*abort;
   // D (128 lanes x N0 columns) -> shared memory S over the tile sets, which
   // no MMA reads any more; warp w reads TMEM lanes 32w..32w+31
-  constexpr int SP = 193;  // S row pitch (floats)
+  const int SP = N0 + 1;  // S row pitch (floats)
   float* S = (float*)tiles;
   if (warp < 4) {
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -784,19 +807,23 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   if (warp == 0) ptx::tmem_dealloc(dt_base, tmem_cols);
 }
 
-size_t tg_smem_bytes(int es) {
-  return 2 * (size_t)TG_SET + TG_NS * ((size_t)64 * TG_COLS * es + sizeof(TgMeta)) +
-         (2 * TG_NS + 4) * sizeof(uint64_t) + 2 * sizeof(int) + 16;
+size_t tg_smem_bytes(int I, int kc, int es, int ns) {
+  const TgLayout L = tg_layout(I, kc, es);
+  return 2 * (size_t)L.set + (size_t)ns * (L.stage + sizeof(TgMeta)) + (2 * TG_NS_MAX + 4) * sizeof(uint64_t) +
+         2 * sizeof(int) + 16;
 }
 
 struct TcGramGeom {
   int64_t A, I, B, nchunk, chunks_per_split;
-  int nsplit, mode, slabs;
+  int nsplit, mode, slabs, kc, ns;
 };
 
 constexpr int TG_MAX_SPLITS = 148;  // one CTA per SM
+constexpr size_t TG_SMEM_LIMIT = 227 * 1024 - 1024;  // the opt-in maximum less the static part
 
-// How mode n's unfolding is staged (see gram_tc_kernel) and split over CTAs.
+// How mode n's unfolding is staged (see gram_tc_kernel) and split over CTAs:
+// the mode, the chunk capacity (64 columns for blocks of whole slabs when it
+// fits, else 32) and the most stages (up to four) that fit.
 TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned16) {
   TcGramGeom g;
   g.A = 1;
@@ -805,21 +832,37 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned
   for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
   g.I = dims[n];
   g.slabs = 1;
+  g.kc = TG_COLS;
+  const int I = (int)g.I;
   const int64_t total_bytes = g.A * g.I * g.B * es;
   // TMA coordinates are 32-bit: the column (in 4-byte units for 8-byte
   // elements) and the slab
   const bool tma_ok = g.A < (1ll << 31) && 2 * g.B < (1ll << 31);
-  if (aligned16 && g.B < TG_COLS && (TG_COLS / g.B) * g.I * g.B * es % 16 == 0 && total_bytes % 16 == 0) {
+  auto slabs_ok = [&](int kc) {
+    return aligned16 && g.B < kc && (kc / g.B) * g.I * g.B * es % 16 == 0 && total_bytes % 16 == 0;
+  };
+  auto fits = [&](int kc, int ns) { return tg_smem_bytes(I, kc, es, ns) <= TG_SMEM_LIMIT; };
+  // (a 64-column block of I <= 32 rows needs at most 65 of the mask words)
+  if (I <= 32 && g.B < TG_COLS && slabs_ok(TG_KC_MAX) && fits(TG_KC_MAX, 2)) {
     g.mode = TG_SLABS;
-    g.slabs = (int)(TG_COLS / g.B);
-    g.nchunk = ceil_div(g.A, (int64_t)g.slabs);
+    g.kc = TG_KC_MAX;
+  } else if (slabs_ok(TG_COLS)) {
+    g.mode = TG_SLABS;
   } else if (aligned16 && tma_ok && g.B % TG_COLS == 0) {
     g.mode = TG_ROWS;
-    g.nchunk = g.A * g.B / TG_COLS;
   } else {
     g.mode = TG_ELEMS;
+  }
+  if (g.mode == TG_SLABS) {
+    g.slabs = (int)(g.kc / g.B);
+    g.nchunk = ceil_div(g.A, (int64_t)g.slabs);
+  } else if (g.mode == TG_ROWS) {
+    g.nchunk = g.A * g.B / TG_COLS;
+  } else {
     g.nchunk = ceil_div(g.A * g.B, (int64_t)TG_COLS);
   }
+  g.ns = TG_NS_MAX;
+  while (g.ns > 2 && !fits(g.kc, g.ns)) --g.ns;
   const int64_t ns = std::max<int64_t>(1, std::min<int64_t>(TG_MAX_SPLITS, g.nchunk));
   g.chunks_per_split = ceil_div(g.nchunk, ns);
   g.nsplit = (int)ceil_div(g.nchunk, g.chunks_per_split);
@@ -843,6 +886,18 @@ __device__ double block_sum(double v, double* red) {
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
   __syncthreads();
   return t;
+}
+
+// Block-wide maximum (every thread gets it); red as for block_sum.
+__device__ double block_max(double v, double* red) {
+  for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double m = -INFINITY;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmax(m, red[w]);
+  __syncthreads();
+  return m;
 }
 
 __global__ void __launch_bounds__(ET) eig_kernel(const EigJob* jobs) {
@@ -1253,6 +1308,260 @@ __global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
     for (int e = threadIdx.x; e < n * n; e += blockDim.x) ((double2*)J.vprev)[e] = Vt[e];
 }
 
+// Hermitian Jacobi for n <= 64, the same rotations and ordering as
+// eig_block_kernel, laid out for speed: A and the eigenvector rows Vt both
+// whole in shared memory with an odd row pitch (a column walk by 32 lanes
+// touches 32 different banks), one warp per rotation pair, and each round
+// in two phases (J^H on the pairs' rows, then J on their columns and on V)
+// so that every access is a plain load or store of one entry.
+constexpr int ES_MAXN = 64;
+
+__global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
+  const EigJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  if (n > ES_MAXN) return;
+  const int NP = n + 1 + (n & 1);  // odd row pitch
+  extern __shared__ double2 dyn[];
+  double2* A = dyn;                // [n][NP]
+  double2* Vt = dyn + n * NP;      // [n][NP]: row k = eigenvector k
+  __shared__ int rp[ES_MAXN / 2], rq[ES_MAXN / 2], rrot[ES_MAXN / 2];
+  __shared__ double rcs[ES_MAXN / 2], rsn[ES_MAXN / 2];
+  __shared__ double2 rph[ES_MAXN / 2];
+  __shared__ double red[ET / 32];
+  __shared__ double ev[ES_MAXN];
+  __shared__ int col_of_rank[ES_MAXN];
+  __shared__ uint8_t lead[ES_MAXN];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  const double2* G = (const double2*)J.gram;
+  if (J.warm) {
+    // Start from the previous refresh's eigenvectors V (rows of Vt): A =
+    // V^H G V is nearly diagonal when the subspaces move little between
+    // refreshes. Jacobi converges from any unitary start.
+    const double2* Vp = (const double2*)J.vprev;
+    double2* W = (double2*)J.work + (size_t)n * n;  // W = G V (n x n)
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int k = e / n, i = e - k * n;
+      Vt[k * NP + i] = Vp[e];
+    }
+    __syncthreads();
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int i = e / n, l = e - i * n;
+      double2 acc = make_double2(0.0, 0.0);
+      for (int j = 0; j < n; ++j) {
+        const double2 g = G[i * n + j], v = Vt[l * NP + j];
+        acc.x += g.x * v.x - g.y * v.y;
+        acc.y += g.x * v.y + g.y * v.x;
+      }
+      W[e] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int k = e / n, l = e - k * n;
+      if (l < k) continue;
+      double2 acc = make_double2(0.0, 0.0);  // sum_i conj(V[i][k]) W[i][l]
+      for (int i = 0; i < n; ++i) {
+        const double2 v = Vt[k * NP + i], w = W[i * n + l];
+        acc.x += v.x * w.x + v.y * w.y;
+        acc.y += v.x * w.y - v.y * w.x;
+      }
+      if (l == k) acc.y = 0.0;  // Hermitian: a real diagonal
+      A[k * NP + l] = acc;
+      A[l * NP + k] = make_double2(acc.x, -acc.y);
+    }
+  } else {
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int i = e / n, j = e - i * n;
+      // the upper triangle of G, mirrored (G is Hermitian up to rounding)
+      const double2 g = i <= j ? G[i * n + j] : G[j * n + i];
+      A[i * NP + j] = i <= j ? g : make_double2(g.x, -g.y);
+      if (i == j) A[i * NP + j].y = 0.0;
+      Vt[i * NP + j] = make_double2(i == j ? 1.0 : 0.0, 0.0);
+    }
+  }
+  __syncthreads();
+  double part = 0;
+  for (int e = tid; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e - i * n;
+    part += zabs2(A[i * NP + j]);
+  }
+  const double fro = block_sum(part, red);
+  const int m = n + (n & 1);
+  const int npairs = m / 2;
+  const int r = J.r;
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    // Stop when A is diagonal to 1e-24 of its squared Frobenius norm, or
+    // when the r rows of the largest diagonal entries are (their off-diagonal
+    // mass below the same bound: those diagonal entries and rows of Vt are
+    // eigenpairs) and a Gershgorin bound puts every eigenvalue of the other
+    // rows' block below the smallest of them (so they are the r leading).
+    for (int i = tid; i < n; i += blockDim.x) {
+      const double di = A[i * NP + i].x;
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const double dj = A[j * NP + j].x;
+        rank += (dj > di) || (dj == di && j < i);
+      }
+      lead[i] = rank < r;
+    }
+    __syncthreads();
+    double off_part = 0, lead_part = 0, ger_part = -INFINITY, low_part = INFINITY;
+    for (int i = wid; i < n; i += nw) {
+      double row = 0, rad = 0;
+      for (int j = lane; j < n; j += 32) {
+        if (j == i) continue;
+        const double a2 = zabs2(A[i * NP + j]);
+        row += a2;
+        if (!lead[j]) rad += sqrt(a2);
+      }
+      for (int o = 16; o; o >>= 1) {
+        row += __shfl_xor_sync(0xffffffffu, row, o);
+        rad += __shfl_xor_sync(0xffffffffu, rad, o);
+      }
+      if (lane == 0) {
+        const double di = A[i * NP + i].x;
+        off_part += row;
+        if (lead[i]) {
+          lead_part += row;
+          low_part = fmin(low_part, di);
+        } else {
+          ger_part = fmax(ger_part, di + rad);
+        }
+      }
+    }
+    const double off = block_sum(off_part, red);
+    const double lead_off = block_sum(lead_part, red);
+    const double ger = block_max(ger_part, red);
+    const double low = -block_max(-low_part, red);
+    if (off <= 1e-24 * fro || off == 0.0) break;
+    // (the rows' coupling, at most sqrt(lead_off), moves no eigenvalue further)
+    if (r < n && lead_off <= 1e-24 * fro && ger + 2.0 * sqrt(lead_off) < low) break;
+    for (int round = 0; round < m - 1; ++round) {
+      // the round's disjoint pairs (round-robin) and their rotations
+      for (int k = tid; k < npairs; k += blockDim.x) {
+        int p, q;
+        if (k == 0) {
+          p = round;
+          q = m - 1;
+        } else {
+          p = (round + k) % (m - 1);
+          q = (round - k + (m - 1)) % (m - 1);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        rp[k] = p;
+        rq[k] = q;
+        rrot[k] = 0;
+        if (q < n) {  // the dummy index of odd n is absent
+          const double2 apq = A[p * NP + q];
+          const double r2 = zabs2(apq);
+          if (r2 > 0.0) {
+            // the same rotation with one reciprocal square root per quantity:
+            // 1/r, then t = sign(tau) / (|tau| + sqrt(1 + tau^2)), c = 1/sqrt(1 + t^2)
+            const double app = A[p * NP + p].x, aqq = A[q * NP + q].x;
+            const double rinv = rsqrt(r2);
+            const double tau = (aqq - app) * 0.5 * rinv;
+            const double t = (tau >= 0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+            const double c = rsqrt(1.0 + t * t);
+            rrot[k] = 1;
+            rcs[k] = c;
+            rsn[k] = t * c;
+            rph[k] = make_double2(apq.x * rinv, apq.y * rinv);
+          }
+        }
+      }
+      __syncthreads();
+      // rows p, q <- J^H (rows p, q)
+      for (int k = wid; k < npairs; k += nw) {
+        if (!rrot[k]) continue;
+        const int p = rp[k], q = rq[k];
+        const double c = rcs[k], s = rsn[k];
+        const double2 e = rph[k];
+        for (int j = lane; j < n; j += 32) {
+          const double2 xp = A[p * NP + j], xq = zmul(A[q * NP + j], e);
+          A[p * NP + j] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          A[q * NP + j] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+      }
+      __syncthreads();
+      // columns p, q <- (columns p, q) J, and V <- V J on the rows of Vt;
+      // the rotation leaves (p, q) zero and the diagonal real
+      for (int k = wid; k < npairs; k += nw) {
+        if (!rrot[k]) continue;
+        const int p = rp[k], q = rq[k];
+        const double c = rcs[k], s = rsn[k];
+        const double2 ec = make_double2(rph[k].x, -rph[k].y);
+        for (int i = lane; i < n; i += 32) {
+          double2 xp = A[i * NP + p], xq = zmul(A[i * NP + q], ec);
+          double2 np = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          double2 nq = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          if (i == p) {
+            np.y = 0.0;
+            nq = make_double2(0.0, 0.0);
+          } else if (i == q) {
+            np = make_double2(0.0, 0.0);
+            nq.y = 0.0;
+          }
+          A[i * NP + p] = np;
+          A[i * NP + q] = nq;
+          xp = Vt[p * NP + i];
+          xq = zmul(Vt[q * NP + i], ec);
+          Vt[p * NP + i] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          Vt[q * NP + i] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < n; i += blockDim.x) ev[i] = A[i * NP + i].x;
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const double li = ev[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += (ev[j] > li) || (ev[j] == li && j < i);
+    col_of_rank[rank] = i;
+    J.evals[rank] = li;
+  }
+  __syncthreads();
+  // the leading r vectors, each scaled by the unit phase that makes its
+  // largest-magnitude entry (ties to the lowest row) real and positive
+  for (int rr = wid; rr < J.r; rr += nw) {
+    const int c = col_of_rank[rr];
+    double best = -1.0;
+    int bi = 0;
+    for (int row = lane; row < n; row += 32) {
+      const double mg = zabs2(Vt[c * NP + row]);
+      if (mg > best) {
+        best = mg;
+        bi = row;
+      }
+    }
+    for (int o = 16; o; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    const double2 piv = Vt[c * NP + bi];
+    const double pm = sqrt(zabs2(piv));
+    const double2 ph = pm > 0 ? make_double2(piv.x / pm, -piv.y / pm) : make_double2(1.0, 0.0);
+    for (int row = lane; row < n; row += 32) {
+      const double2 u = zmul(Vt[c * NP + row], ph);
+      ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
+    }
+  }
+  // the eigenvectors, the start of the next refresh
+  if (J.vprev)
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int k = e / n, i = e - k * n;
+      ((double2*)J.vprev)[e] = Vt[k * NP + i];
+    }
+}
+
 // ------------------------------------------------------- DCT column selection
 // The dynamic column selection of the Trion / DCT-AdamW page as a factor
 // basis: thread j holds column q_j of the orthonormal DCT matrix (entry (k, j)
@@ -1371,6 +1680,8 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
   a.chunks_per_split = t.chunks_per_split;
   a.mode = t.mode;
   a.slabs = t.slabs;
+  a.kc = t.kc;
+  a.ns = t.ns;
   a.partial = partial;
   a.err = err;
   CUtensorMap map;
@@ -1379,7 +1690,8 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
     const cudaError_t e = rows_tensor_map(&map, g, es, t);
     if (e != cudaSuccess) return e;
   }
-  const size_t smem = tg_smem_bytes(es);
+  const size_t smem = tg_smem_bytes((int)t.I, t.kc, es, t.ns);
+  if (smem > TG_SMEM_LIMIT) return cudaErrorInvalidValue;
   const dim3 grid(t.nsplit);
   cudaError_t e = cudaSuccess;
   switch (dt) {
@@ -1445,6 +1757,27 @@ size_t eig_work_doubles(int n) { return (size_t)4 * n * n; }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
+  // every matrix n <= 64: the whole-matrix kernel
+  bool all_64 = true;
+  size_t ssmem = 16;
+  for (int j = 0; j < njobs; ++j) {
+    const int n = jobs_host[j].n;
+    if (n > ES_MAXN || jobs_host[j].r > n) {
+      all_64 = false;
+      break;
+    }
+    const size_t np = (size_t)n + 1 + (n & 1);
+    ssmem = std::max(ssmem, 2 * sizeof(double2) * (size_t)n * np);
+  }
+  if (all_64) {
+    cudaError_t e = cudaFuncSetAttribute(eig_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ssmem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    eig_small_kernel<<<njobs, ET, ssmem, s>>>(jobs_dev);
+    return cudaGetLastError();
+  }
   bool all_small = true;
   size_t bsmem = 16;
   for (int j = 0; j < njobs; ++j) {
