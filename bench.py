@@ -314,8 +314,11 @@ class Bench:
         nt = wl.n_tensors
         self.concurrent = nt > 1 and not args.sequential and concurrent_default
         n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        sm_budget = max(1, n_sms // nt) if self.concurrent else 0
-        self.streams = [torch.cuda.Stream(device=dev) for _ in range(nt)] if self.concurrent else None
+        # tensors go round-robin onto ns streams, each with 1/ns of the SMs
+        ns = min(nt, args.tensor_streams) if args.tensor_streams > 0 else nt
+        self.n_streams = ns if self.concurrent else 1
+        sm_budget = max(1, n_sms // ns) if self.concurrent else 0
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(ns)] if self.concurrent else None
         self.tensors = []
         for gseed, wseed in tensor_seeds(rank, nt):
             gs = GradientStream(wl.shape, wl.gen_ranks, wl.dtype, seed=gseed,
@@ -346,9 +349,10 @@ class Bench:
         main = torch.cuda.current_stream()
         fork = torch.cuda.Event()
         fork.record(main)
-        for (opt, grads, w), st in zip(self.tensors, self.streams):
+        for st in self.streams:
             st.wait_event(fork)
-            with torch.cuda.stream(st):
+        for j, (opt, grads, w) in enumerate(self.tensors):
+            with torch.cuda.stream(self.streams[j % len(self.streams)]):
                 opt.step(grads[i % 2], w)
         for st in self.streams:
             join = torch.cuda.Event()
@@ -445,7 +449,7 @@ def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs, opts=N
            "shape": list(wl.shape), "ranks": list(wl.ranks), "tensors_per_gpu": len(b.tensors),
            "T": wl.T, "grad_dtype": wl.dtype, "kernel_path": b.tensors[0][0].info["path"],
            "l2": "flushed between steps" if b.flush else "inputs larger than L2",
-           "tensor_streams": ("one stream per tensor, 1/%d of the SMs each" % wl.n_tensors)
+           "tensor_streams": ("%d streams, tensors round-robin, 1/%d of the SMs each" % (b.n_streams, b.n_streams))
            if b.concurrent else "one stream",
            "roofline": dict(step_roofline(wl, len(b.tensors), step_ms, hbm_gbs), peak=hbm_gbs,
                             unit="GB/s", bound="hbm"),
@@ -506,6 +510,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--out-dir", default=os.path.join(ROOT, "bench_out"),
                     help="directory for the per-rank clock records")
+    ap.add_argument("--tensor-streams", type=int, default=0,
+                    help="streams the tensors of a multi-tensor workload are spread over "
+                         "(each with that share of the SMs); 0 = one per tensor")
     ap.add_argument("--sequential", action="store_true",
                     help="step the tensors of a multi-tensor workload one after another on one "
                          "stream (default: each on its own stream with an equal share of the SMs)")
@@ -598,7 +605,7 @@ def main():
                    "kernel_path": tensors[0][0].info["path"],
                    "l2": "flushed between steps" if b.flush else "inputs larger than L2",
                    "parallelism": f"independent tensors per rank x{world}",
-                   "tensor_streams": "one stream per tensor, 1/%d of the SMs each" % wl.n_tensors
+                   "tensor_streams": "%d streams, tensors round-robin, 1/%d of the SMs each" % (b.n_streams, b.n_streams)
                    if b.concurrent else "one stream"},
         "roofline": dict({"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
                           "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,

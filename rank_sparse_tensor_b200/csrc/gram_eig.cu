@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
   }
 }
 
-// ------------------------------------------------ tensor-core Gram (I_n <= 64)
+// ------------------------------------------------ tensor-core Gram (I_n <= 128)
 // The Gram as tcgen05 GEMMs over chunks of at most 32 unfolding columns
 // (K = (column, re/im) pairs: 64 bf16 values). Each fp32 value is split into
 // three bf16 parts h + m + l (each the bf16 rounding of what the earlier
@@ -333,7 +333,7 @@ constexpr int TG_COLS = 32;                 // columns of a TG_ROWS / TG_ELEMS c
 constexpr int TG_KC_MAX = 64;               // column capacity of a chunk (TG_SLABS may take 64)
 constexpr int TG_NS_MAX = 4;                // staging stages
 constexpr uint32_t TG_LBO_A = 2048;         // A tile: 128 rows x 16 B between K core matrices
-constexpr int TG_MASK_WORDS = 128;          // two per row, or a block of <= 2048 bits + 1
+constexpr int TG_MASK_WORDS = 256;          // two per row, or a block of <= 4096 bits + 1
 constexpr uint64_t TG_WAIT_NS = 2000000000ull;
 
 enum TgMode { TG_ROWS = 0, TG_SLABS = 1, TG_ELEMS = 2 };
@@ -346,8 +346,9 @@ struct TcGramArgs {
   int64_t chunks_per_split;
   int mode;                   // TgMode
   int slabs;                  // slabs per chunk (TG_SLABS)
-  int kc;                     // column capacity of a chunk: 32, or 64 (TG_SLABS)
+  int kc;                     // column capacity of a chunk: 16, 32, or 64 (TG_SLABS)
   int ns;                     // staging stages
+  int parts;                  // bf16 parts per value: 3, or 2 for 16-bit inputs (I > 64)
   float* partial;             // [split][I][I] complex, interleaved
   int* err;
 };
@@ -393,17 +394,25 @@ __host__ __device__ constexpr int tg_n_of(int I, int a) { return ((3 - a * tg_pa
 // Shared-memory layout for mode size I, chunk capacity kc and element size
 // es: a tile set holds the A tiles (128 rows x 2 kc bf16 values each) and Y
 // (N0 rows); a stage holds a chunk (the swizzled boxes, or a block).
+// For 64 < I <= 128 (wide) a tile set holds, per part, an x tile and (for
+// complex values) a J x tile of 128 rows each, and no Y (the x tile of part q
+// is the B operand).
 struct TgLayout {
   uint32_t tile_a, lbo_b, set, stage;
 };
-__host__ __device__ inline TgLayout tg_layout(int I, int kc, int es) {
+__host__ __device__ inline TgLayout tg_layout(int I, int kc, int es, int parts, bool cplx) {
   TgLayout L;
   const uint32_t kg = (uint32_t)kc / 4;
   L.tile_a = kg * TG_LBO_A;
-  L.lbo_b = (uint32_t)tg_n_of(I, 0) * 16;
-  L.set = (uint32_t)tg_a_tiles(I) * L.tile_a + kg * L.lbo_b;
+  if (I > 64) {
+    L.lbo_b = 0;
+    L.set = (cplx ? 2u : 1u) * parts * L.tile_a;
+  } else {
+    L.lbo_b = (uint32_t)tg_n_of(I, 0) * 16;
+    L.set = (uint32_t)tg_a_tiles(I) * L.tile_a + kg * L.lbo_b;
+  }
   uint32_t st = (uint32_t)kc * I * es;
-  if (es == 8 && 2 * tg_boxb(I) > st) st = 2 * tg_boxb(I);
+  if (es == 8 && ((uint32_t)kc / 16) * tg_boxb(I) > st) st = ((uint32_t)kc / 16) * tg_boxb(I);
   L.stage = (st + 1023) / 1024 * 1024;
   return L;
 }
@@ -486,7 +495,8 @@ template <int DT>
 __global__ void __launch_bounds__(TG_THREADS, 1)
     gram_tc_kernel(const TcGramArgs p, const __grid_constant__ CUtensorMap rows_map) {
   constexpr int ES = Dt<DT>::bytes;
-  const TgLayout L = tg_layout((int)p.I, p.kc, ES);
+  constexpr bool CPLX = DT == TGD_C64 || DT == TGD_C32H;
+  const TgLayout L = tg_layout((int)p.I, p.kc, ES, p.parts, CPLX);
   const int NS = p.ns;
   const uint32_t STAGE = L.stage;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -503,9 +513,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   volatile int* abort = &s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int I = (int)p.I;
+  const bool wide = I > 64;
+  const int P = p.parts;
   const int PA = tg_parts_per_a(I), NA = tg_a_tiles(I);
-  const int N0 = tg_n_of(I, 0);
-  const uint32_t tmem_cols = N0 <= 32 ? 32u : (N0 <= 64 ? 64u : (N0 <= 128 ? 128u : 256u));
+  // D: narrow, 128 lanes x N0 columns; wide, the x rows' block at column 0
+  // and the J x rows' block at column 128, N = I rounded up to 16 each
+  const int N0 = wide ? (I + 15) / 16 * 16 : tg_n_of(I, 0);
+  const uint32_t tmem_cols = wide ? 256u : (N0 <= 32 ? 32u : (N0 <= 64 ? 64u : (N0 <= 128 ? 128u : 256u)));
   const int64_t IB = p.I * p.B;
   const int64_t q_begin = (int64_t)blockIdx.x * p.chunks_per_split;
   const int64_t q_end = q_begin + p.chunks_per_split < p.nchunk ? q_begin + p.chunks_per_split : p.nchunk;
@@ -569,7 +583,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
           ptx::bulk_g2s(st, gb + blk * ES, bytes, &full[slot]);
         }
       } else if (p.mode == TG_ROWS) {
-        const int64_t c0 = q * TG_COLS;
+        const int64_t c0 = q * p.kc;
         const int64_t a = c0 / p.B;
         const int64_t b0 = c0 - a * p.B;
         const int64_t base0 = a * IB + b0;
@@ -583,7 +597,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
           }
         m->colofs[lane] = lane;
         if (lane == 0) {
-          m->ncols = TG_COLS;
+          m->ncols = p.kc;
           m->rs = TG_COLS;
           m->sh = (int)(base0 & 31);
           m->bsh = (int)(p.B & 31);
@@ -591,20 +605,20 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
         cp_async_arrive(&full[slot]);
         __syncwarp();
         if (lane == 0) {
-          ptx::mbar_expect_tx(&full[slot], (uint32_t)(I * TG_COLS * ES));
-          // the I rows x 32 columns at column b0 of slab a; 8-byte elements
-          // are addressed as pairs of 4-byte ones, in two boxes of 16 columns
+          ptx::mbar_expect_tx(&full[slot], (uint32_t)(I * p.kc * ES));
+          // the I rows x kc columns at column b0 of slab a; 8-byte elements
+          // are addressed as pairs of 4-byte ones, in boxes of 16 columns
           if constexpr (ES == 8) {
             tma_load_3d(st, &rows_map, (int)(2 * b0), 0, (int)a, &full[slot]);
-            tma_load_3d(st + tg_boxb(I), &rows_map, (int)(2 * b0 + 32), 0, (int)a, &full[slot]);
+            if (p.kc == 32) tma_load_3d(st + tg_boxb(I), &rows_map, (int)(2 * b0 + 32), 0, (int)a, &full[slot]);
           } else {
             tma_load_3d(st, &rows_map, (int)b0, 0, (int)a, &full[slot]);
           }
         }
       } else {
-        const int64_t c0 = q * TG_COLS;
+        const int64_t c0 = q * p.kc;
         const int64_t ncol = p.A * p.B;
-        const int ncols = (int)(ncol - c0 < TG_COLS ? ncol - c0 : TG_COLS);
+        const int ncols = (int)(ncol - c0 < p.kc ? ncol - c0 : p.kc);
         const bool valid = lane < ncols;
         int64_t cb = 0;
         if (valid) {
@@ -649,13 +663,35 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
       if (lane == 0) {
         const int nks = tks[t];
         const uint32_t set = (uint32_t)t * L.set;
-        for (int kk = 0; kk < nks; ++kk) {
-          const uint64_t dy = dy_base + ((set + kk * 2 * L.lbo_b) >> 4);
+        if (wide) {
+          // every product (part pa of A, part qb of the x tile as B, pa + qb
+          // <= 2) into one block: the x rows' at column 0, the J x rows' at 128
+          const uint32_t idw = ptx::idesc_f16(1, 128, N0);
+          for (int kk = 0; kk < nks; ++kk) {
+            const uint32_t koff = set + kk * 2 * TG_LBO_A;
 #pragma unroll
-          for (int a = 0; a < 3; ++a)
-            if (a < NA)
-              ptx::mma_f16(dt_base, da_base + ((set + a * L.tile_a + kk * 2 * TG_LBO_A) >> 4), dy, idesc[a],
-                           (kc > 0 || kk > 0 || a > 0) ? 1u : 0u);
+            for (int xj = 0; xj < (CPLX ? 2 : 1); ++xj) {
+              int np = 0;
+#pragma unroll
+              for (int pa = 0; pa < 3; ++pa)
+#pragma unroll
+                for (int qb = 0; qb < 3; ++qb) {
+                  if (pa >= P || qb >= P || pa + qb > 2) continue;
+                  ptx::mma_f16(dt_base + xj * 128, da_base + ((koff + (xj * P + pa) * L.tile_a) >> 4),
+                               da_base + ((koff + qb * L.tile_a) >> 4), idw, (kc > 0 || kk > 0 || np > 0) ? 1u : 0u);
+                  ++np;
+                }
+            }
+          }
+        } else {
+          for (int kk = 0; kk < nks; ++kk) {
+            const uint64_t dy = dy_base + ((set + kk * 2 * L.lbo_b) >> 4);
+#pragma unroll
+            for (int a = 0; a < 3; ++a)
+              if (a < NA)
+                ptx::mma_f16(dt_base, da_base + ((set + a * L.tile_a + kk * 2 * TG_LBO_A) >> 4), dy, idesc[a],
+                             (kc > 0 || kk > 0 || a > 0) ? 1u : 0u);
+          }
         }
         ptx::mma_commit(&tfree[t]);
       }
@@ -751,6 +787,24 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
 #pragma unroll
           for (int part = 0; part < 3; ++part) jr[part][u] = __byte_perm(xr[part][u], 0u, 0x1032) ^ 0x8000u;
         }
+        if (wide) {
+          // part p: x row i of tile p, J x row i of tile P + p
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            if (part >= P) break;
+            uint8_t* xp = set + (size_t)part * L.tile_a + (uint32_t)g * TG_LBO_A + (uint32_t)i * 16;
+            uint8_t* jp = set + (size_t)(P + part) * L.tile_a + (uint32_t)g * TG_LBO_A + (uint32_t)i * 16;
+            const uint4 vx = part == 0 ? make_uint4(xr[0][0], xr[0][1], xr[0][2], xr[0][3])
+                             : part == 1 ? make_uint4(xr[1][0], xr[1][1], xr[1][2], xr[1][3])
+                                         : make_uint4(xr[2][0], xr[2][1], xr[2][2], xr[2][3]);
+            const uint4 vj = part == 0 ? make_uint4(jr[0][0], jr[0][1], jr[0][2], jr[0][3])
+                             : part == 1 ? make_uint4(jr[1][0], jr[1][1], jr[1][2], jr[1][3])
+                                         : make_uint4(jr[2][0], jr[2][1], jr[2][2], jr[2][3]);
+            *(uint4*)xp = vx;
+            if (CPLX) *(uint4*)jp = vj;
+          }
+          continue;
+        }
 #pragma unroll
         for (int part = 0; part < 3; ++part) {
           const int at = part / PA, arow = 2 * I * (part % PA);
@@ -775,6 +829,39 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const bool ok = !*abort;
+  float* out = p.partial + (size_t)blockIdx.x * p.I * p.I * 2;
+  if (wide) {
+    // lane = row i: the real part in the x block, the negated imaginary
+    // part in the J x block
+    if (warp < 4) {
+      const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+      const int row = tid;
+      for (int c0 = 0; c0 < N0; c0 += 16) {
+        float yx[16], yj[16];
+        ptx::tmem_ld16(dt_base + lane_base + c0, yx);
+        if (CPLX) {
+          ptx::tmem_ld16(dt_base + lane_base + 128 + c0, yj);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) yj[u] = 0.f;
+        }
+        if (row < I) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int j = c0 + u;
+            if (j < I) {
+              out[((int64_t)row * I + j) * 2] = ok && nch > 0 ? yx[u] : 0.f;
+              out[((int64_t)row * I + j) * 2 + 1] = ok && nch > 0 ? -yj[u] : 0.f;
+            }
+          }
+        }
+      }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) ptx::tmem_dealloc(dt_base, tmem_cols);
+    return;
+  }
   // D (128 lanes x N0 columns) -> shared memory S over the tile sets, which
   // no MMA reads any more; warp w reads TMEM lanes 32w..32w+31
   const int SP = N0 + 1;  // S row pitch (floats)
@@ -792,7 +879,6 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   // stacked row r < 2I (x rows: the real part of row r; J x rows: the
   // negated imaginary part of row r - I), column j < I: the sum over the A
   // tile's part slots s and Y's column blocks q, in that order
-  float* out = p.partial + (size_t)blockIdx.x * p.I * p.I * 2;
   for (int e = tid; e < 2 * I * I; e += TG_THREADS) {
     const int r = e / I, j = e % I;
     float v = 0.f;
@@ -807,15 +893,15 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   if (warp == 0) ptx::tmem_dealloc(dt_base, tmem_cols);
 }
 
-size_t tg_smem_bytes(int I, int kc, int es, int ns) {
-  const TgLayout L = tg_layout(I, kc, es);
+size_t tg_smem_bytes(int I, int kc, int es, int ns, int parts, bool cplx) {
+  const TgLayout L = tg_layout(I, kc, es, parts, cplx);
   return 2 * (size_t)L.set + (size_t)ns * (L.stage + sizeof(TgMeta)) + (2 * TG_NS_MAX + 4) * sizeof(uint64_t) +
          2 * sizeof(int) + 16;
 }
 
 struct TcGramGeom {
   int64_t A, I, B, nchunk, chunks_per_split;
-  int nsplit, mode, slabs, kc, ns;
+  int nsplit, mode, slabs, kc, ns, parts;
 };
 
 constexpr int TG_MAX_SPLITS = 148;  // one CTA per SM
@@ -823,8 +909,11 @@ constexpr size_t TG_SMEM_LIMIT = 227 * 1024 - 1024;  // the opt-in maximum less 
 
 // How mode n's unfolding is staged (see gram_tc_kernel) and split over CTAs:
 // the mode, the chunk capacity (64 columns for blocks of whole slabs when it
-// fits, else 32) and the most stages (up to four) that fit.
-TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned16) {
+// fits and I <= 32, 16 for 8-byte elements when I > 64, else 32), the bf16
+// parts per value (two represent a 16-bit input exactly; used when I > 64)
+// and the most stages (up to four) that fit.
+TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int dt, bool aligned16) {
+  const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
   TcGramGeom g;
   g.A = 1;
   g.B = 1;
@@ -832,8 +921,10 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned
   for (int q = n + 1; q < nd; ++q) g.B *= dims[q];
   g.I = dims[n];
   g.slabs = 1;
-  g.kc = TG_COLS;
   const int I = (int)g.I;
+  const bool wide = I > 64;
+  g.parts = wide && (dt == TGD_C32H || dt == TGD_R16) ? 2 : 3;
+  g.kc = wide && es == 8 ? 16 : TG_COLS;
   const int64_t total_bytes = g.A * g.I * g.B * es;
   // TMA coordinates are 32-bit: the column (in 4-byte units for 8-byte
   // elements) and the slab
@@ -841,14 +932,15 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned
   auto slabs_ok = [&](int kc) {
     return aligned16 && g.B < kc && (kc / g.B) * g.I * g.B * es % 16 == 0 && total_bytes % 16 == 0;
   };
-  auto fits = [&](int kc, int ns) { return tg_smem_bytes(I, kc, es, ns) <= TG_SMEM_LIMIT; };
+  const bool cplx = dt == TGD_C64 || dt == TGD_C32H;
+  auto fits = [&](int kc, int ns) { return tg_smem_bytes(I, kc, es, ns, g.parts, cplx) <= TG_SMEM_LIMIT; };
   // (a 64-column block of I <= 32 rows needs at most 65 of the mask words)
   if (I <= 32 && g.B < TG_COLS && slabs_ok(TG_KC_MAX) && fits(TG_KC_MAX, 2)) {
     g.mode = TG_SLABS;
     g.kc = TG_KC_MAX;
-  } else if (slabs_ok(TG_COLS)) {
+  } else if (slabs_ok(g.kc)) {
     g.mode = TG_SLABS;
-  } else if (aligned16 && tma_ok && g.B % TG_COLS == 0) {
+  } else if (aligned16 && tma_ok && g.B % g.kc == 0) {
     g.mode = TG_ROWS;
   } else {
     g.mode = TG_ELEMS;
@@ -857,9 +949,9 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int es, bool aligned
     g.slabs = (int)(g.kc / g.B);
     g.nchunk = ceil_div(g.A, (int64_t)g.slabs);
   } else if (g.mode == TG_ROWS) {
-    g.nchunk = g.A * g.B / TG_COLS;
+    g.nchunk = g.A * g.B / g.kc;
   } else {
-    g.nchunk = ceil_div(g.A * g.B, (int64_t)TG_COLS);
+    g.nchunk = ceil_div(g.A * g.B, (int64_t)g.kc);
   }
   g.ns = TG_NS_MAX;
   while (g.ns > 2 && !fits(g.kc, g.ns)) --g.ns;
@@ -1308,13 +1400,15 @@ __global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
     for (int e = threadIdx.x; e < n * n; e += blockDim.x) ((double2*)J.vprev)[e] = Vt[e];
 }
 
-// Hermitian Jacobi for n <= 64, the same rotations and ordering as
-// eig_block_kernel, laid out for speed: A and the eigenvector rows Vt both
-// whole in shared memory with an odd row pitch (a column walk by 32 lanes
-// touches 32 different banks), one warp per rotation pair, and each round
-// in two phases (J^H on the pairs' rows, then J on their columns and on V)
-// so that every access is a plain load or store of one entry.
-constexpr int ES_MAXN = 64;
+// Hermitian Jacobi for n <= 128, the same rotations and ordering as
+// eig_block_kernel: A and the eigenvector rows Vt both whole, with an odd
+// row pitch (a column walk by 32 lanes touches 32 different banks), in
+// shared memory for n <= 64 and in the job's global scratch above that; one
+// warp per rotation pair, and each round in two phases (J^H on the pairs'
+// rows, then J on their columns and on V) so that every access is a plain
+// load or store of one entry.
+constexpr int ES_MAXN = 128;
+constexpr int ES_SMEM_MAXN = 64;
 
 __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
   const EigJob J = jobs[blockIdx.x];
@@ -1322,8 +1416,10 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
   if (n > ES_MAXN) return;
   const int NP = n + 1 + (n & 1);  // odd row pitch
   extern __shared__ double2 dyn[];
-  double2* A = dyn;                // [n][NP]
-  double2* Vt = dyn + n * NP;      // [n][NP]: row k = eigenvector k
+  const bool in_smem = n <= ES_SMEM_MAXN;
+  double2* scratch = (double2*)J.work;
+  double2* A = in_smem ? dyn : scratch;                            // [n][NP]
+  double2* Vt = in_smem ? dyn + n * NP : scratch + (size_t)n * NP;  // [n][NP]: row k = eigenvector k
   __shared__ int rp[ES_MAXN / 2], rq[ES_MAXN / 2], rrot[ES_MAXN / 2];
   __shared__ double rcs[ES_MAXN / 2], rsn[ES_MAXN / 2];
   __shared__ double2 rph[ES_MAXN / 2];
@@ -1338,7 +1434,7 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
     // V^H G V is nearly diagonal when the subspaces move little between
     // refreshes. Jacobi converges from any unitary start.
     const double2* Vp = (const double2*)J.vprev;
-    double2* W = (double2*)J.work + (size_t)n * n;  // W = G V (n x n)
+    double2* W = scratch + (size_t)2 * n * NP;  // W = G V (n x n)
     for (int e = tid; e < n * n; e += blockDim.x) {
       const int k = e / n, i = e - k * n;
       Vt[k * NP + i] = Vp[e];
@@ -1621,7 +1717,7 @@ cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);
   size_t b = sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
-  if (g.I <= 64) b = std::max(b, sizeof(float2) * (size_t)TG_MAX_SPLITS * g.I * g.I);
+  if (g.I <= 128) b = std::max(b, sizeof(float2) * (size_t)TG_MAX_SPLITS * g.I * g.I);
   return b;
 }
 
@@ -1669,7 +1765,7 @@ static cudaError_t rows_tensor_map(CUtensorMap* map, const void* g, int es, cons
 cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
                          int n, float* partial, double* gram, int* err, cudaStream_t s) {
   const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
-  const TcGramGeom t = tc_gram_geom(nd, dims, n, es, ((uintptr_t)g & 15) == 0);
+  const TcGramGeom t = tc_gram_geom(nd, dims, n, dt, ((uintptr_t)g & 15) == 0);
   TcGramArgs a;
   a.g = g;
   a.bits = bits;
@@ -1682,6 +1778,7 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
   a.slabs = t.slabs;
   a.kc = t.kc;
   a.ns = t.ns;
+  a.parts = t.parts;
   a.partial = partial;
   a.err = err;
   CUtensorMap map;
@@ -1690,7 +1787,7 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
     const cudaError_t e = rows_tensor_map(&map, g, es, t);
     if (e != cudaSuccess) return e;
   }
-  const size_t smem = tg_smem_bytes((int)t.I, t.kc, es, t.ns);
+  const size_t smem = tg_smem_bytes((int)t.I, t.kc, es, t.ns, t.parts, dt == TGD_C64 || dt == TGD_C32H);
   if (smem > TG_SMEM_LIMIT) return cudaErrorInvalidValue;
   const dim3 grid(t.nsplit);
   cudaError_t e = cudaSuccess;
@@ -1727,7 +1824,7 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
 
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
                       int n, float* partial, double* gram, int* err, cudaStream_t s) {
-  if (dims[n] <= 64) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s);
+  if (dims[n] <= 128) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s);
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
   const size_t smem = gram_smem_bytes(geo);
@@ -1753,11 +1850,12 @@ cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const
   return cudaGetLastError();
 }
 
-size_t eig_work_doubles(int n) { return (size_t)4 * n * n; }
+// (Jacobi scratch: A, Vt and W of n x (n + 2) complex each)
+size_t eig_work_doubles(int n) { return (size_t)6 * n * (n + 2); }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
-  // every matrix n <= 64: the whole-matrix kernel
+  // every matrix n <= 128: the whole-matrix kernel
   bool all_64 = true;
   size_t ssmem = 16;
   for (int j = 0; j < njobs; ++j) {
@@ -1767,7 +1865,7 @@ cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, c
       break;
     }
     const size_t np = (size_t)n + 1 + (n & 1);
-    ssmem = std::max(ssmem, 2 * sizeof(double2) * (size_t)n * np);
+    if (n <= ES_SMEM_MAXN) ssmem = std::max(ssmem, 2 * sizeof(double2) * (size_t)n * np);
   }
   if (all_64) {
     cudaError_t e = cudaFuncSetAttribute(eig_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -30,14 +30,14 @@ cudaError_t build_tile_index(const int64_t* omega, int64_t k, int64_t tile_elems
 // Omega bitmask `bits`), accumulated in fp32 partials and summed in fp64
 // into gram (I_n x I_n complex, interleaved doubles).
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n);
-// Modes with I_n <= 64 run on the tensor cores; err is the device error word
+// Modes with I_n <= 128 run on the tensor cores; err is the device error word
 // a bounded wait sets when it gives up.
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
                       int n, float* partial, double* gram, int* err, cudaStream_t s);
 
 struct EigJob {
   const double* gram;  // n x n complex (interleaved doubles)
-  double* work;        // 2 * n * n complex doubles of global scratch
+  double* work;        // eig_work_doubles(n) doubles of global scratch
   float* U;            // out: n x r complex fp32, row-major
   double* evals;       // out: n eigenvalues, descending
   double* vprev;       // n x n complex: a unitary basis to start from (rows = vectors), and

@@ -48,6 +48,15 @@ CASES = {
     # and tile edges above I_n (9 -> 12, 5 -> 8)
     "c64_gram_pairs_130x20x9": ((130, 20, 9), (8, 5, 3), (8, 5, 3), "c64", 0.05),
     "c32h_gram_pairs_70x66x5": ((70, 66, 5), (6, 9, 2), (6, 9, 2), "c32h", 0.05),
+    # tensor-core Grams of modes 64 < I_n <= 128: row boxes (B a multiple of
+    # the chunk), whole slabs (B = 1), element copies (B = 48), for complex
+    # and real, 32- and 16-bit values
+    "c64_wide_96x32x8": ((96, 32, 8), (8, 4, 2), (8, 4, 2), "c64", 0.05),
+    "c32h_wide_128x64": ((128, 64), (16, 8), (16, 8), "c32h", 0.05),
+    "r32_wide_80x16x4": ((80, 16, 4), (8, 4, 2), (8, 4, 2), "r32", 0.05),
+    "r16_wide_100x32": ((100, 32), (8, 4), (8, 4), "r16", 0.05),
+    "r16_wide_72x48": ((72, 48), (6, 5), (6, 5), "r16", 0.05),
+    "c64_wide_inner_5x100": ((5, 100), (2, 8), (2, 8), "c64", 0.05),
 }
 
 
