@@ -992,422 +992,14 @@ __device__ double block_max(double v, double* red) {
   return m;
 }
 
-__global__ void __launch_bounds__(ET) eig_kernel(const EigJob* jobs) {
-  const EigJob J = jobs[blockIdx.x];
-  const int n = J.n;
-  extern __shared__ double2 dyn[];
-  __shared__ int rp[MAXN / 2], rq[MAXN / 2];
-  __shared__ double rcs[MAXN / 2], rsn[MAXN / 2];
-  __shared__ double2 rph[MAXN / 2];
-  __shared__ double red[ET / 32];
-  __shared__ double ev[MAXN];
-  __shared__ int col_of_rank[MAXN];
-  double2* A;
-  double2* V;
-  if (n <= 64) {
-    A = dyn;
-    V = dyn + n * n;
-  } else {
-    A = (double2*)J.work;
-    V = A + (int64_t)n * n;
-  }
-  const double2* G = (const double2*)J.gram;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    A[e] = G[e];
-    V[e] = make_double2((e / n) == (e % n) ? 1.0 : 0.0, 0.0);
-  }
-  __syncthreads();
-  double fro_part = 0;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) fro_part += zabs2(A[e]);
-  const double fro = block_sum(fro_part, red);
-  const int m = n + (n & 1);
-  const int npairs = m / 2;
-  for (int sweep = 0; sweep < 40; ++sweep) {
-    double off_part = 0;
-    for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-      int i = e / n, j = e - i * n;
-      if (i < j) off_part += zabs2(A[e]);
-    }
-    double off = block_sum(off_part, red);
-    if (off <= 1e-24 * fro || off == 0.0) break;
-    for (int round = 0; round < m - 1; ++round) {
-      for (int k = threadIdx.x; k < npairs; k += blockDim.x) {
-        int p, q;
-        if (k == 0) {
-          p = round;
-          q = m - 1;
-        } else {
-          p = (round + k) % (m - 1);
-          q = (round - k + (m - 1)) % (m - 1);
-        }
-        if (p > q) {
-          int t = p;
-          p = q;
-          q = t;
-        }
-        rp[k] = -1;
-        if (q < n) {
-          double2 apq = A[p * n + q];
-          double r = sqrt(zabs2(apq));
-          if (r > 0.0) {
-            double app = A[p * n + p].x, aqq = A[q * n + q].x;
-            double tau = (aqq - app) / (2.0 * r);
-            double t = (tau >= 0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-            double c = 1.0 / sqrt(1.0 + t * t);
-            rp[k] = p;
-            rq[k] = q;
-            rcs[k] = c;
-            rsn[k] = t * c;
-            rph[k] = make_double2(apq.x / r, apq.y / r);  // e = apq / |apq|
-          }
-        }
-      }
-      __syncthreads();
-      // A <- A J and V <- V J: columns p, q of every row.
-      for (int w = threadIdx.x; w < n * npairs; w += blockDim.x) {
-        int i = w / npairs, k = w - i * npairs;
-        int p = rp[k];
-        if (p < 0) continue;
-        int q = rq[k];
-        double c = rcs[k], s = rsn[k];
-        double2 ec = make_double2(rph[k].x, -rph[k].y);
-        double2 xp = A[i * n + p], xq = zmul(A[i * n + q], ec);
-        A[i * n + p] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-        A[i * n + q] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-        xp = V[i * n + p];
-        xq = zmul(V[i * n + q], ec);
-        V[i * n + p] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-        V[i * n + q] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-      }
-      __syncthreads();
-      // A <- J^H A: rows p, q of every column.
-      for (int w = threadIdx.x; w < npairs * n; w += blockDim.x) {
-        int k = w / n, j = w - k * n;
-        int p = rp[k];
-        if (p < 0) continue;
-        int q = rq[k];
-        double c = rcs[k], s = rsn[k];
-        double2 xp = A[p * n + j], xq = zmul(A[q * n + j], rph[k]);
-        A[p * n + j] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-        A[q * n + j] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-      }
-      __syncthreads();
-      for (int k = threadIdx.x; k < npairs; k += blockDim.x) {
-        int p = rp[k];
-        if (p < 0) continue;
-        int q = rq[k];
-        A[p * n + q] = make_double2(0.0, 0.0);
-        A[q * n + p] = make_double2(0.0, 0.0);
-        A[p * n + p].y = 0.0;
-        A[q * n + q].y = 0.0;
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < n; i += blockDim.x) ev[i] = A[i * n + i].x;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    double li = ev[i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) rank += (ev[j] > li) || (ev[j] == li && j < i);
-    col_of_rank[rank] = i;
-    J.evals[rank] = li;
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int rr = wid; rr < J.r; rr += nw) {
-    int c = col_of_rank[rr];
-    double best = -1.0;
-    int bi = 0;
-    for (int row = lane; row < n; row += 32) {
-      double mg = zabs2(V[row * n + c]);
-      if (mg > best) {
-        best = mg;
-        bi = row;
-      }
-    }
-    for (int o = 16; o; o >>= 1) {
-      double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ob > best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
-      }
-    }
-    double2 piv = V[bi * n + c];
-    double pm = sqrt(zabs2(piv));
-    double2 ph = pm > 0 ? make_double2(piv.x / pm, -piv.y / pm) : make_double2(1.0, 0.0);
-    for (int row = lane; row < n; row += 32) {
-      double2 u = zmul(V[row * n + c], ph);
-      ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
-    }
-  }
-}
-
-// Block form of the same parallel Jacobi for n <= 128: A is Hermitian, so only
-// its upper triangle is kept (packed, in shared memory: 132 KB at n = 128).
-// In a round the n/2 rotations are disjoint; the 2 x 2 block of A at the rows
-// of pair k1 and the columns of pair k2 becomes J1^H B J2 (the column rotation
-// of k2, then the row rotation of k1, as in eig_kernel), and each unordered
-// block (k1 <= k2) is one thread's work, so every stored entry has one writer
-// per round and a round needs two barriers. V is kept transposed (a row per
-// eigenvector): in shared memory for n <= 64, in the job's scratch otherwise.
-constexpr int EB_MAXN = 128;
-
-__device__ __forceinline__ int tri_idx(int i, int j, int n) {  // i <= j
-  return i * n - (i * (i - 1)) / 2 + (j - i);
-}
-
-__global__ void __launch_bounds__(ET) eig_block_kernel(const EigJob* jobs) {
-  const EigJob J = jobs[blockIdx.x];
-  const int n = J.n;
-  if (n > EB_MAXN) return;
-  extern __shared__ double2 dyn[];
-  __shared__ int rp[EB_MAXN / 2], rq[EB_MAXN / 2], rrot[EB_MAXN / 2];
-  __shared__ double rcs[EB_MAXN / 2], rsn[EB_MAXN / 2];
-  __shared__ double2 rph[EB_MAXN / 2];
-  __shared__ uint8_t bk1[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2], bk2[EB_MAXN / 2 * (EB_MAXN / 2 + 1) / 2];
-  __shared__ double red[ET / 32];
-  __shared__ double ev[EB_MAXN];
-  __shared__ int col_of_rank[EB_MAXN];
-  const int ntri = n * (n + 1) / 2;
-  double2* T = dyn;  // packed upper triangle of A
-  double2* Vt = n <= 64 ? dyn + ntri : (double2*)J.work;
-  const double2* G = (const double2*)J.gram;
-  if (J.warm) {
-    // Start from the previous refresh's eigenvectors V (rows of Vt): the
-    // rotated matrix V^H A V is nearly diagonal when the subspaces move
-    // little between refreshes, so the sweeps below end after one or two.
-    // Jacobi converges from any unitary start; the results are the
-    // eigenpairs of A either way.
-    const double2* Vp = (const double2*)J.vprev;
-    double2* W = (double2*)J.work + (size_t)n * n;  // W = A V (n x n)
-    for (int e = threadIdx.x; e < n * n; e += blockDim.x) Vt[e] = Vp[e];
-    __syncthreads();
-    for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-      const int i = e / n, l = e - i * n;
-      double2 acc = make_double2(0.0, 0.0);
-      for (int j = 0; j < n; ++j) {
-        const double2 g = G[i * n + j], v = Vt[l * n + j];
-        acc.x += g.x * v.x - g.y * v.y;
-        acc.y += g.x * v.y + g.y * v.x;
-      }
-      W[e] = acc;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
-      int k = 0, r = e;
-      while (r >= n - k) {
-        r -= n - k;
-        ++k;
-      }
-      const int l = k + r;
-      double2 acc = make_double2(0.0, 0.0);  // sum_i conj(V[i][k]) W[i][l]
-      for (int i = 0; i < n; ++i) {
-        const double2 v = Vt[k * n + i], w = W[i * n + l];
-        acc.x += v.x * w.x + v.y * w.y;
-        acc.y += v.x * w.y - v.y * w.x;
-      }
-      if (l == k) acc.y = 0.0;  // Hermitian: a real diagonal
-      T[e] = acc;
-    }
-  } else {
-    for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-      const int i = e / n, j = e - i * n;
-      if (i <= j) T[tri_idx(i, j, n)] = G[e];
-      Vt[e] = make_double2(i == j ? 1.0 : 0.0, 0.0);
-    }
-  }
-  const int m = n + (n & 1);
-  const int npairs = m / 2;
-  const int nblk = npairs * (npairs + 1) / 2;
-  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
-    int k1 = 0, r = b;
-    while (r >= npairs - k1) {
-      r -= npairs - k1;
-      ++k1;
-    }
-    bk1[b] = (uint8_t)k1;
-    bk2[b] = (uint8_t)(k1 + r);
-  }
-  __syncthreads();
-  auto get = [&](int i, int j) -> double2 {
-    if (i <= j) return T[tri_idx(i, j, n)];
-    const double2 v = T[tri_idx(j, i, n)];
-    return make_double2(v.x, -v.y);
-  };
-  auto put = [&](int i, int j, double2 v) {
-    if (i <= j)
-      T[tri_idx(i, j, n)] = v;
-    else
-      T[tri_idx(j, i, n)] = make_double2(v.x, -v.y);
-  };
-  double part = 0;
-  for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
-    int i = 0, r = e;
-    while (r >= n - i) {
-      r -= n - i;
-      ++i;
-    }
-    part += (r == 0 ? 1.0 : 2.0) * zabs2(T[e]);  // r == 0: the diagonal entry of row i
-  }
-  const double fro = block_sum(part, red);
-  for (int sweep = 0; sweep < 40; ++sweep) {
-    double off_part = 0;
-    for (int e = threadIdx.x; e < ntri; e += blockDim.x) {
-      int i = 0, r = e;
-      while (r >= n - i) {
-        r -= n - i;
-        ++i;
-      }
-      if (r > 0) off_part += zabs2(T[e]);
-    }
-    const double off = block_sum(off_part, red);
-    if (off <= 1e-24 * fro || off == 0.0) break;
-    for (int round = 0; round < m - 1; ++round) {
-      for (int k = threadIdx.x; k < npairs; k += blockDim.x) {
-        int p, q;
-        if (k == 0) {
-          p = round;
-          q = m - 1;
-        } else {
-          p = (round + k) % (m - 1);
-          q = (round - k + (m - 1)) % (m - 1);
-        }
-        if (p > q) {
-          const int t = p;
-          p = q;
-          q = t;
-        }
-        rp[k] = p;
-        rq[k] = q;
-        rrot[k] = 0;
-        if (q < n) {
-          const double2 apq = get(p, q);
-          const double r = sqrt(zabs2(apq));
-          if (r > 0.0) {
-            const double app = get(p, p).x, aqq = get(q, q).x;
-            const double tau = (aqq - app) / (2.0 * r);
-            const double t = (tau >= 0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-            const double c = 1.0 / sqrt(1.0 + t * t);
-            rrot[k] = 1;
-            rcs[k] = c;
-            rsn[k] = t * c;
-            rph[k] = make_double2(apq.x / r, apq.y / r);
-          }
-        }
-      }
-      __syncthreads();
-      for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
-        const int k1 = bk1[b], k2 = bk2[b];
-        const int p1 = rp[k1], q1 = rq[k1], p2 = rp[k2], q2 = rq[k2];
-        const bool rot1 = rrot[k1], rot2 = rrot[k2];
-        if (!rot1 && !rot2) continue;
-        const bool h1 = q1 < n, h2 = q2 < n;  // the dummy index of odd n is absent
-        double2 b00 = get(p1, p2), b01 = h2 ? get(p1, q2) : make_double2(0, 0);
-        double2 b10 = h1 ? get(q1, p2) : make_double2(0, 0);
-        double2 b11 = h1 && h2 ? get(q1, q2) : make_double2(0, 0);
-        if (rot2) {  // columns p2, q2: B <- B J2
-          const double c = rcs[k2], s = rsn[k2];
-          const double2 ec = make_double2(rph[k2].x, -rph[k2].y);
-          double2 xp = b00, xq = zmul(b01, ec);
-          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          b01 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-          xp = b10;
-          xq = zmul(b11, ec);
-          b10 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-        }
-        if (rot1) {  // rows p1, q1: B <- J1^H B
-          const double c = rcs[k1], s = rsn[k1];
-          const double2 e = rph[k1];
-          double2 xp = b00, xq = zmul(b10, e);
-          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          b10 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-          xp = b01;
-          xq = zmul(b11, e);
-          b01 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-        }
-        if (k1 == k2) {
-          // the diagonal block: the rotation zeroes (p, q); the diagonal is real
-          put(p1, p1, make_double2(b00.x, 0.0));
-          if (h1) {
-            put(p1, q1, make_double2(0.0, 0.0));
-            put(q1, q1, make_double2(b11.x, 0.0));
-          }
-        } else {
-          put(p1, p2, b00);
-          if (h2) put(p1, q2, b01);
-          if (h1) put(q1, p2, b10);
-          if (h1 && h2) put(q1, q2, b11);
-        }
-      }
-      // V <- V J on the rows of V^T (no other thread touches them this round)
-      for (int w = threadIdx.x; w < npairs * n; w += blockDim.x) {
-        const int k = w / n, i = w - k * n;
-        if (!rrot[k]) continue;
-        const int p = rp[k], q = rq[k];
-        const double c = rcs[k], s = rsn[k];
-        const double2 ec = make_double2(rph[k].x, -rph[k].y);
-        const double2 xp = Vt[p * n + i], xq = zmul(Vt[q * n + i], ec);
-        Vt[p * n + i] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-        Vt[q * n + i] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < n; i += blockDim.x) ev[i] = T[tri_idx(i, i, n)].x;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const double li = ev[i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) rank += (ev[j] > li) || (ev[j] == li && j < i);
-    col_of_rank[rank] = i;
-    J.evals[rank] = li;
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int rr = wid; rr < J.r; rr += nw) {
-    const int c = col_of_rank[rr];
-    double best = -1.0;
-    int bi = 0;
-    for (int row = lane; row < n; row += 32) {
-      const double mg = zabs2(Vt[c * n + row]);
-      if (mg > best) {
-        best = mg;
-        bi = row;
-      }
-    }
-    for (int o = 16; o; o >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ob > best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
-      }
-    }
-    const double2 piv = Vt[c * n + bi];
-    const double pm = sqrt(zabs2(piv));
-    const double2 ph = pm > 0 ? make_double2(piv.x / pm, -piv.y / pm) : make_double2(1.0, 0.0);
-    for (int row = lane; row < n; row += 32) {
-      const double2 u = zmul(Vt[c * n + row], ph);
-      ((float2*)J.U)[(int64_t)row * J.r + rr] = make_float2((float)u.x, (float)u.y);
-    }
-  }
-  // the eigenvectors, the start of the next refresh
-  if (J.vprev)
-    for (int e = threadIdx.x; e < n * n; e += blockDim.x) ((double2*)J.vprev)[e] = Vt[e];
-}
-
-// Hermitian Jacobi for n <= 128, the same rotations and ordering as
-// eig_block_kernel: A and the eigenvector rows Vt both whole, with an odd
-// row pitch (a column walk by 32 lanes touches 32 different banks), in
-// shared memory for n <= 64 and in the job's global scratch above that; one
-// warp per rotation pair, and each round in two phases (J^H on the pairs'
-// rows, then J on their columns and on V) so that every access is a plain
-// load or store of one entry.
-constexpr int ES_MAXN = 128;
+// Hermitian Jacobi for n <= 256: two-sided rotations in the round-robin
+// parallel ordering (n/2 disjoint pairs per round). A and the eigenvector
+// rows Vt are both whole, with an odd row pitch (a column walk by 32 lanes
+// touches 32 different banks), in shared memory for n <= 64 and in the job's
+// global scratch above that; one warp per rotation pair, and each round in
+// two phases (J^H on the pairs' rows, then J on their columns and on V) so
+// that every access is a plain load or store of one entry.
+constexpr int ES_MAXN = MAXN;
 constexpr int ES_SMEM_MAXN = 64;
 
 __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
@@ -1855,59 +1447,18 @@ size_t eig_work_doubles(int n) { return (size_t)6 * n * (n + 2); }
 
 cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
-  // every matrix n <= 128: the whole-matrix kernel
-  bool all_64 = true;
   size_t ssmem = 16;
   for (int j = 0; j < njobs; ++j) {
     const int n = jobs_host[j].n;
-    if (n > ES_MAXN || jobs_host[j].r > n) {
-      all_64 = false;
-      break;
-    }
+    if (n < 1 || n > ES_MAXN || jobs_host[j].r > n) return cudaErrorInvalidValue;
     const size_t np = (size_t)n + 1 + (n & 1);
     if (n <= ES_SMEM_MAXN) ssmem = std::max(ssmem, 2 * sizeof(double2) * (size_t)n * np);
   }
-  if (all_64) {
-    cudaError_t e = cudaFuncSetAttribute(eig_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ssmem);
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return e;
-    eig_small_kernel<<<njobs, ET, ssmem, s>>>(jobs_dev);
-    return cudaGetLastError();
-  }
-  bool all_small = true;
-  size_t bsmem = 16;
-  for (int j = 0; j < njobs; ++j) {
-    const int n = jobs_host[j].n;
-    if (n > EB_MAXN || jobs_host[j].r > n) {
-      all_small = false;
-      break;
-    }
-    const size_t need = sizeof(double2) * ((size_t)n * (n + 1) / 2 + (n <= 64 ? (size_t)n * n : 0));
-    bsmem = std::max(bsmem, need);
-  }
-  if (all_small) {
-    cudaError_t e = cudaFuncSetAttribute(eig_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)bsmem);
-    if (e != cudaSuccess) return e;
-    e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return e;
-    eig_block_kernel<<<njobs, ET, bsmem, s>>>(jobs_dev);
-    return cudaGetLastError();
-  }
-  int smem_n = 0;
-  for (int j = 0; j < njobs; ++j) {
-    if (jobs_host[j].n > MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;
-    if (jobs_host[j].n <= 64 && jobs_host[j].n > smem_n) smem_n = jobs_host[j].n;
-  }
-  size_t smem = (size_t)2 * smem_n * smem_n * sizeof(double2);
-  cudaError_t e = cudaFuncSetAttribute(eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(smem > 0 ? smem : 1));
+  cudaError_t e = cudaFuncSetAttribute(eig_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
   if (e != cudaSuccess) return e;
   e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return e;
-  eig_kernel<<<njobs, ET, smem, s>>>(jobs_dev);
+  eig_small_kernel<<<njobs, ET, ssmem, s>>>(jobs_dev);
   return cudaGetLastError();
 }
 
