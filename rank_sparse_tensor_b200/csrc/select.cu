@@ -196,11 +196,21 @@ __global__ void __launch_bounds__(CT) write_kernel(KeyF kf, const void* g, int64
   long long run_eq = eq_before[blockIdx.x];
   long long run_out = out_off[blockIdx.x];
   const unsigned lt_mask = (1u << lane) - 1u;
+  // all of this thread's keys first (independent loads in flight), kept as
+  // two flags each; the compaction below then waits on no global load
+  static_assert(CHUNK / CT <= 32, "flags are packed in 32-bit words");
+  uint32_t ltm = 0, eqm = 0;
+#pragma unroll
+  for (int r = 0; r < CHUNK / CT; ++r) {
+    const int64_t i = base + r * CT + threadIdx.x;
+    const bool valid = i < n;
+    const uint64_t key = valid ? kf(i) : ~0ull;
+    ltm |= (uint32_t)(valid && key < K) << r;
+    eqm |= (uint32_t)(valid && key == K) << r;
+  }
   for (int r = 0; r < CHUNK / CT; ++r) {
     int64_t i = base + r * CT + threadIdx.x;
-    bool valid = i < n;
-    uint64_t key = valid ? kf(i) : ~0ull;
-    bool lt = valid && key < K, eq = valid && key == K;
+    const bool lt = (ltm >> r) & 1u, eq = (eqm >> r) & 1u;
     unsigned be = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) s_eq[wid] = __popc(be);
     __syncthreads();

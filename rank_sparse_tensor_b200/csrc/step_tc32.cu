@@ -88,8 +88,23 @@ struct MG32Args {
   // contiguous range each; they then move by bulk copy through shared memory
   // at these offsets (0: not staged)
   uint32_t xs_off, os_off;
+  // ... and Omega's mask words over those ranges (with the output range's
+  // word ranks when the weights are updated), by cp.async (0: not staged)
+  uint32_t xm_off, om_off;
+  int64_t tile0;          // first 128-row tile of the launch (the grid's x counts from it)
   int* err;
 };
+
+// Asynchronous 4- and 8-byte copies global -> shared.
+__device__ __forceinline__ void cpa4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
 // Y[a][j][b] = sum_k X[a][k][b] M[k][j] over one 128-row block of the
 // unfolding and one NT-wide block of (j, re/im) columns. K advances in chunks
@@ -117,18 +132,19 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int64_t rho = (int64_t)blockIdx.x * G32T + tid;
+  const int64_t tile = p.tile0 + blockIdx.x;
+  const int64_t rho = tile * G32T + tid;
   const bool valid = rho < p.rows;
   const int64_t a = valid ? rho / p.B : 0, b = valid ? rho - a * p.B : 0;
   const int64_t xbase = a * p.K * p.B + b;  // element index of (a, k = 0, b)
   // staging applies to CTAs whose 128 rows all exist
-  const bool full_cta = ((int64_t)blockIdx.x + 1) * G32T <= p.rows;
+  const bool full_cta = (tile + 1) * G32T <= p.rows;
   const bool st_in = p.xs_off != 0 && full_cta;
   const bool st_out = p.os_off != 0 && full_cta;
   constexpr int ESZ = CPLX ? 8 : 4;
   float* xs = (float*)(smem + p.xs_off);
   float* os = (float*)(smem + p.os_off);
-  const int64_t a0 = (int64_t)blockIdx.x * G32T;  // first row (B == 1 when staged)
+  const int64_t a0 = tile * G32T;  // first row (B == 1 when staged)
   if (tid == 0) {
     s_abort = 0;
     for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
@@ -142,6 +158,24 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       if (wb) bulk_g2s(os, (const uint8_t*)p.W + a0 * p.J * ESZ, wb, &bars[4]);
     }
   }
+  // Omega's words over the staged ranges (the CTA's rows are contiguous)
+  const bool xm = p.xm_off != 0 && st_in && p.bits;
+  const bool om = p.om_off != 0 && st_out && WUPD;
+  const int64_t xw0 = (a0 * p.K) >> 5, ow0 = (a0 * p.J) >> 5;
+  uint32_t* xmw = (uint32_t*)(smem + p.xm_off);
+  uint32_t* omw = (uint32_t*)(smem + p.om_off);
+  const int onw = (int)((((a0 + G32T) * p.J - 1) >> 5) - ow0 + 1);
+  int64_t* omr = (int64_t*)(omw + ((onw + 1) & ~1));
+  if (xm) {
+    const int nw = (int)((((a0 + G32T) * p.K - 1) >> 5) - xw0 + 1);
+    for (int w = tid; w < nw; w += G32T) cpa4(xmw + w, p.bits + xw0 + w);
+  }
+  if (om)
+    for (int w = tid; w < onw; w += G32T) {
+      cpa4(omw + w, p.wbits + ow0 + w);
+      cpa8(omr + w, p.wrank + ow0 + w);
+    }
+  if (xm || om) cpa_wait_all();
   __syncthreads();
   if (warp == 0) tmem_alloc(tslot, p.tmem_cols);
   tc_fence_before();
@@ -182,7 +216,8 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       float2 x = make_float2(0.f, 0.f);
       if (i < p.K) {
         const int64_t idx = xbase + i;
-        if (!(p.bits && ((__ldg(p.bits + (idx >> 5)) >> (idx & 31)) & 1u))) {
+        const uint32_t word = !p.bits ? 0u : (xm ? xmw[(idx >> 5) - xw0] : __ldg(p.bits + (idx >> 5)));
+        if (!((word >> (idx & 31)) & 1u)) {
           if (CPLX)
             x = ((const float2*)xs)[tid * p.K + i];
           else
@@ -316,10 +351,10 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
             os[so] = dr;
         } else {
           const int64_t o = (a0 + tid) * p.J + j;
-          const uint32_t word = __ldg(p.wbits + (o >> 5));
+          const uint32_t word = om ? omw[(o >> 5) - ow0] : __ldg(p.wbits + (o >> 5));
           const uint32_t bit = (uint32_t)(o & 31);
           if ((word >> bit) & 1u) {
-            const int64_t e = __ldg(p.wrank + (o >> 5)) + __popc(word & ((1u << bit) - 1u));
+            const int64_t e = (om ? omr[(o >> 5) - ow0] : __ldg(p.wrank + (o >> 5))) + __popc(word & ((1u << bit) - 1u));
             if (CPLX) {
               const float2 sv = __ldg((const float2*)p.S + e);
               dr += sv.x;
@@ -343,7 +378,7 @@ __global__ void __launch_bounds__(G32T) mode_gemm32_kernel(const MG32Args p) {
       uint8_t* dst = WUPD ? (uint8_t*)p.W : (uint8_t*)p.Y;
       bulk_s2g(dst + a0 * p.J * ESZ, os, (uint32_t)(G32T * p.J * ESZ));
       bulk_commit();
-      bulk_wait_all0();
+      bulk_wait_read0();  // the source read; the writes complete with the kernel
     }
   } else if (!s_abort) {
     const int64_t j0 = (int64_t)blockIdx.y * (CPLX ? p.NT / 2 : p.NT);
@@ -484,6 +519,262 @@ int pow2_cols32(int n) {
   return c;
 }
 // stages x (three A tiles + three B blocks) + barriers
+// The innermost mode (B = 1, one K chunk, one column block): a persistent
+// version of mode_gemm32_kernel. Each CTA takes whole 128-row tiles t =
+// blockIdx.x, + gridDim.x, ...; a tile's rows of X (and of W when the
+// weights are updated) are one contiguous range each and arrive by bulk copy,
+// Omega's mask words (and word ranks) by cp.async, into a ring of NB buffers,
+// NB - 1 tiles ahead of the one whose rows are split into bf16 parts,
+// multiplied and written back (one bulk store per tile). The operand image
+// of the mode is loaded once per CTA.
+struct Inner32Layout {
+  uint32_t bimg, xs, os, xm, om, bars;  // offsets; buffer 1 of each at + its size
+  uint32_t xs_size, os_size, xm_size, om_size, total;
+};
+__host__ __device__ inline uint32_t al128u(uint32_t x) { return (x + 127u) / 128u * 128u; }
+constexpr int I32_NB_MAX = 4;
+__host__ __device__ inline Inner32Layout inner32_layout(int NT, int kp, int64_t K, int64_t J, int esz, bool masked,
+                                                        bool wupd, int nb) {
+  Inner32Layout L;
+  const uint32_t atile = (uint32_t)(kp / 8) * G32_LBO;
+  L.bimg = 3 * atile;
+  L.xs = al128u(L.bimg + 3u * (uint32_t)NT * (uint32_t)kp * 2u);
+  L.xs_size = al128u((uint32_t)(G32T * K * esz));
+  L.os = L.xs + nb * L.xs_size;
+  L.os_size = al128u((uint32_t)(G32T * J * esz));
+  L.xm = L.os + nb * L.os_size;
+  L.xm_size = masked ? al128u(4u * (uint32_t)(G32T * K / 32 + 2)) : 0u;
+  L.om = L.xm + nb * L.xm_size;
+  const uint32_t nw = (uint32_t)(G32T * J / 32 + 2);
+  L.om_size = wupd ? al128u(4u * (nw + 1) + 8u * nw) : 0u;
+  L.bars = L.om + nb * L.om_size;
+  L.total = L.bars + 8 * (I32_NB_MAX + 2) + 16;
+  return L;
+}
+
+template <bool CPLX, bool WUPD>
+__global__ void __launch_bounds__(G32T) inner32_kernel(const MG32Args p, const int64_t ntiles, const int NB) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int ESZ = CPLX ? 8 : 4;
+  const int kq = p.kp / 8;
+  const uint32_t atile = (uint32_t)kq * G32_LBO;
+  const uint32_t b_bytes = (uint32_t)p.NT * p.kp * 2;
+  const Inner32Layout L = inner32_layout(p.NT, p.kp, p.K, p.J, ESZ, p.bits != nullptr, WUPD, NB);
+  uint64_t* full = (uint64_t*)(smem + L.bars);  // [NB] a tile's rows (and mask words) landed
+  uint64_t* mbar = full + I32_NB_MAX;          // the tile's MMAs done
+  uint64_t* bbar = mbar + 1;                   // the operand image landed
+  uint32_t* tslot = (uint32_t*)(bbar + 1);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const bool masked = p.bits != nullptr;
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < I32_NB_MAX + 2; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tslot, p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t dt = *tslot;
+  const int64_t nloc = ntiles > blockIdx.x ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  if (tid == 0) {
+    mbar_expect_tx(bbar, 3 * b_bytes);
+    bulk_g2s(smem + L.bimg, p.img, 3 * b_bytes, bbar);
+  }
+  // the rows of local tile it into buffer bf: mask words by every thread,
+  // then (after a barrier, so that their pending arrivals are counted first)
+  // the bulk copies
+  auto issue = [&](int64_t it, int bf) {
+    const int64_t a0 = ((int64_t)blockIdx.x + it * gridDim.x) * G32T;
+    if (masked) {
+      uint32_t* xm = (uint32_t*)(smem + L.xm + bf * L.xm_size);
+      const int64_t w0 = (a0 * p.K) >> 5, nw = (((a0 + G32T) * p.K - 1) >> 5) - w0 + 1;
+      for (int w = tid; w < nw; w += G32T) cpa4(xm + w, p.bits + w0 + w);
+    }
+    if (WUPD) {
+      uint32_t* om = (uint32_t*)(smem + L.om + bf * L.om_size);
+      const int64_t w0 = (a0 * p.J) >> 5, nw = (((a0 + G32T) * p.J - 1) >> 5) - w0 + 1;
+      int64_t* orank = (int64_t*)(om + ((nw + 1) & ~1ll));
+      for (int w = tid; w < nw; w += G32T) {
+        cpa4(om + w, p.wbits + w0 + w);
+        cpa8(orank + w, p.wrank + w0 + w);
+      }
+    }
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[bf])) : "memory");
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t xb = (uint32_t)(G32T * p.K * ESZ), wb = WUPD ? (uint32_t)(G32T * p.J * ESZ) : 0u;
+      mbar_expect_tx(&full[bf], xb + wb);
+      bulk_g2s(smem + L.xs + bf * L.xs_size, (const uint8_t*)p.X + a0 * p.K * ESZ, xb, &full[bf]);
+      if (WUPD) bulk_g2s(smem + L.os + bf * L.os_size, (const uint8_t*)p.W + a0 * p.J * ESZ, wb, &full[bf]);
+    }
+  };
+  auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (!mbar_wait(bar, parity, G32_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    return s_abort == 0;
+  };
+  int64_t issued = 0;
+  for (; issued < NB - 1 && issued < nloc; ++issued) issue(issued, (int)issued);
+  bool ok = nloc == 0 || wait_bar(bbar, 0);
+  const uint32_t idesc = idesc_f16(1, 128, p.NT);
+  const uint32_t lbo_b = (uint32_t)(p.NT / 8) * 128;
+  constexpr int KE = CPLX ? G32_KMAX / 2 : G32_KMAX;
+  const int ke = CPLX ? p.kp / 2 : p.kp;
+  for (int64_t it = 0; ok && it < nloc; ++it) {
+    const int bf = (int)(it % NB);
+    const int64_t a0 = ((int64_t)blockIdx.x + it * gridDim.x) * G32T;
+    if (it + NB - 1 < nloc) {
+      // the buffer of tile it + NB - 1 held tile it - 1: its store must have
+      // read it out
+      if (tid == 0) bulk_wait_read0();
+      issue(it + NB - 1, (int)((it + NB - 1) % NB));
+      issued = it + NB;
+    }
+    if (!wait_bar(&full[bf], (uint32_t)((it / NB) & 1))) break;
+    // this row's K values (Omega's entries zero) -> the h, m, l A tiles
+    {
+      const float* xs = (const float*)(smem + L.xs + bf * L.xs_size);
+      const uint32_t* xm = (const uint32_t*)(smem + L.xm + bf * L.xm_size);
+      const int64_t w0 = (a0 * p.K) >> 5;
+      float v[G32_KMAX];
+#pragma unroll
+      for (int i = 0; i < KE; ++i) {
+        if (i >= ke) break;
+        float2 x = make_float2(0.f, 0.f);
+        if (i < p.K) {
+          const int64_t idx = (a0 + tid) * p.K + i;
+          const uint32_t word = masked ? xm[(idx >> 5) - w0] : 0u;
+          if (!((word >> (idx & 31)) & 1u)) {
+            if (CPLX)
+              x = ((const float2*)xs)[tid * p.K + i];
+            else
+              x.x = xs[tid * p.K + i];
+          }
+        }
+        if (CPLX) {
+          v[2 * i] = x.x;
+          v[2 * i + 1] = x.y;
+        } else {
+          v[i] = x.x;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < G32_KMAX / 8; ++q) {
+        if (q >= kq) break;
+        uint32_t h[4], m[4], l[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) split3(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], h[u], m[u], l[u]);
+        *(uint4*)(smem + 0 * atile + q * G32_LBO + tid * 16) = make_uint4(h[0], h[1], h[2], h[3]);
+        *(uint4*)(smem + 1 * atile + q * G32_LBO + tid * 16) = make_uint4(m[0], m[1], m[2], m[3]);
+        *(uint4*)(smem + 2 * atile + q * G32_LBO + tid * 16) = make_uint4(l[0], l[1], l[2], l[3]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t a_base = smem_u32(smem), b_base = smem_u32(smem + L.bimg);
+      for (int kk = 0; kk < kq / 2; ++kk) {
+        // (A part, B part): hh, hm, mh, hl, lh, mm
+#pragma unroll
+        for (int pr = 0; pr < 6; ++pr) {
+          const uint32_t pa = (0x120100u >> (4 * pr)) & 0xFu, pb = (0x102010u >> (4 * pr)) & 0xFu;
+          const uint64_t da = sdesc(a_base + pa * atile + kk * 2 * G32_LBO, G32_LBO, 128);
+          const uint64_t db = sdesc(b_base + pb * b_bytes + kk * 2 * lbo_b, lbo_b, 128);
+          mma_f16(dt, da, db, idesc, (kk > 0 || pr > 0) ? 1u : 0u);
+        }
+      }
+      mma_commit(mbar);
+    }
+    if (!wait_bar(mbar, (uint32_t)(it & 1))) break;
+    tc_fence_after();
+    // the tile's rows of Y, or W updated in place, in buffer bf
+    {
+      float* os = (float*)(smem + L.os + bf * L.os_size);
+      const uint32_t* omw = (const uint32_t*)(smem + L.om + bf * L.om_size);
+      const int64_t ow0 = (a0 * p.J) >> 5;
+      const int onw = (int)((((a0 + G32T) * p.J - 1) >> 5) - ow0 + 1);
+      const int64_t* omr = (const int64_t*)(omw + ((onw + 1) & ~1));
+      for (int c0 = 0; c0 < p.NT; c0 += 16) {
+        constexpr int PER = CPLX ? 8 : 16;
+        // the block's S~ values first (independent loads, in flight together)
+        float2 sv[PER];
+        if (WUPD) {
+#pragma unroll
+          for (int u = 0; u < PER; ++u) {
+            sv[u] = make_float2(0.f, 0.f);
+            const int64_t j = (CPLX ? c0 / 2 : c0) + u;
+            if (j >= p.J) continue;
+            const int64_t o = (a0 + tid) * p.J + j;
+            const uint32_t word = omw[(o >> 5) - ow0];
+            const uint32_t bit = (uint32_t)(o & 31);
+            if ((word >> bit) & 1u) {
+              const int64_t e = omr[(o >> 5) - ow0] + __popc(word & ((1u << bit) - 1u));
+              if (CPLX)
+                sv[u] = __ldg((const float2*)p.S + e);
+              else
+                sv[u].x = __ldg(p.S + e);
+            }
+          }
+        }
+        float y[16];
+        tmem_ld16(dt + lane_base + c0, y);
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const int64_t j = (CPLX ? c0 / 2 : c0) + u;
+          if (j >= p.J) continue;
+          const int64_t so = (int64_t)tid * p.J + j;
+          float dr = CPLX ? y[2 * u] : y[u], di = CPLX ? y[2 * u + 1] : 0.f;
+          if (!WUPD) {
+            if (CPLX)
+              ((float2*)os)[so] = make_float2(dr, di);
+            else
+              os[so] = dr;
+          } else {
+            dr += sv[u].x;
+            di += sv[u].y;
+            if (CPLX) {
+              const float2 w = ((float2*)os)[so];
+              ((float2*)os)[so] = make_float2(__fmaf_rn(-p.lr, dr, w.x * p.decay), __fmaf_rn(-p.lr, di, w.y * p.decay));
+            } else {
+              os[so] = __fmaf_rn(-p.lr, dr, os[so] * p.decay);
+            }
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        uint8_t* dst = WUPD ? (uint8_t*)p.W : (uint8_t*)p.Y;
+        bulk_s2g(dst + a0 * p.J * ESZ, os, (uint32_t)(G32T * p.J * ESZ));
+        bulk_commit();
+      }
+    }
+  }
+  if (tid == 0) {
+    bulk_wait_read0();  // no store still reads this CTA's shared memory
+    if (s_abort) {
+      // bounded waits for copies still in flight
+      for (int64_t i = issued > NB ? issued - NB : 0; i < issued; ++i)
+        mbar_wait(&full[i % NB], (uint32_t)((i / NB) & 1), G32_WAIT_NS / 4);
+      mbar_wait(bbar, 0, G32_WAIT_NS / 4);
+      mbar_wait(mbar, 0, G32_WAIT_NS / 4);
+      mbar_wait(mbar, 1, G32_WAIT_NS / 4);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(dt, p.tmem_cols);
+}
+
 size_t g32_smem(int NT, int nstage, int kp) {
   return (size_t)nstage * (3 * (size_t)(kp / 8) * G32_LBO + 3 * (size_t)NT * kp * 2) + 64;
 }
@@ -511,9 +802,46 @@ void mode_geom(int64_t Kc, int64_t Jc, bool cplx, int& NT, int& nnt, int& nkc, i
 template <bool CPLX, bool WUPD>
 cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
   const size_t esz = CPLX ? 8 : 4;
+  a.tile0 = 0;
+  // the innermost mode with one K chunk and one column block: the persistent
+  // kernel over the whole 128-row tiles, this kernel for a ragged last tile
+  const void* outp = WUPD ? (const void*)a.W : (const void*)a.Y;
+  if (a.B == 1 && a.nkc == 1 && nnt == 1 && a.rows >= G32T && ((uintptr_t)a.X % 16) == 0 &&
+      ((uintptr_t)outp % 16) == 0) {
+    // the most CTAs per SM (a tile's latency chain bounds each CTA), then the
+    // deepest ring those leave room for
+    int nb = 0, cps = 0;
+    Inner32Layout L{};
+    for (int b = 2; b <= I32_NB_MAX; ++b) {
+      const Inner32Layout Lb = inner32_layout(a.NT, a.kp, a.K, a.J, (int)esz, a.bits != nullptr, WUPD, b);
+      if (Lb.total > G32_SMEM_LIMIT) break;
+      const int c = std::min(4, (int)(232448 / (Lb.total + 1024)));
+      if (c >= cps) {
+        nb = b;
+        cps = c;
+        L = Lb;
+      }
+    }
+    if (nb > 0) {
+      int dev = 0, nsm = 148;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      const int64_t ntiles = a.rows / G32T;
+      const int64_t grid = std::min<int64_t>(ntiles, (int64_t)nsm * cps);
+      cudaError_t e = cudaFuncSetAttribute(inner32_kernel<CPLX, WUPD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)L.total);
+      if (e != cudaSuccess) return e;
+      inner32_kernel<CPLX, WUPD><<<(unsigned)grid, G32T, L.total, s>>>(a, ntiles, nb);
+      e = cudaGetLastError();
+      if (e != cudaSuccess || a.rows % G32T == 0) return e;
+      a.tile0 = ntiles;
+    }
+  }
   size_t sm = g32_smem(a.NT, a.nstage, a.kp);
   a.xs_off = 0;
   a.os_off = 0;
+  a.xm_off = 0;
+  a.om_off = 0;
   if (a.B == 1) {
     size_t off = al128(sm);
     if (a.nkc == 1 && ((uintptr_t)a.X % 16) == 0) {
@@ -531,12 +859,29 @@ cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
         off = need;
       }
     }
+    // mask words of a staged range: at most 128 K / 32 + 2 (X), and for the
+    // update that many words and as many 8-byte ranks (output)
+    if (a.xs_off && a.bits) {
+      const size_t need = off + al128(4 * ((size_t)G32T * a.K / 32 + 2));
+      if (need <= G32_SMEM_LIMIT) {
+        a.xm_off = (uint32_t)off;
+        off = need;
+      }
+    }
+    if (a.os_off && WUPD) {
+      const size_t nw = (size_t)G32T * a.J / 32 + 2;
+      const size_t need = off + al128(4 * (nw + 1) + 8 * nw);
+      if (need <= G32_SMEM_LIMIT) {
+        a.om_off = (uint32_t)off;
+        off = need;
+      }
+    }
     sm = off;
   }
   cudaError_t e = cudaFuncSetAttribute(mode_gemm32_kernel<CPLX, WUPD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)ceil_div(a.rows, G32T), (unsigned)nnt);
+  dim3 grid((unsigned)(ceil_div(a.rows, G32T) - a.tile0), (unsigned)nnt);
   mode_gemm32_kernel<CPLX, WUPD><<<grid, G32T, sm, s>>>(a);
   return cudaGetLastError();
 }

@@ -45,6 +45,9 @@ CASES = {
     "r32_16x16x8x8": ((16, 16, 8, 8), (4, 4, 2, 2), "r32", 0.05),
     "r32_3way": ((7, 6, 9), (3, 2, 4), "r32", 0.05),
     "r32_two_chunks_70x66x5": ((70, 66, 5), (6, 9, 2), "r32", 0.05),
+    # innermost-mode launches over whole 128-row tiles plus a ragged one (300 rows)
+    "c64_ragged_tail_10x30x17": ((10, 30, 17), (3, 6, 5), "c64", 0.05),
+    "r32_ragged_tail_5x52x33": ((5, 52, 33), (2, 6, 7), "r32", 0.05),
 }
 
 
