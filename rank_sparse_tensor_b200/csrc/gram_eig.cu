@@ -318,14 +318,14 @@ __global__ void __launch_bounds__(RC * RS) gram_reduce_kernel(const float2* part
 //   words of Omega's bitmask the chunk needs (two per row, or the block's)
 //   come by asynchronous copies beside it (TG_ELEMS, the fallback, reads the
 //   bits where it converts);
-// - two groups of four converter warps take alternate chunks, each group
+// - two groups of eight converter warps take alternate chunks, each group
 //   turning its chunk into the bf16 tiles of its own tile set (one thread:
 //   one row, four columns), the entries of Omega read as zero (the
 //   residual);
 // - one thread issues the chunk's MMAs and commits them to the tile set's
 //   free barrier.
-constexpr int TG_CONV_WARPS = 8;
-constexpr int TG_GROUP_WARPS = 4;           // converter warps per tile set
+constexpr int TG_CONV_WARPS = 16;
+constexpr int TG_GROUP_WARPS = 8;           // converter warps per tile set
 constexpr int TG_PROD_WARP = TG_CONV_WARPS;
 constexpr int TG_MMA_WARP = TG_CONV_WARPS + 1;
 constexpr int TG_THREADS = 32 * (TG_CONV_WARPS + 2);
