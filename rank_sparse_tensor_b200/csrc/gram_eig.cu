@@ -967,7 +967,7 @@ __device__ __forceinline__ double2 zmul(double2 a, double2 b) {
 }
 __device__ __forceinline__ double zabs2(double2 a) { return a.x * a.x + a.y * a.y; }
 
-constexpr int ET = 512;  // threads per eigensolver block
+constexpr int ET = 1024;  // threads per eigensolver block
 constexpr int MAXN = 256;
 
 __device__ double block_sum(double v, double* red) {
