@@ -317,7 +317,7 @@ class Bench:
         # tensors go round-robin onto ns streams, each with 1/ns of the SMs
         ns = min(nt, args.tensor_streams) if args.tensor_streams > 0 else nt
         self.n_streams = ns if self.concurrent else 1
-        sm_budget = max(1, n_sms // ns) if self.concurrent else 0
+        sm_budget = max(1, n_sms // ns) if self.concurrent and not args.full_sms else 0
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(ns)] if self.concurrent else None
         self.tensors = []
         for gseed, wseed in tensor_seeds(rank, nt):
@@ -449,7 +449,7 @@ def other_workload(name, args, dev, world, rank, local, barrier, hbm_gbs, opts=N
            "shape": list(wl.shape), "ranks": list(wl.ranks), "tensors_per_gpu": len(b.tensors),
            "T": wl.T, "grad_dtype": wl.dtype, "kernel_path": b.tensors[0][0].info["path"],
            "l2": "flushed between steps" if b.flush else "inputs larger than L2",
-           "tensor_streams": ("%d streams, tensors round-robin, 1/%d of the SMs each" % (b.n_streams, b.n_streams))
+           "tensor_streams": ("%d streams, tensors round-robin, %s" % (b.n_streams, "all SMs each" if b.args.full_sms else "1/%d of the SMs each" % b.n_streams))
            if b.concurrent else "one stream",
            "roofline": dict(step_roofline(wl, len(b.tensors), step_ms, hbm_gbs), peak=hbm_gbs,
                             unit="GB/s", bound="hbm"),
@@ -513,6 +513,8 @@ def main():
     ap.add_argument("--tensor-streams", type=int, default=0,
                     help="streams the tensors of a multi-tensor workload are spread over "
                          "(each with that share of the SMs); 0 = one per tensor")
+    ap.add_argument("--full-sms", action="store_true",
+                    help="concurrent tensors' kernels each sized for all SMs (no SM budget)")
     ap.add_argument("--sequential", action="store_true",
                     help="step the tensors of a multi-tensor workload one after another on one "
                          "stream (default: each on its own stream with an equal share of the SMs)")
@@ -605,7 +607,7 @@ def main():
                    "kernel_path": tensors[0][0].info["path"],
                    "l2": "flushed between steps" if b.flush else "inputs larger than L2",
                    "parallelism": f"independent tensors per rank x{world}",
-                   "tensor_streams": "%d streams, tensors round-robin, 1/%d of the SMs each" % (b.n_streams, b.n_streams)
+                   "tensor_streams": "%d streams, tensors round-robin, %s" % (b.n_streams, "all SMs each" if args.full_sms else "1/%d of the SMs each" % b.n_streams)
                    if b.concurrent else "one stream"},
         "roofline": dict({"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm_gbs,
                           "unit": "GB/s", "frac": (achieved / hbm_gbs) if achieved else None,
