@@ -183,69 +183,79 @@ __global__ void __launch_bounds__(1024) block_offsets_kernel(const int* blk_lt, 
   }
 }
 
+// Ordered compaction of one block of CHUNK keys. Key r CT + t of the block
+// belongs to thread t (coalesced loads), so index order is (r, warp, lane).
+// Each thread loads its CHUNK / CT keys first and keeps two flags each (below
+// / equal to the threshold); per (r, warp) counts of equal keys, then of taken
+// keys, go through one block scan each, and every key's rank follows from its
+// warp's ballot. Ties go to the lower index.
 template <class KeyF, int DT>
-__global__ void __launch_bounds__(CT) write_kernel(KeyF kf, const void* g, int64_t n,
+__global__ void __launch_bounds__(CT, 4) write_kernel(KeyF kf, const void* g, int64_t n,
                                                    const SelState* st, const long long* out_off,
                                                    const long long* eq_before, int64_t* out_idx,
                                                    float* out_val) {
+  constexpr int PER = CHUNK / CT, NW = CT / 32;
+  static_assert(PER <= 32 && PER * NW <= CT, "flags in 32-bit words, one scan entry per thread");
+  __shared__ int s_cnt[PER * NW];
+  __shared__ long long s_ex[PER * NW];
   const uint64_t K = st->prefix;
   const long long need = st->need;
   const int64_t base = (int64_t)blockIdx.x * CHUNK;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  __shared__ int s_eq[CT / 32], s_tk[CT / 32];
-  long long run_eq = eq_before[blockIdx.x];
-  long long run_out = out_off[blockIdx.x];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
-  // all of this thread's keys first (independent loads in flight), kept as
-  // two flags each; the compaction below then waits on no global load
-  static_assert(CHUNK / CT <= 32, "flags are packed in 32-bit words");
   uint32_t ltm = 0, eqm = 0;
 #pragma unroll
-  for (int r = 0; r < CHUNK / CT; ++r) {
-    const int64_t i = base + r * CT + threadIdx.x;
+  for (int r = 0; r < PER; ++r) {
+    const int64_t i = base + r * CT + tid;
     const bool valid = i < n;
     const uint64_t key = valid ? kf(i) : ~0ull;
     ltm |= (uint32_t)(valid && key < K) << r;
     eqm |= (uint32_t)(valid && key == K) << r;
   }
-  for (int r = 0; r < CHUNK / CT; ++r) {
-    int64_t i = base + r * CT + threadIdx.x;
-    const bool lt = (ltm >> r) & 1u, eq = (eqm >> r) & 1u;
-    unsigned be = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_eq[wid] = __popc(be);
-    __syncthreads();
-    int eq_w = 0, eq_tot = 0;
-    for (int w = 0; w < CT / 32; ++w) {
-      eq_tot += s_eq[w];
-      if (w < wid) eq_w += s_eq[w];
+  // exclusive prefix, in (r, warp) order, of per-(r, warp) counts of flags f
+  auto rank_base = [&](uint32_t f) {
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const unsigned b = __ballot_sync(0xffffffffu, (f >> r) & 1u);
+      if (lane == 0) s_cnt[r * NW + wid] = __popc(b);
     }
-    long long eq_rank = run_eq + eq_w + __popc(be & lt_mask);
-    bool take = lt || (eq && eq_rank < need);
-    unsigned bt = __ballot_sync(0xffffffffu, take);
-    if (lane == 0) s_tk[wid] = __popc(bt);
     __syncthreads();
-    int tk_w = 0, tk_tot = 0;
-    for (int w = 0; w < CT / 32; ++w) {
-      tk_tot += s_tk[w];
-      if (w < wid) tk_w += s_tk[w];
+    const unsigned long long v = tid < PER * NW ? (unsigned long long)s_cnt[tid] : 0ull;
+    const unsigned long long ex = block_excl_scan(v, nullptr);
+    if (tid < PER * NW) s_ex[tid] = (long long)ex;
+    __syncthreads();
+  };
+  rank_base(eqm);
+  uint32_t take = ltm;
+  const long long eq0 = eq_before[blockIdx.x];
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    const unsigned b = __ballot_sync(0xffffffffu, (eqm >> r) & 1u);
+    if ((eqm >> r) & 1u) {
+      const long long rank = eq0 + s_ex[r * NW + wid] + __popc(b & lt_mask);
+      if (rank < need) take |= 1u << r;
     }
-    if (take) {
-      long long pos = run_out + tk_w + __popc(bt & lt_mask);
-      out_idx[pos] = i;
-      if (out_val) {
-        if constexpr (DT >= 0) {
-          float2 v = load_elem<DT>(g, i);
-          if constexpr (Dt<DT>::cplx) {
-            ((float2*)out_val)[pos] = v;
-          } else {
-            out_val[pos] = v.x;
-          }
+  }
+  __syncthreads();  // s_ex is rewritten below
+  rank_base(take);
+  const long long off0 = out_off[blockIdx.x];
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    const unsigned b = __ballot_sync(0xffffffffu, (take >> r) & 1u);
+    if (!((take >> r) & 1u)) continue;
+    const long long pos = off0 + s_ex[r * NW + wid] + __popc(b & lt_mask);
+    const int64_t i = base + r * CT + tid;
+    out_idx[pos] = i;
+    if (out_val) {
+      if constexpr (DT >= 0) {
+        const float2 v = load_elem<DT>(g, i);
+        if constexpr (Dt<DT>::cplx) {
+          ((float2*)out_val)[pos] = v;
+        } else {
+          out_val[pos] = v.x;
         }
       }
     }
-    run_eq += eq_tot;
-    run_out += tk_tot;
-    __syncthreads();
   }
 }
 
