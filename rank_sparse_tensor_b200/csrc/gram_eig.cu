@@ -996,9 +996,9 @@ __device__ double block_max(double v, double* red) {
 // parallel ordering (n/2 disjoint pairs per round). A and the eigenvector
 // rows Vt are both whole, with an odd row pitch (a column walk by 32 lanes
 // touches 32 different banks), in shared memory for n <= 64 and in the job's
-// global scratch above that; one warp per rotation pair, and each round in
-// two phases (J^H on the pairs' rows, then J on their columns and on V) so
-// that every access is a plain load or store of one entry.
+// global scratch above that. A round applies its rotations to A on 2 x 2
+// blocks of pairs, a thread per block (each entry is read and written once,
+// the mirror half from the upper one), and to V a warp per pair.
 constexpr int ES_MAXN = MAXN;
 constexpr int ES_SMEM_MAXN = 64;
 
@@ -1019,6 +1019,7 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
   __shared__ double ev[ES_MAXN];
   __shared__ int col_of_rank[ES_MAXN];
   __shared__ uint8_t lead[ES_MAXN];
+  __shared__ uint8_t bk1[ES_MAXN / 2 * (ES_MAXN / 2 + 1) / 2], bk2[ES_MAXN / 2 * (ES_MAXN / 2 + 1) / 2];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
   const double2* G = (const double2*)J.gram;
   if (J.warm) {
@@ -1075,6 +1076,18 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
   const double fro = block_sum(part, red);
   const int m = n + (n & 1);
   const int npairs = m / 2;
+  // the 2 x 2 blocks of pairs (k1 <= k2), row by row
+  const int nblk = npairs * (npairs + 1) / 2;
+  for (int b = tid; b < nblk; b += blockDim.x) {
+    int k1 = 0, rr = b;
+    while (rr >= npairs - k1) {
+      rr -= npairs - k1;
+      ++k1;
+    }
+    bk1[b] = (uint8_t)k1;
+    bk2[b] = (uint8_t)(k1 + rr);
+  }
+  __syncthreads();
   const int r = J.r;
   for (int sweep = 0; sweep < 40; ++sweep) {
     // Stop when A is diagonal to 1e-24 of its squared Frobenius norm, or
@@ -1161,41 +1174,73 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
         }
       }
       __syncthreads();
-      // rows p, q <- J^H (rows p, q)
-      for (int k = wid; k < npairs; k += nw) {
-        if (!rrot[k]) continue;
-        const int p = rp[k], q = rq[k];
-        const double c = rcs[k], s = rsn[k];
-        const double2 e = rph[k];
-        for (int j = lane; j < n; j += 32) {
-          const double2 xp = A[p * NP + j], xq = zmul(A[q * NP + j], e);
-          A[p * NP + j] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          A[q * NP + j] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+      // A <- J^H A J on 2 x 2 blocks of pairs (k1 <= k2): a thread reads the
+      // block's four entries once, applies J_k2 to its columns and J_k1^H to
+      // its rows, and writes it and its mirror (A is Hermitian); the diagonal
+      // blocks come out with (p, q) zero and a real diagonal
+      for (int b = tid; b < nblk; b += blockDim.x) {
+        const int k1 = bk1[b], k2 = bk2[b];
+        const bool rot1 = rrot[k1], rot2 = rrot[k2];
+        if (!rot1 && !rot2) continue;
+        const int p1 = rp[k1], q1 = rq[k1], p2 = rp[k2], q2 = rq[k2];
+        const bool h1 = q1 < n, h2 = q2 < n;  // the dummy index of odd n is absent
+        const double2 z = make_double2(0.0, 0.0);
+        double2 b00 = A[p1 * NP + p2], b01 = h2 ? A[p1 * NP + q2] : z;
+        double2 b10 = h1 ? A[q1 * NP + p2] : z, b11 = h1 && h2 ? A[q1 * NP + q2] : z;
+        if (rot2) {
+          const double c = rcs[k2], s = rsn[k2];
+          const double2 ec = make_double2(rph[k2].x, -rph[k2].y);
+          double2 xp = b00, xq = zmul(b01, ec);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b01 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b10;
+          xq = zmul(b11, ec);
+          b10 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (rot1) {
+          const double c = rcs[k1], s = rsn[k1];
+          const double2 e = rph[k1];
+          double2 xp = b00, xq = zmul(b10, e);
+          b00 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b10 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+          xp = b01;
+          xq = zmul(b11, e);
+          b01 = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
+          b11 = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
+        }
+        if (k1 == k2) {
+          A[p1 * NP + p1] = make_double2(b00.x, 0.0);
+          if (h1) {
+            A[p1 * NP + q1] = z;
+            A[q1 * NP + p1] = z;
+            A[q1 * NP + q1] = make_double2(b11.x, 0.0);
+          }
+        } else {
+          A[p1 * NP + p2] = b00;
+          A[p2 * NP + p1] = make_double2(b00.x, -b00.y);
+          if (h2) {
+            A[p1 * NP + q2] = b01;
+            A[q2 * NP + p1] = make_double2(b01.x, -b01.y);
+          }
+          if (h1) {
+            A[q1 * NP + p2] = b10;
+            A[p2 * NP + q1] = make_double2(b10.x, -b10.y);
+          }
+          if (h1 && h2) {
+            A[q1 * NP + q2] = b11;
+            A[q2 * NP + q1] = make_double2(b11.x, -b11.y);
+          }
         }
       }
-      __syncthreads();
-      // columns p, q <- (columns p, q) J, and V <- V J on the rows of Vt;
-      // the rotation leaves (p, q) zero and the diagonal real
+      // V <- V J on the rows of Vt, a warp per pair
       for (int k = wid; k < npairs; k += nw) {
         if (!rrot[k]) continue;
         const int p = rp[k], q = rq[k];
         const double c = rcs[k], s = rsn[k];
         const double2 ec = make_double2(rph[k].x, -rph[k].y);
         for (int i = lane; i < n; i += 32) {
-          double2 xp = A[i * NP + p], xq = zmul(A[i * NP + q], ec);
-          double2 np = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
-          double2 nq = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
-          if (i == p) {
-            np.y = 0.0;
-            nq = make_double2(0.0, 0.0);
-          } else if (i == q) {
-            np = make_double2(0.0, 0.0);
-            nq.y = 0.0;
-          }
-          A[i * NP + p] = np;
-          A[i * NP + q] = nq;
-          xp = Vt[p * NP + i];
-          xq = zmul(Vt[q * NP + i], ec);
+          const double2 xp = Vt[p * NP + i], xq = zmul(Vt[q * NP + i], ec);
           Vt[p * NP + i] = make_double2(c * xp.x - s * xq.x, c * xp.y - s * xq.y);
           Vt[q * NP + i] = make_double2(s * xp.x + c * xq.x, s * xp.y + c * xq.y);
         }
