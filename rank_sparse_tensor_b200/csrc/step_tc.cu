@@ -524,7 +524,14 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
           tmem_ld32(tmem + p.d1_col[b] + lane_base + c0, v);
         else
           tmem_ld16(tmem + p.d1_col[b] + lane_base + c0, v);
-        if (valid) {
+        const int jb0 = m2base + c0 / 2;
+        if (valid && (jb0 & 7) == 0 && c0 / 2 + 16 <= p.rb) {
+          // 16 whole rows from an 8-row boundary: offsets from one base
+          uint8_t* dst = A2 + kmaj_off((uint32_t)jb0, (uint32_t)(2 * ia_row), p.lbo_a2);
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            *(uint32_t*)(dst + (u & 7) * 16 + (u >> 3) * 128) = f2_to_bf2(v[2 * u], v[2 * u + 1]);
+        } else if (valid) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             int jb = c0 / 2 + u;
@@ -761,6 +768,33 @@ __device__ __forceinline__ float2 wload(const __half2* p) { return __half22float
 __device__ __forceinline__ void wstore(__half2* p, float x, float y) { *p = __floats2half2_rn(x, y); }
 __device__ __forceinline__ float2 wload(const float2* p) { return *p; }
 __device__ __forceinline__ void wstore(float2* p, float x, float y) { *p = make_float2(x, y); }
+// v + d for an fp16 pair d by mixed-precision adds (no separate conversion;
+// the same value as converting d and adding in fp32)
+__device__ __forceinline__ float2 add_f2_h2(float2 v, uint32_t d) {
+  float2 x;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %3;\n\tadd.rn.f32.f16 %1, hi, %4;\n\t}"
+      : "=f"(x.x), "=f"(x.y)
+      : "r"(d), "f"(v.x), "f"(v.y));
+  return x;
+}
+// a * b + c on a pair (packed fp32: two fmaf_rn in one instruction)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 
 constexpr int R3T = 512;
 constexpr int PREP_ITEMS = 2;  // B1 items per prep thread whose addressing is precomputed
@@ -1156,19 +1190,19 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
         if (!valid) continue;
         const int ib0 = c * 8;
         if (ib0 + 8 <= Ib) {
-          float2 w[8], d[8];
+          float2 w[8];
+          uint32_t d[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             w[u] = wload(wrow + ib0 + u);
-            d[u] = h2_to_f2(drow[ib0 + u]);
+            d[u] = drow[ib0 + u];
           }
+          const float2 nlr2 = make_float2(nlr, nlr), dec2 = make_float2(decay, decay);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float xr = v[2 * u] + d[u].x, xi = v[2 * u + 1] + d[u].y;
-            if (UNIT_DECAY)
-              wstore(wrow + ib0 + u, __fmaf_rn(nlr, xr, w[u].x), __fmaf_rn(nlr, xi, w[u].y));
-            else
-              wstore(wrow + ib0 + u, __fmaf_rn(nlr, xr, w[u].x * decay), __fmaf_rn(nlr, xi, w[u].y * decay));
+            const float2 x = add_f2_h2(make_float2(v[2 * u], v[2 * u + 1]), d[u]);
+            const float2 y = ffma2(nlr2, x, UNIT_DECAY ? w[u] : fmul2(w[u], dec2));
+            wstore(wrow + ib0 + u, y.x, y.y);
           }
         } else {
 #pragma unroll
