@@ -406,10 +406,6 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
         sw[l] = 0u;
       }
       if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
-      cur_e0 = nx_e0;
-      cur_e1 = nx_e1;
-      nx_e0 = nn_e0;
-      nx_e1 = nn_e1;
       named_sync(1, 256);  // every zeroed entry is in place before conversion
       if (!waitw(&a1empty[b], par ^ 1u, s_abort, p.err, p.wait_ns)) {
         dead_from = it + 1;
@@ -440,6 +436,12 @@ __global__ void __launch_bounds__(P1T, 1) proj_stream_kernel(const P1Args p) {
       tc_fence_before();
       mbar_arrive(&a1full[b]);
       mbar_arrive(&sempty[s]);
+      // move to the next tile's ranges at the end of the tile, well after
+      // the loads of the one two ahead were issued
+      cur_e0 = nx_e0;
+      cur_e1 = nx_e1;
+      nx_e0 = nn_e0;
+      nx_e1 = nn_e1;
       cur.next(q);
       ahead.next(q);
       if (++s == ns) {
@@ -1172,6 +1174,11 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
         if (e < cur_e1) ds[pf_loc[j]] = pf_val[j];
       }
       for (int64_t e = cur_e0 + 256 * EPF + et; e < cur_e1; e += 256) ds[p.loc[e]] = p.sp_upd[e];
+      // the next tile's entries, a whole tile ahead of their use
+      uint32_t zl[EPF];
+#pragma unroll
+      for (int j = 0; j < EPF; ++j) zl[j] = pf_loc[j];
+      if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
       named_sync(2, 256);
       if (!waitw(&d2full[b], par, s_abort, p.err) || !waitw(&full[s], sph, s_abort, p.err)) {
         named_sync(2, 256);
@@ -1224,11 +1231,10 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
 #pragma unroll
       for (int j = 0; j < EPF; ++j) {
         int64_t e = cur_e0 + et + 256 * j;
-        if (e < cur_e1) ds[pf_loc[j]] = 0u;
+        if (e < cur_e1) ds[zl[j]] = 0u;
       }
       for (int64_t e = cur_e0 + 256 * EPF + et; e < cur_e1; e += 256) ds[p.loc[e]] = 0u;
       named_sync(2, 256);  // zeroed before the next tile scatters
-      if (it + 1 < n_it) load_entries(nx_e0, nx_e1);
       cur_e0 = nx_e0;
       cur_e1 = nx_e1;
       nx_e0 = nn_e0;
