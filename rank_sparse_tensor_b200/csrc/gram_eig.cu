@@ -1000,6 +1000,11 @@ __device__ double block_max(double v, double* red) {
 // blocks of pairs, a thread per block (each entry is read and written once,
 // the mirror half from the upper one), and to V a warp per pair.
 constexpr int ES_MAXN = MAXN;
+// Off-diagonal mass, relative to |A|_F^2, below which the rotations stop:
+// entries under 1e-9 |A|_F move the eigenvectors by less than the Gram's own
+// error (fp32 accumulation, ~1e-7 relative), and the eigenvalues by their
+// square.
+constexpr double JAC_TOL = 1e-18;
 constexpr int ES_SMEM_MAXN = 64;
 
 __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
@@ -1090,7 +1095,7 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
   __syncthreads();
   const int r = J.r;
   for (int sweep = 0; sweep < 40; ++sweep) {
-    // Stop when A is diagonal to 1e-24 of its squared Frobenius norm, or
+    // Stop when A is diagonal to JAC_TOL of its squared Frobenius norm, or
     // when the r rows of the largest diagonal entries are (their off-diagonal
     // mass below the same bound: those diagonal entries and rows of Vt are
     // eigenpairs) and a Gershgorin bound puts every eigenvalue of the other
@@ -1133,9 +1138,9 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
     const double lead_off = block_sum(lead_part, red);
     const double ger = block_max(ger_part, red);
     const double low = -block_max(-low_part, red);
-    if (off <= 1e-24 * fro || off == 0.0) break;
+    if (off <= JAC_TOL * fro || off == 0.0) break;
     // (the rows' coupling, at most sqrt(lead_off), moves no eigenvalue further)
-    if (r < n && lead_off <= 1e-24 * fro && ger + 2.0 * sqrt(lead_off) < low) break;
+    if (r < n && lead_off <= JAC_TOL * fro && ger + 2.0 * sqrt(lead_off) < low) break;
     for (int round = 0; round < m - 1; ++round) {
       // the round's disjoint pairs (round-robin) and their rotations
       for (int k = tid; k < npairs; k += blockDim.x) {
