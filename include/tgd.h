@@ -301,12 +301,9 @@ TGD_API tgd_status tgd_topk_select(const void* grad, tgd_dtype dtype, int64_t n,
  *  - n must not exceed TGD_TOPK_STATIC_MAX_N, else TGD_ERR_INVALID_ARG.
  *  - The array (TGD_TOPK_STATIC_SCRATCH_BYTES bytes) exists once per GPU
  *    that loads the library and stays allocated until the process exits.
- *  - The first call on each device looks up the array's device address on
- *    that device (the current device); make that first call before any
- *    stream capture. This note is about that set-up only.
- *  - The address is looked up once per device and kept until the process
- *    exits: after cudaDeviceReset on a device, this entry point must not be
- *    called on that device again in the same process.
+ *  - Every call looks up the array's device address on the current device
+ *    (a host-side query, no stream work), so calls may be captured into a
+ *    CUDA graph, and a device reset leaves nothing stale behind.
  *  - All calls share the array: calls whose work overlaps on the GPU (on
  *    different streams, or from different threads) race and give wrong
  *    results. Calls in one stream are ordered and safe; the array keeps the

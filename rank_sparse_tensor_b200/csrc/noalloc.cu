@@ -5,7 +5,6 @@
 // scratch space (digit histograms, selection state, per-block counts) lives
 // in `g_topk_scratch` below instead of a caller workspace.
 
-#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -16,9 +15,6 @@ namespace {
 // One copy per device, allocated with the module and kept until exit.
 static __device__ __align__(256) unsigned char g_topk_scratch[TGD_TOPK_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};  // device address of the array, per device
 tgd_status fail(tgd_status st, const std::string& msg) {
   tgd::set_global_error(msg);
   return st;
@@ -38,24 +34,13 @@ extern "C" tgd_status tgd_topk_select_static(const void* grad, tgd_dtype dtype, 
     return fail(TGD_ERR_INVALID_ARG, "scratch array too small for n");
   if (k == 0) return TGD_OK;
   if (!grad || !omega_out) return fail(TGD_ERR_INVALID_ARG, "grad or omega_out is NULL");
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(TGD_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return fail(TGD_ERR_UNSUPPORTED, "device index out of range");
+  // The array's device address in the current device's context, looked up
+  // on every call (a host-side query): nothing stale survives a device reset
+  // or a change of the current device.
   void* ws = nullptr;
-  {
-    // Set-up, once per device with that device current: the host-side name
-    // of the array is a stand-in, its device address comes from the runtime.
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-      void* ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, g_topk_scratch);
-      if (e != cudaSuccess || !ptr)
-        return fail(TGD_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-      g_scratch_ptr[dev] = ptr;
-    }
-    ws = g_scratch_ptr[dev];
-  }
+  cudaError_t e = cudaGetSymbolAddress(&ws, g_topk_scratch);
+  if (e != cudaSuccess || !ws)
+    return fail(TGD_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
   // The selection clears its histograms and initialises its state on the
   // stream before use, so the array's previous contents do not matter.
   e = tgd::select_topk(grad, dtype, n, k, omega_out, val_out, ws, (cudaStream_t)stream);
