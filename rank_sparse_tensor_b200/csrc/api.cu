@@ -59,6 +59,11 @@ struct tgd_ctx {
   bool eig_warm = false;             // eig_v holds them (every projected mode <= 128)
   EigJob* jobs_dev = nullptr;
   std::vector<EigJob> jobs;
+  // the refresh runs each mode's eigensolve on a side stream beside the next
+  // mode's Gram (fork and join by events)
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  int num_sms = 0;
   // generic step scratch
   float* P[TGD_MAX_NDIM] = {};  // projection coefficients (r x I)
   float* E[TGD_MAX_NDIM] = {};  // expansion coefficients (I x r)
@@ -189,6 +194,11 @@ bool dalloc_t(tgd_ctx* h, T** p, size_t count) {
 void free_all(tgd_ctx* h) {
   tc_release(h->tc);
   tc32_release(h->tc32);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
+  h->ev_fork = h->ev_join = nullptr;
+  h->side = nullptr;
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   h->ev_pool.clear();
   for (void* p : h->allocs) cudaFree(p);
@@ -420,10 +430,18 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
   }
   TGD_CUDA(h, build_mask_bits(h->omega, h->k, h->N, h->bits, s));
   h->jobs.clear();
+  // Each mode's eigensolve (one CTA, latency-bound) starts on the side stream
+  // as soon as its Gram is done and runs beside the next mode's Gram, which
+  // leaves one SM free for it; the main stream waits for the last one. Not
+  // for a handle given an SM budget: it shares the GPU with other streams.
+  const bool overlap = h->opt.basis != 1 && h->side && h->num_sms > 1 && h->opt.sm_budget == 0;
   for (int n = 0; n < h->d; ++n) {
     if (!mode_active(h, n)) continue;
-    TIMED(h, s, "mode_gram");
-    TGD_CUDA(h, mode_gram(g, h->gdt, h->bits, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s));
+    {
+      TIMED(h, s, "mode_gram");
+      TGD_CUDA(h, mode_gram(g, h->gdt, h->bits, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s,
+                            overlap ? h->num_sms - 1 : 0));
+    }
     EigJob j;
     j.gram = h->gram[n];
     j.work = h->eig_work[n];
@@ -434,8 +452,18 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.n = (int)h->I[n];
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
+    if (overlap) {
+      TGD_CUDA(h, cudaEventRecord(h->ev_fork, s));
+      TGD_CUDA(h, cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+      TIMED(h, h->side, "eigh");
+      TGD_CUDA(h, batched_eigh(&h->jobs.back(), 1, h->jobs_dev + (h->jobs.size() - 1), h->side));
+    }
   }
-  if (h->opt.basis == 1) {
+  if (overlap) {
+    TGD_CUDA(h, cudaEventRecord(h->ev_join, h->side));
+    TGD_CUDA(h, cudaStreamWaitEvent(s, h->ev_join, 0));
+    h->eig_warm = eig_keeps_vectors(h);
+  } else if (h->opt.basis == 1) {
     TIMED(h, s, "dct_select");
     TGD_CUDA(h, batched_dct_select(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
   } else {
@@ -750,6 +778,24 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
     free_all(h);
     delete h;
     return fail(nullptr, TGD_ERR_OOM, "device allocation failed");
+  }
+  {
+    // the refresh's side stream (see do_refresh); without it the refresh
+    // runs on the caller's stream alone
+    bool have = false;
+    for (int n = 0; n < ndim; ++n) have |= h->gram[n] != nullptr;
+    const bool made = have &&
+                      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) == cudaSuccess &&
+                      cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
+    if (!made) {
+      if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+      if (h->side) cudaStreamDestroy(h->side);
+      h->ev_fork = h->ev_join = nullptr;
+      h->side = nullptr;
+      cudaGetLastError();
+    }
   }
   cudaStream_t s = 0;
   cudaError_t e = cudaSuccess;

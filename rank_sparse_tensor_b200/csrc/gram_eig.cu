@@ -912,7 +912,7 @@ constexpr size_t TG_SMEM_LIMIT = 227 * 1024 - 1024;  // the opt-in maximum less 
 // fits and I <= 32, 16 for 8-byte elements when I > 64, else 32), the bf16
 // parts per value (two represent a 16-bit input exactly; used when I > 64)
 // and the most stages (up to four) that fit.
-TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int dt, bool aligned16) {
+TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int dt, bool aligned16, int max_splits) {
   const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
   TcGramGeom g;
   g.A = 1;
@@ -955,7 +955,8 @@ TcGramGeom tc_gram_geom(int nd, const int64_t* dims, int n, int dt, bool aligned
   }
   g.ns = TG_NS_MAX;
   while (g.ns > 2 && !fits(g.kc, g.ns)) --g.ns;
-  const int64_t ns = std::max<int64_t>(1, std::min<int64_t>(TG_MAX_SPLITS, g.nchunk));
+  const int cap = max_splits > 0 && max_splits < TG_MAX_SPLITS ? max_splits : TG_MAX_SPLITS;
+  const int64_t ns = std::max<int64_t>(1, std::min<int64_t>(cap, g.nchunk));
   g.chunks_per_split = ceil_div(g.nchunk, ns);
   g.nsplit = (int)ceil_div(g.nchunk, g.chunks_per_split);
   return g;
@@ -1405,9 +1406,9 @@ static cudaError_t rows_tensor_map(CUtensorMap* map, const void* g, int es, cons
 // Tensor-core Gram for I_n <= 64 (see gram_tc_kernel); the split partials are
 // summed by the same fixed-order fp64 reduction.
 cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                         int n, float* partial, double* gram, int* err, cudaStream_t s) {
+                         int n, float* partial, double* gram, int* err, cudaStream_t s, int max_ctas) {
   const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
-  const TcGramGeom t = tc_gram_geom(nd, dims, n, dt, ((uintptr_t)g & 15) == 0);
+  const TcGramGeom t = tc_gram_geom(nd, dims, n, dt, ((uintptr_t)g & 15) == 0, max_ctas);
   TcGramArgs a;
   a.g = g;
   a.bits = bits;
@@ -1465,8 +1466,8 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
 }
 
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                      int n, float* partial, double* gram, int* err, cudaStream_t s) {
-  if (dims[n] <= 128) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s);
+                      int n, float* partial, double* gram, int* err, cudaStream_t s, int max_ctas) {
+  if (dims[n] <= 128) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s, max_ctas);
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
   const size_t smem = gram_smem_bytes(geo);

@@ -31,9 +31,10 @@ cudaError_t build_tile_index(const int64_t* omega, int64_t k, int64_t tile_elems
 // into gram (I_n x I_n complex, interleaved doubles).
 size_t gram_partial_bytes(int nd, const int64_t* dims, int n);
 // Modes with I_n <= 128 run on the tensor cores; err is the device error word
-// a bounded wait sets when it gives up.
+// a bounded wait sets when it gives up. max_ctas > 0 caps the tensor-core
+// Gram's CTAs (one per SM), leaving SMs free for work on another stream.
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
-                      int n, float* partial, double* gram, int* err, cudaStream_t s);
+                      int n, float* partial, double* gram, int* err, cudaStream_t s, int max_ctas = 0);
 
 struct EigJob {
   const double* gram;  // n x n complex (interleaved doubles)
