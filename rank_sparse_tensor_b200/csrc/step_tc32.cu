@@ -92,6 +92,10 @@ struct MG32Args {
   // word ranks when the weights are updated), by cp.async (0: not staged)
   uint32_t xm_off, om_off;
   int64_t tile0;          // first 128-row tile of the launch (the grid's x counts from it)
+  // the factor itself (I x ur, complex pairs or reals) for the CUDA-core
+  // innermost-mode kernel: M = conj(U) (ukind 0) or U^T (ukind 1)
+  const float* Uf;
+  int ur, ukind;
   int* err;
 };
 
@@ -495,6 +499,7 @@ struct Mode32 {
   bool active = false;
   uint16_t* img_p = nullptr;  // projection image
   uint16_t* img_e = nullptr;  // expansion image
+  const float* U = nullptr;   // the factor (the caller's buffer, refreshed in place)
   int NTp = 0, nntp = 0, nkcp = 0, NTe = 0, nnte = 0, nkce = 0;
   int kpp = 64, kpe = 64;     // bf16 K values per chunk
 };
@@ -775,6 +780,215 @@ __global__ void __launch_bounds__(G32T) inner32_kernel(const MG32Args p, const i
   if (warp == 0) tmem_dealloc(dt, p.tmem_cols);
 }
 
+// The innermost mode on CUDA cores, for factors small enough that the
+// product is bound by the rows' bytes (4 K J fp32 FMAs per complex row: 340
+// for K = 17, J = 5, against 136 + 40 bytes): the staging ring of
+// inner32_kernel (whole 128-row tiles, rows and Omega's words arriving NB - 1
+// tiles ahead, one bulk store per tile), with y = x M computed per thread in
+// fp32 FMAs from the masked row in registers and M (K x J, from U) in shared
+// memory. M[k][j] = conj(U[k][j]) for a projection (ukind 0, K = I, J = r),
+// U[j][k] for an expansion (ukind 1, K = r, J = I).
+__host__ __device__ inline Inner32Layout ffma32_layout(int64_t K, int64_t J, int esz, bool masked, bool wupd,
+                                                       int nb) {
+  Inner32Layout L;
+  L.bimg = 0;  // M
+  L.xs = al128u((uint32_t)(K * J * esz));
+  L.xs_size = al128u((uint32_t)(G32T * K * esz));
+  L.os = L.xs + nb * L.xs_size;
+  L.os_size = al128u((uint32_t)(G32T * J * esz));
+  L.xm = L.os + nb * L.os_size;
+  L.xm_size = masked ? al128u(4u * (uint32_t)(G32T * K / 32 + 2)) : 0u;
+  L.om = L.xm + nb * L.xm_size;
+  const uint32_t nw = (uint32_t)(G32T * J / 32 + 2);
+  L.om_size = wupd ? al128u(4u * (nw + 1) + 8u * nw) : 0u;
+  L.bars = L.om + nb * L.om_size;
+  L.total = L.bars + 8 * (I32_NB_MAX + 2) + 16;
+  return L;
+}
+constexpr int F32_KMAX = 32;  // K entries of a row held in registers
+constexpr int F32_JMAX = 32;  // outputs of a row
+
+template <bool CPLX, bool WUPD>
+__global__ void __launch_bounds__(G32T) inner32_ffma_kernel(const MG32Args p, const int64_t ntiles, const int NB) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int ESZ = CPLX ? 8 : 4;
+  const Inner32Layout L = ffma32_layout(p.K, p.J, ESZ, p.bits != nullptr, WUPD, NB);
+  uint64_t* full = (uint64_t*)(smem + L.bars);  // [NB] a tile's rows (and mask words) landed
+  __shared__ int s_abort;
+  const int tid = threadIdx.x;
+  const bool masked = p.bits != nullptr;
+  const int K = (int)p.K, J = (int)p.J;
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < I32_NB_MAX; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  // M from U (I x ur, complex pairs or reals)
+  for (int e = tid; e < K * J; e += G32T) {
+    const int k = e / J, j = e - k * J;
+    const int64_t ui = p.ukind == 0 ? (int64_t)k * p.ur + j : (int64_t)j * p.ur + k;
+    if (CPLX) {
+      const float2 u = ((const float2*)p.Uf)[ui];
+      ((float2*)(smem + L.bimg))[e] = make_float2(u.x, p.ukind == 0 ? -u.y : u.y);
+    } else {
+      ((float*)(smem + L.bimg))[e] = p.Uf[2 * ui];
+    }
+  }
+  __syncthreads();
+  const int64_t nloc = ntiles > blockIdx.x ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  auto issue = [&](int64_t it, int bf) {
+    const int64_t a0 = ((int64_t)blockIdx.x + it * gridDim.x) * G32T;
+    if (masked) {
+      uint32_t* xm = (uint32_t*)(smem + L.xm + bf * L.xm_size);
+      const int64_t w0 = (a0 * p.K) >> 5, nw = (((a0 + G32T) * p.K - 1) >> 5) - w0 + 1;
+      for (int w = tid; w < nw; w += G32T) cpa4(xm + w, p.bits + w0 + w);
+    }
+    if (WUPD) {
+      uint32_t* om = (uint32_t*)(smem + L.om + bf * L.om_size);
+      const int64_t w0 = (a0 * p.J) >> 5, nw = (((a0 + G32T) * p.J - 1) >> 5) - w0 + 1;
+      int64_t* orank = (int64_t*)(om + ((nw + 1) & ~1ll));
+      for (int w = tid; w < nw; w += G32T) {
+        cpa4(om + w, p.wbits + w0 + w);
+        cpa8(orank + w, p.wrank + w0 + w);
+      }
+    }
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[bf])) : "memory");
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t xb = (uint32_t)(G32T * p.K * ESZ), wb = WUPD ? (uint32_t)(G32T * p.J * ESZ) : 0u;
+      mbar_expect_tx(&full[bf], xb + wb);
+      bulk_g2s(smem + L.xs + bf * L.xs_size, (const uint8_t*)p.X + a0 * p.K * ESZ, xb, &full[bf]);
+      if (WUPD) bulk_g2s(smem + L.os + bf * L.os_size, (const uint8_t*)p.W + a0 * p.J * ESZ, wb, &full[bf]);
+    }
+  };
+  auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (!mbar_wait(bar, parity, G32_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    __syncthreads();
+    return s_abort == 0;
+  };
+  int64_t issued = 0;
+  for (; issued < NB - 1 && issued < nloc; ++issued) issue(issued, (int)issued);
+  const float2* M2 = (const float2*)(smem + L.bimg);
+  const float* M1 = (const float*)(smem + L.bimg);
+  for (int64_t it = 0; it < nloc; ++it) {
+    const int bf = (int)(it % NB);
+    const int64_t a0 = ((int64_t)blockIdx.x + it * gridDim.x) * G32T;
+    if (it + NB - 1 < nloc) {
+      // the buffer of tile it + NB - 1 held tile it - 1: its store must have
+      // read it out
+      if (tid == 0) bulk_wait_read0();
+      issue(it + NB - 1, (int)((it + NB - 1) % NB));
+      issued = it + NB;
+    }
+    if (!wait_bar(&full[bf], (uint32_t)((it / NB) & 1))) break;
+    // this row's K values, Omega's entries zero
+    float2 v[F32_KMAX];
+    {
+      const float* xs = (const float*)(smem + L.xs + bf * L.xs_size);
+      const uint32_t* xm = (const uint32_t*)(smem + L.xm + bf * L.xm_size);
+      const int64_t w0 = (a0 * p.K) >> 5;
+#pragma unroll
+      for (int i = 0; i < F32_KMAX; ++i) {
+        if (i >= K) break;
+        float2 x = make_float2(0.f, 0.f);
+        const int64_t idx = (a0 + tid) * p.K + i;
+        const uint32_t word = masked ? xm[(idx >> 5) - w0] : 0u;
+        if (!((word >> (idx & 31)) & 1u)) {
+          if (CPLX)
+            x = ((const float2*)xs)[tid * K + i];
+          else
+            x.x = xs[tid * K + i];
+        }
+        v[i] = x;
+      }
+    }
+    // the row's outputs, then its rows of Y or W updated in place, in buffer bf
+    {
+      float* os = (float*)(smem + L.os + bf * L.os_size);
+      const uint32_t* omw = (const uint32_t*)(smem + L.om + bf * L.om_size);
+      const int64_t ow0 = (a0 * p.J) >> 5;
+      const int onw = (int)((((a0 + G32T) * p.J - 1) >> 5) - ow0 + 1);
+      const int64_t* omr = (const int64_t*)(omw + ((onw + 1) & ~1));
+      // eight outputs at a time; for the update their S~ values are loaded
+      // first (independent loads, in flight together)
+#pragma unroll 1
+      for (int j0 = 0; j0 < J; j0 += 8) {
+        float2 sv[8];
+        if (WUPD) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            sv[u] = make_float2(0.f, 0.f);
+            const int j = j0 + u;
+            if (j >= J) continue;
+            const int64_t o = (a0 + tid) * p.J + j;
+            const uint32_t word = omw[(o >> 5) - ow0];
+            const uint32_t bit = (uint32_t)(o & 31);
+            if ((word >> bit) & 1u) {
+              const int64_t e = omr[(o >> 5) - ow0] + __popc(word & ((1u << bit) - 1u));
+              if (CPLX)
+                sv[u] = __ldg((const float2*)p.S + e);
+              else
+                sv[u].x = __ldg(p.S + e);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          if (j >= J) break;
+          float dr = 0.f, di = 0.f;
+#pragma unroll
+          for (int i = 0; i < F32_KMAX; ++i) {
+            if (i >= K) break;
+            if (CPLX) {
+              const float2 m = M2[i * J + j];
+              dr = __fmaf_rn(v[i].x, m.x, __fmaf_rn(-v[i].y, m.y, dr));
+              di = __fmaf_rn(v[i].x, m.y, __fmaf_rn(v[i].y, m.x, di));
+            } else {
+              dr = __fmaf_rn(v[i].x, M1[i * J + j], dr);
+            }
+          }
+          const int64_t so = (int64_t)tid * p.J + j;
+          if (!WUPD) {
+            if (CPLX)
+              ((float2*)os)[so] = make_float2(dr, di);
+            else
+              os[so] = dr;
+          } else {
+            dr += sv[u].x;
+            di += sv[u].y;
+            if (CPLX) {
+              const float2 w = ((float2*)os)[so];
+              ((float2*)os)[so] = make_float2(__fmaf_rn(-p.lr, dr, w.x * p.decay), __fmaf_rn(-p.lr, di, w.y * p.decay));
+            } else {
+              os[so] = __fmaf_rn(-p.lr, dr, os[so] * p.decay);
+            }
+          }
+        }
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        uint8_t* dst = WUPD ? (uint8_t*)p.W : (uint8_t*)p.Y;
+        bulk_s2g(dst + a0 * p.J * ESZ, os, (uint32_t)(G32T * p.J * ESZ));
+        bulk_commit();
+      }
+    }
+  }
+  if (tid == 0) {
+    bulk_wait_read0();  // no store still reads this CTA's shared memory
+    if (s_abort) {
+      // bounded waits for copies still in flight
+      for (int64_t i = issued > NB ? issued - NB : 0; i < issued; ++i)
+        mbar_wait(&full[i % NB], (uint32_t)((i / NB) & 1), G32_WAIT_NS / 4);
+    }
+  }
+  __syncthreads();
+}
+
 size_t g32_smem(int NT, int nstage, int kp) {
   return (size_t)nstage * (3 * (size_t)(kp / 8) * G32_LBO + 3 * (size_t)NT * kp * 2) + 64;
 }
@@ -806,7 +1020,41 @@ cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
   // the innermost mode with one K chunk and one column block: the persistent
   // kernel over the whole 128-row tiles, this kernel for a ragged last tile
   const void* outp = WUPD ? (const void*)a.W : (const void*)a.Y;
-  if (a.B == 1 && a.nkc == 1 && nnt == 1 && a.rows >= G32T && ((uintptr_t)a.X % 16) == 0 &&
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  // a small factor (K, J <= 32, K J <= 512): CUDA cores over whole tiles
+  // (at most 4 K J fp32 FMAs per complex row, bound by the rows' bytes), this
+  // kernel for a ragged last tile
+  bool tiles_done = false;
+  if (a.B == 1 && a.Uf && a.K <= F32_KMAX && a.J <= F32_JMAX && a.K * a.J <= 512 && a.rows >= G32T &&
+      ((uintptr_t)a.X % 16) == 0 && ((uintptr_t)outp % 16) == 0) {
+    int nb = 0, cps = 0;
+    Inner32Layout L{};
+    for (int b = 2; b <= I32_NB_MAX; ++b) {
+      const Inner32Layout Lb = ffma32_layout(a.K, a.J, (int)esz, a.bits != nullptr, WUPD, b);
+      if (Lb.total > G32_SMEM_LIMIT) break;
+      const int c = std::min(8, (int)(232448 / (Lb.total + 1024)));
+      if (c >= cps) {
+        nb = b;
+        cps = c;
+        L = Lb;
+      }
+    }
+    if (nb > 0) {
+      const int64_t ntiles = a.rows / G32T;
+      const int64_t grid = std::min<int64_t>(ntiles, (int64_t)nsm * cps);
+      cudaError_t e = cudaFuncSetAttribute(inner32_ffma_kernel<CPLX, WUPD>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+      if (e != cudaSuccess) return e;
+      inner32_ffma_kernel<CPLX, WUPD><<<(unsigned)grid, G32T, L.total, s>>>(a, ntiles, nb);
+      e = cudaGetLastError();
+      if (e != cudaSuccess || a.rows % G32T == 0) return e;
+      a.tile0 = ntiles;
+      tiles_done = true;
+    }
+  }
+  if (!tiles_done && a.B == 1 && a.nkc == 1 && nnt == 1 && a.rows >= G32T && ((uintptr_t)a.X % 16) == 0 &&
       ((uintptr_t)outp % 16) == 0) {
     // the most CTAs per SM (a tile's latency chain bounds each CTA), then the
     // deepest ring those leave room for
@@ -823,9 +1071,6 @@ cudaError_t launch32(MG32Args a, int nnt, cudaStream_t s) {
       }
     }
     if (nb > 0) {
-      int dev = 0, nsm = 148;
-      cudaGetDevice(&dev);
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
       const int64_t ntiles = a.rows / G32T;
       const int64_t grid = std::min<int64_t>(ntiles, (int64_t)nsm * cps);
       cudaError_t e = cudaFuncSetAttribute(inner32_kernel<CPLX, WUPD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -977,6 +1222,7 @@ cudaError_t tc32_rebuild(Tc32Plan& p, const int64_t* omega, int64_t k, const flo
   word_rank_kernel<<<blocks(g->nwords), 256, 0, s>>>(omega, k, g->nwords, g->wrank);
   for (auto& m : g->modes) {
     if (!m.active) continue;
+    m.U = U[m.n];
     const float2* Un = (const float2*)U[m.n];
     int Np = m.nntp * m.NTp, Kp = m.nkcp * m.kpp;
     embed32_kernel<<<blocks((int64_t)Np * Kp), 256, 0, s>>>(Un, (int)m.I, (int)m.r, 0, g->cplx ? 1 : 0, Np, Kp,
@@ -1027,6 +1273,9 @@ cudaError_t tc32_project(Tc32Plan& p, const void* grad, const uint32_t* bits, in
     a.kp = m.kpp;
     a.nstage = m.nkcp > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTp);
+    a.Uf = m.U;
+    a.ur = (int)m.r;
+    a.ukind = 0;
     a.err = d_err;
     if (hook) hook(hook_ctx, 0, "mode_gemm32", s);
     cudaError_t e = launch_mode32(g->cplx, false, a, m.nntp, s);
@@ -1074,6 +1323,9 @@ cudaError_t tc32_expand_update(Tc32Plan& p, void* w, const uint32_t* bits, float
     a.kp = m.kpe;
     a.nstage = m.nkce > 1 ? 2 : 1;
     a.tmem_cols = (uint32_t)pow2_cols32(m.NTe);
+    a.Uf = m.U;
+    a.ur = (int)m.r;
+    a.ukind = 1;
     a.W = (float*)w;
     a.S = g->S;
     a.wrank = g->wrank;
