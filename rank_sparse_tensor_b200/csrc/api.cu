@@ -59,10 +59,10 @@ struct tgd_ctx {
   bool eig_warm = false;             // eig_v holds them (every projected mode <= 128)
   EigJob* jobs_dev = nullptr;
   std::vector<EigJob> jobs;
-  // the refresh runs each mode's eigensolve on a side stream beside the next
-  // mode's Gram (fork and join by events)
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  // the refresh runs each mode's eigensolve on one of two side streams beside
+  // the next modes' Grams (fork and join by events)
+  cudaStream_t side[2] = {};
+  cudaEvent_t ev_fork = nullptr, ev_join[2] = {};
   int num_sms = 0;
   // generic step scratch
   float* P[TGD_MAX_NDIM] = {};  // projection coefficients (r x I)
@@ -195,10 +195,13 @@ void free_all(tgd_ctx* h) {
   tc_release(h->tc);
   tc32_release(h->tc32);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-  if (h->ev_join) cudaEventDestroy(h->ev_join);
-  if (h->side) cudaStreamDestroy(h->side);
-  h->ev_fork = h->ev_join = nullptr;
-  h->side = nullptr;
+  h->ev_fork = nullptr;
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_join[i]) cudaEventDestroy(h->ev_join[i]);
+    if (h->side[i]) cudaStreamDestroy(h->side[i]);
+    h->ev_join[i] = nullptr;
+    h->side[i] = nullptr;
+  }
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   h->ev_pool.clear();
   for (void* p : h->allocs) cudaFree(p);
@@ -430,17 +433,19 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
   }
   TGD_CUDA(h, build_mask_bits(h->omega, h->k, h->N, h->bits, s));
   h->jobs.clear();
-  // Each mode's eigensolve (one CTA, latency-bound) starts on the side stream
-  // as soon as its Gram is done and runs beside the next mode's Gram, which
-  // leaves one SM free for it; the main stream waits for the last one. Not
-  // for a handle given an SM budget: it shares the GPU with other streams.
-  const bool overlap = h->opt.basis != 1 && h->side && h->num_sms > 1 && h->opt.sm_budget == 0;
+  // Each mode's eigensolve (one CTA, latency-bound) starts on a side stream
+  // (the two in turn) as soon as its Gram is done and runs beside the next
+  // modes' Grams, which leave two SMs free for them; the main stream waits
+  // for both. Not for a handle given an SM budget: it shares the GPU with
+  // other streams.
+  const bool overlap = h->opt.basis != 1 && h->side[1] && h->num_sms > 2 && h->opt.sm_budget == 0;
+  int nside = 0;
   for (int n = 0; n < h->d; ++n) {
     if (!mode_active(h, n)) continue;
     {
       TIMED(h, s, "mode_gram");
       TGD_CUDA(h, mode_gram(g, h->gdt, h->bits, h->d, h->I, n, h->gram_part, h->gram[n], h->d_err, s,
-                            overlap ? h->num_sms - 1 : 0));
+                            overlap ? h->num_sms - 2 : 0));
     }
     EigJob j;
     j.gram = h->gram[n];
@@ -453,15 +458,19 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     j.r = (int)h->r[n];
     h->jobs.push_back(j);
     if (overlap) {
+      cudaStream_t ss = h->side[nside & 1];
+      ++nside;
       TGD_CUDA(h, cudaEventRecord(h->ev_fork, s));
-      TGD_CUDA(h, cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-      TIMED(h, h->side, "eigh");
-      TGD_CUDA(h, batched_eigh(&h->jobs.back(), 1, h->jobs_dev + (h->jobs.size() - 1), h->side));
+      TGD_CUDA(h, cudaStreamWaitEvent(ss, h->ev_fork, 0));
+      TIMED(h, ss, "eigh");
+      TGD_CUDA(h, batched_eigh(&h->jobs.back(), 1, h->jobs_dev + (h->jobs.size() - 1), ss));
     }
   }
   if (overlap) {
-    TGD_CUDA(h, cudaEventRecord(h->ev_join, h->side));
-    TGD_CUDA(h, cudaStreamWaitEvent(s, h->ev_join, 0));
+    for (int i = 0; i < 2; ++i) {
+      TGD_CUDA(h, cudaEventRecord(h->ev_join[i], h->side[i]));
+      TGD_CUDA(h, cudaStreamWaitEvent(s, h->ev_join[i], 0));
+    }
     h->eig_warm = eig_keeps_vectors(h);
   } else if (h->opt.basis == 1) {
     TIMED(h, s, "dct_select");
@@ -780,20 +789,24 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
     return fail(nullptr, TGD_ERR_OOM, "device allocation failed");
   }
   {
-    // the refresh's side stream (see do_refresh); without it the refresh
+    // the refresh's side streams (see do_refresh); without them the refresh
     // runs on the caller's stream alone
     bool have = false;
     for (int n = 0; n < ndim; ++n) have |= h->gram[n] != nullptr;
-    const bool made = have &&
-                      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) == cudaSuccess &&
-                      cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess &&
-                      cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
-                      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
+    bool made = have && cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) == cudaSuccess &&
+                cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2; ++i)
+      made = made && cudaStreamCreateWithFlags(&h->side[i], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h->ev_join[i], cudaEventDisableTiming) == cudaSuccess;
     if (!made) {
       if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-      if (h->side) cudaStreamDestroy(h->side);
-      h->ev_fork = h->ev_join = nullptr;
-      h->side = nullptr;
+      h->ev_fork = nullptr;
+      for (int i = 0; i < 2; ++i) {
+        if (h->ev_join[i]) cudaEventDestroy(h->ev_join[i]);
+        if (h->side[i]) cudaStreamDestroy(h->side[i]);
+        h->ev_join[i] = nullptr;
+        h->side[i] = nullptr;
+      }
       cudaGetLastError();
     }
   }

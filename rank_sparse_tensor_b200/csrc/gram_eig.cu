@@ -1361,6 +1361,8 @@ size_t gram_partial_bytes(int nd, const int64_t* dims, int n) {
   GramGeom g = gram_geom(nd, dims, n);
   size_t b = sizeof(float2) * (size_t)g.nsplit * g.I * g.I;
   if (g.I <= 128) b = std::max(b, sizeof(float2) * (size_t)TG_MAX_SPLITS * g.I * g.I);
+  // the small-mode Gram: at most 8 CTAs per SM of up to 256 SMs
+  if (g.I <= 32) b = std::max(b, sizeof(float2) * (size_t)(8 * 256) * g.I * g.I);
   return b;
 }
 
@@ -1402,6 +1404,276 @@ static cudaError_t rows_tensor_map(CUtensorMap* map, const void* g, int es, cons
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+
+// ---------------------------------------------- small-mode Gram, CUDA cores
+// Modes with I_n <= 32 whose slab (I_n x B, contiguous) is small: the Gram
+// needs 4 I_n fp32 FMAs per complex element at most (I_n <= 32), which the
+// CUDA cores sustain at the rate G streams in, while a tensor-core Gram of
+// such a mode is bound by its MMA count (a 128-row tile mostly padding).
+// A CTA takes a range of chunks of whole slabs: each chunk arrives by one
+// bulk copy (plain loads for a tail or an unaligned tensor) with Omega's
+// mask words beside it (cp.async), Omega's entries are zeroed in shared
+// memory, and thread (tile pair, column lane) accumulates the 4 x 4 block
+// (ti <= tj) of sum_c x_i(c) conj(x_j(c)) over its columns c = lane, lane +
+// 16, ... of the chunk. At the end the 16 column lanes of a pair are summed
+// by shuffles and the CTA writes its whole I_n x I_n partial (the lower
+// blocks as conjugates), which the fixed-order fp64 reduction then sums.
+constexpr int SG_CL = 16;      // column lanes per tile pair
+constexpr int SG_MAXI = 32;    // I_n at most
+constexpr int SG_MAXT = 36 * SG_CL;  // threads: tile pairs of I_n = 32 (8 x 9 / 2) x lanes
+constexpr int SG_CHUNK = 32768;      // bytes of a chunk, at most (two in flight)
+
+struct SmallGramArgs {
+  const void* g;
+  const uint32_t* bits;
+  int64_t A, B;        // slabs, columns per slab row
+  int I, IP, ntp;      // rows, 4-row tiles, tile pairs
+  int spc;             // slabs per chunk
+  int64_t nchunk, cpc; // chunks, chunks per CTA
+  int bulk;            // whole chunks by bulk copy (aligned tensor, chunk bytes % 16 == 0)
+  float2* partial;     // [gridDim.x][I][I]
+  int* err;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(SG_MAXT) gram_small_kernel(const SmallGramArgs p) {
+  constexpr int ES = Dt<DT>::bytes;
+  extern __shared__ __align__(128) uint8_t sg_smem[];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int64_t IB = (int64_t)p.I * p.B;
+  const int64_t chunk_elems = (int64_t)p.spc * IB;
+  const size_t xbytes = (size_t)((chunk_elems * ES + 127) / 128) * 128;
+  const size_t mbytes = (size_t)((4 * (chunk_elems / 32 + 2) + 127) / 128) * 128;
+  // two buffers: the chunk (raw) and its mask words
+  auto xbuf = [&](int b) { return sg_smem + (size_t)b * (xbytes + mbytes); };
+  auto mwb = [&](int b) { return (uint32_t*)(sg_smem + (size_t)b * (xbytes + mbytes) + xbytes); };
+  // this thread's tile pair (ti <= tj) and column lane
+  const int pi = tid / SG_CL, lc = tid - pi * SG_CL;
+  int ti = 0, rem = pi;
+  while (rem >= p.IP - ti) {
+    rem -= p.IP - ti;
+    ++ti;
+  }
+  const int tj = ti + rem;
+  const bool active = pi < p.ntp;
+  float2 acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = make_float2(0.f, 0.f);
+  if (tid == 0) {
+    s_abort = 0;
+    ptx::mbar_init(&bar[0], 1);
+    ptx::mbar_init(&bar[1], 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t c_begin = (int64_t)blockIdx.x * p.cpc;
+  const int64_t c_end = c_begin + p.cpc < p.nchunk ? c_begin + p.cpc : p.nchunk;
+  auto geom = [&](int64_t ch, int& nsl, int64_t& e0, int64_t& ne, int64_t& w0, int64_t& nw) {
+    const int64_t a0 = ch * p.spc;
+    nsl = (int)(p.A - a0 < p.spc ? p.A - a0 : p.spc);
+    e0 = a0 * IB;
+    ne = (int64_t)nsl * IB;
+    w0 = e0 >> 5;
+    nw = p.bits ? ((e0 + ne - 1) >> 5) - w0 + 1 : 0;
+  };
+  // chunk ch into buffer b: mask words by cp.async (their arrivals counted
+  // before the copy's), then the chunk by one bulk copy, or by plain loads
+  // (a tail chunk or an unaligned tensor)
+  auto issue = [&](int64_t ch, int b) {
+    int nsl;
+    int64_t e0, ne, w0, nw;
+    geom(ch, nsl, e0, ne, w0, nw);
+    const bool whole = p.bulk && nsl == p.spc;
+    uint32_t* mw = mwb(b);
+    uint8_t* xb = xbuf(b);
+    for (int64_t w = tid; w < nw; w += nthr) cp_async_elem<4>(mw + w, p.bits + w0 + w);
+    if (!whole) {
+      for (int64_t e = tid; e < ne; e += nthr) {
+        if constexpr (ES == 8)
+          ((uint2*)xb)[e] = __ldg((const uint2*)p.g + e0 + e);
+        else if constexpr (ES == 4)
+          ((uint32_t*)xb)[e] = __ldg((const uint32_t*)p.g + e0 + e);
+        else
+          ((uint16_t*)xb)[e] = __ldg((const unsigned short*)p.g + e0 + e);
+      }
+    }
+    cp_async_arrive(&bar[b]);
+    __syncthreads();
+    if (tid == 0) {
+      if (whole) {
+        ptx::mbar_expect_tx(&bar[b], (uint32_t)(ne * ES));
+        ptx::bulk_g2s(xb, (const uint8_t*)p.g + e0 * ES, (uint32_t)(ne * ES), &bar[b]);
+      } else {
+        tg_arrive(&bar[b]);
+      }
+    }
+  };
+  uint32_t phbits = 0;  // bit b: the parity buffer b's next phase completes with
+  int64_t issued = 0;
+  if (c_begin < c_end) {
+    issue(c_begin, 0);
+    issued = 1;
+  }
+  for (int64_t ch = c_begin; ch < c_end; ++ch) {
+    const int b = (int)((ch - c_begin) & 1);
+    // the next chunk goes into the other buffer (read out by the barrier
+    // that ended the previous iteration)
+    if (ch + 1 < c_end) {
+      issue(ch + 1, b ^ 1);
+      ++issued;
+    }
+    if (tid == 0 && !ptx::mbar_wait(&bar[b], (phbits >> b) & 1u, TG_WAIT_NS)) {
+      atomicOr(p.err, DEV_ERR_TIMEOUT);
+      s_abort = 1;
+    }
+    phbits ^= 1u << b;
+    __syncthreads();
+    if (s_abort) break;
+    int nsl;
+    int64_t e0, ne, w0, nw;
+    geom(ch, nsl, e0, ne, w0, nw);
+    uint8_t* xb = xbuf(b);
+    const uint32_t* mw = mwb(b);
+    // Omega's entries of the chunk -> zero (the residual)
+    for (int64_t w = tid; w < nw; w += nthr) {
+      uint32_t word = mw[w];
+      const int64_t base = (w0 + w) * 32 - e0;
+      while (word) {
+        const int bt = __ffs(word) - 1;
+        word &= word - 1;
+        const int64_t e = base + bt;
+        if (e >= 0 && e < ne) {
+          if constexpr (ES == 8)
+            ((uint2*)xb)[e] = make_uint2(0u, 0u);
+          else if constexpr (ES == 4)
+            ((uint32_t*)xb)[e] = 0u;
+          else
+            ((uint16_t*)xb)[e] = 0;
+        }
+      }
+    }
+    __syncthreads();
+    if (active) {
+      const int64_t ncol = (int64_t)nsl * p.B;
+      int64_t al = lc / p.B, bb = lc - al * p.B;
+      const int64_t dA = SG_CL / p.B, dB = SG_CL - dA * p.B;  // a step of SG_CL columns
+      for (int64_t c = lc; c < ncol; c += SG_CL) {
+        const int64_t base = al * IB + bb;
+        float2 xa[4], xc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * ti + u;
+          xa[u] = i < p.I ? load_rw<DT>(xb, base + (int64_t)i * p.B) : make_float2(0.f, 0.f);
+        }
+        if (tj == ti) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) xc[v] = xa[v];
+        } else {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int jj = 4 * tj + v;
+            xc[v] = jj < p.I ? load_rw<DT>(xb, base + (int64_t)jj * p.B) : make_float2(0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            // xa * conj(xc)
+            acc[u][v].x = __fmaf_rn(xa[u].x, xc[v].x, acc[u][v].x);
+            if constexpr (Dt<DT>::cplx) {
+              acc[u][v].x = __fmaf_rn(xa[u].y, xc[v].y, acc[u][v].x);
+              acc[u][v].y = __fmaf_rn(xa[u].y, xc[v].x, __fmaf_rn(-xa[u].x, xc[v].y, acc[u][v].y));
+            }
+          }
+        bb += dB;
+        al += dA;
+        if (bb >= p.B) {
+          bb -= p.B;
+          ++al;
+        }
+      }
+    }
+    __syncthreads();  // this buffer is read before it is refilled
+  }
+  // the 16 column lanes of each pair (aligned lanes of one warp), summed
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+#pragma unroll
+      for (int o = SG_CL / 2; o; o >>= 1) {
+        acc[u][v].x += __shfl_xor_sync(0xffffffffu, acc[u][v].x, o);
+        acc[u][v].y += __shfl_xor_sync(0xffffffffu, acc[u][v].y, o);
+      }
+  if (active && lc == 0) {
+    float2* out = p.partial + (int64_t)blockIdx.x * p.I * p.I;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int i = 4 * ti + u, jj = 4 * tj + v;
+        if (i < p.I && jj < p.I) {
+          out[(int64_t)i * p.I + jj] = acc[u][v];
+          if (ti != tj) out[(int64_t)jj * p.I + i] = make_float2(acc[u][v].x, -acc[u][v].y);
+        }
+      }
+  }
+  if (tid == 0 && s_abort) {
+    // bounded waits for the copies still in flight (both buffers' last phases)
+    for (int b = 0; b < 2; ++b)
+      if ((int64_t)b < issued) ptx::mbar_wait(&bar[b], (phbits >> b) & 1u, TG_WAIT_NS / 4);
+  }
+}
+
+// The small-mode Gram's plan, or false when the mode does not fit it.
+bool small_gram_plan(int nd, const int64_t* dims, int n, int dt, bool aligned16, int max_ctas, SmallGramArgs& a,
+                     size_t& smem, int& threads) {
+  const int es = dt == TGD_C64 ? 8 : (dt == TGD_R16 ? 2 : 4);
+  int64_t A = 1, B = 1;
+  for (int q = 0; q < n; ++q) A *= dims[q];
+  for (int q = n + 1; q < nd; ++q) B *= dims[q];
+  const int I = (int)dims[n];
+  if (I > SG_MAXI || I < 1) return false;
+  const int64_t slab = (int64_t)I * B * es;
+  if (slab > SG_CHUNK) return false;
+  // slabs per chunk: as many as fit, a multiple of what keeps chunks 16-byte sized
+  int step = 1;
+  while ((slab * step) % 16 != 0 && step < 16) step *= 2;
+  int spc = (int)(SG_CHUNK / slab) / step * step;
+  if (spc < step) spc = step;
+  if (spc > A) spc = (int)A;
+  a.A = A;
+  a.B = B;
+  a.I = I;
+  a.IP = (I + 3) / 4;
+  a.ntp = a.IP * (a.IP + 1) / 2;
+  a.spc = spc;
+  a.nchunk = ceil_div(A, (int64_t)spc);
+  a.bulk = aligned16 && (slab * spc) % 16 == 0;
+  threads = a.ntp * SG_CL;
+  const int64_t chunk_elems = (int64_t)spc * I * B;
+  smem = 2 * ((size_t)((chunk_elems * es + 127) / 128) * 128 + (size_t)((4 * (chunk_elems / 32 + 2) + 127) / 128) * 128);
+  // CTAs: as many as the SMs hold (threads and shared memory), each at least
+  // two chunks
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (max_ctas > 0 && max_ctas < nsm) nsm = max_ctas;
+  // resident CTAs per SM: threads, shared memory and registers (up to 96 a thread)
+  int per = std::min(2048 / threads, (int)(220 * 1024 / (smem + 1024)));
+  per = std::min(per, 65536 / (threads * 96));
+  per = std::max(1, std::min(per, 8));
+  const int64_t want = std::max<int64_t>(1, std::min<int64_t>((int64_t)nsm * per, ceil_div(a.nchunk, (int64_t)2)));
+  a.cpc = ceil_div(a.nchunk, want);
+  return true;
+}
+
+int small_gram_ctas(const SmallGramArgs& a) { return (int)ceil_div(a.nchunk, a.cpc); }
 
 // Tensor-core Gram for I_n <= 64 (see gram_tc_kernel); the split partials are
 // summed by the same fixed-order fp64 reduction.
@@ -1467,6 +1739,50 @@ cudaError_t mode_gram_tc(const void* g, int dt, const uint32_t* bits, int nd, co
 
 cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const int64_t* dims,
                       int n, float* partial, double* gram, int* err, cudaStream_t s, int max_ctas) {
+  {
+    SmallGramArgs a{};
+    size_t smem = 0;
+    int threads = 0;
+    if (small_gram_plan(nd, dims, n, dt, ((uintptr_t)g & 15) == 0, max_ctas, a, smem, threads)) {
+      a.g = g;
+      a.bits = bits;
+      a.partial = (float2*)partial;
+      a.err = err;
+      const int grid = small_gram_ctas(a);
+      auto launch = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, threads, smem, s>>>(a);
+        return cudaGetLastError();
+      };
+      cudaError_t e = cudaErrorInvalidValue;
+      switch (dt) {
+        case TGD_R32:
+          e = launch(gram_small_kernel<TGD_R32>);
+          break;
+        case TGD_C64:
+          e = launch(gram_small_kernel<TGD_C64>);
+          break;
+        case TGD_C32H:
+          e = launch(gram_small_kernel<TGD_C32H>);
+          break;
+        case TGD_R16:
+          e = launch(gram_small_kernel<TGD_R16>);
+          break;
+        default:
+          break;
+      }
+      if (e != cudaSuccess) return e;
+      GramGeom geo{};
+      geo.I = a.I;
+      geo.TI = 64;  // every cell of the partials is written
+      geo.nsplit = grid;
+      const int64_t cells = (int64_t)a.I * a.I;
+      gram_reduce_kernel<<<(int)ceil_div(cells, RC), RC * RS, 0, s>>>((const float2*)partial, geo,
+                                                                       (double2*)gram);
+      return cudaGetLastError();
+    }
+  }
   if (dims[n] <= 128) return mode_gram_tc(g, dt, bits, nd, dims, n, partial, gram, err, s, max_ctas);
   GramGeom geo = gram_geom(nd, dims, n);
   dim3 grid(geo.npairs, geo.nsplit);
