@@ -80,6 +80,10 @@ struct tgd_ctx {
   // host-buffer step
   void* stage_g = nullptr;
   void* stage_w = nullptr;
+  // the tensor-core path's host-buffer step moves the weights in chunks of
+  // tiles on two copy streams (in, out), overlapped with the reconstruction
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t hev[2 * 8 + 2] = {};
   std::vector<void*> allocs;
   size_t bytes = 0;
   std::string last_error;
@@ -196,6 +200,13 @@ void free_all(tgd_ctx* h) {
   tc32_release(h->tc32);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   h->ev_fork = nullptr;
+  for (cudaEvent_t& e : h->hev) {
+    if (e) cudaEventDestroy(e);
+    e = nullptr;
+  }
+  if (h->cin) cudaStreamDestroy(h->cin);
+  if (h->cout) cudaStreamDestroy(h->cout);
+  h->cin = h->cout = nullptr;
   for (int i = 0; i < 2; ++i) {
     if (h->ev_join[i]) cudaEventDestroy(h->ev_join[i]);
     if (h->side[i]) cudaStreamDestroy(h->side[i]);
@@ -901,6 +912,62 @@ tgd_status tgd_step_end(tgd_handle h, void* weight, void* stream) {
   return step_end(h, weight, (cudaStream_t)stream);
 }
 
+// The host-buffer step of the tensor-core path (complex fp16): G in on the
+// caller's stream; W in, in HC chunks of whole tiles, on the input copy
+// stream behind G; the projection, the core AdamW and the expansions on the
+// caller's stream while W arrives; then per chunk the reconstruction stream
+// over its tiles once they have landed, and the chunk back to the host on the
+// output copy stream while the next chunks are still coming in (the link
+// carries both directions at once).
+constexpr int HC = 8;
+tgd_status step_host_tc(tgd_ctx* h, const void* grad_host, void* weight_host, cudaStream_t s) {
+  const size_t gb = (size_t)h->N * dt_bytes(h->gdt), ws = dt_bytes(h->wdt);
+  TGD_CUDA(h, cudaMemcpyAsync(h->stage_g, grad_host, gb, cudaMemcpyHostToDevice, s));
+  cudaEvent_t* ev_w = h->hev;           // [HC] chunk i of W landed
+  cudaEvent_t* ev_r = h->hev + HC;      // [HC] chunk i of W updated
+  cudaEvent_t ev_g = h->hev[2 * HC], ev_out = h->hev[2 * HC + 1];
+  TGD_CUDA(h, cudaEventRecord(ev_g, s));
+  TGD_CUDA(h, cudaStreamWaitEvent(h->cin, ev_g, 0));
+  const int64_t T = tc_tiles(h->tc), te = tc_tile_elems(h->tc);
+  const int C = (int)std::min<int64_t>(HC, T);
+  auto tile_of = [&](int i) { return T * i / C; };
+  auto elem_of = [&](int64_t t) { return std::min<int64_t>(t * te, h->N); };
+  for (int i = 0; i < C; ++i) {
+    const int64_t e0 = elem_of(tile_of(i)), e1 = elem_of(tile_of(i + 1));
+    TGD_CUDA(h, cudaMemcpyAsync((uint8_t*)h->stage_w + e0 * ws, (const uint8_t*)weight_host + e0 * ws,
+                                (size_t)(e1 - e0) * ws, cudaMemcpyHostToDevice, h->cin));
+    TGD_CUDA(h, cudaEventRecord(ev_w[i], h->cin));
+  }
+  if (h->opt.auto_refresh && h->T > 0 && h->t % h->T == 0) {
+    tgd_status st = do_refresh(h, h->stage_g, s);
+    if (st != TGD_OK) return st;
+  }
+  if (!h->has_subspace) return fail(h, TGD_ERR_STATE, "no refresh has run: call tgd_refresh first");
+  tgd_status st = step_begin(h, h->stage_g, s);
+  if (st != TGD_OK) return st;
+  AdamConst acore = adam_const(h, 1.0);
+  const float decay = (float)(1.0 - (double)h->lr * (double)h->wd);
+  cudaError_t e = tc_step_finish(h->tc, h->stage_w, h->core_m, h->core_v, acore, decay, h->lr, h->d_err, s,
+                                 timer_hook, h, false);
+  if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core reconstruction");
+  for (int i = 0; i < C; ++i) {
+    const int64_t t0 = tile_of(i), t1 = tile_of(i + 1);
+    const int64_t e0 = elem_of(t0), e1 = elem_of(t1);
+    TGD_CUDA(h, cudaStreamWaitEvent(s, ev_w[i], 0));
+    e = tc_recon(h->tc, h->stage_w, t0, t1 - t0, decay, h->lr, h->d_err, s, timer_hook, h);
+    if (e != cudaSuccess) return cuda_fail(h, e, "tensor-core reconstruction");
+    TGD_CUDA(h, cudaEventRecord(ev_r[i], s));
+    TGD_CUDA(h, cudaStreamWaitEvent(h->cout, ev_r[i], 0));
+    TGD_CUDA(h, cudaMemcpyAsync((uint8_t*)weight_host + e0 * ws, (const uint8_t*)h->stage_w + e0 * ws,
+                                (size_t)(e1 - e0) * ws, cudaMemcpyDeviceToHost, h->cout));
+  }
+  TGD_CUDA(h, cudaEventRecord(ev_out, h->cout));
+  TGD_CUDA(h, cudaStreamWaitEvent(s, ev_out, 0));
+  h->pending = false;
+  h->t += 1;
+  return check_device_error(h, s, true);
+}
+
 tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host, void* stream) {
   if (!h) return fail(nullptr, TGD_ERR_INVALID_ARG, "NULL handle");
   if (!grad_host || !weight_host) return fail(h, TGD_ERR_INVALID_ARG, "grad or weight is NULL");
@@ -908,6 +975,25 @@ tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host,
   size_t gb = (size_t)h->N * dt_bytes(h->gdt), wb = (size_t)h->N * dt_bytes(h->wdt);
   if (!h->stage_g && !dalloc(h, &h->stage_g, gb)) return fail(h, TGD_ERR_OOM, "staging allocation failed");
   if (!h->stage_w && !dalloc(h, &h->stage_w, wb)) return fail(h, TGD_ERR_OOM, "staging allocation failed");
+  if (h->pending) return fail(h, TGD_ERR_STATE, "tgd_step_begin is waiting for tgd_step_end");
+  if (h->path == TGD_PATH_TCGEN05 && !h->use_tc32 && h->opt.order == 0 && h->mode0_total == 0) {
+    if (!h->cin) {
+      bool made = cudaStreamCreateWithFlags(&h->cin, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&h->cout, cudaStreamNonBlocking) == cudaSuccess;
+      for (cudaEvent_t& ev : h->hev) made = made && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+      if (!made) {
+        for (cudaEvent_t& ev : h->hev) {
+          if (ev) cudaEventDestroy(ev);
+          ev = nullptr;
+        }
+        if (h->cin) cudaStreamDestroy(h->cin);
+        if (h->cout) cudaStreamDestroy(h->cout);
+        h->cin = h->cout = nullptr;
+        cudaGetLastError();
+      }
+    }
+    if (h->cin) return step_host_tc(h, grad_host, weight_host, s);
+  }
   TGD_CUDA(h, cudaMemcpyAsync(h->stage_g, grad_host, gb, cudaMemcpyHostToDevice, s));
   TGD_CUDA(h, cudaMemcpyAsync(h->stage_w, weight_host, wb, cudaMemcpyHostToDevice, s));
   tgd_status st = tgd_step(h, h->stage_g, h->stage_w, stream);

@@ -809,6 +809,7 @@ struct R3Args {
   void* W;
   int w_c64;
   int64_t N, n_slabs, n_tiles, tile_elems;
+  int64_t tile0, tiles;  // this launch: tiles [tile0, tile0 + tiles)
   int Ia, Ib, ra, rb, spb, log2Ia;
   int K1, N1, K2, N2;
   uint32_t d1_col[2], d2_col[2], a1_col, a2_col[2];  // TMEM columns
@@ -861,8 +862,8 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
   __shared__ int s_abort_storage;
   volatile int* s_abort = &s_abort_storage;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n_it =
-      p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t n_it = p.tiles > (int64_t)blockIdx.x ? (p.tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t tb = p.tile0 + blockIdx.x;  // this CTA's first tile
   const int64_t G = gridDim.x;
   const int ns = p.nstage;
   auto wst = [&](int s) { return smem + p.off_w + (uint32_t)s * p.w_tile_bytes; };
@@ -929,7 +930,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       bulk_g2s(B2, p.B2img, b2b, opnd);
       auto load = [&](int64_t it) {
         const int s = (int)(it % ns);
-        const int64_t t = blockIdx.x + it * G;
+        const int64_t t = tb + it * G;
         const uint32_t nw = tile_wbytes(t), ny = tile_ybytes(t);
         mbar_expect_tx(&full[s], nw + ny);
         bulk_g2s(wst(s), (const uint8_t*)p.W + t * p.tile_elems * wb, nw, &full[s]);
@@ -941,7 +942,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       uint32_t ph = 0;
       for (int64_t it = 0; it < n_it; ++it) {
         if (!wait1(&wdone[s], ph, s_abort, p.err)) break;
-        const int64_t t = blockIdx.x + it * G;
+        const int64_t t = tb + it * G;
         bulk_s2g((uint8_t*)p.W + t * p.tile_elems * wb, wst(s), tile_wbytes(t));
         bulk_commit();
         if (loaded < n_it) {
@@ -1037,7 +1038,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
     auto build = [&](int64_t it) -> bool {
       const int b = (int)(it & 1), s = (int)(it % ns);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
-      const int64_t t = blockIdx.x + it * G;
+      const int64_t t = tb + it * G;
       if (!waitw(&full[s], (uint32_t)((it / ns) & 1), s_abort, p.err)) return false;
       if (!waitw(&b1empty[b], par ^ 1u, s_abort, p.err)) return false;
       // B1: rows (j_b, re/im), K = (slab, j_a, re/im), entries [[Yr, -Yi], [Yi, Yr]];
@@ -1138,11 +1139,11 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       }
     };
     if (n_it > 0) {
-      cur_e0 = p.tile_off[blockIdx.x];
-      cur_e1 = p.tile_off[blockIdx.x + 1];
+      cur_e0 = p.tile_off[tb];
+      cur_e1 = p.tile_off[tb + 1];
       if (n_it > 1) {
-        nx_e0 = p.tile_off[blockIdx.x + G];
-        nx_e1 = p.tile_off[blockIdx.x + G + 1];
+        nx_e0 = p.tile_off[tb + G];
+        nx_e1 = p.tile_off[tb + G + 1];
       }
       load_entries(cur_e0, cur_e1);
     }
@@ -1162,7 +1163,7 @@ __global__ void __launch_bounds__(R3T, 1) recon_stream_kernel(const R3Args p) {
       }
       const int b = (int)(it & 1);
       const uint32_t par = (uint32_t)((it >> 1) & 1);
-      const int64_t t = blockIdx.x + it * G;
+      const int64_t t = tb + it * G;
       if (it + 2 < n_it) {
         nn_e0 = p.tile_off[t + 2 * G];
         nn_e1 = p.tile_off[t + 2 * G + 1];
@@ -1747,7 +1748,7 @@ cudaError_t tc_step_project(TcPlan& p, const void* grad, float* sp_m, float* sp_
 
 cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, const AdamConst& acore,
                            float decay, float lr, int* d_err, cudaStream_t s, TimerHook hook,
-                           void* hook_ctx) {
+                           void* hook_ctx, bool recon) {
   TcImpl* g = impl_of(p);
   if (!g) return cudaErrorNotReady;
   auto H = [&](int ph, const char* name) {
@@ -1800,6 +1801,28 @@ cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, con
     cur = out;
     which ^= 1;
   }
+  if (!recon) return cudaSuccess;
+  return tc_recon(p, w, 0, g->n_tiles, decay, lr, d_err, s, hook, hook_ctx);
+}
+
+int64_t tc_tiles(TcPlan& p) {
+  TcImpl* g = impl_of(p);
+  return g ? g->n_tiles : 0;
+}
+int64_t tc_tile_elems(TcPlan& p) {
+  TcImpl* g = impl_of(p);
+  return g ? g->tile_elems : 0;
+}
+
+cudaError_t tc_recon(TcPlan& p, void* w, int64_t tile0, int64_t tiles, float decay, float lr, int* d_err,
+                     cudaStream_t s, TimerHook hook, void* hook_ctx) {
+  TcImpl* g = impl_of(p);
+  if (!g) return cudaErrorNotReady;
+  if (tile0 < 0 || tiles < 1 || tile0 + tiles > g->n_tiles) return cudaErrorInvalidValue;
+  auto H = [&](int ph, const char* name) {
+    if (hook) hook(hook_ctx, ph, name, s);
+  };
+  cudaError_t e = cudaSuccess;
   // ---- reconstruction stream over W
   R3Args& r = g->r3;
   const int wbytes = g->wdt == TGD_C64 ? 8 : 4;
@@ -1824,6 +1847,8 @@ cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, con
   r.N = p.N;
   r.n_slabs = g->n_slabs;
   r.n_tiles = g->n_tiles;
+  r.tile0 = tile0;
+  r.tiles = tiles;
   r.tile_elems = g->tile_elems;
   r.Ia = g->Ia;
   r.Ib = g->Ib;
@@ -1844,7 +1869,7 @@ cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, con
   r.lr = lr;
   r.err = d_err;
   const size_t r3_launch_smem = std::max(g->r3_smem, ONE_CTA_SMEM);
-  const unsigned r3_grid = (unsigned)std::min<int64_t>(g->n_tiles, g->num_sms);
+  const unsigned r3_grid = (unsigned)std::min<int64_t>(tiles, g->num_sms);
   auto launch_r3 = [&](auto kern) -> cudaError_t {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r3_launch_smem);
     if (err != cudaSuccess) return err;

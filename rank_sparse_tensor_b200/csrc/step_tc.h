@@ -41,9 +41,17 @@ cudaError_t tc_step(TcPlan& p, const void* g, void* w, float* sp_m, float* sp_v,
 // AdamW, the expansion and the weight update.
 cudaError_t tc_step_project(TcPlan& p, const void* grad, float* sp_m, float* sp_v, const AdamConst& asp,
                             int* d_err, cudaStream_t s, TimerHook hook, void* hook_ctx);
+// recon false: stop before the reconstruction stream (run it with tc_recon).
 cudaError_t tc_step_finish(TcPlan& p, void* w, float* core_m, float* core_v, const AdamConst& acore,
                            float decay, float lr, int* d_err, cudaStream_t s, TimerHook hook,
-                           void* hook_ctx);
+                           void* hook_ctx, bool recon = true);
+// The reconstruction stream alone, over tiles [tile0, tile0 + tiles) of the
+// weights (tile_elems elements each, the last one possibly partial), after
+// tc_step_finish's earlier stages; tc_step_finish runs it over all tiles.
+cudaError_t tc_recon(TcPlan& p, void* w, int64_t tile0, int64_t tiles, float decay, float lr, int* d_err,
+                     cudaStream_t s, TimerHook hook, void* hook_ctx);
+int64_t tc_tiles(TcPlan& p);
+int64_t tc_tile_elems(TcPlan& p);
 float* tc_core(TcPlan& p);
 // Core moments are stored in the path's internal layout; these convert
 // to/from the canonical row-major r_1 x ... x r_d layout (host buffers).
