@@ -164,7 +164,10 @@ TGD_API tgd_status tgd_refresh(tgd_handle h, const void* grad, void* stream);
  *  and weight (host, N elements) to the device, steps, copies weight back.
  *  Synchronises the stream before returning, then returns any device-side
  *  error recorded since the last check (TIMEOUT) as tgd_sync does. Lazily
- *  allocates device staging for both tensors on first use. */
+ *  allocates device staging for both tensors on first use. On the tensor-core
+ *  path the weights move in chunks of tiles on two copy streams of the
+ *  handle's own, overlapped with the reconstruction of earlier chunks; pinned
+ *  host buffers let those copies run asynchronously. */
 TGD_API tgd_status tgd_step_host(tgd_handle h, const void* grad_host, void* weight_host, void* stream);
 
 /* Waits for the handle's work on `stream` and returns any device-side error
