@@ -1415,10 +1415,11 @@ static cudaError_t rows_tensor_map(CUtensorMap* map, const void* g, int es, cons
 // mask words beside it (cp.async), Omega's entries are zeroed in shared
 // memory, and thread (tile pair, column lane) accumulates the 4 x 4 block
 // (ti <= tj) of sum_c x_i(c) conj(x_j(c)) over its columns c = lane, lane +
-// 16, ... of the chunk. At the end the 16 column lanes of a pair are summed
-// by shuffles and the CTA writes its whole I_n x I_n partial (the lower
-// blocks as conjugates), which the fixed-order fp64 reduction then sums.
-constexpr int SG_CL = 16;      // column lanes per tile pair
+// CL, ... of the chunk (CL = 16 column lanes a pair up to I_n = 16, 8 above,
+// so that two CTAs fit an SM). At the end the column lanes of a pair are
+// summed by shuffles and the CTA writes its whole I_n x I_n partial (the
+// lower blocks as conjugates), which the fixed-order fp64 reduction sums.
+constexpr int SG_CL = 16;      // column lanes per tile pair, at most
 constexpr int SG_MAXI = 32;    // I_n at most
 constexpr int SG_MAXT = 36 * SG_CL;  // threads: tile pairs of I_n = 32 (8 x 9 / 2) x lanes
 constexpr int SG_CHUNK = 32768;      // bytes of a chunk, at most (two in flight)
@@ -1428,6 +1429,7 @@ struct SmallGramArgs {
   const uint32_t* bits;
   int64_t A, B;        // slabs, columns per slab row
   int I, IP, ntp;      // rows, 4-row tiles, tile pairs
+  int cl;              // column lanes per tile pair (8 or 16)
   int spc;             // slabs per chunk
   int64_t nchunk, cpc; // chunks, chunks per CTA
   int bulk;            // whole chunks by bulk copy (aligned tensor, chunk bytes % 16 == 0)
@@ -1450,7 +1452,8 @@ __global__ void __launch_bounds__(SG_MAXT) gram_small_kernel(const SmallGramArgs
   auto xbuf = [&](int b) { return sg_smem + (size_t)b * (xbytes + mbytes); };
   auto mwb = [&](int b) { return (uint32_t*)(sg_smem + (size_t)b * (xbytes + mbytes) + xbytes); };
   // this thread's tile pair (ti <= tj) and column lane
-  const int pi = tid / SG_CL, lc = tid - pi * SG_CL;
+  const int CL = p.cl;
+  const int pi = tid / CL, lc = tid - pi * CL;
   int ti = 0, rem = pi;
   while (rem >= p.IP - ti) {
     rem -= p.IP - ti;
@@ -1560,8 +1563,8 @@ __global__ void __launch_bounds__(SG_MAXT) gram_small_kernel(const SmallGramArgs
     if (active) {
       const int64_t ncol = (int64_t)nsl * p.B;
       int64_t al = lc / p.B, bb = lc - al * p.B;
-      const int64_t dA = SG_CL / p.B, dB = SG_CL - dA * p.B;  // a step of SG_CL columns
-      for (int64_t c = lc; c < ncol; c += SG_CL) {
+      const int64_t dA = CL / p.B, dB = CL - dA * p.B;  // a step of CL columns
+      for (int64_t c = lc; c < ncol; c += CL) {
         const int64_t base = al * IB + bb;
         float2 xa[4], xc[4];
 #pragma unroll
@@ -1606,7 +1609,8 @@ __global__ void __launch_bounds__(SG_MAXT) gram_small_kernel(const SmallGramArgs
 #pragma unroll
     for (int v = 0; v < 4; ++v)
 #pragma unroll
-      for (int o = SG_CL / 2; o; o >>= 1) {
+      for (int o = 8; o; o >>= 1) {
+        if (o >= CL) continue;
         acc[u][v].x += __shfl_xor_sync(0xffffffffu, acc[u][v].x, o);
         acc[u][v].y += __shfl_xor_sync(0xffffffffu, acc[u][v].y, o);
       }
@@ -1652,10 +1656,11 @@ bool small_gram_plan(int nd, const int64_t* dims, int n, int dt, bool aligned16,
   a.I = I;
   a.IP = (I + 3) / 4;
   a.ntp = a.IP * (a.IP + 1) / 2;
+  a.cl = a.IP > 4 ? 8 : SG_CL;
   a.spc = spc;
   a.nchunk = ceil_div(A, (int64_t)spc);
   a.bulk = aligned16 && (slab * spc) % 16 == 0;
-  threads = a.ntp * SG_CL;
+  threads = a.ntp * a.cl;
   const int64_t chunk_elems = (int64_t)spc * I * B;
   smem = 2 * ((size_t)((chunk_elems * es + 127) / 128) * 128 + (size_t)((4 * (chunk_elems / 32 + 2) + 127) / 128) * 128);
   // CTAs: as many as the SMs hold (threads and shared memory), each at least
