@@ -792,7 +792,7 @@ __host__ __device__ inline Inner32Layout ffma32_layout(int64_t K, int64_t J, int
                                                        int nb) {
   Inner32Layout L;
   L.bimg = 0;  // M
-  L.xs = al128u((uint32_t)(K * J * esz));
+  L.xs = al128u((uint32_t)(K * ((J + 7) / 8 * 8) * esz));  // M, rows padded to 8 outputs
   L.xs_size = al128u((uint32_t)(G32T * K * esz));
   L.os = L.xs + nb * L.xs_size;
   L.os_size = al128u((uint32_t)(G32T * J * esz));
@@ -823,15 +823,17 @@ __global__ void __launch_bounds__(G32T) inner32_ffma_kernel(const MG32Args p, co
     for (int i = 0; i < I32_NB_MAX; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
-  // M from U (I x ur, complex pairs or reals)
-  for (int e = tid; e < K * J; e += G32T) {
-    const int k = e / J, j = e - k * J;
+  // M from U (I x ur, complex pairs or reals), rows of Jp (J rounded up to
+  // 8) outputs, zero padded: eight outputs of a row are 16-byte aligned
+  const int Jp = (J + 7) / 8 * 8;
+  for (int e = tid; e < K * Jp; e += G32T) {
+    const int k = e / Jp, j = e - k * Jp;
     const int64_t ui = p.ukind == 0 ? (int64_t)k * p.ur + j : (int64_t)j * p.ur + k;
     if (CPLX) {
-      const float2 u = ((const float2*)p.Uf)[ui];
+      const float2 u = j < J ? ((const float2*)p.Uf)[ui] : make_float2(0.f, 0.f);
       ((float2*)(smem + L.bimg))[e] = make_float2(u.x, p.ukind == 0 ? -u.y : u.y);
     } else {
-      ((float*)(smem + L.bimg))[e] = p.Uf[2 * ui];
+      ((float*)(smem + L.bimg))[e] = j < J ? p.Uf[2 * ui] : 0.f;
     }
   }
   __syncthreads();
@@ -935,22 +937,41 @@ __global__ void __launch_bounds__(G32T) inner32_ffma_kernel(const MG32Args p, co
             }
           }
         }
+        // the block's eight outputs together: per K entry, one row of M
+        // (four 16-byte loads) and eight independent accumulations
+        float ar[8], ai[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ar[u] = ai[u] = 0.f;
+#pragma unroll
+        for (int i = 0; i < F32_KMAX; ++i) {
+          if (i >= K) break;
+          if (CPLX) {
+            const float4* mr = (const float4*)(M2 + i * Jp + j0);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float4 m = mr[h];
+              ar[2 * h] = __fmaf_rn(v[i].x, m.x, __fmaf_rn(-v[i].y, m.y, ar[2 * h]));
+              ai[2 * h] = __fmaf_rn(v[i].x, m.y, __fmaf_rn(v[i].y, m.x, ai[2 * h]));
+              ar[2 * h + 1] = __fmaf_rn(v[i].x, m.z, __fmaf_rn(-v[i].y, m.w, ar[2 * h + 1]));
+              ai[2 * h + 1] = __fmaf_rn(v[i].x, m.w, __fmaf_rn(v[i].y, m.z, ai[2 * h + 1]));
+            }
+          } else {
+            const float4* mr = (const float4*)(M1 + i * Jp + j0);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 m = mr[h];
+              ar[4 * h] = __fmaf_rn(v[i].x, m.x, ar[4 * h]);
+              ar[4 * h + 1] = __fmaf_rn(v[i].x, m.y, ar[4 * h + 1]);
+              ar[4 * h + 2] = __fmaf_rn(v[i].x, m.z, ar[4 * h + 2]);
+              ar[4 * h + 3] = __fmaf_rn(v[i].x, m.w, ar[4 * h + 3]);
+            }
+          }
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int j = j0 + u;
           if (j >= J) break;
-          float dr = 0.f, di = 0.f;
-#pragma unroll
-          for (int i = 0; i < F32_KMAX; ++i) {
-            if (i >= K) break;
-            if (CPLX) {
-              const float2 m = M2[i * J + j];
-              dr = __fmaf_rn(v[i].x, m.x, __fmaf_rn(-v[i].y, m.y, dr));
-              di = __fmaf_rn(v[i].x, m.y, __fmaf_rn(v[i].y, m.x, di));
-            } else {
-              dr = __fmaf_rn(v[i].x, M1[i * J + j], dr);
-            }
-          }
+          float dr = ar[u], di = ai[u];
           const int64_t so = (int64_t)tid * p.J + j;
           if (!WUPD) {
             if (CPLX)
