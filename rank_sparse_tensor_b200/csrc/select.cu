@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(1024) block_offsets_kernel(const int* blk_lt, 
 // keys, go through one block scan each, and every key's rank follows from its
 // warp's ballot. Ties go to the lower index.
 template <class KeyF, int DT>
-__global__ void __launch_bounds__(CT, 4) write_kernel(KeyF kf, const void* g, int64_t n,
+__global__ void __launch_bounds__(CT, 6) write_kernel(KeyF kf, const void* g, int64_t n,
                                                    const SelState* st, const long long* out_off,
                                                    const long long* eq_before, int64_t* out_idx,
                                                    float* out_val) {
