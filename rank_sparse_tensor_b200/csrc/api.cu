@@ -57,7 +57,6 @@ struct tgd_ctx {
   double* eig_work[TGD_MAX_NDIM] = {};
   double* eig_v[TGD_MAX_NDIM] = {};  // each mode's eigenvectors of the last refresh
   bool eig_warm = false;             // eig_v holds them (every projected mode <= 128)
-  EigJob* jobs_dev = nullptr;
   std::vector<EigJob> jobs;
   // the refresh runs each mode's eigensolve on one of two side streams beside
   // the next modes' Grams (fork and join by events)
@@ -361,7 +360,7 @@ tgd_status do_refresh_lowrank_first(tgd_ctx* h, const void* g, cudaStream_t s) {
   }
   {
     TIMED(h, s, "eigh");
-    TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+    TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), s));
     h->eig_warm = eig_keeps_vectors(h);
   }
   for (int n = 0; n < h->d; ++n)
@@ -474,7 +473,7 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
       TGD_CUDA(h, cudaEventRecord(h->ev_fork, s));
       TGD_CUDA(h, cudaStreamWaitEvent(ss, h->ev_fork, 0));
       TIMED(h, ss, "eigh");
-      TGD_CUDA(h, batched_eigh(&h->jobs.back(), 1, h->jobs_dev + (h->jobs.size() - 1), ss));
+      TGD_CUDA(h, batched_eigh(&h->jobs.back(), 1, ss));
     }
   }
   if (overlap) {
@@ -485,10 +484,10 @@ tgd_status do_refresh(tgd_ctx* h, const void* g, cudaStream_t s) {
     h->eig_warm = eig_keeps_vectors(h);
   } else if (h->opt.basis == 1) {
     TIMED(h, s, "dct_select");
-    TGD_CUDA(h, batched_dct_select(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+    TGD_CUDA(h, batched_dct_select(h->jobs.data(), (int)h->jobs.size(), s));
   } else {
     TIMED(h, s, "eigh");
-    TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), h->jobs_dev, s));
+    TGD_CUDA(h, batched_eigh(h->jobs.data(), (int)h->jobs.size(), s));
     h->eig_warm = eig_keeps_vectors(h);
   }
   tgd_status st = rebuild_derived(h, s);
@@ -770,7 +769,6 @@ tgd_status tgd_create(tgd_handle* out, int ndim, const int64_t* shape, const int
       ok &= dalloc_t(h, &h->eig_v[n], (size_t)2 * shape[n] * shape[n]);
     }
   ok &= dalloc(h, (void**)&h->gram_part, gp);
-  ok &= dalloc_t(h, &h->jobs_dev, TGD_MAX_NDIM);
   ok &= dalloc_t(h, &h->d_err, 1);
   if (ok && h->path == TGD_PATH_GENERIC) {
     for (int n = 0; n < ndim; ++n)

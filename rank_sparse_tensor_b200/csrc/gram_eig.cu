@@ -1008,8 +1008,8 @@ constexpr int ES_MAXN = MAXN;
 constexpr double JAC_TOL = 1e-18;
 constexpr int ES_SMEM_MAXN = 64;
 
-__global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
-  const EigJob J = jobs[blockIdx.x];
+__global__ void __launch_bounds__(ET) eig_small_kernel(const EigJobs jobs) {
+  const EigJob J = jobs.j[blockIdx.x];
   const int n = J.n;
   if (n > ES_MAXN) return;
   const int NP = n + 1 + (n & 1);  // odd row pitch
@@ -1309,8 +1309,8 @@ __global__ void __launch_bounds__(ET) eig_small_kernel(const EigJob* jobs) {
 // alignment (ties to the lower column) and the first r written to U.
 constexpr int DCT_MAXN = 256;
 
-__global__ void __launch_bounds__(DCT_MAXN) dct_select_kernel(const EigJob* jobs) {
-  const EigJob J = jobs[blockIdx.x];
+__global__ void __launch_bounds__(DCT_MAXN) dct_select_kernel(const EigJobs jobs) {
+  const EigJob J = jobs.j[blockIdx.x];
   const int n = J.n;
   __shared__ double score[DCT_MAXN];
   __shared__ int col_of_rank[DCT_MAXN];
@@ -1347,13 +1347,15 @@ __global__ void __launch_bounds__(DCT_MAXN) dct_select_kernel(const EigJob* jobs
 
 }  // namespace
 
-cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
-  for (int j = 0; j < njobs; ++j)
+  if (njobs > TGD_MAX_NDIM) return cudaErrorInvalidValue;
+  EigJobs jobs{};
+  for (int j = 0; j < njobs; ++j) {
     if (jobs_host[j].n > DCT_MAXN || jobs_host[j].r > jobs_host[j].n) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return e;
-  dct_select_kernel<<<njobs, DCT_MAXN, 0, s>>>(jobs_dev);
+    jobs.j[j] = jobs_host[j];
+  }
+  dct_select_kernel<<<njobs, DCT_MAXN, 0, s>>>(jobs);
   return cudaGetLastError();
 }
 
@@ -1817,20 +1819,21 @@ cudaError_t mode_gram(const void* g, int dt, const uint32_t* bits, int nd, const
 // (Jacobi scratch: A, Vt and W of n x (n + 2) complex each)
 size_t eig_work_doubles(int n) { return (size_t)6 * n * (n + 2); }
 
-cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s) {
+cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, cudaStream_t s) {
   if (njobs <= 0) return cudaSuccess;
+  if (njobs > TGD_MAX_NDIM) return cudaErrorInvalidValue;
+  EigJobs jobs{};
   size_t ssmem = 16;
   for (int j = 0; j < njobs; ++j) {
     const int n = jobs_host[j].n;
     if (n < 1 || n > ES_MAXN || jobs_host[j].r > n) return cudaErrorInvalidValue;
     const size_t np = (size_t)n + 1 + (n & 1);
     if (n <= ES_SMEM_MAXN) ssmem = std::max(ssmem, 2 * sizeof(double2) * (size_t)n * np);
+    jobs.j[j] = jobs_host[j];
   }
   cudaError_t e = cudaFuncSetAttribute(eig_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
   if (e != cudaSuccess) return e;
-  e = cudaMemcpyAsync(jobs_dev, jobs_host, sizeof(EigJob) * njobs, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return e;
-  eig_small_kernel<<<njobs, ET, ssmem, s>>>(jobs_dev);
+  eig_small_kernel<<<njobs, ET, ssmem, s>>>(jobs);
   return cudaGetLastError();
 }
 

@@ -6,6 +6,8 @@
 
 #include <string>
 
+#include "../../include/tgd.h"
+
 namespace tgd {
 
 struct AdamConst;
@@ -46,11 +48,16 @@ struct EigJob {
   int n, r;
   int warm;            // 1: start from vprev, 0: from the identity
 };
+// The jobs of one batched launch, passed to the kernel by value (no copy
+// from host memory on the stream).
+struct EigJobs {
+  EigJob j[TGD_MAX_NDIM];
+};
 size_t eig_work_doubles(int n);
-cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
+cudaError_t batched_eigh(const EigJob* jobs_host, int njobs, cudaStream_t s);
 // DCT basis instead of eigenvectors: U = the r columns of the orthonormal DCT
 // matrix most aligned with the Gram (evals: the alignments, descending).
-cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, EigJob* jobs_dev, cudaStream_t s);
+cudaError_t batched_dct_select(const EigJob* jobs_host, int njobs, cudaStream_t s);
 
 // ---- step_generic.cu: CUDA-core path of the step
 // L (optional, fp32 like the chain buffers): Adam on G[Omega] - L[Omega].
